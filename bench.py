@@ -1,0 +1,521 @@
+#!/usr/bin/env python
+"""Throughput of the NVFP4 routed-expert MoE block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole chain over one batch: the activation global
+scale (nvfp4_global_scale) and nvfp4_moe_forward (route, quantise+permute,
+L1 gate_up GEMM with fused SiLU*up re-quantisation, L2 down GEMM, combine).
+Headline workload: the 384-expert prefill MoE (T=4096, top-6, H=7168,
+I=3072, Zipf-skewed routing with empty experts) -> tokens/s, TFLOP/s and the
+fraction of the FP4 peak; the 48-expert decode MoE (T=64) is measured in the
+same run -> GB/s and the fraction of HBM bandwidth.  Inputs are seeded
+synthetic data of those shapes (nvfp4_moe_expert_topk_b200.workloads).
+
+With torchrun (N > 1) every rank runs its own replica of the workload (data
+parallel over token batches, weights replicated, no collective on the data
+path); timing is the max over ranks; value = all ranks' tokens / that time.
+
+--impl reference times the CPU oracle (oracle/, plain C) on this host's
+cores on a bounded sample of the same workload (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from nvfp4_moe_expert_topk_b200 import (nvfp4_global_scale, nvfp4_moe_calibrate, nvfp4_moe_forward,  # noqa: E402
+                                        nvfp4_moe_forward_timed, nvfp4_moe_get_error)
+from nvfp4_moe_expert_topk_b200 import prep  # noqa: E402
+from nvfp4_moe_expert_topk_b200 import workloads as W  # noqa: E402
+
+FP4_NOMINAL_TFLOPS = 9000.0            # dense FP4, NVIDIA public B200 figure
+BF16_TO_FP4_NOMINAL_RATIO = 4.0        # 9 / 2.25 PFLOP/s dense
+STAGES = ["global_scale", "route", "quantize_permute", "l1_gate_up_swiglu_quant", "l2_down", "combine"]
+KERNELS_PER_STEP = 7                   # amax + finalize (global scale), route, quantise, L1, L2, combine
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SOURCES = ["gemm.cu", "ptx.cuh", "quant.cuh", "internal.h"]
+
+
+# ---------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def gemm_source_sha():
+    h = hashlib.sha256()
+    for name in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "nvfp4_moe_expert_topk_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current GEMM sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    rows = {}
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                key, _, val = line.partition(":")
+                rows[key.strip()] = val.strip()
+    if rows.get("source_sha") != gemm_source_sha():
+        return None
+    v = rows.get(f"{workload}.{kernel}.dram_bytes_per_launch")
+    return float(v) if v else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.device = device
+        self.proc = None
+        self.samples = []
+
+    def _id(self):
+        try:
+            return "GPU-" + str(torch.cuda.get_device_properties(self.device).uuid)
+        except Exception:
+            return None
+
+    def start(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
+        gid = self._id()
+        if gid:
+            cmd[1:1] = ["-i", gid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.seek(0)
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+        self.file.close()
+        os.unlink(self.file.name)
+        self.proc = None
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- workloads
+class Workload:
+    """A MoE config resident on the device: NVFP4 weights, one batch, inter_gs
+    from the library's own warmup (nvfp4_moe_calibrate on the warmup batch)."""
+
+    def __init__(self, cfg, dev):
+        self.cfg = cfg
+        self.dev = dev
+        self.weights = prep.MoeWeights.synthetic(cfg, dev)
+        x, ids, w = W.batch(cfg)
+        self.x_cpu, self.ids_cpu, self.w_cpu = x, ids, w
+        self.x, self.ids, self.w = x.to(dev), ids.to(dev), w.to(dev)
+        self.x_gs = torch.empty(1, dtype=torch.float32, device=dev)
+        self.ws = prep.workspace(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I, dev)
+        self.out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
+        xw, idw, ww = W.batch(cfg, warmup=True)
+        xw = xw.to(dev)
+        gsw = torch.empty(1, dtype=torch.float32, device=dev)
+        nvfp4_global_scale(xw, gsw)
+        wsw = prep.workspace(cfg.warmup_T, cfg.k, cfg.E, cfg.H, cfg.I, dev)
+        self.inter_gs = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+        nvfp4_moe_calibrate(xw, idw.to(dev), ww.to(dev), gsw, **self.weights.args(), inter_gs_out=self.inter_gs,
+                            workspace=wsw)
+        del wsw
+        counts = np.bincount(ids.numpy().reshape(-1), minlength=cfg.E)
+        self.rows = int(counts.sum())
+        self.nonempty = int((counts > 0).sum())
+
+    def step(self, events=None):
+        nvfp4_global_scale(self.x, self.x_gs)
+        if events is None:
+            nvfp4_moe_forward(self.x, self.ids, self.w, self.x_gs, **self.weights.args(), inter_gs=self.inter_gs,
+                              out=self.out, workspace=self.ws)
+        else:
+            nvfp4_moe_forward_timed(self.x, self.ids, self.w, self.x_gs, **self.weights.args(),
+                                    inter_gs=self.inter_gs, out=self.out, workspace=self.ws, events=events)
+
+    # algorithmic work (real rows only; weights of non-empty experts once)
+    def flops(self):
+        c = self.cfg
+        return 2.0 * self.rows * 3 * c.H * c.I
+
+    def kernel_bytes(self):
+        c = self.cfg
+        fp4 = 0.5 + 1.0 / 16                # code + scale bytes per element
+        R, T, H, I, k = self.rows, c.T, c.H, c.I, c.k
+        w13 = self.nonempty * 2 * I * H * fp4
+        w2 = self.nonempty * H * I * fp4
+        return {
+            "global_scale": T * H * 2.0,
+            "route": T * k * 4.0 * 2 + c.E * 16.0,
+            "quantize_permute": T * H * 2.0 + R * H * fp4 + T * k * 4.0,
+            "l1_gate_up_swiglu_quant": w13 + R * H * fp4 + R * I * fp4,
+            "l2_down": w2 + R * I * fp4 + R * H * 2.0,
+            "combine": R * H * 2.0 + T * H * 2.0 + T * k * 12.0,
+        }
+
+    def step_bytes(self):
+        """Algorithmic bytes of one step: non-empty experts' weights + x in + out + ids/weights."""
+        c = self.cfg
+        fp4 = 0.5 + 1.0 / 16
+        return self.nonempty * 3 * c.H * c.I * fp4 + 2 * c.T * c.H * 2.0 + c.T * c.k * 8.0
+
+
+def time_steps(wl, steps, warmup, world, timed_events=True):
+    """Device time of `steps` steps (events on the launching stream, barrier +
+    synchronize on both sides), and per-stage mean durations."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        wl.step()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)] if timed_events else None
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        if ev is not None:
+            ev[i][0].record(stream)
+            wl.step(events=ev[i][1:])
+        else:
+            wl.step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = t0.elapsed_time(t1)
+    stage_ms = None
+    if ev is not None:
+        stage_ms = {name: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in ev])) for j, name in enumerate(STAGES)}
+    return max_over_ranks(world, ms), stage_ms
+
+
+def time_e2e(wl, steps, warmup, world):
+    """Same step through the public API from pinned host buffers: H2D of x,
+    ids and weights, the step, D2H of the output, all inside the timed region."""
+    stream = torch.cuda.current_stream()
+    hx = wl.x_cpu.pin_memory()
+    hids = wl.ids_cpu.pin_memory()
+    hw = wl.w_cpu.pin_memory()
+    hout = torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True)
+
+    def one():
+        wl.x.copy_(hx, non_blocking=True)
+        wl.ids.copy_(hids, non_blocking=True)
+        wl.w.copy_(hw, non_blocking=True)
+        wl.step()
+        hout.copy_(wl.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        one()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(world, t0.elapsed_time(t1))
+    h2d = hx.numel() * hx.element_size() + hids.numel() * 4 + hw.numel() * 4
+    d2h = hout.numel() * hout.element_size()
+    if not torch.isfinite(hout.float()).all():
+        raise RuntimeError("non-finite output in the end-to-end run")
+    return ms, h2d, d2h
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(cfg, tokens, dev, inter_gs_dev):
+    """Oracle inputs for a token sample of a workload: the sampled tokens'
+    experts regenerated from their seeds and quantised by the oracle."""
+    import oracle as O
+    x, ids, w = W.batch(cfg)
+    xb = W.bf16_bits(x)
+    x_gs = O.global_scale_bf16(xb)
+    sub_ids = ids.numpy()[tokens]
+    experts = sorted(set(sub_ids.reshape(-1).tolist()))
+    lut = {e: i for i, e in enumerate(experts)}
+    H, I, n = cfg.H, cfg.I, len(experts)
+    w13c = np.empty((n, 2 * I, H // 2), np.uint8)
+    w13s = np.empty((n, 2 * I, H // 16), np.uint8)
+    w13g = np.empty((n, 2), np.float32)
+    w2c = np.empty((n, H, I // 2), np.uint8)
+    w2s = np.empty((n, H, I // 16), np.uint8)
+    w2g = np.empty(n, np.float32)
+    for i, e in enumerate(experts):
+        b13 = W.bf16_bits(W.expert_w13(cfg, e, dev))
+        for h in range(2):
+            part = b13[h * I:(h + 1) * I]
+            w13g[i, h] = O.global_scale_bf16(part)
+            w13c[i, h * I:(h + 1) * I], w13s[i, h * I:(h + 1) * I] = O.quantize_bf16(part, w13g[i, h])
+        b2 = W.bf16_bits(W.expert_w2(cfg, e, dev))
+        w2g[i] = O.global_scale_bf16(b2)
+        w2c[i], w2s[i] = O.quantize_bf16(b2, w2g[i])
+    inter = inter_gs_dev.cpu().numpy()[experts]
+    remap = np.vectorize(lambda e: lut[e])(sub_ids).astype(np.int32)
+    return dict(x_bits=xb[tokens], topk_ids=remap, topk_weights=w.numpy()[tokens], x_gs=x_gs,
+                w13_codes=w13c, w13_scales=w13s, w13_gs=w13g, w2_codes=w2c, w2_scales=w2s, w2_gs=w2g,
+                inter_gs=inter)
+
+
+def run_oracle_tokens(sample, token_idx):
+    import oracle as O
+    sel = np.atleast_1d(token_idx)
+    kw = dict(sample)
+    kw["x_bits"] = sample["x_bits"][sel]
+    kw["topk_ids"] = sample["topk_ids"][sel]
+    kw["topk_weights"] = sample["topk_weights"][sel]
+    t0 = time.perf_counter()
+    O.moe_forward(**kw)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(cfg, dev, inter_gs_dev, n_tokens=8):
+    import oracle as O
+    tokens = np.sort(np.random.default_rng(123).choice(cfg.T, n_tokens, replace=False))
+    sample = oracle_sample(cfg, tokens, dev, inter_gs_dev)
+    secs = run_oracle_tokens(sample, np.arange(n_tokens))
+    return {"value": n_tokens / secs, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"{n_tokens} tokens of the {cfg.name} batch (their {sample['w13_codes'].shape[0]} experts), "
+                      f"{secs:.1f} s of CPU work; weight generation and quantisation excluded"}
+
+
+# ---------------------------------------------------------------- arms
+def config_block(cfg, world):
+    return {"workload": f"{cfg.name}_moe_E{cfg.E}_k{cfg.k}_T{cfg.T}_H{cfg.H}_I{cfg.I}"
+                        + ("_zipf1.1_16empty" if cfg.routing == "zipf" else ""),
+            "experts": cfg.E, "top_k": cfg.k, "tokens_per_gpu": cfg.T, "hidden": cfg.H, "intermediate": cfg.I,
+            "global_batch": cfg.T * world, "routing": cfg.routing, "outlier_channels": cfg.outliers,
+            "weights": "NVFP4 (E2M1 + E4M3 per 16 + fp32 per tensor) from seeded N(0,0.02) bf16",
+            "l2": "no flush: every step streams >= 1.7 GB of weights (> 126 MB L2)",
+            "parallelism": "replicas" if world == 1 else f"dp{world} replicas (no data-path collective)"}
+
+
+def run_ours(args):
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    steps, warmup = args.steps, max(3, args.warmup)
+
+    pre = Workload(W.MOE_CONFIGS["prefill"], dev)
+    dec = Workload(W.MOE_CONFIGS["decode"], dev)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(dev)
+    clocks.start()
+    ms_pre, stages_pre = time_steps(pre, steps, warmup, world)
+    ms_dec, stages_dec = time_steps(dec, steps, warmup, world)
+    clocks.stop()
+    for wl in (pre, dec):
+        err = nvfp4_moe_get_error(wl.ws)
+        if err != 0:
+            raise RuntimeError(f"device error word {err} after the {wl.cfg.name} run")
+        if not torch.isfinite(wl.out.float()).all():
+            raise RuntimeError(f"non-finite output in the {wl.cfg.name} run")
+    e2e_ms, h2d, d2h = time_e2e(pre, steps, warmup, world)
+
+    t_step = ms_pre / steps / 1e3
+    tokens_s = world * pre.cfg.T / t_step
+    tflops = pre.flops() / t_step / 1e12
+    fp4_measured = peaks["bf16_tflops_sustained"] * BF16_TO_FP4_NOMINAL_RATIO
+    kb = pre.kernel_bytes()
+    dominant = max(STAGES, key=lambda s: stages_pre[s])
+    dom_ms = stages_pre[dominant]
+    achieved = kb[dominant] / (dom_ms / 1e3) / 1e9
+    hbm = peaks["hbm_gbs"]
+    traffic = ncu_traffic(dominant, "prefill")
+
+    t_dec = ms_dec / steps / 1e3
+    dec_gbs = dec.step_bytes() / t_dec / 1e9
+    dec_kb = dec.kernel_bytes()
+    dec_dom = max(STAGES, key=lambda s: stages_dec[s])
+
+    line = {
+        "metric": "moe_prefill_tokens_per_s",
+        "value": tokens_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": ms_pre / steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4",
+        "data": "synthetic",
+        "config": config_block(pre.cfg, world),
+        "tflops": tflops,
+        "fp4_peak_frac": {"of_nominal_9000": tflops / FP4_NOMINAL_TFLOPS,
+                          f"of_{peak_src}_bf16_sustained_x4": tflops / fp4_measured},
+        "hbm_gbs_step": pre.step_bytes() / t_step / 1e9,
+        "hbm_frac_step": pre.step_bytes() / t_step / 1e9 / hbm,
+        "stage_ms": stages_pre,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "peak_source": f"{peak_src} hbm_gbs",
+                     "algorithmic_bytes": kb[dominant], "traffic": traffic},
+        "decode": {
+            "workload": config_block(dec.cfg, world)["workload"],
+            "metric": "moe_decode_GB_per_s", "value": dec_gbs, "unit": "GB/s", "ms_per_step": ms_dec / steps,
+            "hbm_frac": dec_gbs / hbm, "tokens_per_s": world * dec.cfg.T / t_dec,
+            "algorithmic_bytes_per_step": dec.step_bytes(), "stage_ms": stages_dec,
+            "roofline": {"bound": "hbm", "kernel": dec_dom,
+                         "achieved": dec_kb[dec_dom] / (stages_dec[dec_dom] / 1e3) / 1e9, "peak": hbm,
+                         "unit": "GB/s", "frac": dec_kb[dec_dom] / (stages_dec[dec_dom] / 1e3) / 1e9 / hbm,
+                         "traffic": ncu_traffic(dec_dom, "decode")},
+        },
+        "e2e": {"value": world * pre.cfg.T * steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / steps},
+        "gpu_launches": KERNELS_PER_STEP * steps * 2,
+        "clocks": clocks.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(pre.cfg, dev, pre.inter_gs)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The CPU oracle on this host's cores, one token of the prefill batch per
+    step (cycling through a fixed sample), rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle as O
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    cfg = W.MOE_CONFIGS["prefill"]
+    steps, warmup = args.steps, max(3, args.warmup)
+    tokens = np.sort(np.random.default_rng(321).choice(cfg.T, 4, replace=False))
+    # warmup inter_gs is the library's; it only sets the arithmetic's scale, not the work
+    if dev.type == "cuda":
+        inter = Workload.__new__(Workload)
+        inter_gs = _calibrated_inter_gs(cfg, dev)
+    else:
+        inter_gs = torch.full((cfg.E,), 1000.0)
+    sample = oracle_sample(cfg, tokens, dev, inter_gs)
+    for i in range(warmup):
+        run_oracle_tokens(sample, i % len(tokens))
+    total = 0.0
+    for i in range(steps):
+        total += run_oracle_tokens(sample, i % len(tokens))
+    value = steps / total
+    line = {"impl": "reference", "metric": "moe_prefill_tokens_per_s", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": total / steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64",
+            "data": "synthetic", "config": config_block(cfg, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": O.num_threads(), "kind": "oracle",
+                             "sample": f"one token of the prefill batch per step, cycling over {len(tokens)} tokens"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _calibrated_inter_gs(cfg, dev):
+    wts = prep.MoeWeights.synthetic(cfg, dev)
+    xw, idw, ww = W.batch(cfg, warmup=True)
+    xw = xw.to(dev)
+    gs = torch.empty(1, dtype=torch.float32, device=dev)
+    nvfp4_global_scale(xw, gs)
+    ws = prep.workspace(cfg.warmup_T, cfg.k, cfg.E, cfg.H, cfg.I, dev)
+    out = torch.empty(cfg.E, dtype=torch.float32, device=dev)
+    nvfp4_moe_calibrate(xw, idw.to(dev), ww.to(dev), gs, **wts.args(), inter_gs_out=out, workspace=ws)
+    torch.cuda.synchronize()
+    del wts
+    return out.cpu()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

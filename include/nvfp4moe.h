@@ -1,0 +1,187 @@
+/*
+ * nvfp4moe.h -- C ABI of libnvfp4moe.so: the NVFP4 (W4A4) routed-expert MoE
+ * block of a DeepSeek-V4-style layer on one B200 (sm_100a).
+ *
+ * Source of the operations: "nvfp4-megamoe-kernel / CURRENT_BUG.md" (three
+ * snapshots of one page).  Page 1 "Phase 1: CuTeDSL Shared Expert Kernel"
+ * gives the chain L1 gate_up GEMM -> SiLU -> re-quantise -> L2 GEMM with the
+ * gate and up weights stacked; page 1 "Phase 2" gives the dual global scales
+ * of a stacked projection; page 2 "What the quant method does" gives the
+ * global-scale convention; page 3 "Architecture Notes" gives 384 experts,
+ * top-6 and expert intermediate 3072; page 1 "Phase 1" asks for a
+ * cudagraph-safe runner with pre-allocated buffers and warmup global scales.
+ *
+ * Conventions for every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller, unless a
+ *    parameter says "host".  The library allocates no memory, never
+ *    synchronises the device (except nvfp4_moe_get_error) and launches only
+ *    on the given stream (a cudaStream_t passed as void*; NULL = legacy
+ *    default stream).  Nothing is JIT-compiled at run time.
+ *  - Launches are asynchronous: the return code reports argument checks and
+ *    launch errors only.  Faults inside a kernel surface later, as CUDA
+ *    errors on the stream.
+ *  - bf16 tensors are passed as uint16_t bit patterns.
+ *  - NVFP4 tensor = codes + scales + one fp32 global scale gs:
+ *      codes  [rows, cols/2] uint8, row-major; element 2i of a row in the low
+ *             nibble of byte i, element 2i+1 in the high nibble; each nibble is
+ *             an E2M1 value (sign bit 3, magnitudes 0,.5,1,1.5,2,3,4,6).
+ *      scales one E4M3 byte per 16 consecutive elements of a row, in one of
+ *             two layouts:
+ *             NVFP4_SCALES_ROWMAJOR  [rows, cols/16] row-major;
+ *             NVFP4_SCALES_MMA       the tensor-core tile layout: rows padded
+ *             to a multiple of 128, stored as [rows/128][cols/64][512 bytes]
+ *             where byte (r % 32)*16 + ((r % 128)/32)*4 + j of a 512-byte
+ *             atom holds the scale of row r, 16-column block 4*kb + j.
+ *      value  = e2m1(code) * e4m3(scale) / gs.
+ *  - Quantisation of a 16-element block (bit-exact contract):
+ *      a = max|x_i| (fp32); v = (a / 6) * gs; s = E4M3(v) (round to nearest
+ *      even, saturating at 448); r = (s == 0) ? 0 : gs / value(s);
+ *      q_i = E2M1(x_i * r) (round to nearest even, saturating at 6, sign of
+ *      zero kept).  Every fp32 step rounds to nearest.
+ *  - Global scale: gs = 2688 / amax (= 448 * 6 / amax) in fp32; 1 if amax = 0.
+ *  - Inputs must be finite.
+ */
+#ifndef NVFP4MOE_H
+#define NVFP4MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every int-valued entry point. */
+#define NVFP4_OK                       0
+#define NVFP4_ERR_INVALID_ARG         -1  /* null pointer, negative size, bad enum   */
+#define NVFP4_ERR_UNSUPPORTED_SHAPE   -2  /* size outside the documented constraints */
+#define NVFP4_ERR_MISALIGNED          -3  /* pointer or leading dim not 16-B aligned */
+#define NVFP4_ERR_WORKSPACE_TOO_SMALL -4
+#define NVFP4_ERR_CUDA                -5  /* a CUDA runtime or driver call failed   */
+#define NVFP4_ERR_UNSUPPORTED_DEVICE  -6  /* current device is not sm_100           */
+#define NVFP4_ERR_TIMEOUT             -7  /* device error word: a bounded wait gave up */
+#define NVFP4_ERR_BAD_EXPERT_ID       -8  /* device error word: a top-k id >= E      */
+
+#define NVFP4_SCALES_ROWMAJOR 0
+#define NVFP4_SCALES_MMA      1
+
+/* Human-readable name of a status code (static string; never NULL). */
+const char *nvfp4_status_string(int status);
+
+/* Global scale of a bf16 tensor (page 2, "What the quant method does": the
+ * global scale is a multiplier applied before FP4 conversion).
+ * x: [n] bf16; gs_out: device float, receives 2688 / max|x| (1 if all zero).
+ * gs_out is also used as the reduction's scratch word.  n >= 1. */
+int nvfp4_global_scale(const uint16_t *x, int64_t n, float *gs_out, void *stream);
+
+/* Bytes needed for the scales of a [rows, cols] NVFP4 tensor in a layout. */
+int64_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int scale_layout);
+
+/* NVFP4 quantisation of a bf16 matrix (page 3 test table: activation
+ * quantisation; page 1 "Confirmed working": NVFP4 weights).
+ * x: [rows, ldx] bf16, ldx >= cols, ldx % 8 == 0; gs: device float [1];
+ * codes: [rows, cols/2]; scales: see scale_layout (NVFP4_SCALES_MMA needs
+ * cols % 64 == 0 and nvfp4_scales_bytes() bytes; pad rows of the last
+ * 128-row block are not written).  cols % 16 == 0.  x, codes, scales 16-B
+ * aligned. */
+int nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs,
+                   uint8_t *codes, uint8_t *scales, int scale_layout, void *stream);
+
+/* Row-major scales [batch, rows, cols/16] -> NVFP4_SCALES_MMA layout, per
+ * batch entry (weight preparation, page 3 "Next Steps" 2: weight packing).
+ * cols % 64 == 0.  Pad rows of the last 128-row block are written as 0.
+ * out: batch * nvfp4_scales_bytes(rows, cols, NVFP4_SCALES_MMA) bytes. */
+int nvfp4_swizzle_scales(const uint8_t *in, int64_t batch, int64_t rows, int64_t cols,
+                         uint8_t *out, void *stream);
+
+/* Dense NVFP4 GEMM, out[m, n] = bf16( sum_k A[m,k] * B[n,k] ), i.e. the
+ * grouped engine with one group (page 1 "Phase 1": ScaledGroupedGemm with
+ * num_groups=1 is a regular GEMM; page 1 "Phase 2": one NVFP4 GEMM per
+ * attention projection, with two global scales for fused_wqa_wkv).
+ * a_codes [M, K/2], a_scales NVFP4_SCALES_MMA, a_gs device [1];
+ * b_codes [N, K/2], b_scales NVFP4_SCALES_MMA, b_gs device [nseg];
+ * seg_end HOST [nseg]: increasing column ends of the B segments, the last
+ * equal to N, each a multiple of 32; rows of B in segment s use b_gs[s].
+ * out [M, ldo] bf16, ldo >= N, ldo % 8 == 0.
+ * Constraints: M >= 1, N % 128 == 0, K % 64 == 0, 1 <= nseg <= 4. */
+int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs, int64_t M,
+               const uint8_t *b_codes, const uint8_t *b_scales, const float *b_gs,
+               const int64_t *seg_end, int nseg, int64_t N, int64_t K,
+               uint16_t *out, int64_t ldo, void *stream);
+
+/* The routed-expert MoE block (page 1 "Phase 1" chain; page 3
+ * "Architecture Notes" routing).  Shapes: T tokens, hidden H, expert
+ * intermediate I, E experts, top-k.
+ * Constraints: T >= 0, H % 128 == 0, I % 128 == 0, 1 <= E <= 1024,
+ * 1 <= k <= 32, T*k < 2^31.  All pointers 16-B aligned. */
+typedef struct {
+    const uint16_t *x;            /* [T, H] bf16 activations                          */
+    int64_t T, H, I;
+    int32_t E, k;
+    const int32_t *topk_ids;      /* [T, k]; id < 0: slot skipped; id >= E: error word set, slot skipped */
+    const float *topk_weights;    /* [T, k] fp32                                      */
+    const float *x_gs;            /* [1] global scale of x (nvfp4_global_scale, or warmup) */
+    const uint8_t *w13_codes;     /* [E, 2I, H/2]: rows 0..I-1 gate, rows I..2I-1 up   */
+    const uint8_t *w13_scales;    /* NVFP4_SCALES_MMA of [E*2I, H]                     */
+    const float *w13_gs;          /* [E, 2]: global scale of (gate, up) of each expert */
+    const uint8_t *w2_codes;      /* [E, H, I/2]                                       */
+    const uint8_t *w2_scales;     /* NVFP4_SCALES_MMA of [E*H, I]                      */
+    const float *w2_gs;           /* [E]                                               */
+    const float *inter_gs;        /* [E] global scale of h = SiLU(gate)*up, from warmup */
+    uint16_t *out;                /* [T, H] bf16 output                                */
+} nvfp4_moe_args;
+
+/* Workspace bytes nvfp4_moe_forward / nvfp4_moe_calibrate need.  The
+ * workspace is caller-owned device memory; zero it once after allocation
+ * (it holds the sticky device error word). */
+size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
+
+/* out = sum_j topk_weights[t,j] * Expert_{ids[t,j]}(x[t]) with
+ * Expert_e(x) = W2_e . q(SiLU(W13g_e . q(x)) * (W13u_e . q(x))), all GEMMs
+ * in NVFP4 on the tensor cores, q() the NVFP4 quantiser (x with x_gs, h with
+ * inter_gs[e]).  Launches route, quantise+permute, L1 (fused SiLU*up
+ * re-quantise epilogue), L2 and combine on `stream`; no host sync, no
+ * allocation, so the call can be captured in a CUDA graph (make one eager
+ * call per device first: it sets per-kernel attributes). */
+int nvfp4_moe_forward(const nvfp4_moe_args *args, void *workspace, size_t ws_bytes, void *stream);
+
+/* nvfp4_moe_forward with a CUDA event recorded on `stream` before each of
+ * its five kernels (route, quantise+permute, L1, L2, combine) and after the
+ * last: events = 6 cudaEvent_t handles created by the caller.  Otherwise
+ * identical; for per-stage timing. */
+int nvfp4_moe_forward_timed(const nvfp4_moe_args *args, void *workspace, size_t ws_bytes, void *stream,
+                            void *const *events);
+
+/* Warmup (page 1 "Phase 1": warmup-based gs; page 2 "Option A": compute the
+ * scale from a warmup pass): runs the chain up to h on args (a warmup batch;
+ * inter_gs and out are ignored) and writes inter_gs_out[e] = 2688 / max|h|
+ * over expert e's rows; experts without rows get 2688 / (max over experts).
+ * inter_gs_out: device [E]. */
+int nvfp4_moe_calibrate(const nvfp4_moe_args *args, float *inter_gs_out, void *workspace,
+                        size_t ws_bytes, void *stream);
+
+/* Routing step alone, for inspection: counts [E], padded_offsets [E+1]
+ * (expert segments padded to 128 rows), inv [T*k] (padded row of each slot,
+ * -1 if skipped).  Slot f = t*k + j of expert e lands at
+ * padded_offsets[e] + #{f' < f : ids[f'] == e} (a stable counting sort). */
+int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *counts,
+                          int32_t *padded_offsets, int32_t *inv, void *workspace, size_t ws_bytes,
+                          void *stream);
+
+/* Byte offset and size of a workspace region (for inspection and tests).
+ * region: 0 A codes, 1 A scales (MMA layout), 2 h codes, 3 h scales
+ * (MMA layout), 4 y (bf16 [T*k, H], rows in expert-major routing order),
+ * 5 inv, 6 counts, 7 padded offsets. */
+int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, int region,
+                               int64_t *offset, int64_t *bytes);
+
+/* Reads and clears the sticky device error word of a workspace (host
+ * err_host receives NVFP4_OK or a device error code).  Synchronises
+ * `stream`. */
+int nvfp4_moe_get_error(void *workspace, int32_t *err_host, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4MOE_H */

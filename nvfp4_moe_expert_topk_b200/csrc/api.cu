@@ -1,0 +1,554 @@
+// api.cu -- the C ABI of libnvfp4moe.so (declared in include/nvfp4moe.h):
+// argument checks, workspace layout, tensor-map creation and the launch
+// sequence of each entry point.  No allocation, no host synchronisation
+// (except nvfp4_moe_get_error), everything on the caller's stream.
+#include <mutex>
+
+#include "internal.h"
+
+using namespace nvfp4;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int checked = 0;      // 1 ok, -1 unsupported
+    int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Current device must be sm_100 (B200).  Caches the SM count.
+int device_check(int *num_sms)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return NVFP4_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (d.checked == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        d.checked = (major == 10 && minor == 0) ? 1 : -1;
+        d.num_sms = sms;
+    }
+    if (d.checked < 0)
+        return NVFP4_ERR_UNSUPPORTED_DEVICE;
+    if (num_sms)
+        *num_sms = d.num_sms;
+    if (g_encode == nullptr) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return NVFP4_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    return NVFP4_OK;
+}
+
+// 2-D uint8 tensor map over a row-major code matrix [rows, cols_bytes]
+// (row stride cols_bytes), box 128 rows x 128 bytes, 128-byte swizzle; rows
+// and columns outside the matrix read as zero.
+int make_code_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols_bytes)
+{
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols_bytes), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols_bytes)};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15) == 0;
+}
+
+int cuda_status(cudaError_t e)
+{
+    return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+int64_t round_up(int64_t v, int64_t m)
+{
+    return (v + m - 1) / m * m;
+}
+
+// ---------------------------------------------------------------- workspace
+struct Layout {
+    int64_t mt_max = 0, rpad = 0;
+    int64_t counts = 0, off = 0, poff = 0, mtiles = 0, inv = 0, amax = 0;
+    int64_t a_codes = 0, a_sf = 0, h_codes = 0, h_sf = 0, y = 0, total = 0;
+};
+
+// Header (256 B): int32 error word at 0, int32 m-tile count at 4.
+Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
+{
+    Layout L;
+    const int64_t R = T * k;
+    const int64_t ne = std::min<int64_t>(E, R);
+    L.mt_max = (R + 127 * ne) / 128;          // >= sum_e ceil(count_e / 128)
+    L.rpad = 128 * L.mt_max;
+    int64_t o = 256;
+    auto take = [&](int64_t bytes) {
+        const int64_t at = o;
+        o = round_up(o + bytes, 1024);
+        return at;
+    };
+    L.counts = take(4 * E);
+    L.off = take(4 * (E + 1));
+    L.poff = take(4 * (E + 1));
+    L.amax = take(4 * E);
+    L.mtiles = take(16 * std::max<int64_t>(L.mt_max, 1));
+    L.inv = take(4 * std::max<int64_t>(R, 1));
+    L.a_codes = take(L.rpad * (H / 2));
+    L.a_sf = take(L.rpad * (H / 16));
+    L.h_codes = take(L.rpad * (I / 2));
+    L.h_sf = take(L.rpad * (I / 16));
+    L.y = take(R * H * 2);
+    L.total = o;
+    return L;
+}
+
+int check_moe_shape(int64_t T, int k, int E, int64_t H, int64_t I)
+{
+    if (T < 0 || H <= 0 || I <= 0 || E < 1 || k < 1)
+        return NVFP4_ERR_INVALID_ARG;
+    if (H % 128 != 0 || I % 128 != 0 || E > 1024 || k > 32 || T * k >= (1LL << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (H > (1LL << 20) || I > (1LL << 20) || static_cast<int64_t>(E) * 2 * I >= (1LL << 31) ||
+        static_cast<int64_t>(E) * H >= (1LL << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    return NVFP4_OK;
+}
+
+int check_moe_args(const nvfp4_moe_args *a, bool need_out)
+{
+    if (a == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    int st = check_moe_shape(a->T, a->k, a->E, a->H, a->I);
+    if (st != NVFP4_OK)
+        return st;
+    const void *ptrs[] = {a->x, a->topk_ids, a->topk_weights, a->x_gs, a->w13_codes, a->w13_scales,
+                          a->w13_gs, a->w2_codes, a->w2_scales, a->w2_gs};
+    for (const void *p : ptrs)
+        if (p == nullptr)
+            return NVFP4_ERR_INVALID_ARG;
+    if (need_out && (a->out == nullptr || a->inter_gs == nullptr))
+        return NVFP4_ERR_INVALID_ARG;
+    const void *al[] = {a->x, a->w13_codes, a->w13_scales, a->w2_codes, a->w2_scales};
+    for (const void *p : al)
+        if (!aligned16(p))
+            return NVFP4_ERR_MISALIGNED;
+    if (need_out && !aligned16(a->out))
+        return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+// Routing + quantise/permute + L1 (given epilogue).  Shared by forward and calibrate.
+// Records events[i] on s when events is non-null (per-stage timing).
+int mark(void *const *events, int i, cudaStream_t s)
+{
+    if (events == nullptr)
+        return NVFP4_OK;
+    return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s));
+}
+
+int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi, void *const *events,
+              cudaStream_t s, int num_sms, CUtensorMap *map_a1, CUtensorMap *map_b1)
+{
+    const int64_t T = a->T, H = a->H, I = a->I, R = T * a->k;
+    const int E = a->E, k = a->k;
+    int32_t *err = reinterpret_cast<int32_t *>(ws);
+    int32_t *num_mt = reinterpret_cast<int32_t *>(ws + 4);
+    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    int32_t *off = reinterpret_cast<int32_t *>(ws + L.off);
+    int32_t *poff = reinterpret_cast<int32_t *>(ws + L.poff);
+    int4 *mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
+    int32_t *inv = reinterpret_cast<int32_t *>(ws + L.inv);
+
+    if (mark(events, 0, s) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
+    cudaError_t e = launch_route(a->topk_ids, R, E, counts, off, poff, num_mt, mtiles, inv, err, s);
+    if (e != cudaSuccess || mark(events, 1, s) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
+    e = launch_quantize(reinterpret_cast<const __nv_bfloat16 *>(a->x), T, H, H, a->x_gs, ws + L.a_codes,
+                        ws + L.a_sf, NVFP4_SCALES_MMA, inv, k, s);
+    if (e != cudaSuccess || mark(events, 2, s) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
+
+    int st = make_code_map(map_a1, ws + L.a_codes, L.rpad, H / 2);
+    if (st == NVFP4_OK)
+        st = make_code_map(map_b1, a->w13_codes, static_cast<int64_t>(E) * 2 * I, H / 2);
+    if (st != NVFP4_OK)
+        return st;
+    GemmArgs g{};
+    g.sfa = ws + L.a_sf;
+    g.sfa_block_stride = (H / 64) * 512;
+    g.sfb = a->w13_scales;
+    g.sfb_block_stride = (H / 64) * 512;
+    g.K = static_cast<int>(H);
+    g.num_k_tiles = static_cast<int>((H + 255) / 256);
+    g.num_mtiles_dev = num_mt;
+    g.mtiles = mtiles;
+    g.n_tiles = static_cast<int>(I / 128);
+    g.b_rows_per_expert = 2 * I;
+    g.b_tile_rows = 128;
+    g.b_half_offset = static_cast<int>(I);
+    g.a_gs = a->x_gs;
+    g.a_gs_per_expert = 0;
+    g.b_gs = a->w13_gs;
+    g.b_gs_stride = 2;
+    g.nseg = 1;
+    g.inter_gs = a->inter_gs;
+    g.h_codes = ws + L.h_codes;
+    g.h_ld_bytes = I / 2;
+    g.h_sf = ws + L.h_sf;
+    g.h_sf_block_stride = (I / 64) * 512;
+    g.amax_bits = reinterpret_cast<unsigned int *>(ws + L.amax);
+    g.err = err;
+    return cuda_status(launch_gemm(256, l1_epi, *map_a1, *map_b1, g, num_sms, s));
+}
+
+} // namespace
+
+extern "C" {
+
+const char *nvfp4_status_string(int status)
+{
+    switch (status) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "NVFP4_ERR_UNSUPPORTED_SHAPE";
+    case NVFP4_ERR_MISALIGNED: return "NVFP4_ERR_MISALIGNED";
+    case NVFP4_ERR_WORKSPACE_TOO_SMALL: return "NVFP4_ERR_WORKSPACE_TOO_SMALL";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+    case NVFP4_ERR_UNSUPPORTED_DEVICE: return "NVFP4_ERR_UNSUPPORTED_DEVICE";
+    case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT";
+    case NVFP4_ERR_BAD_EXPERT_ID: return "NVFP4_ERR_BAD_EXPERT_ID";
+    default: return "NVFP4_ERR_UNKNOWN";
+    }
+}
+
+int nvfp4_global_scale(const uint16_t *x, int64_t n, float *gs_out, void *stream)
+{
+    if (x == nullptr || gs_out == nullptr || n < 1)
+        return NVFP4_ERR_INVALID_ARG;
+    int sms = 0;
+    int st = device_check(&sms);
+    if (st != NVFP4_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(gs_out, 0, sizeof(float), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (launch_amax_bf16(reinterpret_cast<const __nv_bfloat16 *>(x), n, gs_out, sms, s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return cuda_status(launch_finalize_gs(gs_out, s));
+}
+
+int64_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int scale_layout)
+{
+    if (rows < 0 || cols < 0 || cols % 16 != 0)
+        return -1;
+    if (scale_layout == NVFP4_SCALES_ROWMAJOR)
+        return rows * (cols / 16);
+    if (scale_layout == NVFP4_SCALES_MMA) {
+        if (cols % 64 != 0)
+            return -1;
+        return round_up(rows, 128) * (cols / 16);
+    }
+    return -1;
+}
+
+int nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs, uint8_t *codes,
+                   uint8_t *scales, int scale_layout, void *stream)
+{
+    if (x == nullptr || gs == nullptr || codes == nullptr || scales == nullptr || rows < 0 || cols <= 0 || ldx < cols)
+        return NVFP4_ERR_INVALID_ARG;
+    if (scale_layout != NVFP4_SCALES_ROWMAJOR && scale_layout != NVFP4_SCALES_MMA)
+        return NVFP4_ERR_INVALID_ARG;
+    if (cols % 16 != 0 || (scale_layout == NVFP4_SCALES_MMA && cols % 64 != 0))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || ldx % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    if (rows > (1LL << 31) / 8)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    int st = device_check(nullptr);
+    if (st != NVFP4_OK)
+        return st;
+    if (rows == 0)
+        return NVFP4_OK;
+    return cuda_status(launch_quantize(reinterpret_cast<const __nv_bfloat16 *>(x), rows, cols, ldx, gs, codes, scales,
+                                       scale_layout, nullptr, 1, static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_swizzle_scales(const uint8_t *in, int64_t batch, int64_t rows, int64_t cols, uint8_t *out, void *stream)
+{
+    if (in == nullptr || out == nullptr || batch < 0 || rows < 0 || cols <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (cols % 64 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(in) & 3) != 0 || (reinterpret_cast<uintptr_t>(out) & 3) != 0)
+        return NVFP4_ERR_MISALIGNED;
+    int st = device_check(nullptr);
+    if (st != NVFP4_OK)
+        return st;
+    if (batch == 0 || rows == 0)
+        return NVFP4_OK;
+    return cuda_status(launch_swizzle(in, batch, rows, cols, out, static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs, int64_t M, const uint8_t *b_codes,
+               const uint8_t *b_scales, const float *b_gs, const int64_t *seg_end, int nseg, int64_t N, int64_t K,
+               uint16_t *out, int64_t ldo, void *stream)
+{
+    if (a_codes == nullptr || a_scales == nullptr || a_gs == nullptr || b_codes == nullptr || b_scales == nullptr ||
+        b_gs == nullptr || seg_end == nullptr || out == nullptr || M < 1 || N < 1 || K < 1 || nseg < 1 || ldo < N)
+        return NVFP4_ERR_INVALID_ARG;
+    if (N % 128 != 0 || K % 64 != 0 || nseg > 4 || M >= (1LL << 31) || N >= (1LL << 31) || K > (1LL << 20))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    int64_t prev = 0;
+    for (int i = 0; i < nseg; ++i) {
+        if (seg_end[i] <= prev || seg_end[i] % 32 != 0)
+            return NVFP4_ERR_INVALID_ARG;
+        prev = seg_end[i];
+    }
+    if (prev != N)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(b_codes) || !aligned16(b_scales) ||
+        !aligned16(out) || ldo % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    int st = device_check(&sms);
+    if (st != NVFP4_OK)
+        return st;
+    CUtensorMap ma, mb;
+    st = make_code_map(&ma, a_codes, M, K / 2);
+    if (st == NVFP4_OK)
+        st = make_code_map(&mb, b_codes, N, K / 2);
+    if (st != NVFP4_OK)
+        return st;
+    const int bn = (N % 256 == 0) ? 256 : 128;
+    GemmArgs g{};
+    g.sfa = a_scales;
+    g.sfa_block_stride = (K / 64) * 512;
+    g.sfb = b_scales;
+    g.sfb_block_stride = (K / 64) * 512;
+    g.K = static_cast<int>(K);
+    g.num_k_tiles = static_cast<int>((K + 255) / 256);
+    g.num_mtiles_dev = nullptr;
+    g.mtiles = nullptr;
+    g.dense_m_tiles = static_cast<int>((M + 127) / 128);
+    g.dense_M = static_cast<int>(M);
+    g.n_tiles = static_cast<int>(N / bn);
+    g.b_rows_per_expert = N;
+    g.b_tile_rows = bn;
+    g.b_half_offset = 128;
+    g.a_gs = a_gs;
+    g.a_gs_per_expert = 0;
+    g.b_gs = b_gs;
+    g.b_gs_stride = 0;
+    g.nseg = nseg;
+    for (int i = 0; i < nseg; ++i)
+        g.seg_end[i] = static_cast<int>(seg_end[i]);
+    g.out = reinterpret_cast<__nv_bfloat16 *>(out);
+    g.ldo = ldo;
+    g.err = nullptr;            // no workspace: a timed-out wait ends the kernel without a report
+    int64_t tiles = static_cast<int64_t>(g.dense_m_tiles) * g.n_tiles;
+    const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+    return cuda_status(launch_gemm(bn, EPI_BF16, ma, mb, g, grid, static_cast<cudaStream_t>(stream)));
+}
+
+size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I)
+{
+    if (check_moe_shape(T, k, E, H, I) != NVFP4_OK)
+        return 0;
+    return static_cast<size_t>(ws_layout(T, k, E, H, I).total);
+}
+
+int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, int region, int64_t *offset,
+                               int64_t *bytes)
+{
+    if (offset == nullptr || bytes == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    int st = check_moe_shape(T, k, E, H, I);
+    if (st != NVFP4_OK)
+        return st;
+    const Layout L = ws_layout(T, k, E, H, I);
+    const int64_t R = T * k;
+    switch (region) {
+    case 0: *offset = L.a_codes; *bytes = L.rpad * (H / 2); break;
+    case 1: *offset = L.a_sf; *bytes = L.rpad * (H / 16); break;
+    case 2: *offset = L.h_codes; *bytes = L.rpad * (I / 2); break;
+    case 3: *offset = L.h_sf; *bytes = L.rpad * (I / 16); break;
+    case 4: *offset = L.y; *bytes = R * H * 2; break;
+    case 5: *offset = L.inv; *bytes = R * 4; break;
+    case 6: *offset = L.counts; *bytes = 4LL * E; break;
+    case 7: *offset = L.poff; *bytes = 4LL * (E + 1); break;
+    default: return NVFP4_ERR_INVALID_ARG;
+    }
+    return NVFP4_OK;
+}
+
+static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_bytes, void *stream,
+                            void *const *events)
+{
+    int st = check_moe_args(a, true);
+    if (st != NVFP4_OK)
+        return st;
+    if (workspace == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(workspace))
+        return NVFP4_ERR_MISALIGNED;
+    const Layout L = ws_layout(a->T, a->k, a->E, a->H, a->I);
+    if (ws_bytes < static_cast<size_t>(L.total))
+        return NVFP4_ERR_WORKSPACE_TOO_SMALL;
+    int sms = 0;
+    st = device_check(&sms);
+    if (st != NVFP4_OK)
+        return st;
+    if (a->T == 0)
+        return NVFP4_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    CUtensorMap ma1, mb1, ma2, mb2;
+    st = run_front(a, ws, L, EPI_SWIGLU_QUANT, events, s, sms, &ma1, &mb1);
+    if (st != NVFP4_OK)
+        return st;
+
+    const int64_t H = a->H, I = a->I;
+    const int E = a->E;
+    st = make_code_map(&ma2, ws + L.h_codes, L.rpad, I / 2);
+    if (st == NVFP4_OK)
+        st = make_code_map(&mb2, a->w2_codes, static_cast<int64_t>(E) * H, I / 2);
+    if (st != NVFP4_OK)
+        return st;
+    const int bn = (H % 256 == 0) ? 256 : 128;
+    GemmArgs g{};
+    g.sfa = ws + L.h_sf;
+    g.sfa_block_stride = (I / 64) * 512;
+    g.sfb = a->w2_scales;
+    g.sfb_block_stride = (I / 64) * 512;
+    g.K = static_cast<int>(I);
+    g.num_k_tiles = static_cast<int>((I + 255) / 256);
+    g.num_mtiles_dev = reinterpret_cast<int32_t *>(ws + 4);
+    g.mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
+    g.n_tiles = static_cast<int>(H / bn);
+    g.b_rows_per_expert = H;
+    g.b_tile_rows = bn;
+    g.b_half_offset = 128;
+    g.a_gs = a->inter_gs;
+    g.a_gs_per_expert = 1;
+    g.b_gs = a->w2_gs;
+    g.b_gs_stride = 1;
+    g.nseg = 1;
+    g.seg_end[0] = static_cast<int>(H);
+    g.out = reinterpret_cast<__nv_bfloat16 *>(ws + L.y);
+    g.ldo = H;
+    g.err = reinterpret_cast<int32_t *>(ws);
+    if (mark(events, 3, s) != NVFP4_OK || launch_gemm(bn, EPI_BF16, ma2, mb2, g, sms, s) != cudaSuccess ||
+        mark(events, 4, s) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
+
+    if (launch_combine(reinterpret_cast<const __nv_bfloat16 *>(ws + L.y),
+                       reinterpret_cast<const int32_t *>(ws + L.inv), a->topk_ids, a->topk_weights,
+                       reinterpret_cast<const int32_t *>(ws + L.off), reinterpret_cast<const int32_t *>(ws + L.poff),
+                       a->T, a->k, H, reinterpret_cast<__nv_bfloat16 *>(a->out), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return mark(events, 5, s);
+}
+
+int nvfp4_moe_forward(const nvfp4_moe_args *a, void *workspace, size_t ws_bytes, void *stream)
+{
+    return moe_forward_impl(a, workspace, ws_bytes, stream, nullptr);
+}
+
+int nvfp4_moe_forward_timed(const nvfp4_moe_args *a, void *workspace, size_t ws_bytes, void *stream,
+                            void *const *events)
+{
+    if (events == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    for (int i = 0; i < 6; ++i)
+        if (events[i] == nullptr)
+            return NVFP4_ERR_INVALID_ARG;
+    return moe_forward_impl(a, workspace, ws_bytes, stream, events);
+}
+
+int nvfp4_moe_calibrate(const nvfp4_moe_args *a, float *inter_gs_out, void *workspace, size_t ws_bytes, void *stream)
+{
+    int st = check_moe_args(a, false);
+    if (st != NVFP4_OK)
+        return st;
+    if (workspace == nullptr || inter_gs_out == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(workspace))
+        return NVFP4_ERR_MISALIGNED;
+    const Layout L = ws_layout(a->T, a->k, a->E, a->H, a->I);
+    if (ws_bytes < static_cast<size_t>(L.total))
+        return NVFP4_ERR_WORKSPACE_TOO_SMALL;
+    int sms = 0;
+    st = device_check(&sms);
+    if (st != NVFP4_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    if (cudaMemsetAsync(ws + L.amax, 0, 4 * static_cast<size_t>(a->E), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (a->T > 0) {
+        CUtensorMap ma1, mb1;
+        st = run_front(a, ws, L, EPI_SWIGLU_AMAX, nullptr, s, sms, &ma1, &mb1);
+        if (st != NVFP4_OK)
+            return st;
+    }
+    return cuda_status(
+        launch_finalize_inter_gs(reinterpret_cast<const unsigned int *>(ws + L.amax), a->E, inter_gs_out, s));
+}
+
+int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int32_t *counts, int32_t *padded_offsets,
+                          int32_t *inv, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (topk_ids == nullptr || counts == nullptr || padded_offsets == nullptr || inv == nullptr ||
+        workspace == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (T < 0 || k < 1 || E < 1)
+        return NVFP4_ERR_INVALID_ARG;
+    if (E > 1024 || k > 32 || T * k >= (1LL << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const Layout L = ws_layout(T, k, E, 128, 128);
+    if (ws_bytes < static_cast<size_t>(L.total))
+        return NVFP4_ERR_WORKSPACE_TOO_SMALL;
+    int st = device_check(nullptr);
+    if (st != NVFP4_OK)
+        return st;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    return cuda_status(launch_route(topk_ids, T * k, E, counts, reinterpret_cast<int32_t *>(ws + L.off),
+                                    padded_offsets, reinterpret_cast<int32_t *>(ws + 4),
+                                    reinterpret_cast<int4 *>(ws + L.mtiles), inv, reinterpret_cast<int32_t *>(ws),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_moe_get_error(void *workspace, int32_t *err_host, void *stream)
+{
+    if (workspace == nullptr || err_host == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(err_host, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (cudaMemsetAsync(workspace, 0, sizeof(int32_t), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return cuda_status(cudaStreamSynchronize(s));
+}
+
+} // extern "C"

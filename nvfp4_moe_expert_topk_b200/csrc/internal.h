@@ -1,0 +1,75 @@
+// internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nvfp4moe.h"
+
+namespace nvfp4 {
+
+// Arguments of the persistent block-scaled FP4 GEMM engine (gemm.cu).
+struct GemmArgs {
+    // scale factors, NVFP4_SCALES_MMA layout: one 128-row block = (K/64) atoms of 512 bytes
+    const uint8_t *sfa;
+    int64_t sfa_block_stride;
+    const uint8_t *sfb;
+    int64_t sfb_block_stride;
+    int K;                    // reduction length in elements, multiple of 64
+    int num_k_tiles;          // ceil(K / 256)
+    // tile space: grouped (m-tile table written on the device) or dense
+    const int32_t *num_mtiles_dev;
+    const int4 *mtiles;       // {expert, first padded row, valid rows, first output row}
+    int dense_m_tiles;
+    int dense_M;
+    int n_tiles;
+    int64_t b_rows_per_expert;
+    int b_tile_rows;          // B rows advanced per n-tile
+    int b_half_offset;        // row offset of the second 128-row half of a 256-wide B tile
+    // global scales: alpha = 1 / (a_gs * b_gs)
+    const float *a_gs;
+    int a_gs_per_expert;
+    const float *b_gs;
+    int b_gs_stride;          // b_gs index = expert * b_gs_stride + segment
+    int nseg;
+    int seg_end[4];           // column ends of the B segments (dense GEMM)
+    // SwiGLU epilogues
+    const float *inter_gs;
+    uint8_t *h_codes;
+    int64_t h_ld_bytes;
+    uint8_t *h_sf;
+    int64_t h_sf_block_stride;
+    unsigned int *amax_bits;
+    // bf16 epilogue
+    __nv_bfloat16 *out;
+    int64_t ldo;
+    int32_t *err;             // device error word
+};
+
+enum Epilogue { EPI_SWIGLU_QUANT = 0, EPI_BF16 = 1, EPI_SWIGLU_AMAX = 2 };
+
+// Launches the GEMM engine.  map_a / map_b: 2-D uint8 tensor maps over the
+// code matrices (box 128 x 128 bytes, 128-byte swizzle).
+cudaError_t launch_gemm(int bn, int epi, const CUtensorMap &map_a, const CUtensorMap &map_b, const GemmArgs &args,
+                        int grid, cudaStream_t stream);
+
+int gemm_smem_bytes(int bn);
+
+// Memory-bound kernels (kernels.cu).
+cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s);
+cudaError_t launch_finalize_gs(float *gs, cudaStream_t s);
+cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs,
+                            uint8_t *codes, uint8_t *scales, int layout, const int32_t *inv, int k,
+                            cudaStream_t s);
+cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64_t cols, uint8_t *out,
+                           cudaStream_t s);
+cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
+                         int32_t *num_mtiles, int4 *mtiles, int32_t *inv, int32_t *err, cudaStream_t s);
+cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int32_t *ids, const float *w,
+                           const int32_t *off, const int32_t *poff, int64_t T, int k, int64_t H,
+                           __nv_bfloat16 *out, cudaStream_t s);
+cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float *inter_gs, cudaStream_t s);
+
+} // namespace nvfp4

@@ -1,0 +1,433 @@
+// kernels.cu -- the memory-bound steps of the chain: global scale, activation
+// quantisation (plain and fused with the expert permutation), scale-layout
+// conversion, routing (histogram, prefix sums, stable permutation, m-tile
+// table) and the top-k weighted combine.
+#include "internal.h"
+#include "quant.cuh"
+
+namespace nvfp4 {
+
+// ------------------------------------------------------------ global scale
+// amax of a bf16 tensor, accumulated into *out_bits (the float bit pattern;
+// non-negative floats order like their bits).  *out_bits must start at 0.
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t n,
+                                                        unsigned int *__restrict__ out_bits)
+{
+    float m = 0.0f;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    int64_t start_scalar = 0;
+    if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+        const int64_t n8 = n / 8;
+        const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+        for (int64_t i = tid; i < n8; i += nth) {
+            const uint4 v = __ldg(xv + i);
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = __bfloat1622float2(h[j]);
+                m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+        start_scalar = n8 * 8;
+    }
+    for (int64_t i = start_scalar + tid; i < n; i += nth)
+        m = fmaxf(m, fabsf(__bfloat162float(x[i])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __shared__ float wmax[8];
+    if ((threadIdx.x & 31) == 0)
+        wmax[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+            m = fmaxf(m, wmax[w]);
+        atomicMax(out_bits, __float_as_uint(m));
+    }
+}
+
+// gs = 2688 / amax (fp32, round to nearest), 1 if amax == 0; in place.
+__global__ void finalize_gs_kernel(float *gs)
+{
+    const float a = __uint_as_float(*reinterpret_cast<unsigned int *>(gs));
+    *gs = (a == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, a);
+}
+
+cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s)
+{
+    int64_t blocks = (n / 8 + 255) / 256;
+    if (blocks < 1)
+        blocks = 1;
+    if (blocks > 8LL * num_sms)
+        blocks = 8LL * num_sms;
+    amax_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, n, reinterpret_cast<unsigned int *>(gs_out));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_gs(float *gs, cudaStream_t s)
+{
+    finalize_gs_kernel<<<1, 1, 0, s>>>(gs);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ quantisation
+// One warp per source row; each lane handles 64 consecutive elements (4
+// blocks) per step.  With inv != nullptr the row is token t of a routed batch
+// and its codes and scales are written to each padded destination row
+// inv[t*k + j] >= 0 (the expert permutation); otherwise to row t.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
+                                                            int64_t cols, int64_t ldx, const float *__restrict__ gs_ptr,
+                                                            uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                                                            int layout, const int32_t *__restrict__ inv, int k)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+    if (row >= rows)
+        return;
+    const float gs = __ldg(gs_ptr);
+    int my_dst = -1;                         // lane j < k holds destination j
+    int ndst = 1;
+    if (inv != nullptr) {
+        ndst = k;
+        if (lane < k)
+            my_dst = __ldg(inv + row * k + lane);
+    }
+    const int64_t kb_per_block = cols / 64;
+    const __nv_bfloat16 *xr = x + row * ldx;
+    for (int64_t c0 = static_cast<int64_t>(lane) * 64; c0 < cols; c0 += 32 * 64) {
+        const int64_t nb_left = (cols - c0) / 16;
+        const int nb = nb_left < 4 ? static_cast<int>(nb_left) : 4;
+        uint32_t cw[8];
+        uint32_t sw = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            cw[2 * b] = cw[2 * b + 1] = 0;
+            if (b < nb) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(xr + c0 + 16 * b);
+                const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+                const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&v0);
+                const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&v1);
+                float f[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 a = __bfloat1622float2(h0[j]);
+                    const float2 c = __bfloat1622float2(h1[j]);
+                    f[2 * j] = a.x;
+                    f[2 * j + 1] = a.y;
+                    f[8 + 2 * j] = c.x;
+                    f[8 + 2 * j + 1] = c.y;
+                }
+                const uint32_t sb = quantize16(f, gs, cw[2 * b], cw[2 * b + 1]);
+                sw |= sb << (8 * b);
+            }
+        }
+        for (int d = 0; d < ndst; ++d) {
+            int64_t dst = row;
+            if (inv != nullptr) {
+                dst = __shfl_sync(0xffffffffu, my_dst, d);
+                if (dst < 0)
+                    continue;
+            }
+            uint8_t *crow = codes + dst * (cols / 2) + c0 / 2;
+            if (nb == 4) {
+                reinterpret_cast<uint4 *>(crow)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                reinterpret_cast<uint4 *>(crow)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            } else {
+                for (int b = 0; b < nb; ++b)
+                    reinterpret_cast<uint2 *>(crow)[b] = make_uint2(cw[2 * b], cw[2 * b + 1]);
+            }
+            if (layout == NVFP4_SCALES_MMA) {
+                *reinterpret_cast<uint32_t *>(scales + mma_scale_offset(dst, c0 / 64, kb_per_block)) = sw;
+            } else {
+                uint8_t *srow = scales + dst * (cols / 16) + c0 / 16;
+                if (nb == 4 && (cols % 64) == 0)
+                    *reinterpret_cast<uint32_t *>(srow) = sw;
+                else
+                    for (int b = 0; b < nb; ++b)
+                        srow[b] = static_cast<uint8_t>(sw >> (8 * b));
+            }
+        }
+    }
+}
+
+cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs,
+                            uint8_t *codes, uint8_t *scales, int layout, const int32_t *inv, int k, cudaStream_t s)
+{
+    const int64_t blocks = (rows + 7) / 8;
+    quantize_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, rows, cols, ldx, gs, codes, scales, layout,
+                                                                     inv, k);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ scale layout
+// One thread per 4-byte word of the MMA layout: row r, 64-element block kb.
+__global__ void swizzle_scales_kernel(const uint8_t *__restrict__ in, int64_t batch, int64_t rows, int64_t cols,
+                                      uint8_t *__restrict__ out)
+{
+    const int64_t kbs = cols / 64;
+    const int64_t rblocks = (rows + 127) / 128;
+    const int64_t per_batch_words = rblocks * kbs * 128;
+    const int64_t total = batch * per_batch_words;
+    for (int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; w < total;
+         w += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t b = w / per_batch_words;
+        int64_t rem = w - b * per_batch_words;
+        const int64_t atom = rem / 128;
+        const int64_t word = rem - atom * 128;
+        const int64_t rb = atom / kbs, kb = atom - rb * kbs;
+        const int64_t r = rb * 128 + (word & 3) * 32 + (word >> 2);
+        uint32_t v = 0;
+        if (r < rows)
+            v = *reinterpret_cast<const uint32_t *>(in + (b * rows + r) * (cols / 16) + kb * 4);
+        reinterpret_cast<uint32_t *>(out)[w] = v;
+    }
+}
+
+cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64_t cols, uint8_t *out,
+                           cudaStream_t s)
+{
+    const int64_t words = batch * ((rows + 127) / 128) * (cols / 64) * 128;
+    int64_t blocks = (words + 255) / 256;
+    if (blocks > 65535)
+        blocks = 65535;
+    if (blocks < 1)
+        blocks = 1;
+    swizzle_scales_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(in, batch, rows, cols, out);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ routing
+// One block of 1024 threads.  Warp w owns the contiguous slot range
+// [w*chunk, (w+1)*chunk) of the flattened ids (slot f = t*k + j):
+//  1. per-warp histograms in shared memory;
+//  2. per expert: exclusive prefix over warps (so warp w starts after all
+//     earlier warps' slots of that expert) and the total count;
+//  3. exclusive scans over experts of the counts and of the 128-row m-tile
+//     counts -> unpadded offsets, padded offsets, the m-tile table;
+//  4. each warp walks its range in order; lanes with equal ids find each
+//     other with match_any, so a slot's rank is the number of earlier slots
+//     of its expert: position = padded_offset[e] + rank (a stable counting
+//     sort, deterministic for a given input).
+__global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__ ids, int R, int E,
+                                                     int32_t *__restrict__ counts, int32_t *__restrict__ off,
+                                                     int32_t *__restrict__ poff, int32_t *__restrict__ num_mtiles,
+                                                     int4 *__restrict__ mtiles, int32_t *__restrict__ inv,
+                                                     int32_t *__restrict__ err)
+{
+    extern __shared__ int32_t sm[];
+    int32_t *wcnt = sm;                // [32][E]
+    int32_t *poff_s = sm + 32 * E;     // [E]
+    __shared__ int32_t warp_sum_c[32], warp_sum_t[32];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    for (int i = tid; i < 32 * E; i += blockDim.x)
+        wcnt[i] = 0;
+    __syncthreads();
+
+    const int chunk = (R + 31) / 32;
+    const int f0 = min(R, warp * chunk), f1 = min(R, f0 + chunk);
+    int bad = 0;
+    for (int f = f0 + lane; f < f1; f += 32) {
+        const int e = __ldg(ids + f);
+        if (e >= E)
+            bad = 1;
+        else if (e >= 0)
+            atomicAdd(&wcnt[warp * E + e], 1);
+    }
+    if (bad)
+        atomicCAS(err, 0, NVFP4_ERR_BAD_EXPERT_ID);
+    __syncthreads();
+
+    // 2 + 3: thread e owns expert e (E <= 1024)
+    int cnt = 0, tiles = 0;
+    if (tid < E) {
+        for (int w = 0; w < 32; ++w) {
+            const int c = wcnt[w * E + tid];
+            wcnt[w * E + tid] = cnt;
+            cnt += c;
+        }
+        tiles = (cnt + 127) / 128;
+    }
+    // block-wide exclusive scan of (cnt, tiles) over thread index
+    int ic = cnt, it = tiles;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, ic, o);
+        const int b = __shfl_up_sync(0xffffffffu, it, o);
+        if (lane >= o) {
+            ic += a;
+            it += b;
+        }
+    }
+    if (lane == 31) {
+        warp_sum_c[warp] = ic;
+        warp_sum_t[warp] = it;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int c = warp_sum_c[lane], t = warp_sum_t[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(0xffffffffu, c, o);
+            const int b = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) {
+                c += a;
+                t += b;
+            }
+        }
+        warp_sum_c[lane] = c;   // inclusive over warps
+        warp_sum_t[lane] = t;
+    }
+    __syncthreads();
+    const int base_c = (warp > 0 ? warp_sum_c[warp - 1] : 0) + ic - cnt;   // exclusive
+    const int base_t = (warp > 0 ? warp_sum_t[warp - 1] : 0) + it - tiles;
+    if (tid < E) {
+        counts[tid] = cnt;
+        off[tid] = base_c;
+        poff[tid] = base_t * 128;
+        poff_s[tid] = base_t * 128;
+        for (int i = 0; i < tiles; ++i)
+            mtiles[base_t + i] = make_int4(tid, base_t * 128 + 128 * i, min(128, cnt - 128 * i), base_c + 128 * i);
+        if (tid == E - 1) {
+            off[E] = base_c + cnt;
+            poff[E] = (base_t + tiles) * 128;
+            *num_mtiles = base_t + tiles;
+        }
+    }
+    __syncthreads();
+
+    // 4: stable positions
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int base = f0; base < f1; base += 32) {
+        const int f = base + lane;
+        const bool act = f < f1;
+        const int e = act ? __ldg(ids + f) : -1;
+        const bool valid = act && e >= 0 && e < E;
+        const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+        const int rank = __popc(peers & lt_mask);
+        if (valid)
+            inv[f] = poff_s[e] + wcnt[warp * E + e] + rank;
+        else if (act)
+            inv[f] = -1;
+        __syncwarp();
+        if (valid && rank == 0)
+            wcnt[warp * E + e] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
+                         int32_t *num_mtiles, int4 *mtiles, int32_t *inv, int32_t *err, cudaStream_t s)
+{
+    const size_t smem = sizeof(int32_t) * (33 * static_cast<size_t>(E));
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * 1024 * 4);
+        if (e != cudaSuccess)
+            return e;
+        attr_set = true;
+    }
+    route_kernel<<<1, 1024, smem, s>>>(ids, static_cast<int>(R), E, counts, off, poff, num_mtiles, mtiles, inv, err);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ combine
+// out[t] = bf16( sum_{j ascending} w[t,j] * y[row(t,j)] ) in fp32, where
+// row(t,j) is the slot's row in the unpadded expert-major y buffer.  One
+// block per token, 8 bf16 (16 bytes) per thread per step.
+__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__restrict__ y,
+                                                      const int32_t *__restrict__ inv,
+                                                      const int32_t *__restrict__ ids, const float *__restrict__ w,
+                                                      const int32_t *__restrict__ off,
+                                                      const int32_t *__restrict__ poff, int k, int64_t H,
+                                                      __nv_bfloat16 *__restrict__ out)
+{
+    __shared__ int64_t s_row[32];
+    __shared__ float s_w[32];
+    const int64_t t = blockIdx.x;
+    if (threadIdx.x < k) {
+        const int64_t f = t * k + threadIdx.x;
+        const int p = __ldg(inv + f);
+        int64_t row = -1;
+        if (p >= 0) {
+            const int e = __ldg(ids + f);
+            row = static_cast<int64_t>(p) - __ldg(poff + e) + __ldg(off + e);
+        }
+        s_row[threadIdx.x] = row;
+        s_w[threadIdx.x] = __ldg(w + f);
+    }
+    __syncthreads();
+    for (int64_t c = static_cast<int64_t>(threadIdx.x) * 8; c < H; c += static_cast<int64_t>(blockDim.x) * 8) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            acc[i] = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            const int64_t row = s_row[j];
+            if (row < 0)
+                continue;
+            const float wj = s_w[j];
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + row * H + c));
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h[i]);
+                acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wj, f.x));
+                acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wj, f.y));
+            }
+        }
+        uint4 o;
+        __nv_bfloat162 *oh = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            oh[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        *reinterpret_cast<uint4 *>(out + t * H + c) = o;
+    }
+}
+
+cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int32_t *ids, const float *w,
+                           const int32_t *off, const int32_t *poff, int64_t T, int k, int64_t H,
+                           __nv_bfloat16 *out, cudaStream_t s)
+{
+    combine_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(y, inv, ids, w, off, poff, k, H, out);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ warmup scales
+// inter_gs[e] = 2688 / amax_e; experts with amax 0 use the largest amax.
+__global__ void finalize_inter_gs_kernel(const unsigned int *__restrict__ amax_bits, int E, float *inter_gs)
+{
+    __shared__ float wmax[32];
+    const int tid = threadIdx.x;
+    const float a = tid < E ? __uint_as_float(amax_bits[tid]) : 0.0f;
+    float m = a;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0)
+        wmax[tid >> 5] = m;
+    __syncthreads();
+    if (tid < 32) {
+        m = tid < static_cast<int>(blockDim.x >> 5) ? wmax[tid] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (tid == 0)
+            wmax[0] = m;
+    }
+    __syncthreads();
+    const float gmax = wmax[0];
+    if (tid < E) {
+        const float use = a > 0.0f ? a : gmax;
+        inter_gs[tid] = use == 0.0f ? 1.0f : __fdiv_rn(2688.0f, use);
+    }
+}
+
+cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float *inter_gs, cudaStream_t s)
+{
+    finalize_inter_gs_kernel<<<1, 1024, 0, s>>>(amax_bits, E, inter_gs);
+    return cudaGetLastError();
+}
+
+} // namespace nvfp4

@@ -1,0 +1,110 @@
+"""The C-ABI library builds, loads and exports every entry point of
+include/nvfp4moe.h; host-only entry points and argument checks work without a
+GPU (no kernel is launched here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "nvfp4moe.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from nvfp4_moe_expert_topk_b200 import build, lib
+    build.build()
+    return lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ ]*?\s*\*?\s*(nvfp4_[a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for want in ["nvfp4_quantize", "nvfp4_gemm", "nvfp4_moe_forward", "nvfp4_global_scale",
+                 "nvfp4_swizzle_scales", "nvfp4_moe_workspace_size", "nvfp4_moe_get_error",
+                 "nvfp4_moe_route_debug", "nvfp4_moe_calibrate", "nvfp4_status_string"]:
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from nvfp4_moe_expert_topk_b200 import LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(line.split()[-1] for line in out.splitlines() if line.strip())
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_status_strings(L):
+    from nvfp4_moe_expert_topk_b200 import nvfp4_status_string
+    assert nvfp4_status_string(0) == "NVFP4_OK"
+    for code in range(-1, -9, -1):
+        assert nvfp4_status_string(code).startswith("NVFP4_ERR_")
+    assert nvfp4_status_string(-99) == "NVFP4_ERR_UNKNOWN"
+
+
+def test_sizes_host_only(L):
+    from nvfp4_moe_expert_topk_b200 import nvfp4_moe_workspace_region, nvfp4_moe_workspace_size, nvfp4_scales_bytes
+    assert nvfp4_scales_bytes(100, 256, 0) == 100 * 16
+    assert nvfp4_scales_bytes(100, 256, 1) == 128 * 16
+    assert nvfp4_scales_bytes(100, 48, 1) == -1
+    assert nvfp4_scales_bytes(100, 40, 0) == -1
+    ws = nvfp4_moe_workspace_size(4096, 6, 384, 7168, 3072)
+    R = 4096 * 6
+    mt_max = (R + 127 * 384) // 128
+    assert ws >= mt_max * 128 * (7168 // 2 + 7168 // 16 + 3072 // 2 + 3072 // 16) + R * 7168 * 2
+    assert nvfp4_moe_workspace_size(64, 6, 48, 7168, 3000) == 0          # I % 128 != 0
+    assert nvfp4_moe_workspace_size(64, 33, 48, 7168, 3072) == 0         # k > 32
+    assert nvfp4_moe_workspace_size(0, 6, 48, 7168, 3072) > 0
+    off, n = nvfp4_moe_workspace_region(64, 6, 48, 7168, 3072, 4)
+    assert off % 1024 == 0 and n == 64 * 6 * 7168 * 2
+    end = 0
+    for region in range(8):
+        o, n = nvfp4_moe_workspace_region(64, 6, 48, 7168, 3072, region)
+        assert o + n <= nvfp4_moe_workspace_size(64, 6, 48, 7168, 3072)
+
+
+def test_argument_checks_before_any_launch(L):
+    P = ctypes.c_void_p
+    fake = P(1 << 40)                          # never dereferenced: the checks fail first
+    assert L.nvfp4_quantize(None, 4, 64, 64, fake, fake, fake, 0, None) == -1
+    assert L.nvfp4_quantize(fake, 4, 40, 64, fake, fake, fake, 0, None) == -2          # cols % 16
+    assert L.nvfp4_quantize(fake, 4, 48, 48, fake, fake, fake, 1, None) == -2          # MMA layout, cols % 64
+    assert L.nvfp4_quantize(fake, 4, 64, 64, fake, fake, fake, 7, None) == -1          # bad layout
+    assert L.nvfp4_quantize(P((1 << 40) + 4), 4, 64, 64, fake, fake, fake, 0, None) == -3
+    seg = (ctypes.c_int64 * 1)(256)
+    cseg = ctypes.cast(seg, P)
+    assert L.nvfp4_gemm(fake, fake, fake, 8, fake, fake, fake, cseg, 1, 256, 100, fake, 256, None) == -2   # K % 64
+    assert L.nvfp4_gemm(fake, fake, fake, 8, fake, fake, fake, cseg, 1, 200, 128, fake, 256, None) == -2   # N % 128
+    bad = (ctypes.c_int64 * 2)(100, 256)
+    assert L.nvfp4_gemm(fake, fake, fake, 8, fake, fake, fake, ctypes.cast(bad, P), 2, 256, 128, fake, 256,
+                        None) == -1                                                     # segment end % 32
+    assert L.nvfp4_gemm(fake, fake, fake, 8, fake, fake, fake, cseg, 1, 256, 128, fake, 100, None) == -1   # ldo < N
+    assert L.nvfp4_moe_forward(None, fake, 1 << 30, None) == -1
+    assert L.nvfp4_moe_get_error(None, None, None) == -1
+
+
+def test_moe_forward_checks(L):
+    from nvfp4_moe_expert_topk_b200 import MoeArgs
+    a = MoeArgs()
+    F = 1 << 40
+    a.x = a.topk_ids = a.topk_weights = a.x_gs = a.w13_codes = a.w13_scales = F
+    a.w13_gs = a.w2_codes = a.w2_scales = a.w2_gs = a.inter_gs = a.out = F
+    a.T, a.H, a.I, a.E, a.k = 64, 7168, 3072, 48, 6
+    assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1024, None) == -4     # workspace too small
+    a.I = 3000
+    assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None) == -2
+    a.I = 3072
+    a.w2_codes = F + 8
+    assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None) == -3
+    a.w2_codes = None
+    assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None) == -1

@@ -1,0 +1,96 @@
+"""GPU parity of the dense NVFP4 GEMM (the grouped engine with one group):
+one-hot probes that pin nibble order, scale placement and the B halves, then
+random problems against the oracle, including ragged M, a partial last
+k-tile and dual global scales."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from helpers import bf16_to_np, cosine, row_rel_l2, to_mma_layout
+from nvfp4_moe_expert_topk_b200 import nvfp4_gemm
+from nvfp4_moe_expert_topk_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+E2M1 = [0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6]
+
+
+def run_gemm(a_codes, a_sc, a_gs, b_codes, b_sc, b_gs, seg_end):
+    M, N = a_codes.shape[0], b_codes.shape[0]
+    out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    nvfp4_gemm(torch.from_numpy(a_codes).to(DEV), torch.from_numpy(to_mma_layout(a_sc)).to(DEV),
+               torch.tensor([a_gs], dtype=torch.float32, device=DEV), torch.from_numpy(b_codes).to(DEV),
+               torch.from_numpy(to_mma_layout(b_sc)).to(DEV),
+               torch.tensor(np.asarray(b_gs, np.float32), device=DEV), seg_end, out)
+    torch.cuda.synchronize()
+    return bf16_to_np(out)
+
+
+def set_code(codes, r, k, c):
+    b = codes[r, k // 2]
+    codes[r, k // 2] = (b & 0xF0) | c if k % 2 == 0 else (b & 0x0F) | (c << 4)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (128, 128, 512), (200, 512, 1024)])
+def test_one_hot_probes(M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    for trial in range(6):
+        m0, n0, k0 = int(rng.integers(M)), int(rng.integers(N)), int(rng.integers(K))
+        ca, cb = int(rng.integers(1, 16)), int(rng.integers(1, 16))
+        a = np.zeros((M, K // 2), np.uint8)
+        b = np.zeros((N, K // 2), np.uint8)
+        set_code(a, m0, k0, ca)
+        set_code(b, n0, k0, cb)
+        a_sc = np.full((M, K // 16), 0x38, np.uint8)        # 1.0
+        b_sc = np.full((N, K // 16), 0x38, np.uint8)
+        sa, sb = [0x30, 0x40, 0x48][trial % 3], [0x38, 0x44, 0x2C][trial % 3]   # 0.5/2/4, 1/3/0.1875
+        a_sc[m0, k0 // 16] = sa
+        b_sc[n0, k0 // 16] = sb
+        out = run_gemm(a, a_sc, 1.0, b, b_sc, [2.0], [N])
+        want = np.zeros((M, N), np.float32)
+        want[m0, n0] = E2M1[ca] * O.e4m3_decode(sa) * E2M1[cb] * O.e4m3_decode(sb) / 2.0
+        np.testing.assert_array_equal(out, want.astype(np.float32))
+
+
+def quantized_operands(M, N, K, seed, segs):
+    g = torch.Generator().manual_seed(seed)
+    a = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    b = torch.randn(N, K, generator=g) * 0.02
+    start = 0
+    for i, end in enumerate(segs):
+        b[start:end] *= (1.0, 30.0, 0.1, 3.0)[i]
+        start = end
+    b = b.to(torch.bfloat16)
+    ab = W.bf16_bits(a)
+    a_gs = O.global_scale_bf16(ab)
+    ac, asc = O.quantize_bf16(ab, a_gs)
+    bc, bsc, bgs = [], [], []
+    start = 0
+    for end in segs:
+        part = W.bf16_bits(b[start:end])
+        gs = O.global_scale_bf16(part)
+        c, s = O.quantize_bf16(part, gs)
+        bc.append(c), bsc.append(s), bgs.append(gs)
+        start = end
+    return ac, asc, a_gs, np.concatenate(bc), np.concatenate(bsc), np.array(bgs, np.float32)
+
+
+@pytest.mark.parametrize("M,N,K,segs", [
+    (128, 256, 256, [256]),
+    (1, 128, 64, [128]),            # single row, one k-block
+    (64, 256, 192, [256]),          # partial last k-tile (3 of 4 k-blocks)
+    (200, 384, 512, [128, 384]),    # ragged M, N % 256 != 0, two global scales
+    (257, 512, 1536, [256, 512]),   # q_b-like K
+    (130, 2048, 7168, [1536, 2048]),  # fused_wqa_wkv-like: dual global scales split at 1536
+    (300, 1024, 8192, [1024]),      # o_b-like K
+])
+def test_gemm_matches_oracle(M, N, K, segs):
+    ac, asc, a_gs, bc, bsc, bgs = quantized_operands(M, N, K, M * 7 + N, segs)
+    ref = O.gemm(ac, asc, a_gs, bc, bsc, bgs, segs)
+    out = run_gemm(ac, asc, a_gs, bc, bsc, bgs, segs)
+    assert np.all(np.isfinite(out))
+    err = row_rel_l2(out, ref)
+    assert err.max() <= 5e-3, err.max()
+    assert cosine(out, ref) >= 0.99999

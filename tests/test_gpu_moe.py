@@ -1,0 +1,263 @@
+"""GPU parity of the whole routed-expert chain (nvfp4_moe_forward) against
+the oracle on the same quantised operands.
+
+Bars: routing, x codes and x scales bit-exact; output per row
+||gpu - ref||_2 / ||ref||_2 <= 2e-2 and cosine >= 0.9995; h codes (which
+depend on fp32 accumulation order) >= 99% identical with every mismatch an
+adjacent code; the L2 GEMM fed the GPU's own h within 5e-3 per row."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from helpers import OracleWeights, bf16_to_np, cosine, from_mma_layout, row_max_rel, row_rel_l2
+from nvfp4_moe_expert_topk_b200 import (nvfp4_global_scale, nvfp4_moe_calibrate, nvfp4_moe_forward,
+                                        nvfp4_moe_get_error, nvfp4_moe_workspace_region)
+from nvfp4_moe_expert_topk_b200 import prep
+from nvfp4_moe_expert_topk_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+ROW_TOL = 2e-2
+COS_TOL = 0.9995
+
+
+class Problem:
+    """A config's batch on the device plus oracle-side weights of the experts
+    it touches; inter_gs from the oracle's warmup (reading R8)."""
+
+    def __init__(self, cfg, oracle_tokens=None):
+        self.cfg = cfg
+        x, ids, w = W.batch(cfg)
+        self.x, self.ids, self.w = x, ids, w
+        xw, idw, ww = W.batch(cfg, warmup=True)
+        if oracle_tokens is None:
+            experts = list(range(cfg.E))
+        else:                   # oracle weights only for the experts the oracle will touch
+            used = set(np.unique(ids.numpy()[oracle_tokens]).tolist()) | set(np.unique(idw.numpy()).tolist())
+            experts = sorted(used)
+        self.ow = OracleWeights(cfg, experts, DEV)
+        self.dw = prep.MoeWeights.synthetic(cfg, DEV)
+        # warmup: per-expert max|h| on the warmup batch, 2688/amax, fallback for experts without rows
+        xwb = W.bf16_bits(xw)
+        _, inter = O.moe_forward(xwb, self.ow.remap_ids(idw.numpy()), ww.numpy(), O.global_scale_bf16(xwb),
+                                 **self.ow.oracle_kwargs(), inter_gs=None, intermediates=True)
+        amax = inter["h_amax"]
+        full = np.zeros(cfg.E, np.float32)
+        full[self.ow.experts] = amax
+        gmax = full.max()
+        self.inter_gs = np.array([O.global_scale_from_amax(a if a > 0 else gmax) for a in full], np.float32)
+        self.x_gs = O.global_scale_bf16(W.bf16_bits(x))
+
+    def oracle(self, intermediates=False):
+        return O.moe_forward(W.bf16_bits(self.x), self.ow.remap_ids(self.ids.numpy()), self.w.numpy(), self.x_gs,
+                             **self.ow.oracle_kwargs(), inter_gs=self.inter_gs[self.ow.experts],
+                             intermediates=intermediates)
+
+    def device_inputs(self):
+        return dict(x=self.x.to(DEV), topk_ids=self.ids.to(DEV), topk_weights=self.w.to(DEV),
+                    x_gs=torch.tensor([self.x_gs], device=DEV), **self.dw.args(),
+                    inter_gs=torch.from_numpy(self.inter_gs).to(DEV))
+
+    def run(self, inputs=None, ws=None):
+        cfg = self.cfg
+        T = self.x.shape[0]
+        inputs = inputs or self.device_inputs()
+        ws = prep.workspace(T, cfg.k, cfg.E, cfg.H, cfg.I, DEV) if ws is None else ws
+        out = torch.full((T, cfg.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+        nvfp4_moe_forward(**inputs, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        return out, ws
+
+
+def check_output(out, ref):
+    got = bf16_to_np(out)
+    assert np.all(np.isfinite(got))
+    err = row_rel_l2(got, ref)
+    assert err.max() <= ROW_TOL, (err.max(), err.argmax())
+    assert row_max_rel(got, ref).max() <= ROW_TOL
+    assert cosine(got, ref) >= COS_TOL
+
+
+def region(p, r):
+    cfg = p.cfg
+    T = p.x.shape[0]
+    return nvfp4_moe_workspace_region(T, cfg.k, cfg.E, cfg.H, cfg.I, r)
+
+
+def check_weights_bitexact(p, experts):
+    """The device-quantised weights equal the oracle's for these experts."""
+    cfg = p.cfg
+    H, I = cfg.H, cfg.I
+    for i, e in enumerate(experts):
+        j = p.ow.experts.index(e)
+        np.testing.assert_array_equal(p.dw.w13_codes[e].cpu().numpy(), p.ow.w13_codes[j])
+        np.testing.assert_array_equal(p.dw.w13_gs[e].cpu().numpy(), p.ow.w13_gs[j])
+        s13 = 2 * I * (H // 16)
+        np.testing.assert_array_equal(
+            from_mma_layout(p.dw.w13_scales[e * s13:(e + 1) * s13].cpu().numpy(), 2 * I, H), p.ow.w13_scales[j])
+        np.testing.assert_array_equal(p.dw.w2_codes[e].cpu().numpy(), p.ow.w2_codes[j])
+        assert p.dw.w2_gs[e].item() == p.ow.w2_gs[j]
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    return Problem(W.MOE_CONFIGS["tiny"])
+
+
+def test_tiny_end_to_end_and_intermediates(tiny):
+    p = tiny
+    cfg = p.cfg
+    T, k, H, I = p.x.shape[0], cfg.k, cfg.H, cfg.I
+    check_weights_bitexact(p, range(cfg.E))
+    out, ws = p.run()
+    ref, inter = p.oracle(intermediates=True)
+    check_output(out, ref)
+    assert nvfp4_moe_get_error(ws) == 0
+    wsn = ws.cpu().numpy()
+
+    route = O.route(p.ids.numpy(), cfg.E)
+    o, n = region(p, 5)
+    inv = wsn[o:o + n].view(np.int32)
+    np.testing.assert_array_equal(inv, route["pos_padded"])
+    o, n = region(p, 6)
+    np.testing.assert_array_equal(wsn[o:o + n].view(np.int32), route["counts"])
+
+    # x codes / scales at every slot's padded row: bit-exact
+    xc, xs = O.quantize_bf16(W.bf16_bits(p.x), p.x_gs)
+    o, n = region(p, 0)
+    a_codes = wsn[o:o + n].reshape(-1, H // 2)
+    o, n = region(p, 1)
+    a_sc = from_mma_layout(wsn[o:o + n], a_codes.shape[0], H)
+    tok = np.arange(T * k) // k
+    np.testing.assert_array_equal(a_codes[inv], xc[tok])
+    np.testing.assert_array_equal(a_sc[inv], xs[tok])
+
+    # h codes: fp32 accumulation order may move a value across a rounding edge
+    o, n = region(p, 2)
+    h_codes = wsn[o:o + n].reshape(-1, I // 2)[inv]
+    o, n = region(p, 3)
+    h_sc = from_mma_layout(wsn[o:o + n], a_codes.shape[0], I)[inv]
+    ref_q = np.stack([inter["h_codes"] & 15, inter["h_codes"] >> 4], -1).reshape(T * k, I)
+    got_q = np.stack([h_codes & 15, h_codes >> 4], -1).reshape(T * k, I)
+    same = got_q == ref_q
+    assert same.mean() >= 0.99, same.mean()
+    mag = lambda c: np.where(c & 8, -(c & 7).astype(int), (c & 7).astype(int))
+    assert np.all(np.abs(mag(got_q) - mag(ref_q))[~same] <= 1)
+    assert (h_sc == inter["h_scales"]).mean() >= 0.99
+
+    # staged: oracle L2 on the GPU's own h, per expert, against the GPU's y
+    o, n = region(p, 4)
+    y = wsn[o:o + n].view(np.uint16).reshape(T * k, H)
+    y = (y.astype(np.uint32) << 16).view(np.float32)
+    yrow = route["offsets"][p.ids.numpy().reshape(-1)] + route["rank"]
+    for e in range(cfg.E):
+        sl = np.nonzero(p.ids.numpy().reshape(-1) == e)[0]
+        if sl.size == 0:
+            continue
+        ye = O.gemm(h_codes[sl], h_sc[sl], p.inter_gs[e], p.ow.w2_codes[e], p.ow.w2_scales[e], p.ow.w2_gs[e:e + 1])
+        err = row_rel_l2(y[yrow[sl]], ye)
+        assert err.max() <= 5e-3, (e, err.max())
+
+
+def test_tiny_with_skipped_slots(tiny):
+    p = tiny
+    inputs = p.device_inputs()
+    ids = p.ids.clone()
+    ids[::3, 1] = -1
+    inputs["topk_ids"] = ids.to(DEV)
+    out, ws = p.run(inputs)
+    ref = O.moe_forward(W.bf16_bits(p.x), ids.numpy(), p.w.numpy(), p.x_gs, **p.ow.oracle_kwargs(),
+                        inter_gs=p.inter_gs)
+    check_output(out, ref)
+    assert nvfp4_moe_get_error(ws) == 0
+
+
+def test_tiny_bad_ids_set_error_word(tiny):
+    p = tiny
+    inputs = p.device_inputs()
+    ids = p.ids.clone()
+    ids[5, 0] = p.cfg.E + 3
+    inputs["topk_ids"] = ids.to(DEV)
+    out, ws = p.run(inputs)
+    assert nvfp4_moe_get_error(ws) == -8
+    ids_skip = ids.numpy().copy()
+    ids_skip[5, 0] = -1
+    ref = O.moe_forward(W.bf16_bits(p.x), ids_skip, p.w.numpy(), p.x_gs, **p.ow.oracle_kwargs(),
+                        inter_gs=p.inter_gs)
+    check_output(out, ref)
+
+
+def test_calibrate_matches_oracle_warmup(tiny):
+    p = tiny
+    cfg = p.cfg
+    xw, idw, ww = W.batch(cfg, warmup=True)
+    gs = torch.empty(1, dtype=torch.float32, device=DEV)
+    nvfp4_global_scale(xw.to(DEV), gs)
+    ws = prep.workspace(xw.shape[0], cfg.k, cfg.E, cfg.H, cfg.I, DEV)
+    got = torch.empty(cfg.E, dtype=torch.float32, device=DEV)
+    nvfp4_moe_calibrate(xw.to(DEV), idw.to(DEV), ww.to(DEV), gs, **p.dw.args(), inter_gs_out=got, workspace=ws)
+    got = got.cpu().numpy()
+    np.testing.assert_allclose(got, p.inter_gs, rtol=2e-6)
+
+
+def test_cuda_graph_replay_with_new_inputs(tiny):
+    """Capture once, replay with new x and topk ids of the same shape
+    (page 1 "Phase 1": cudagraph-safe runner, pre-allocated buffers)."""
+    p = tiny
+    cfg = p.cfg
+    T = p.x.shape[0]
+    inputs = p.device_inputs()
+    ws = prep.workspace(T, cfg.k, cfg.E, cfg.H, cfg.I, DEV)
+    out = torch.empty(T, cfg.H, dtype=torch.bfloat16, device=DEV)
+    nvfp4_moe_forward(**inputs, out=out, workspace=ws)          # eager call first (per-kernel attributes)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            nvfp4_moe_forward(**inputs, out=out, workspace=ws, stream=s)
+    g2 = torch.Generator().manual_seed(99)
+    x2 = torch.randn(T, cfg.H, generator=g2).to(torch.bfloat16)
+    ids2 = torch.stack([torch.randperm(cfg.E, generator=g2)[:cfg.k] for _ in range(T)]).to(torch.int32)
+    inputs["x"].copy_(x2.to(DEV))
+    inputs["topk_ids"].copy_(ids2.to(DEV))
+    g.replay()
+    torch.cuda.synchronize()
+    ref = O.moe_forward(W.bf16_bits(x2), ids2.numpy(), p.w.numpy(), p.x_gs, **p.ow.oracle_kwargs(),
+                        inter_gs=p.inter_gs)
+    check_output(out, ref)
+    eager = torch.empty_like(out)
+    nvfp4_moe_forward(**inputs, out=eager, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(eager, out)
+
+
+@pytest.mark.parametrize("name", ["decode", "shared"])
+def test_full_size_configs(name):
+    cfg = W.MOE_CONFIGS[name]
+    p = Problem(cfg)
+    check_weights_bitexact(p, [0, cfg.E - 1])
+    out, ws = p.run()
+    ref = p.oracle()
+    check_output(out, ref)
+    assert nvfp4_moe_get_error(ws) == 0
+
+
+def test_prefill_sampled_tokens():
+    """384 experts, Zipf-skewed routing with empty experts: the whole batch on
+    the GPU, sampled tokens through the oracle."""
+    cfg = W.MOE_CONFIGS["prefill"]
+    tokens = np.sort(np.random.default_rng(0).choice(cfg.T, 6, replace=False))
+    p = Problem(cfg, oracle_tokens=tokens)
+    route = O.route(p.ids.numpy(), cfg.E)
+    assert (route["counts"] == 0).sum() >= 16                  # some experts are empty
+    check_weights_bitexact(p, p.ow.experts[:2])
+    out, ws = p.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    ref = O.moe_forward(W.bf16_bits(p.x[tokens]), p.ow.remap_ids(p.ids.numpy()[tokens]), p.w.numpy()[tokens],
+                        p.x_gs, **p.ow.oracle_kwargs(), inter_gs=p.inter_gs[p.ow.experts])
+    check_output(out[torch.from_numpy(tokens).to(DEV)], ref)
+    # every routed row of the batch: inv matches the oracle's stable positions
+    o, n = region(p, 5)
+    np.testing.assert_array_equal(ws[o:o + n].cpu().numpy().view(np.int32), route["pos_padded"])
