@@ -236,7 +236,7 @@ class Workload:
         return self.nonempty * 3 * c.H * c.I * fp4 + 2 * c.T * c.H * 2.0 + c.T * c.k * 8.0
 
 
-def time_steps(wl, steps, warmup, world, timed_events=True):
+def time_steps(wl, steps, warmup, world, timed_events=True, tag="timed"):
     """Device time of `steps` steps (events on the launching stream, barrier +
     synchronize on both sides), and per-stage mean durations."""
     stream = torch.cuda.current_stream()
@@ -245,8 +245,14 @@ def time_steps(wl, steps, warmup, world, timed_events=True):
     barrier(world)
     torch.cuda.synchronize()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)] if timed_events else None
+    if ev is not None:                  # create the CUDA events outside the timed region
+        for row in ev:
+            for e in row:
+                e.record(stream)
+        torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push(f"{tag}_{wl.cfg.name}")
     t0.record(stream)
     for i in range(steps):
         if ev is not None:
@@ -255,6 +261,7 @@ def time_steps(wl, steps, warmup, world, timed_events=True):
         else:
             wl.step()
     t1.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier(world)
     ms = t0.elapsed_time(t1)
@@ -373,6 +380,8 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     steps, warmup = args.steps, max(3, args.warmup)
 
+    if args.only == "decode":
+        return run_decode_only(args, world, rank, dev, peaks, peak_src, steps, warmup)
     pre = Workload(W.MOE_CONFIGS["prefill"], dev)
     dec = Workload(W.MOE_CONFIGS["decode"], dev)
     torch.cuda.synchronize()
@@ -453,6 +462,33 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_decode_only(args, world, rank, dev, peaks, peak_src, steps, warmup):
+    """The 48-expert decode workload alone (a small case for profiling)."""
+    dec = Workload(W.MOE_CONFIGS["decode"], dev)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    ms_dec, stages = time_steps(dec, steps, warmup, world)
+    clocks.stop()
+    err = nvfp4_moe_get_error(dec.ws)
+    if err != 0:
+        raise RuntimeError(f"device error word {err}")
+    t = ms_dec / steps / 1e3
+    gbs = dec.step_bytes() / t / 1e9
+    kb = dec.kernel_bytes()
+    dom = max(STAGES, key=lambda s: stages[s])
+    achieved = kb[dom] / (stages[dom] / 1e3) / 1e9
+    line = {"metric": "moe_decode_GB_per_s", "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
+            "warmup": warmup, "ms_per_step": ms_dec / steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic", "config": config_block(dec.cfg, world),
+            "hbm_frac": gbs / peaks["hbm_gbs"], "stage_ms": stages,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
+                         "algorithmic_bytes": kb[dom], "traffic": ncu_traffic(dom, "decode")},
+            "gpu_launches": KERNELS_PER_STEP * steps, "clocks": clocks.summary()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_reference(args):
     """The CPU oracle on this host's cores, one token of the prefill batch per
     step (cycling through a fixed sample), rank 0 only."""
@@ -468,7 +504,6 @@ def run_reference(args):
     tokens = np.sort(np.random.default_rng(321).choice(cfg.T, 4, replace=False))
     # warmup inter_gs is the library's; it only sets the arithmetic's scale, not the work
     if dev.type == "cuda":
-        inter = Workload.__new__(Workload)
         inter_gs = _calibrated_inter_gs(cfg, dev)
     else:
         inter_gs = torch.full((cfg.E,), 1000.0)
@@ -510,6 +545,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "decode"], default="all",
+                    help="decode: the 48-expert decode workload alone (small profiling case)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

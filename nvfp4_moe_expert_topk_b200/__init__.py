@@ -180,6 +180,9 @@ def nvfp4_moe_forward_timed(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scal
                   inter_gs, out)
     if len(events) != 6:
         raise ValueError("events must hold 6 torch.cuda.Event objects")
+    for e in events:
+        if e.cuda_event == 0:           # torch creates the CUDA event on its first record()
+            e.record()
     ev = (ctypes.c_void_p * 6)(*[e.cuda_event for e in events])
     _check(lib().nvfp4_moe_forward_timed(ctypes.byref(a), _dev(workspace, "workspace", torch.uint8),
                                          workspace.numel(), _stream(stream), ev), "nvfp4_moe_forward_timed")
