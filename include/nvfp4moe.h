@@ -175,6 +175,25 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
 int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, int region,
                                int64_t *offset, int64_t *bytes);
 
+/* nvfp4_moe_forward without a caller-supplied workspace, for callers that
+ * cannot allocate device memory: code running while a CUDA graph is being
+ * captured (cudaMalloc cannot be captured), plug-ins whose host framework
+ * owns all device memory and forbids side allocations, and latency-critical
+ * paths that cannot take cudaMalloc's implicit synchronisation.  The pages
+ * have no counterpart of this entry point; it is a deployment convenience.
+ * Scratch: one static device array of NVFP4_NOALLOC_SCRATCH_BYTES (32 MiB)
+ * that every device using this entry point holds until the process exits;
+ * shapes whose nvfp4_moe_workspace_size() exceeds it return
+ * NVFP4_ERR_WORKSPACE_TOO_SMALL without launching.  The call allocates
+ * nothing.  Its first call on a device looks up the array's device address
+ * with that device current; make that first call before any stream capture.
+ * All calls on a device share the array (it keeps the last call's contents,
+ * and each call clears its error word), so calls that overlap on the GPU
+ * race: serialise them (one stream, or events).  Device-side errors (a top-k
+ * id >= E) skip the slot as in nvfp4_moe_forward but cannot be read back. */
+#define NVFP4_NOALLOC_SCRATCH_BYTES (32u << 20)
+int nvfp4_moe_forward_noalloc(const nvfp4_moe_args *args, void *stream);
+
 /* Reads and clears the sticky device error word of a workspace (host
  * err_host receives NVFP4_OK or a device error code).  Synchronises
  * `stream`. */

@@ -16,7 +16,7 @@ __all__ = [
     "Nvfp4Error", "lib", "NVFP4_SCALES_ROWMAJOR", "NVFP4_SCALES_MMA",
     "nvfp4_status_string", "nvfp4_global_scale", "nvfp4_scales_bytes", "nvfp4_quantize",
     "nvfp4_swizzle_scales", "nvfp4_gemm", "nvfp4_moe_workspace_size", "nvfp4_moe_forward",
-    "nvfp4_moe_forward_timed",
+    "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
     "nvfp4_moe_get_error", "MoeArgs",
 ]
@@ -68,6 +68,7 @@ def lib():
         L.nvfp4_moe_forward.argtypes = [ctypes.POINTER(MoeArgs), P, ctypes.c_size_t, P]
         L.nvfp4_moe_forward_timed.argtypes = [ctypes.POINTER(MoeArgs), P, ctypes.c_size_t, P,
                                               ctypes.POINTER(ctypes.c_void_p)]
+        L.nvfp4_moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeArgs), P]
         L.nvfp4_moe_calibrate.argtypes = [ctypes.POINTER(MoeArgs), P, P, ctypes.c_size_t, P]
         L.nvfp4_moe_route_debug.argtypes = [P, i64, i32, i32, P, P, P, P, ctypes.c_size_t, P]
         L.nvfp4_moe_workspace_region.argtypes = [i64, i32, i32, i64, i64, i32,
@@ -186,6 +187,16 @@ def nvfp4_moe_forward_timed(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scal
     ev = (ctypes.c_void_p * 6)(*[e.cuda_event for e in events])
     _check(lib().nvfp4_moe_forward_timed(ctypes.byref(a), _dev(workspace, "workspace", torch.uint8),
                                          workspace.numel(), _stream(stream), ev), "nvfp4_moe_forward_timed")
+
+
+def nvfp4_moe_forward_noalloc(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs, w2_codes,
+                              w2_scales, w2_gs, inter_gs, out, stream=None):
+    """nvfp4_moe_forward with the library's own fixed 32 MiB device scratch
+    instead of a workspace (for callers that cannot allocate device memory);
+    calls that overlap on the GPU race for that scratch."""
+    a = _moe_args(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs, w2_codes, w2_scales, w2_gs,
+                  inter_gs, out)
+    _check(lib().nvfp4_moe_forward_noalloc(ctypes.byref(a), _stream(stream)), "nvfp4_moe_forward_noalloc")
 
 
 def nvfp4_moe_calibrate(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs, w2_codes, w2_scales,
