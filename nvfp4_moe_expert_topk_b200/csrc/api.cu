@@ -57,13 +57,13 @@ int device_check(int *num_sms)
 }
 
 // 2-D uint8 tensor map over a row-major code matrix [rows, cols_bytes]
-// (row stride cols_bytes), box 128 rows x 128 bytes, 128-byte swizzle; rows
-// and columns outside the matrix read as zero.
-int make_code_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols_bytes)
+// (row stride cols_bytes), box box_rows rows x 128 bytes, 128-byte swizzle;
+// rows and columns outside the matrix read as zero.
+int make_code_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols_bytes, int box_rows)
 {
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols_bytes), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols_bytes)};
-    cuuint32_t box[2] = {128, 128};
+    cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -167,7 +167,7 @@ int mark(void *const *events, int i, cudaStream_t s)
 }
 
 int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi, void *const *events,
-              cudaStream_t s, int num_sms, CUtensorMap *map_a1, CUtensorMap *map_b1)
+              cudaStream_t s, int num_sms)
 {
     const int64_t T = a->T, H = a->H, I = a->I, R = T * a->k;
     const int E = a->E, k = a->k;
@@ -189,9 +189,12 @@ int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi,
     if (e != cudaSuccess || mark(events, 2, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
 
-    int st = make_code_map(map_a1, ws + L.a_codes, L.rpad, H / 2);
+    CUtensorMap ma, ma32, mb;
+    int st = make_code_map(&ma, ws + L.a_codes, L.rpad, H / 2, 128);
     if (st == NVFP4_OK)
-        st = make_code_map(map_b1, a->w13_codes, static_cast<int64_t>(E) * 2 * I, H / 2);
+        st = make_code_map(&ma32, ws + L.a_codes, L.rpad, H / 2, 32);
+    if (st == NVFP4_OK)
+        st = make_code_map(&mb, a->w13_codes, static_cast<int64_t>(E) * 2 * I, H / 2, 64);
     if (st != NVFP4_OK)
         return st;
     GemmArgs g{};
@@ -203,9 +206,9 @@ int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi,
     g.num_k_tiles = static_cast<int>((H + 255) / 256);
     g.num_mtiles_dev = num_mt;
     g.mtiles = mtiles;
-    g.n_tiles = static_cast<int>(I / 128);
+    g.n_tiles = static_cast<int>(I / 64);
     g.b_rows_per_expert = 2 * I;
-    g.b_tile_rows = 128;
+    g.b_tile_rows = 64;
     g.b_half_offset = static_cast<int>(I);
     g.a_gs = a->x_gs;
     g.a_gs_per_expert = 0;
@@ -219,7 +222,7 @@ int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi,
     g.h_sf_block_stride = (I / 64) * 512;
     g.amax_bits = reinterpret_cast<unsigned int *>(ws + L.amax);
     g.err = err;
-    return cuda_status(launch_gemm(256, l1_epi, *map_a1, *map_b1, g, num_sms, s));
+    return cuda_status(launch_gemm(l1_epi, ma, ma32, mb, g, num_sms, s));
 }
 
 } // namespace
@@ -334,13 +337,15 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_g
     int st = device_check(&sms);
     if (st != NVFP4_OK)
         return st;
-    CUtensorMap ma, mb;
-    st = make_code_map(&ma, a_codes, M, K / 2);
+    CUtensorMap ma, ma32, mb;
+    st = make_code_map(&ma, a_codes, M, K / 2, 128);
     if (st == NVFP4_OK)
-        st = make_code_map(&mb, b_codes, N, K / 2);
+        st = make_code_map(&ma32, a_codes, M, K / 2, 32);
+    if (st == NVFP4_OK)
+        st = make_code_map(&mb, b_codes, N, K / 2, 128);
     if (st != NVFP4_OK)
         return st;
-    const int bn = (N % 256 == 0) ? 256 : 128;
+    const int bn = 128;
     GemmArgs g{};
     g.sfa = a_scales;
     g.sfa_block_stride = (K / 64) * 512;
@@ -368,7 +373,7 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_g
     g.err = nullptr;            // no workspace: a timed-out wait ends the kernel without a report
     int64_t tiles = static_cast<int64_t>(g.dense_m_tiles) * g.n_tiles;
     const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
-    return cuda_status(launch_gemm(bn, EPI_BF16, ma, mb, g, grid, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_gemm(EPI_BF16, ma, ma32, mb, g, grid, static_cast<cudaStream_t>(stream)));
 }
 
 size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I)
@@ -423,19 +428,21 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
         return NVFP4_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    CUtensorMap ma1, mb1, ma2, mb2;
-    st = run_front(a, ws, L, EPI_SWIGLU_QUANT, events, s, sms, &ma1, &mb1);
+    st = run_front(a, ws, L, EPI_SWIGLU_QUANT, events, s, sms);
     if (st != NVFP4_OK)
         return st;
 
     const int64_t H = a->H, I = a->I;
     const int E = a->E;
-    st = make_code_map(&ma2, ws + L.h_codes, L.rpad, I / 2);
+    CUtensorMap ma2, ma2_32, mb2;
+    st = make_code_map(&ma2, ws + L.h_codes, L.rpad, I / 2, 128);
     if (st == NVFP4_OK)
-        st = make_code_map(&mb2, a->w2_codes, static_cast<int64_t>(E) * H, I / 2);
+        st = make_code_map(&ma2_32, ws + L.h_codes, L.rpad, I / 2, 32);
+    if (st == NVFP4_OK)
+        st = make_code_map(&mb2, a->w2_codes, static_cast<int64_t>(E) * H, I / 2, 128);
     if (st != NVFP4_OK)
         return st;
-    const int bn = (H % 256 == 0) ? 256 : 128;
+    const int bn = 128;
     GemmArgs g{};
     g.sfa = ws + L.h_sf;
     g.sfa_block_stride = (I / 64) * 512;
@@ -458,7 +465,7 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
     g.out = reinterpret_cast<__nv_bfloat16 *>(ws + L.y);
     g.ldo = H;
     g.err = reinterpret_cast<int32_t *>(ws);
-    if (mark(events, 3, s) != NVFP4_OK || launch_gemm(bn, EPI_BF16, ma2, mb2, g, sms, s) != cudaSuccess ||
+    if (mark(events, 3, s) != NVFP4_OK || launch_gemm(EPI_BF16, ma2, ma2_32, mb2, g, sms, s) != cudaSuccess ||
         mark(events, 4, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
 
@@ -507,8 +514,7 @@ int nvfp4_moe_calibrate(const nvfp4_moe_args *a, float *inter_gs_out, void *work
     if (cudaMemsetAsync(ws + L.amax, 0, 4 * static_cast<size_t>(a->E), s) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     if (a->T > 0) {
-        CUtensorMap ma1, mb1;
-        st = run_front(a, ws, L, EPI_SWIGLU_AMAX, nullptr, s, sms, &ma1, &mb1);
+        st = run_front(a, ws, L, EPI_SWIGLU_AMAX, nullptr, s, sms);
         if (st != NVFP4_OK)
             return st;
     }

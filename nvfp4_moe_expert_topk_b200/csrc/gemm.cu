@@ -1,6 +1,6 @@
 // gemm.cu -- persistent block-scaled FP4 GEMM engine for sm_100a.
 //
-// D[128 x BN] tiles of  A (E2M1 codes, K-major) x B^T (E2M1 codes, K-major)
+// D[128 x 128] tiles of  A (E2M1 codes, K-major) x B^T (E2M1 codes, K-major)
 // with one E4M3 scale per 16 elements on both sides, on the 5th-generation
 // tensor cores (tcgen05.mma kind::mxf4nvf4, block16 scaling), accumulating in
 // fp32 in tensor memory.  This is the grouped GEMM of the expert chain
@@ -8,28 +8,39 @@
 // GEMM -> SiLU -> re-quantise -> L2 GEMM; with one group it is the plain
 // NVFP4 GEMM of page 1 "Phase 2").
 //
-// Block of 6 warps, one block per SM, persistent over the tile list:
-//   warp 0    TMA producer: per k-tile (256 elements) one 128x128-byte box
-//             of A, one or two 128x128-byte boxes of B (128-byte swizzle),
-//             and the matching 512-byte scale atoms by bulk copy, into a
-//             4-stage shared-memory ring guarded by mbarriers;
-//   warp 1    allocates TMEM, and one thread issues tcgen05.cp (scales ->
-//             TMEM) and tcgen05.mma (4 instructions of K=64 per k-tile);
+// Block of 10 warps, one block per SM, persistent over the tile list:
+//   warp 0    TMA producer: per k-tile (256 elements) the valid 32-row boxes
+//             (or one 128-row box) of A, the 128 rows of B, and the matching
+//             512-byte scale atoms by bulk copy, into a 5- or 6-stage
+//             shared-memory ring guarded by mbarriers;
+//   warps 6-9 scale stagers, one per TMEM lane quarter: move each stage's
+//             E4M3 scales from shared memory into that stage's TMEM scale
+//             slot with tcgen05.st (the layout the MMA reads: lane l, column
+//             4*kb + m holds the 4 scales of row 32*m + l, replicated in all
+//             four quarters), then signal the stage's sf_ready barrier;
+//             scale copies through the tensor pipe (tcgen05.cp) cost more
+//             pipe time than the MMAs they feed at these tile sizes;
+//   warp 1    allocates TMEM; one thread issues the 4 tcgen05.mma (K=64) of
+//             each k-tile into one of two 128-column accumulators, so the
+//             next tile's MMAs run while the epilogue drains the previous;
 //   warps 2-5 epilogue: TMEM -> registers (each thread owns one row of the
-//             128-row tile), then one of
+//             tile), then one of
 //             EPI_SWIGLU_QUANT  h = SiLU(a_g*g) * (a_u*u), NVFP4-quantised
 //                               with the expert's inter_gs (L1),
 //             EPI_SWIGLU_AMAX   same h, max|h| per expert (warmup),
 //             EPI_BF16          y = alpha * acc -> bf16 (L2, dense GEMM).
-// In the L1 tile the B tile is 128 gate rows stacked on the 128 matching up
-// rows, so TMEM columns 0-127 hold gate and 128-255 hold up of the same h
-// columns, and every 16-element block of h is produced by one thread.
+// In the L1 tile the B tile is 64 gate rows stacked on the matching 64 up
+// rows (the weight keeps its [gate; up] layout: two 64-row boxes), so TMEM
+// columns 0-63 hold gate and 64-127 hold up of the same 64 h columns and each
+// 16-element block of h is produced by one thread.  The scales of those two
+// 64-row halves sit in two different 128-row scale atoms; the stagers pair
+// their 32-row groups on the way into TMEM.
 //
-// The tile list is either dense (m-tiles of M) or grouped: an m-tile table
-// written on the device by the routing kernel (expert, first padded row,
-// valid rows, first output row), so the launch needs no host sync and every
-// expert's rows are covered by one tensor map over the padded A buffer and
-// one over all experts' stacked weights.
+// The tile list is either dense (m-tiles of M, n-major) or grouped: an
+// m-tile table written on the device by the routing kernel (expert, first
+// padded row, valid rows, first output row), so the launch needs no host
+// sync and every expert's rows are covered by one tensor map over the padded
+// A buffer and one over all experts' stacked weights.
 //
 // Every mbarrier wait is bounded (ptx.cuh): on a timeout the block records
 // NVFP4_ERR_TIMEOUT in the error word, stops issuing, waits (bounded) for its
@@ -40,36 +51,33 @@
 namespace nvfp4 {
 
 constexpr int kBM = 128;
+constexpr int kBN = 128;
 constexpr int kBK = 256;                        // elements per k-tile
 constexpr int kBKBytes = 128;                   // bytes of codes per row per k-tile
-constexpr int kStages = 4;
-constexpr int kATileBytes = kBM * kBKBytes;     // 16 KB
-constexpr int kBHalfBytes = 128 * kBKBytes;     // 16 KB
-constexpr int kSFAtom = 512;                    // 128 rows x 4 scales
-constexpr int kThreads = 192;
+constexpr int kTileBytes = 128 * kBKBytes;      // 16 KB: 128 rows of one k-tile
+constexpr int kSFAtom = 512;                    // 128 rows x 4 scales (64 elements)
+constexpr int kSFStage = 4 * kSFAtom;           // one 128-row block, 4 k-blocks
+constexpr int kNumAcc = 2;                      // TMEM accumulators
+constexpr int kThreads = 320;
+constexpr int kFirstSFWarp = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSFA = 256;              // 4 k-blocks x 4 columns
-constexpr uint32_t kTmemSFB = 272;              // 4 k-blocks x (4 or 8) columns
+constexpr uint32_t kTmemSF = kNumAcc * kBN;     // 256: per-stage scale slots follow the accumulators
+constexpr uint32_t kSFSlotCols = 32;            // A: 4 k-blocks x 4 columns, then B: the same
 
-template <int BN>
+template <int EPI>
 struct Smem {
-    static constexpr int kHalves = BN / 128;
-    static constexpr int kBTileBytes = BN * kBKBytes;
-    static constexpr int kSFBStageBytes = kHalves * 4 * kSFAtom;
+    static constexpr bool kPaired = EPI != EPI_BF16;
+    static constexpr int kStages = kPaired ? 5 : 6;
     static constexpr int kA = 0;
-    static constexpr int kB = kA + kStages * kATileBytes;
-    static constexpr int kSFA = kB + kStages * kBTileBytes;
-    static constexpr int kSFB = kSFA + kStages * 4 * kSFAtom;
-    static constexpr int kBars = kSFB + kStages * kSFBStageBytes;
-    static constexpr int kBarCount = 2 * kStages + 3;
+    static constexpr int kB = kA + kStages * kTileBytes;
+    static constexpr int kSFA = kB + kStages * kTileBytes;
+    static constexpr int kSFB = kSFA + kStages * kSFStage;              // paired: gate atoms, then up atoms
+    static constexpr int kBars = kSFB + kStages * kSFStage * (kPaired ? 2 : 1);
+    static constexpr int kBarCount = 3 * kStages + 2 * kNumAcc + 1;
     static constexpr int kMisc = kBars + kBarCount * 8;
     static constexpr int kTotal = kMisc + 16 + 1024;   // + tmem slot, abort flag, alignment slack
+    static_assert(kTmemSF + kStages * kSFSlotCols <= kTmemCols, "TMEM scale slots");
 };
-
-int gemm_smem_bytes(int bn)
-{
-    return bn == 256 ? Smem<256>::kTotal : Smem<128>::kTotal;
-}
 
 struct TileInfo {
     int e, row0, valid, row0_out, nt;
@@ -98,24 +106,32 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, int t, int m_
     return ti;
 }
 
+__device__ __forceinline__ int tile_nt(const GemmArgs &p, int t, int m_tiles)
+{
+    return p.mtiles != nullptr ? t % p.n_tiles : t / m_tiles;
+}
+
 __device__ __forceinline__ void record_error(int32_t *err, int code)
 {
     if (err != nullptr)
         atomicCAS(err, 0, code);
 }
 
+// SiLU(g) * u with the fast exponential and division (relative error a few
+// ulp; h is re-quantised to 4 bits right after).
 __device__ __forceinline__ float silu_mul(float g, float u)
 {
-    return g / (1.0f + __expf(-g)) * u;
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-template <int BN, int EPI>
+template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-    nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                      const GemmArgs p)
+    nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a32,
+                      const __grid_constant__ CUtensorMap map_b, const GemmArgs p)
 {
-    using L = Smem<BN>;
-    constexpr int kHalves = L::kHalves;
+    using L = Smem<EPI>;
+    constexpr bool kPaired = L::kPaired;
+    constexpr int kStages = L::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem + L::kA;
@@ -124,9 +140,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sSFB = smem + L::kSFB;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBars);
     uint64_t *empty = full + kStages;
-    uint64_t *acc_full = empty + kStages;
-    uint64_t *acc_empty = acc_full + 1;
-    uint64_t *drain = acc_full + 2;
+    uint64_t *sf_ready = empty + kStages;
+    uint64_t *acc_full = sf_ready + kStages;
+    uint64_t *acc_empty = acc_full + kNumAcc;
+    uint64_t *drain = acc_empty + kNumAcc;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
     __shared__ int never_abort;
@@ -136,14 +153,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sf_ready[s], 4);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4);
+        for (int b = 0; b < kNumAcc; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         never_abort = 0;
         fence_mbar_init();
         tma_prefetch_map(&map_a);
+        tma_prefetch_map(&map_a32);
         tma_prefetch_map(&map_b);
     }
     if (warp == 1) {
@@ -169,6 +190,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const TileInfo ti = decode_tile(p, t, m_tiles);
                 const int64_t brow0 = ti.e * p.b_rows_per_expert + static_cast<int64_t>(ti.nt) * p.b_tile_rows;
                 const int64_t brow1 = brow0 + p.b_half_offset;
+                const int a_boxes = ti.valid >= kBM ? 0 : (ti.valid + 31) / 32;   // 0: one 128-row box
+                const uint32_t a_bytes = a_boxes == 0 ? kTileBytes : a_boxes * (kTileBytes / 4);
                 const uint8_t *sfa = p.sfa + static_cast<int64_t>(ti.row0 / kBM) * p.sfa_block_stride;
                 const uint8_t *sfb0 = p.sfb + (brow0 / 128) * p.sfb_block_stride;
                 const uint8_t *sfb1 = p.sfb + (brow1 / 128) * p.sfb_block_stride;
@@ -179,19 +202,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const int nkb = min(4, (p.K - kt * kBK) / 64);
                     const uint32_t sf_bytes = static_cast<uint32_t>(nkb * kSFAtom);
-                    mbar_arrive_expect_tx(&full[stage],
-                                          kATileBytes + L::kBTileBytes + sf_bytes * (1 + kHalves));
-                    tma_load_2d(sA + stage * kATileBytes, &map_a, kt * kBKBytes, ti.row0, &full[stage]);
-                    tma_load_2d(sB + stage * L::kBTileBytes, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0),
-                                &full[stage]);
-                    bulk_load(sSFA + stage * 4 * kSFAtom, sfa + kt * 4 * kSFAtom, sf_bytes, &full[stage]);
-                    bulk_load(sSFB + stage * L::kSFBStageBytes, sfb0 + kt * 4 * kSFAtom, sf_bytes, &full[stage]);
-                    if (kHalves == 2) {
-                        tma_load_2d(sB + stage * L::kBTileBytes + kBHalfBytes, &map_b, kt * kBKBytes,
-                                    static_cast<int32_t>(brow1), &full[stage]);
-                        bulk_load(sSFB + stage * L::kSFBStageBytes + 4 * kSFAtom, sfb1 + kt * 4 * kSFAtom, sf_bytes,
-                                  &full[stage]);
+                    mbar_arrive_expect_tx(&full[stage], a_bytes + kTileBytes + sf_bytes * (kPaired ? 3 : 2));
+                    uint8_t *a_dst = sA + stage * kTileBytes;
+                    if (a_boxes == 0) {
+                        tma_load_2d(a_dst, &map_a, kt * kBKBytes, ti.row0, &full[stage]);
+                    } else {
+                        for (int i = 0; i < a_boxes; ++i)
+                            tma_load_2d(a_dst + i * (kTileBytes / 4), &map_a32, kt * kBKBytes, ti.row0 + 32 * i,
+                                        &full[stage]);
                     }
+                    uint8_t *b_dst = sB + stage * kTileBytes;
+                    if constexpr (kPaired) {
+                        tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
+                        tma_load_2d(b_dst + kTileBytes / 2, &map_b, kt * kBKBytes, static_cast<int32_t>(brow1),
+                                    &full[stage]);
+                        uint8_t *raw = sSFB + stage * 2 * kSFStage;
+                        bulk_load(raw, sfb0 + kt * kSFStage, sf_bytes, &full[stage]);
+                        bulk_load(raw + kSFStage, sfb1 + kt * kSFStage, sf_bytes, &full[stage]);
+                    } else {
+                        tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
+                        bulk_load(sSFB + stage * kSFStage, sfb0 + kt * kSFStage, sf_bytes, &full[stage]);
+                    }
+                    bulk_load(sSFA + stage * kSFStage, sfa + kt * kSFStage, sf_bytes, &full[stage]);
                     pend_mask |= 1u << stage;
                     pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == kStages) {
@@ -210,40 +242,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait(&full[s], (pend_par >> s) & 1u, &never_abort);
         }
     } else if (warp == 1) {
+        // -------------------------------------------------------- MMA issuer
+        constexpr uint32_t idesc = idesc_nvf4(kBM, kBN);
         if (lane == 0) {
-            // ---------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
-            int stage = 0;
+            int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kBN);
                 for (int kt = 0; kt < p.num_k_tiles; ++kt) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag)) {
+                    if (!mbar_wait(&sf_ready[stage], phase, abort_flag) || !mbar_wait(&full[stage], phase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int nkb = min(4, (p.K - kt * kBK) / 64);
-                    const uint32_t a_addr = smem_u32(sA + stage * kATileBytes);
-                    const uint32_t b_addr = smem_u32(sB + stage * L::kBTileBytes);
-                    const uint32_t sfa_addr = smem_u32(sSFA + stage * 4 * kSFAtom);
-                    const uint32_t sfb_addr = smem_u32(sSFB + stage * L::kSFBStageBytes);
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        tc_cp_32x128b_warpx4(tmem + kTmemSFA + kb * 4, sdesc_scale_block(sfa_addr + kb * kSFAtom));
-#pragma unroll
-                        for (int h = 0; h < kHalves; ++h)
-                            tc_cp_32x128b_warpx4(tmem + kTmemSFB + kb * 4 * kHalves + h * 4,
-                                                 sdesc_scale_block(sfb_addr + h * 4 * kSFAtom + kb * kSFAtom));
-                    }
+                    const uint32_t a_addr = smem_u32(sA + stage * kTileBytes);
+                    const uint32_t b_addr = smem_u32(sB + stage * kTileBytes);
+                    const uint32_t t_sfa = tmem + kTmemSF + static_cast<uint32_t>(stage) * kSFSlotCols;
                     for (int kb = 0; kb < nkb; ++kb)
-                        tc_mma_nvf4(tmem, sdesc_kmajor_sw128(a_addr + kb * 32), sdesc_kmajor_sw128(b_addr + kb * 32),
-                                    idesc, tmem + kTmemSFA + kb * 4, tmem + kTmemSFB + kb * 4 * kHalves,
-                                    (kt | kb) != 0 ? 1u : 0u);
+                        tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(a_addr + kb * 32), sdesc_kmajor_sw128(b_addr + kb * 32),
+                                    idesc, t_sfa + kb * 4, t_sfa + 16 + kb * 4, (kt | kb) != 0 ? 1u : 0u);
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
                         stage = 0;
@@ -252,25 +276,84 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit(acc_full);
-                acc_phase ^= 1u;
+                tc_commit(&acc_full[acc]);
+                if (++acc == kNumAcc) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
             }
             if (!ok) {
                 *abort_flag = 1;
                 record_error(p.err, NVFP4_ERR_TIMEOUT);
             }
-            // all MMAs and scale copies of this thread complete before TMEM is freed
+            // all MMAs of this thread complete before TMEM is freed
             tc_commit(drain);
             mbar_wait(drain, 0, &never_abort);
+        }
+        __syncwarp();
+    } else if (warp >= kFirstSFWarp) {
+        // -------------------------------------------------------- scale stagers
+        const int q = warp & 3;
+        const uint32_t t_q = tmem + (static_cast<uint32_t>(q * 32) << 16) + kTmemSF;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            // paired tiles: byte offset of this tile's two 32-row groups inside a 16-byte scale row
+            const int pair_off = kPaired ? (tile_nt(p, t, m_tiles) & 1) * 8 : 0;
+            for (int kt = 0; kt < p.num_k_tiles; ++kt) {
+                const bool got = mbar_wait(&full[stage], phase, abort_flag);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                const int nkb = min(4, (p.K - kt * kBK) / 64);
+                uint32_t ra[16], rb[16];
+                const uint8_t *sfa = sSFA + stage * kSFStage + lane * 16;
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    uint4 va = make_uint4(0, 0, 0, 0), vb = make_uint4(0, 0, 0, 0);
+                    if (kb < nkb) {
+                        va = *reinterpret_cast<const uint4 *>(sfa + kb * kSFAtom);
+                        if constexpr (kPaired) {
+                            const uint8_t *raw = sSFB + stage * 2 * kSFStage + kb * kSFAtom + lane * 16 + pair_off;
+                            const uint2 g = *reinterpret_cast<const uint2 *>(raw);
+                            const uint2 u = *reinterpret_cast<const uint2 *>(raw + kSFStage);
+                            vb = make_uint4(g.x, g.y, u.x, u.y);
+                        } else {
+                            vb = *reinterpret_cast<const uint4 *>(sSFB + stage * kSFStage + kb * kSFAtom + lane * 16);
+                        }
+                    }
+                    ra[4 * kb] = va.x, ra[4 * kb + 1] = va.y, ra[4 * kb + 2] = va.z, ra[4 * kb + 3] = va.w;
+                    rb[4 * kb] = vb.x, rb[4 * kb + 1] = vb.y, rb[4 * kb + 2] = vb.z, rb[4 * kb + 3] = vb.w;
+                }
+                const uint32_t t_slot = t_q + static_cast<uint32_t>(stage) * kSFSlotCols;
+                tc_st_32x32b_x16(t_slot, ra);
+                tc_st_32x32b_x16(t_slot + 16, rb);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sf_ready[stage]);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            record_error(p.err, NVFP4_ERR_TIMEOUT);
         }
     } else {
         // -------------------------------------------------------- epilogue
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
         const int row = q * 32 + lane;          // row of the tile owned by this thread
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+        int acc = 0;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
-            const bool got = mbar_wait(acc_full, acc_phase, abort_flag);
+            const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, got)) {
                 *abort_flag = 1;
                 record_error(p.err, NVFP4_ERR_TIMEOUT);
@@ -279,26 +362,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const TileInfo ti = decode_tile(p, t, m_tiles);
             const bool valid = row < ti.valid;
+            const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc * kBN);
 
             if constexpr (EPI == EPI_SWIGLU_QUANT || EPI == EPI_SWIGLU_AMAX) {
                 const float a = p.a_gs[0];
                 const float alpha_g = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + 0]));
                 const float alpha_u = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + 1]));
-                float hgs = 1.0f;
-                uint8_t *hrow = nullptr;
-                uint8_t *sfblk = nullptr;
-                if constexpr (EPI == EPI_SWIGLU_QUANT) {
-                    hgs = p.inter_gs[ti.e];
-                    hrow = p.h_codes + static_cast<int64_t>(ti.row0 + row) * p.h_ld_bytes + ti.nt * 64;
-                    sfblk = p.h_sf + static_cast<int64_t>(ti.row0 / kBM) * p.h_sf_block_stride + lane * 16 + q * 4;
-                }
                 float amax = 0.0f;
                 uint32_t sfword = 0;
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                uint32_t codes[8];
+                float hgs = 1.0f;
+                if constexpr (EPI == EPI_SWIGLU_QUANT)
+                    hgs = p.inter_gs[ti.e];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
                     uint32_t g[16], u[16];
-                    tc_ld_32x32b_x16(t_lane + c * 16, g);
-                    tc_ld_32x32b_x16(t_lane + 128 + c * 16, u);
+                    tc_ld_32x32b_x16(t_acc + c * 16, g);
+                    tc_ld_32x32b_x16(t_acc + 64 + c * 16, u);
                     tc_wait_ld();
                     float h[16];
 #pragma unroll
@@ -309,17 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 16; ++i)
                             amax = fmaxf(amax, fabsf(h[i]));
                     } else {
-                        uint32_t lo, hi;
-                        const uint32_t s = quantize16(h, hgs, lo, hi);
-                        sfword |= s << (8 * (c & 3));
-                        if (valid)
-                            *reinterpret_cast<uint2 *>(hrow + c * 8) = make_uint2(lo, hi);
-                        if ((c & 3) == 3) {
-                            const int kb = ti.nt * 2 + (c >> 2);     // 64-column block of h
-                            if (valid)
-                                *reinterpret_cast<uint32_t *>(sfblk + static_cast<int64_t>(kb) * kSFAtom) = sfword;
-                            sfword = 0;
-                        }
+                        const uint32_t s = quantize16(h, hgs, codes[2 * c], codes[2 * c + 1]);
+                        sfword |= s << (8 * c);
                     }
                 }
                 if constexpr (EPI == EPI_SWIGLU_AMAX) {
@@ -330,18 +401,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                     if (lane == 0)
                         atomicMax(p.amax_bits + ti.e, __float_as_uint(amax));
+                } else if (valid) {
+                    // 64 h columns of this row: 32 bytes of codes and one 4-byte scale word (k-block nt)
+                    uint4 *hrow = reinterpret_cast<uint4 *>(p.h_codes + static_cast<int64_t>(ti.row0 + row) * p.h_ld_bytes +
+                                                            ti.nt * 32);
+                    hrow[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                    hrow[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                    *reinterpret_cast<uint32_t *>(p.h_sf + static_cast<int64_t>(ti.row0 / kBM) * p.h_sf_block_stride +
+                                                  static_cast<int64_t>(ti.nt) * kSFAtom + lane * 16 + q * 4) = sfword;
                 }
             } else {
                 const float a = p.a_gs[p.a_gs_per_expert ? ti.e : 0];
                 __nv_bfloat16 *orow = p.out + static_cast<int64_t>(ti.row0_out + row) * p.ldo +
-                                      static_cast<int64_t>(ti.nt) * BN;
-#pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
+                                      static_cast<int64_t>(ti.nt) * kBN;
+#pragma unroll
+                for (int c = 0; c < kBN / 32; ++c) {
                     uint32_t v0[16], v1[16];
-                    tc_ld_32x32b_x16(t_lane + c * 32, v0);
-                    tc_ld_32x32b_x16(t_lane + c * 32 + 16, v1);
+                    tc_ld_32x32b_x16(t_acc + c * 32, v0);
+                    tc_ld_32x32b_x16(t_acc + c * 32 + 16, v1);
                     tc_wait_ld();
-                    const int col = ti.nt * BN + c * 32;
+                    const int col = ti.nt * kBN + c * 32;
                     int seg = 0;
 #pragma unroll
                     for (int i = 0; i < 3; ++i)
@@ -349,8 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             seg = i + 1;
                     const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + seg]));
                     if (valid) {
-                        uint4 o[4];
-                        uint32_t *ow = reinterpret_cast<uint32_t *>(o);
+                        uint32_t ow[16];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(v0[2 * i]) * alpha,
@@ -363,15 +441,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
-                            dst[i] = o[i];
+                            dst[i] = make_uint4(ow[4 * i], ow[4 * i + 1], ow[4 * i + 2], ow[4 * i + 3]);
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(acc_empty);
-            acc_phase ^= 1u;
+                mbar_arrive(&acc_empty[acc]);
+            if (++acc == kNumAcc) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
         }
     }
 
@@ -384,37 +465,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int BN, int EPI>
-static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_b, const GemmArgs &args, int grid,
-                              cudaStream_t stream)
+template <int EPI>
+static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
+                              const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    const int smem = Smem<BN>::kTotal;
+    const int smem = Smem<EPI>::kTotal;
     static int attr_done_device = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
     if (attr_done_device != dev) {
-        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess)
             return e;
         attr_done_device = dev;
     }
-    nvfp4_gemm_kernel<BN, EPI><<<grid, kThreads, smem, stream>>>(map_a, map_b, args);
+    nvfp4_gemm_kernel<EPI><<<grid, kThreads, smem, stream>>>(map_a, map_a32, map_b, args);
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int bn, int epi, const CUtensorMap &map_a, const CUtensorMap &map_b, const GemmArgs &args,
-                        int grid, cudaStream_t stream)
+cudaError_t launch_gemm(int epi, const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
+                        const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    if (bn == 256) {
-        switch (epi) {
-        case EPI_SWIGLU_QUANT: return launch_one<256, EPI_SWIGLU_QUANT>(map_a, map_b, args, grid, stream);
-        case EPI_SWIGLU_AMAX: return launch_one<256, EPI_SWIGLU_AMAX>(map_a, map_b, args, grid, stream);
-        default: return launch_one<256, EPI_BF16>(map_a, map_b, args, grid, stream);
-        }
+    switch (epi) {
+    case EPI_SWIGLU_QUANT: return launch_one<EPI_SWIGLU_QUANT>(map_a, map_a32, map_b, args, grid, stream);
+    case EPI_SWIGLU_AMAX: return launch_one<EPI_SWIGLU_AMAX>(map_a, map_a32, map_b, args, grid, stream);
+    default: return launch_one<EPI_BF16>(map_a, map_a32, map_b, args, grid, stream);
     }
-    return launch_one<128, EPI_BF16>(map_a, map_b, args, grid, stream);
 }
 
 } // namespace nvfp4
