@@ -380,8 +380,8 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     steps, warmup = args.steps, max(3, args.warmup)
 
-    if args.only == "decode":
-        return run_decode_only(args, world, rank, dev, peaks, peak_src, steps, warmup)
+    if args.only != "all":
+        return run_single(args.only, world, rank, dev, peaks, peak_src, steps, warmup)
     pre = Workload(W.MOE_CONFIGS["prefill"], dev)
     dec = Workload(W.MOE_CONFIGS["decode"], dev)
     torch.cuda.synchronize()
@@ -462,9 +462,9 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_decode_only(args, world, rank, dev, peaks, peak_src, steps, warmup):
-    """The 48-expert decode workload alone (a small case for profiling)."""
-    dec = Workload(W.MOE_CONFIGS["decode"], dev)
+def run_single(name, world, rank, dev, peaks, peak_src, steps, warmup):
+    """One MoE workload alone (small cases for profiling: decode, prefill_ep48)."""
+    dec = Workload(W.MOE_CONFIGS[name], dev)
     clocks = ClockSampler(dev)
     clocks.start()
     ms_dec, stages = time_steps(dec, steps, warmup, world)
@@ -477,13 +477,13 @@ def run_decode_only(args, world, rank, dev, peaks, peak_src, steps, warmup):
     kb = dec.kernel_bytes()
     dom = max(STAGES, key=lambda s: stages[s])
     achieved = kb[dom] / (stages[dom] / 1e3) / 1e9
-    line = {"metric": "moe_decode_GB_per_s", "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
+    line = {"metric": f"moe_{name}_GB_per_s", "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,
             "warmup": warmup, "ms_per_step": ms_dec / steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic", "config": config_block(dec.cfg, world),
             "hbm_frac": gbs / peaks["hbm_gbs"], "stage_ms": stages,
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
-                         "algorithmic_bytes": kb[dom], "traffic": ncu_traffic(dom, "decode")},
+                         "algorithmic_bytes": kb[dom], "traffic": ncu_traffic(dom, name)},
             "gpu_launches": KERNELS_PER_STEP * steps, "clocks": clocks.summary()}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -545,8 +545,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "decode"], default="all",
-                    help="decode: the 48-expert decode workload alone (small profiling case)")
+    ap.add_argument("--only", choices=["all", "decode", "prefill_ep48", "shared", "tiny"], default="all",
+                    help="one workload alone (small profiling cases)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -194,7 +194,7 @@ int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi,
     if (st == NVFP4_OK)
         st = make_code_map(&ma32, ws + L.a_codes, L.rpad, H / 2, 32);
     if (st == NVFP4_OK)
-        st = make_code_map(&mb, a->w13_codes, static_cast<int64_t>(E) * 2 * I, H / 2, 64);
+        st = make_code_map(&mb, a->w13_codes, static_cast<int64_t>(E) * 2 * I, H / 2, 128);
     if (st != NVFP4_OK)
         return st;
     GemmArgs g{};
@@ -206,9 +206,9 @@ int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi,
     g.num_k_tiles = static_cast<int>((H + 255) / 256);
     g.num_mtiles_dev = num_mt;
     g.mtiles = mtiles;
-    g.n_tiles = static_cast<int>(I / 64);
+    g.n_tiles = static_cast<int>(I / 128);
     g.b_rows_per_expert = 2 * I;
-    g.b_tile_rows = 64;
+    g.b_tile_rows = 128;
     g.b_half_offset = static_cast<int>(I);
     g.a_gs = a->x_gs;
     g.a_gs_per_expert = 0;
@@ -222,7 +222,7 @@ int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi,
     g.h_sf_block_stride = (I / 64) * 512;
     g.amax_bits = reinterpret_cast<unsigned int *>(ws + L.amax);
     g.err = err;
-    return cuda_status(launch_gemm(l1_epi, ma, ma32, mb, g, num_sms, s));
+    return cuda_status(launch_gemm(256, l1_epi, ma, ma32, mb, g, num_sms, s));
 }
 
 } // namespace
@@ -345,7 +345,7 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_g
         st = make_code_map(&mb, b_codes, N, K / 2, 128);
     if (st != NVFP4_OK)
         return st;
-    const int bn = 128;
+    const int bn = (N % 256 == 0) ? 256 : 128;
     GemmArgs g{};
     g.sfa = a_scales;
     g.sfa_block_stride = (K / 64) * 512;
@@ -373,7 +373,7 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_g
     g.err = nullptr;            // no workspace: a timed-out wait ends the kernel without a report
     int64_t tiles = static_cast<int64_t>(g.dense_m_tiles) * g.n_tiles;
     const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
-    return cuda_status(launch_gemm(EPI_BF16, ma, ma32, mb, g, grid, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_gemm(bn, EPI_BF16, ma, ma32, mb, g, grid, static_cast<cudaStream_t>(stream)));
 }
 
 size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I)
@@ -442,7 +442,7 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
         st = make_code_map(&mb2, a->w2_codes, static_cast<int64_t>(E) * H, I / 2, 128);
     if (st != NVFP4_OK)
         return st;
-    const int bn = 128;
+    const int bn = (H % 256 == 0) ? 256 : 128;
     GemmArgs g{};
     g.sfa = ws + L.h_sf;
     g.sfa_block_stride = (I / 64) * 512;
@@ -465,7 +465,7 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
     g.out = reinterpret_cast<__nv_bfloat16 *>(ws + L.y);
     g.ldo = H;
     g.err = reinterpret_cast<int32_t *>(ws);
-    if (mark(events, 3, s) != NVFP4_OK || launch_gemm(EPI_BF16, ma2, ma2_32, mb2, g, sms, s) != cudaSuccess ||
+    if (mark(events, 3, s) != NVFP4_OK || launch_gemm(bn, EPI_BF16, ma2, ma2_32, mb2, g, sms, s) != cudaSuccess ||
         mark(events, 4, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
 

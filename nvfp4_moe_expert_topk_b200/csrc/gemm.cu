@@ -1,40 +1,39 @@
 // gemm.cu -- persistent block-scaled FP4 GEMM engine for sm_100a.
 //
-// D[128 x 128] tiles of  A (E2M1 codes, K-major) x B^T (E2M1 codes, K-major)
-// with one E4M3 scale per 16 elements on both sides, on the 5th-generation
-// tensor cores (tcgen05.mma kind::mxf4nvf4, block16 scaling), accumulating in
-// fp32 in tensor memory.  This is the grouped GEMM of the expert chain
+// D[128 x BN] tiles (BN = 256, or 128 when N is not a multiple of 256) of
+// A (E2M1 codes, K-major) x B^T (E2M1 codes, K-major) with one E4M3 scale per
+// 16 elements on both sides, on the 5th-generation tensor cores
+// (tcgen05.mma kind::mxf4nvf4, block16 scaling), accumulating in fp32 in
+// tensor memory.  This is the grouped GEMM of the expert chain
 // ("nvfp4-megamoe-kernel / CURRENT_BUG.md", page 1 "Phase 1": L1 gate_up
 // GEMM -> SiLU -> re-quantise -> L2 GEMM; with one group it is the plain
 // NVFP4 GEMM of page 1 "Phase 2").
 //
 // Block of 10 warps, one block per SM, persistent over the tile list:
 //   warp 0    TMA producer: per k-tile (256 elements) the valid 32-row boxes
-//             (or one 128-row box) of A, the 128 rows of B, and the matching
-//             512-byte scale atoms by bulk copy, into a 5- or 6-stage
+//             (or one 128-row box) of A, the BN rows of B as 128-row boxes,
+//             and the matching 512-byte scale atoms by bulk copy, into a
 //             shared-memory ring guarded by mbarriers;
 //   warps 6-9 scale stagers, one per TMEM lane quarter: move each stage's
 //             E4M3 scales from shared memory into that stage's TMEM scale
 //             slot with tcgen05.st (the layout the MMA reads: lane l, column
-//             4*kb + m holds the 4 scales of row 32*m + l, replicated in all
-//             four quarters), then signal the stage's sf_ready barrier;
-//             scale copies through the tensor pipe (tcgen05.cp) cost more
-//             pipe time than the MMAs they feed at these tile sizes;
+//             4*j + m holds the 4 scales of row 128*h + 32*m + l for k-block
+//             j, B half h; replicated in all four quarters), then signal the
+//             stage's sf_ready barrier (copying scales through the tensor
+//             pipe with tcgen05.cp costs more pipe time than the MMAs);
 //   warp 1    allocates TMEM; one thread issues the 4 tcgen05.mma (K=64) of
-//             each k-tile into one of two 128-column accumulators, so the
-//             next tile's MMAs run while the epilogue drains the previous;
+//             each k-tile; the block-scaled FP4 MMA costs about the same pipe
+//             time per instruction at N=128 as at N=256, so tiles are 256 wide;
 //   warps 2-5 epilogue: TMEM -> registers (each thread owns one row of the
-//             tile), then one of
+//             tile), release the accumulator to the MMA thread, then one of
 //             EPI_SWIGLU_QUANT  h = SiLU(a_g*g) * (a_u*u), NVFP4-quantised
 //                               with the expert's inter_gs (L1),
 //             EPI_SWIGLU_AMAX   same h, max|h| per expert (warmup),
 //             EPI_BF16          y = alpha * acc -> bf16 (L2, dense GEMM).
-// In the L1 tile the B tile is 64 gate rows stacked on the matching 64 up
-// rows (the weight keeps its [gate; up] layout: two 64-row boxes), so TMEM
-// columns 0-63 hold gate and 64-127 hold up of the same 64 h columns and each
-// 16-element block of h is produced by one thread.  The scales of those two
-// 64-row halves sit in two different 128-row scale atoms; the stagers pair
-// their 32-row groups on the way into TMEM.
+// In the L1 tile the B tile is 128 gate rows stacked on the matching 128 up
+// rows of the stacked [gate; up] weight (two boxes), so TMEM columns 0-127
+// hold gate and 128-255 hold up of the same 128 h columns, and each
+// 16-element block of h is produced and quantised by one thread.
 //
 // The tile list is either dense (m-tiles of M, n-major) or grouped: an
 // m-tile table written on the device by the routing kernel (expert, first
@@ -51,32 +50,32 @@
 namespace nvfp4 {
 
 constexpr int kBM = 128;
-constexpr int kBN = 128;
 constexpr int kBK = 256;                        // elements per k-tile
 constexpr int kBKBytes = 128;                   // bytes of codes per row per k-tile
 constexpr int kTileBytes = 128 * kBKBytes;      // 16 KB: 128 rows of one k-tile
 constexpr int kSFAtom = 512;                    // 128 rows x 4 scales (64 elements)
 constexpr int kSFStage = 4 * kSFAtom;           // one 128-row block, 4 k-blocks
-constexpr int kNumAcc = 2;                      // TMEM accumulators
 constexpr int kThreads = 320;
 constexpr int kFirstSFWarp = 6;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSF = kNumAcc * kBN;     // 256: per-stage scale slots follow the accumulators
-constexpr uint32_t kSFSlotCols = 32;            // A: 4 k-blocks x 4 columns, then B: the same
 
-template <int EPI>
-struct Smem {
-    static constexpr bool kPaired = EPI != EPI_BF16;
-    static constexpr int kStages = kPaired ? 5 : 6;
+template <int BN>
+struct Cfg {
+    static constexpr int kHalves = BN / 128;                 // 128-row halves of the B tile
+    static constexpr int kNumAcc = BN == 256 ? 1 : 2;        // TMEM accumulators
+    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kSFSlotCols = 16 + 16 * kHalves;    // A: 4 k-blocks x 4 cols; B: 4 x 4 per half
+    static constexpr uint32_t kTmemSF = kNumAcc * BN;        // scale slots follow the accumulators
     static constexpr int kA = 0;
     static constexpr int kB = kA + kStages * kTileBytes;
-    static constexpr int kSFA = kB + kStages * kTileBytes;
-    static constexpr int kSFB = kSFA + kStages * kSFStage;              // paired: gate atoms, then up atoms
-    static constexpr int kBars = kSFB + kStages * kSFStage * (kPaired ? 2 : 1);
+    static constexpr int kSFA = kB + kStages * kTileBytes * kHalves;
+    static constexpr int kSFB = kSFA + kStages * kSFStage;
+    static constexpr int kBars = kSFB + kStages * kSFStage * kHalves;
     static constexpr int kBarCount = 3 * kStages + 2 * kNumAcc + 1;
     static constexpr int kMisc = kBars + kBarCount * 8;
-    static constexpr int kTotal = kMisc + 16 + 1024;   // + tmem slot, abort flag, alignment slack
-    static_assert(kTmemSF + kStages * kSFSlotCols <= kTmemCols, "TMEM scale slots");
+    static constexpr int kSmem = kMisc + 16 + 1024;          // + tmem slot, abort flag, alignment slack
+    static_assert(kTmemSF + kStages * kSFSlotCols <= kTmemCols, "TMEM budget");
+    static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 struct TileInfo {
@@ -106,11 +105,6 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, int t, int m_
     return ti;
 }
 
-__device__ __forceinline__ int tile_nt(const GemmArgs &p, int t, int m_tiles)
-{
-    return p.mtiles != nullptr ? t % p.n_tiles : t / m_tiles;
-}
-
 __device__ __forceinline__ void record_error(int32_t *err, int code)
 {
     if (err != nullptr)
@@ -124,28 +118,36 @@ __device__ __forceinline__ float silu_mul(float g, float u)
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
-template <int EPI>
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a32,
                       const __grid_constant__ CUtensorMap map_b, const GemmArgs p)
 {
-    using L = Smem<EPI>;
-    constexpr bool kPaired = L::kPaired;
-    constexpr int kStages = L::kStages;
+    using C = Cfg<BN>;
+    constexpr int kStages = C::kStages;
+    constexpr int kHalves = C::kHalves;
+    constexpr int kNumAcc = C::kNumAcc;
+    static_assert(EPI == EPI_BF16 || BN == 256, "SwiGLU tiles are 128 gate + 128 up columns");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem + L::kA;
-    uint8_t *sB = smem + L::kB;
-    uint8_t *sSFA = smem + L::kSFA;
-    uint8_t *sSFB = smem + L::kSFB;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::kBars);
+    uint8_t *sA = smem + C::kA;
+    uint8_t *sB = smem + C::kB;
+    uint8_t *sSFA = smem + C::kSFA;
+    uint8_t *sSFB = smem + C::kSFB;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBars);
     uint64_t *empty = full + kStages;
     uint64_t *sf_ready = empty + kStages;
     uint64_t *acc_full = sf_ready + kStages;
     uint64_t *acc_empty = acc_full + kNumAcc;
     uint64_t *drain = acc_empty + kNumAcc;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kMisc);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kMisc + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kMisc + 4);
     __shared__ int never_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const int nkb = min(4, (p.K - kt * kBK) / 64);
                     const uint32_t sf_bytes = static_cast<uint32_t>(nkb * kSFAtom);
-                    mbar_arrive_expect_tx(&full[stage], a_bytes + kTileBytes + sf_bytes * (kPaired ? 3 : 2));
+                    mbar_arrive_expect_tx(&full[stage], a_bytes + kHalves * kTileBytes + sf_bytes * (1 + kHalves));
                     uint8_t *a_dst = sA + stage * kTileBytes;
                     if (a_boxes == 0) {
                         tma_load_2d(a_dst, &map_a, kt * kBKBytes, ti.row0, &full[stage]);
@@ -211,17 +213,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_2d(a_dst + i * (kTileBytes / 4), &map_a32, kt * kBKBytes, ti.row0 + 32 * i,
                                         &full[stage]);
                     }
-                    uint8_t *b_dst = sB + stage * kTileBytes;
-                    if constexpr (kPaired) {
-                        tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
-                        tma_load_2d(b_dst + kTileBytes / 2, &map_b, kt * kBKBytes, static_cast<int32_t>(brow1),
+                    uint8_t *b_dst = sB + stage * kHalves * kTileBytes;
+                    uint8_t *sfb_dst = sSFB + stage * kHalves * kSFStage;
+                    tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
+                    bulk_load(sfb_dst, sfb0 + kt * kSFStage, sf_bytes, &full[stage]);
+                    if constexpr (kHalves == 2) {
+                        tma_load_2d(b_dst + kTileBytes, &map_b, kt * kBKBytes, static_cast<int32_t>(brow1),
                                     &full[stage]);
-                        uint8_t *raw = sSFB + stage * 2 * kSFStage;
-                        bulk_load(raw, sfb0 + kt * kSFStage, sf_bytes, &full[stage]);
-                        bulk_load(raw + kSFStage, sfb1 + kt * kSFStage, sf_bytes, &full[stage]);
-                    } else {
-                        tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
-                        bulk_load(sSFB + stage * kSFStage, sfb0 + kt * kSFStage, sf_bytes, &full[stage]);
+                        bulk_load(sfb_dst + kSFStage, sfb1 + kt * kSFStage, sf_bytes, &full[stage]);
                     }
                     bulk_load(sSFA + stage * kSFStage, sfa + kt * kSFStage, sf_bytes, &full[stage]);
                     pend_mask |= 1u << stage;
@@ -243,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = idesc_nvf4(kBM, kBN);
+        constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
         if (lane == 0) {
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
@@ -254,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kBN);
+                const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * BN);
                 for (int kt = 0; kt < p.num_k_tiles; ++kt) {
                     if (!mbar_wait(&sf_ready[stage], phase, abort_flag) || !mbar_wait(&full[stage], phase, abort_flag)) {
                         ok = false;
@@ -263,11 +262,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const int nkb = min(4, (p.K - kt * kBK) / 64);
                     const uint32_t a_addr = smem_u32(sA + stage * kTileBytes);
-                    const uint32_t b_addr = smem_u32(sB + stage * kTileBytes);
-                    const uint32_t t_sfa = tmem + kTmemSF + static_cast<uint32_t>(stage) * kSFSlotCols;
+                    const uint32_t b_addr = smem_u32(sB + stage * kHalves * kTileBytes);
+                    const uint32_t t_sfa = tmem + C::kTmemSF + static_cast<uint32_t>(stage * C::kSFSlotCols);
                     for (int kb = 0; kb < nkb; ++kb)
                         tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(a_addr + kb * 32), sdesc_kmajor_sw128(b_addr + kb * 32),
-                                    idesc, t_sfa + kb * 4, t_sfa + 16 + kb * 4, (kt | kb) != 0 ? 1u : 0u);
+                                    idesc, t_sfa + kb * 4, t_sfa + 16 + kb * 4 * kHalves, (kt | kb) != 0 ? 1u : 0u);
                     tc_commit(&empty[stage]);
                     if (++stage == kStages) {
                         stage = 0;
@@ -294,13 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= kFirstSFWarp) {
         // -------------------------------------------------------- scale stagers
         const int q = warp & 3;
-        const uint32_t t_q = tmem + (static_cast<uint32_t>(q * 32) << 16) + kTmemSF;
+        const uint32_t t_q = tmem + (static_cast<uint32_t>(q * 32) << 16) + C::kTmemSF;
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            // paired tiles: byte offset of this tile's two 32-row groups inside a 16-byte scale row
-            const int pair_off = kPaired ? (tile_nt(p, t, m_tiles) & 1) * 8 : 0;
             for (int kt = 0; kt < p.num_k_tiles; ++kt) {
                 const bool got = mbar_wait(&full[stage], phase, abort_flag);
                 if (!__all_sync(0xffffffffu, got)) {
@@ -308,28 +305,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const int nkb = min(4, (p.K - kt * kBK) / 64);
-                uint32_t ra[16], rb[16];
-                const uint8_t *sfa = sSFA + stage * kSFStage + lane * 16;
+                const uint32_t t_slot = t_q + static_cast<uint32_t>(stage * C::kSFSlotCols);
+                // A: column 4*kb + m <- row `lane` of atom kb (the 4 scales of rows 32*m + lane)
+                uint32_t r[16];
+                const uint8_t *src = sSFA + stage * kSFStage + lane * 16;
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb) {
-                    uint4 va = make_uint4(0, 0, 0, 0), vb = make_uint4(0, 0, 0, 0);
-                    if (kb < nkb) {
-                        va = *reinterpret_cast<const uint4 *>(sfa + kb * kSFAtom);
-                        if constexpr (kPaired) {
-                            const uint8_t *raw = sSFB + stage * 2 * kSFStage + kb * kSFAtom + lane * 16 + pair_off;
-                            const uint2 g = *reinterpret_cast<const uint2 *>(raw);
-                            const uint2 u = *reinterpret_cast<const uint2 *>(raw + kSFStage);
-                            vb = make_uint4(g.x, g.y, u.x, u.y);
-                        } else {
-                            vb = *reinterpret_cast<const uint4 *>(sSFB + stage * kSFStage + kb * kSFAtom + lane * 16);
-                        }
-                    }
-                    ra[4 * kb] = va.x, ra[4 * kb + 1] = va.y, ra[4 * kb + 2] = va.z, ra[4 * kb + 3] = va.w;
-                    rb[4 * kb] = vb.x, rb[4 * kb + 1] = vb.y, rb[4 * kb + 2] = vb.z, rb[4 * kb + 3] = vb.w;
+                    const uint4 v = kb < nkb ? *reinterpret_cast<const uint4 *>(src + kb * kSFAtom) : make_uint4(0, 0, 0, 0);
+                    r[4 * kb] = v.x, r[4 * kb + 1] = v.y, r[4 * kb + 2] = v.z, r[4 * kb + 3] = v.w;
                 }
-                const uint32_t t_slot = t_q + static_cast<uint32_t>(stage) * kSFSlotCols;
-                tc_st_32x32b_x16(t_slot, ra);
-                tc_st_32x32b_x16(t_slot + 16, rb);
+                tc_st_32x32b_x16(t_slot, r);
+                // B: column 4*(kHalves*kb + h) + m <- row `lane` of atom kb of half h
+                src = sSFB + stage * kHalves * kSFStage + lane * 16;
+#pragma unroll
+                for (int part = 0; part < kHalves; ++part) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int kb = (part * 4 + i) / kHalves, h = (part * 4 + i) % kHalves;
+                        const uint4 v = kb < nkb ? *reinterpret_cast<const uint4 *>(src + h * kSFStage + kb * kSFAtom)
+                                                 : make_uint4(0, 0, 0, 0);
+                        r[4 * i] = v.x, r[4 * i + 1] = v.y, r[4 * i + 2] = v.z, r[4 * i + 3] = v.w;
+                    }
+                    tc_st_32x32b_x16(t_slot + 16 + 16 * part, r);
+                }
                 tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -362,38 +360,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const TileInfo ti = decode_tile(p, t, m_tiles);
             const bool valid = row < ti.valid;
-            const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc * kBN);
+            const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc * BN);
 
             if constexpr (EPI == EPI_SWIGLU_QUANT || EPI == EPI_SWIGLU_AMAX) {
                 const float a = p.a_gs[0];
                 const float alpha_g = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + 0]));
                 const float alpha_u = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + 1]));
-                float amax = 0.0f;
-                uint32_t sfword = 0;
-                uint32_t codes[8];
-                float hgs = 1.0f;
-                if constexpr (EPI == EPI_SWIGLU_QUANT)
-                    hgs = p.inter_gs[ti.e];
+                // drain: h for the tile's 128 columns of this row, then give the accumulator back
+                float h[128];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint32_t g[16], u[16];
                     tc_ld_32x32b_x16(t_acc + c * 16, g);
-                    tc_ld_32x32b_x16(t_acc + 64 + c * 16, u);
+                    tc_ld_32x32b_x16(t_acc + 128 + c * 16, u);
                     tc_wait_ld();
-                    float h[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        h[i] = silu_mul(__uint_as_float(g[i]) * alpha_g, __uint_as_float(u[i]) * alpha_u);
-                    if constexpr (EPI == EPI_SWIGLU_AMAX) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            amax = fmaxf(amax, fabsf(h[i]));
-                    } else {
-                        const uint32_t s = quantize16(h, hgs, codes[2 * c], codes[2 * c + 1]);
-                        sfword |= s << (8 * c);
-                    }
+                        h[c * 16 + i] = silu_mul(__uint_as_float(g[i]) * alpha_g, __uint_as_float(u[i]) * alpha_u);
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&acc_empty[acc]);
                 if constexpr (EPI == EPI_SWIGLU_AMAX) {
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 128; ++i)
+                        amax = fmaxf(amax, fabsf(h[i]));
                     if (!valid)
                         amax = 0.0f;
 #pragma unroll
@@ -401,54 +394,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                     if (lane == 0)
                         atomicMax(p.amax_bits + ti.e, __float_as_uint(amax));
-                } else if (valid) {
-                    // 64 h columns of this row: 32 bytes of codes and one 4-byte scale word (k-block nt)
-                    uint4 *hrow = reinterpret_cast<uint4 *>(p.h_codes + static_cast<int64_t>(ti.row0 + row) * p.h_ld_bytes +
-                                                            ti.nt * 32);
-                    hrow[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                    hrow[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-                    *reinterpret_cast<uint32_t *>(p.h_sf + static_cast<int64_t>(ti.row0 / kBM) * p.h_sf_block_stride +
-                                                  static_cast<int64_t>(ti.nt) * kSFAtom + lane * 16 + q * 4) = sfword;
+                } else {
+                    const float hgs = p.inter_gs[ti.e];
+                    uint32_t codes[16];
+                    uint32_t sfw[2] = {0, 0};
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float blk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            blk[i] = h[c * 16 + i];
+                        const uint32_t s = quantize16(blk, hgs, codes[2 * c], codes[2 * c + 1]);
+                        sfw[c >> 2] |= s << (8 * (c & 3));
+                    }
+                    if (valid) {
+                        // 128 h columns: 64 bytes of codes and two 4-byte scale words (k-blocks 2nt, 2nt+1)
+                        uint4 *hrow = reinterpret_cast<uint4 *>(p.h_codes +
+                                                                static_cast<int64_t>(ti.row0 + row) * p.h_ld_bytes +
+                                                                ti.nt * 64);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            hrow[i] = make_uint4(codes[4 * i], codes[4 * i + 1], codes[4 * i + 2], codes[4 * i + 3]);
+                        uint8_t *sf = p.h_sf + static_cast<int64_t>(ti.row0 / kBM) * p.h_sf_block_stride +
+                                      static_cast<int64_t>(2 * ti.nt) * kSFAtom + lane * 16 + q * 4;
+                        *reinterpret_cast<uint32_t *>(sf) = sfw[0];
+                        *reinterpret_cast<uint32_t *>(sf + kSFAtom) = sfw[1];
+                    }
                 }
             } else {
                 const float a = p.a_gs[p.a_gs_per_expert ? ti.e : 0];
-                __nv_bfloat16 *orow = p.out + static_cast<int64_t>(ti.row0_out + row) * p.ldo +
-                                      static_cast<int64_t>(ti.nt) * kBN;
+                uint32_t o[BN / 2];
 #pragma unroll
-                for (int c = 0; c < kBN / 32; ++c) {
-                    uint32_t v0[16], v1[16];
-                    tc_ld_32x32b_x16(t_acc + c * 32, v0);
-                    tc_ld_32x32b_x16(t_acc + c * 32 + 16, v1);
+                for (int c = 0; c < BN / 16; ++c) {
+                    uint32_t v[16];
+                    tc_ld_32x32b_x16(t_acc + c * 16, v);
                     tc_wait_ld();
-                    const int col = ti.nt * kBN + c * 32;
+                    const int col = ti.nt * BN + c * 16;
                     int seg = 0;
 #pragma unroll
                     for (int i = 0; i < 3; ++i)
                         if (i < p.nseg - 1 && col >= p.seg_end[i])
                             seg = i + 1;
                     const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + seg]));
-                    if (valid) {
-                        uint32_t ow[16];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(v0[2 * i]) * alpha,
-                                                                     __uint_as_float(v0[2 * i + 1]) * alpha);
-                            ow[i] = *reinterpret_cast<uint32_t *>(&b);
-                            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v1[2 * i]) * alpha,
-                                                                      __uint_as_float(v1[2 * i + 1]) * alpha);
-                            ow[8 + i] = *reinterpret_cast<uint32_t *>(&b2);
-                        }
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+                    for (int i = 0; i < 8; ++i)
+                        o[c * 8 + i] = pack_bf16x2(__uint_as_float(v[2 * i]) * alpha, __uint_as_float(v[2 * i + 1]) * alpha);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&acc_empty[acc]);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + static_cast<int64_t>(ti.row0_out + row) * p.ldo +
+                                                           static_cast<int64_t>(ti.nt) * BN);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(ow[4 * i], ow[4 * i + 1], ow[4 * i + 2], ow[4 * i + 3]);
-                    }
+                    for (int i = 0; i < BN / 8; ++i)
+                        dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&acc_empty[acc]);
             if (++acc == kNumAcc) {
                 acc = 0;
                 acc_phase ^= 1u;
@@ -465,33 +468,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int EPI>
+template <int BN, int EPI>
 static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
                               const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    const int smem = Smem<EPI>::kTotal;
+    const int smem = Cfg<BN>::kSmem;
     static int attr_done_device = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
     if (attr_done_device != dev) {
-        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess)
             return e;
         attr_done_device = dev;
     }
-    nvfp4_gemm_kernel<EPI><<<grid, kThreads, smem, stream>>>(map_a, map_a32, map_b, args);
+    nvfp4_gemm_kernel<BN, EPI><<<grid, kThreads, smem, stream>>>(map_a, map_a32, map_b, args);
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm(int epi, const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
-                        const GemmArgs &args, int grid, cudaStream_t stream)
+cudaError_t launch_gemm(int bn, int epi, const CUtensorMap &map_a, const CUtensorMap &map_a32,
+                        const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream)
 {
     switch (epi) {
-    case EPI_SWIGLU_QUANT: return launch_one<EPI_SWIGLU_QUANT>(map_a, map_a32, map_b, args, grid, stream);
-    case EPI_SWIGLU_AMAX: return launch_one<EPI_SWIGLU_AMAX>(map_a, map_a32, map_b, args, grid, stream);
-    default: return launch_one<EPI_BF16>(map_a, map_a32, map_b, args, grid, stream);
+    case EPI_SWIGLU_QUANT: return launch_one<256, EPI_SWIGLU_QUANT>(map_a, map_a32, map_b, args, grid, stream);
+    case EPI_SWIGLU_AMAX: return launch_one<256, EPI_SWIGLU_AMAX>(map_a, map_a32, map_b, args, grid, stream);
+    default:
+        return bn == 256 ? launch_one<256, EPI_BF16>(map_a, map_a32, map_b, args, grid, stream)
+                         : launch_one<128, EPI_BF16>(map_a, map_a32, map_b, args, grid, stream);
     }
 }
 

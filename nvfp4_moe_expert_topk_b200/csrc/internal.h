@@ -26,8 +26,8 @@ struct GemmArgs {
     int dense_M;
     int n_tiles;
     int64_t b_rows_per_expert;
-    int b_tile_rows;          // B rows advanced per n-tile (64 for the paired gate/up tiles, else 128)
-    int b_half_offset;        // paired tiles: row offset of the up half (I)
+    int b_tile_rows;          // B rows advanced per n-tile (128 for the gate/up tiles of L1, else bn)
+    int b_half_offset;        // row offset of the second 128-row box of a 256-wide tile (I for L1: the up half)
     // global scales: alpha = 1 / (a_gs * b_gs)
     const float *a_gs;
     int a_gs_per_expert;
@@ -50,12 +50,13 @@ struct GemmArgs {
 
 enum Epilogue { EPI_SWIGLU_QUANT = 0, EPI_BF16 = 1, EPI_SWIGLU_AMAX = 2 };
 
-// Launches the GEMM engine.  map_a / map_a32: 2-D uint8 tensor maps over
-// the A code matrix with boxes of 128 and 32 rows; map_b: over the B code
-// matrix with 64-row boxes (SwiGLU epilogues: gate and up halves) or 128-row
-// boxes (EPI_BF16); every box is 128 bytes wide with 128-byte swizzle.
-cudaError_t launch_gemm(int epi, const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
-                        const GemmArgs &args, int grid, cudaStream_t stream);
+// Launches the GEMM engine with 128 x bn tiles (bn 256, or 128 for EPI_BF16
+// when N is not a multiple of 256).  map_a / map_a32: 2-D uint8 tensor maps
+// over the A code matrix with boxes of 128 and 32 rows; map_b: over the B
+// code matrix with 128-row boxes; every box is 128 bytes wide with 128-byte
+// swizzle.
+cudaError_t launch_gemm(int bn, int epi, const CUtensorMap &map_a, const CUtensorMap &map_a32,
+                        const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream);
 
 // Memory-bound kernels (kernels.cu).
 cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s);

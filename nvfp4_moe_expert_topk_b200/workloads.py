@@ -50,6 +50,10 @@ MOE_CONFIGS = {
     "shared": MoeConfig("shared", E=1, k=1, T=256, H=7168, I=3072, routing="single", outliers=True, warmup_T=256),
     "decode": MoeConfig("decode", E=48, k=6, T=64, H=7168, I=3072, routing="sigmoid", outliers=False, warmup_T=64),
     "prefill": MoeConfig("prefill", E=384, k=6, T=4096, H=7168, I=3072, routing="zipf", outliers=True, warmup_T=16),
+    # prefill-shaped (64 routed rows per expert on average, Zipf-skewed) on one
+    # expert-parallel slice: small enough to profile and to check in full
+    "prefill_ep48": MoeConfig("prefill_ep48", E=48, k=6, T=512, H=7168, I=3072, routing="zipf", outliers=True,
+                              warmup_T=64, zipf_zero_tail=2),
 }
 
 
