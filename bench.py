@@ -236,38 +236,61 @@ class Workload:
         return self.nonempty * 3 * c.H * c.I * fp4 + 2 * c.T * c.H * 2.0 + c.T * c.k * 8.0
 
 
-def time_steps(wl, steps, warmup, world, timed_events=True, tag="timed"):
-    """Device time of `steps` steps (events on the launching stream, barrier +
-    synchronize on both sides), and per-stage mean durations."""
+def time_steps(wl, steps, warmup, world, graph=True, tag="timed"):
+    """Device time of `steps` steps: events on the launching stream, barrier +
+    synchronize on both sides, max over ranks; per-stage mean durations from
+    events recorded between the kernels of every step.  With graph=True the
+    `steps` steps (events included) are captured once into a CUDA graph and
+    the timed region is one replay of it -- the way a serving runtime issues
+    the block (the pages' runner is cudagraph-safe); otherwise eager launches."""
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         wl.step()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True, external=graph) for _ in range(7)] for _ in range(steps)]
+    for row in ev:                      # create the CUDA events outside the timed region
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+
+    def issue():
+        for i in range(steps):
+            ev[i][0].record()
+            wl.step(events=ev[i][1:])
+
+    g = None
+    if graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                issue()
+        stream.wait_stream(side)
+        g.replay()                      # upload + warm
+        torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)] if timed_events else None
-    if ev is not None:                  # create the CUDA events outside the timed region
-        for row in ev:
-            for e in row:
-                e.record(stream)
-        torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.nvtx.range_push(f"{tag}_{wl.cfg.name}")
     t0.record(stream)
-    for i in range(steps):
-        if ev is not None:
-            ev[i][0].record(stream)
-            wl.step(events=ev[i][1:])
-        else:
-            wl.step()
+    if g is not None:
+        g.replay()
+    else:
+        issue()
     t1.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier(world)
     ms = t0.elapsed_time(t1)
-    stage_ms = None
-    if ev is not None:
+    try:
         stage_ms = {name: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in ev])) for j, name in enumerate(STAGES)}
+    except Exception:                   # graph-recorded events not timeable here: time the stages eagerly
+        stage_ms = None
+    del g
+    if stage_ms is None:
+        _, stage_ms = time_steps(wl, steps, 0, world, graph=False, tag="stages")
     return max_over_ranks(world, ms), stage_ms
 
 
@@ -388,9 +411,11 @@ def run_ours(args):
 
     clocks = ClockSampler(dev)
     clocks.start()
-    ms_pre, stages_pre = time_steps(pre, steps, warmup, world)
-    ms_dec, stages_dec = time_steps(dec, steps, warmup, world)
+    ms_pre, stages_pre = time_steps(pre, steps, warmup, world, graph=not args.eager)
+    ms_dec, stages_dec = time_steps(dec, steps, warmup, world, graph=not args.eager)
     clocks.stop()
+    ms_pre_eager, _ = time_steps(pre, steps, warmup, world, graph=False, tag="eager")
+    ms_dec_eager, _ = time_steps(dec, steps, warmup, world, graph=False, tag="eager")
     for wl in (pre, dec):
         err = nvfp4_moe_get_error(wl.ws)
         if err != 0:
@@ -435,6 +460,8 @@ def run_ours(args):
         "hbm_gbs_step": pre.step_bytes() / t_step / 1e9,
         "hbm_frac_step": pre.step_bytes() / t_step / 1e9 / hbm,
         "stage_ms": stages_pre,
+        "launch": "eager" if args.eager else "cuda_graph",
+        "eager_ms_per_step": ms_pre_eager / steps,
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "peak_source": f"{peak_src} hbm_gbs",
                      "algorithmic_bytes": kb[dominant], "traffic": traffic},
@@ -442,6 +469,7 @@ def run_ours(args):
             "workload": config_block(dec.cfg, world)["workload"],
             "metric": "moe_decode_GB_per_s", "value": dec_gbs, "unit": "GB/s", "ms_per_step": ms_dec / steps,
             "hbm_frac": dec_gbs / hbm, "tokens_per_s": world * dec.cfg.T / t_dec,
+            "eager_ms_per_step": ms_dec_eager / steps,
             "algorithmic_bytes_per_step": dec.step_bytes(), "stage_ms": stages_dec,
             "roofline": {"bound": "hbm", "kernel": dec_dom,
                          "achieved": dec_kb[dec_dom] / (stages_dec[dec_dom] / 1e3) / 1e9, "peak": hbm,
@@ -467,7 +495,7 @@ def run_single(name, world, rank, dev, peaks, peak_src, steps, warmup):
     dec = Workload(W.MOE_CONFIGS[name], dev)
     clocks = ClockSampler(dev)
     clocks.start()
-    ms_dec, stages = time_steps(dec, steps, warmup, world)
+    ms_dec, stages = time_steps(dec, steps, warmup, world, graph=False)
     clocks.stop()
     err = nvfp4_moe_get_error(dec.ws)
     if err != 0:
@@ -545,6 +573,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA-graph replay")
     ap.add_argument("--only", choices=["all", "decode", "prefill_ep48", "shared", "tiny"], default="all",
                     help="one workload alone (small profiling cases)")
     args = ap.parse_args()

@@ -148,7 +148,9 @@ int nvfp4_moe_forward(const nvfp4_moe_args *args, void *workspace, size_t ws_byt
 /* nvfp4_moe_forward with a CUDA event recorded on `stream` before each of
  * its five kernels (route, quantise+permute, L1, L2, combine) and after the
  * last: events = 6 cudaEvent_t handles created by the caller.  Otherwise
- * identical; for per-stage timing. */
+ * identical; for per-stage timing.  While `stream` is being captured into a
+ * CUDA graph the records become external event nodes, so the events can be
+ * timed after each replay. */
 int nvfp4_moe_forward_timed(const nvfp4_moe_args *args, void *workspace, size_t ws_bytes, void *stream,
                             void *const *events);
 

@@ -158,12 +158,18 @@ int check_moe_args(const nvfp4_moe_args *a, bool need_out)
 }
 
 // Routing + quantise/permute + L1 (given epilogue).  Shared by forward and calibrate.
-// Records events[i] on s when events is non-null (per-stage timing).
+// Records events[i] on s when events is non-null (per-stage timing).  While
+// s is being captured into a CUDA graph the record becomes an external event
+// node, so the event can still be timed after the graph is replayed.
 int mark(void *const *events, int i, cudaStream_t s)
 {
     if (events == nullptr)
         return NVFP4_OK;
-    return cuda_status(cudaEventRecord(static_cast<cudaEvent_t>(events[i]), s));
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    const unsigned flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+    return cuda_status(cudaEventRecordWithFlags(static_cast<cudaEvent_t>(events[i]), s, flags));
 }
 
 int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi, void *const *events,

@@ -72,19 +72,25 @@ cudaError_t launch_finalize_gs(float *gs, cudaStream_t s)
 }
 
 // ------------------------------------------------------------ quantisation
-// One warp per source row; each lane handles 64 consecutive elements (4
-// blocks) per step.  With inv != nullptr the row is token t of a routed batch
-// and its codes and scales are written to each padded destination row
-// inv[t*k + j] >= 0 (the expert permutation); otherwise to row t.
+// One warp per (source row, 2048-column chunk); each lane handles 64
+// consecutive elements (4 blocks).  With inv != nullptr the row is token t of
+// a routed batch and its codes and scales are written to each padded
+// destination row inv[t*k + j] >= 0 (the expert permutation); otherwise to
+// row t.
+constexpr int kQuantChunk = 2048;
+
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
                                                             int64_t cols, int64_t ldx, const float *__restrict__ gs_ptr,
                                                             uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
                                                             int layout, const int32_t *__restrict__ inv, int k)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp;
-    if (row >= rows)
+    const int64_t chunks = (cols + kQuantChunk - 1) / kQuantChunk;
+    const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+    if (item >= rows * chunks)
         return;
+    const int64_t row = item / chunks;
+    const int64_t c0 = (item - row * chunks) * kQuantChunk + static_cast<int64_t>(lane) * 64;
     const float gs = __ldg(gs_ptr);
     int my_dst = -1;                         // lane j < k holds destination j
     int ndst = 1;
@@ -93,60 +99,59 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 
         if (lane < k)
             my_dst = __ldg(inv + row * k + lane);
     }
+    // lanes past the end of the row do no work but stay for the shuffles below
+    const bool active = c0 < cols;
     const int64_t kb_per_block = cols / 64;
     const __nv_bfloat16 *xr = x + row * ldx;
-    for (int64_t c0 = static_cast<int64_t>(lane) * 64; c0 < cols; c0 += 32 * 64) {
-        const int64_t nb_left = (cols - c0) / 16;
-        const int nb = nb_left < 4 ? static_cast<int>(nb_left) : 4;
-        uint32_t cw[8];
-        uint32_t sw = 0;
+    const int64_t nb_left = active ? (cols - c0) / 16 : 0;
+    const int nb = nb_left < 4 ? static_cast<int>(nb_left) : 4;
+    uint32_t cw[8];
+    uint32_t sw = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            cw[2 * b] = cw[2 * b + 1] = 0;
-            if (b < nb) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(xr + c0 + 16 * b);
-                const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-                const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&v0);
-                const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&v1);
-                float f[16];
+    for (int b = 0; b < 4; ++b) {
+        cw[2 * b] = cw[2 * b + 1] = 0;
+        if (b < nb) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(xr + c0 + 16 * b);
+            const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+            const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&v0);
+            const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&v1);
+            float f[16];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 a = __bfloat1622float2(h0[j]);
-                    const float2 c = __bfloat1622float2(h1[j]);
-                    f[2 * j] = a.x;
-                    f[2 * j + 1] = a.y;
-                    f[8 + 2 * j] = c.x;
-                    f[8 + 2 * j + 1] = c.y;
-                }
-                const uint32_t sb = quantize16(f, gs, cw[2 * b], cw[2 * b + 1]);
-                sw |= sb << (8 * b);
+            for (int j = 0; j < 4; ++j) {
+                const float2 a = __bfloat1622float2(h0[j]);
+                const float2 c = __bfloat1622float2(h1[j]);
+                f[2 * j] = a.x;
+                f[2 * j + 1] = a.y;
+                f[8 + 2 * j] = c.x;
+                f[8 + 2 * j + 1] = c.y;
             }
+            const uint32_t sb = quantize16(f, gs, cw[2 * b], cw[2 * b + 1]);
+            sw |= sb << (8 * b);
         }
-        for (int d = 0; d < ndst; ++d) {
-            int64_t dst = row;
-            if (inv != nullptr) {
-                dst = __shfl_sync(0xffffffffu, my_dst, d);
-                if (dst < 0)
-                    continue;
-            }
-            uint8_t *crow = codes + dst * (cols / 2) + c0 / 2;
-            if (nb == 4) {
-                reinterpret_cast<uint4 *>(crow)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-                reinterpret_cast<uint4 *>(crow)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-            } else {
+    }
+    for (int d = 0; d < ndst; ++d) {
+        int64_t dst = row;
+        if (inv != nullptr)
+            dst = __shfl_sync(0xffffffffu, my_dst, d);
+        if (!active || dst < 0)
+            continue;
+        uint8_t *crow = codes + dst * (cols / 2) + c0 / 2;
+        if (nb == 4) {
+            reinterpret_cast<uint4 *>(crow)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            reinterpret_cast<uint4 *>(crow)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+        } else {
+            for (int b = 0; b < nb; ++b)
+                reinterpret_cast<uint2 *>(crow)[b] = make_uint2(cw[2 * b], cw[2 * b + 1]);
+        }
+        if (layout == NVFP4_SCALES_MMA) {
+            *reinterpret_cast<uint32_t *>(scales + mma_scale_offset(dst, c0 / 64, kb_per_block)) = sw;
+        } else {
+            uint8_t *srow = scales + dst * (cols / 16) + c0 / 16;
+            if (nb == 4 && (cols % 64) == 0)
+                *reinterpret_cast<uint32_t *>(srow) = sw;
+            else
                 for (int b = 0; b < nb; ++b)
-                    reinterpret_cast<uint2 *>(crow)[b] = make_uint2(cw[2 * b], cw[2 * b + 1]);
-            }
-            if (layout == NVFP4_SCALES_MMA) {
-                *reinterpret_cast<uint32_t *>(scales + mma_scale_offset(dst, c0 / 64, kb_per_block)) = sw;
-            } else {
-                uint8_t *srow = scales + dst * (cols / 16) + c0 / 16;
-                if (nb == 4 && (cols % 64) == 0)
-                    *reinterpret_cast<uint32_t *>(srow) = sw;
-                else
-                    for (int b = 0; b < nb; ++b)
-                        srow[b] = static_cast<uint8_t>(sw >> (8 * b));
-            }
+                    srow[b] = static_cast<uint8_t>(sw >> (8 * b));
         }
     }
 }
@@ -154,7 +159,8 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 
 cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs,
                             uint8_t *codes, uint8_t *scales, int layout, const int32_t *inv, int k, cudaStream_t s)
 {
-    const int64_t blocks = (rows + 7) / 8;
+    const int64_t items = rows * ((cols + kQuantChunk - 1) / kQuantChunk);
+    const int64_t blocks = (items + 7) / 8;
     quantize_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, rows, cols, ldx, gs, codes, scales, layout,
                                                                      inv, k);
     return cudaGetLastError();
@@ -335,7 +341,9 @@ cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, 
 // ------------------------------------------------------------ combine
 // out[t] = bf16( sum_{j ascending} w[t,j] * y[row(t,j)] ) in fp32, where
 // row(t,j) is the slot's row in the unpadded expert-major y buffer.  One
-// block per token, 8 bf16 (16 bytes) per thread per step.
+// block per (token, 1024-column chunk), 8 bf16 (16 bytes) per thread.
+constexpr int kCombineChunk = 1024;
+
 __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__restrict__ y,
                                                       const int32_t *__restrict__ inv,
                                                       const int32_t *__restrict__ ids, const float *__restrict__ w,
@@ -358,39 +366,41 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__res
         s_w[threadIdx.x] = __ldg(w + f);
     }
     __syncthreads();
-    for (int64_t c = static_cast<int64_t>(threadIdx.x) * 8; c < H; c += static_cast<int64_t>(blockDim.x) * 8) {
-        float acc[8];
+    const int64_t c = static_cast<int64_t>(blockIdx.y) * kCombineChunk + static_cast<int64_t>(threadIdx.x) * 8;
+    if (c >= H)
+        return;
+    float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            acc[i] = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            const int64_t row = s_row[j];
-            if (row < 0)
-                continue;
-            const float wj = s_w[j];
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + row * H + c));
-            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+    for (int i = 0; i < 8; ++i)
+        acc[i] = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        const int64_t row = s_row[j];
+        if (row < 0)
+            continue;
+        const float wj = s_w[j];
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + row * H + c));
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = __bfloat1622float2(h[i]);
-                acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wj, f.x));
-                acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wj, f.y));
-            }
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h[i]);
+            acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wj, f.x));
+            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wj, f.y));
         }
-        uint4 o;
-        __nv_bfloat162 *oh = reinterpret_cast<__nv_bfloat162 *>(&o);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            oh[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-        *reinterpret_cast<uint4 *>(out + t * H + c) = o;
     }
+    uint4 o;
+    __nv_bfloat162 *oh = reinterpret_cast<__nv_bfloat162 *>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        oh[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(out + t * H + c) = o;
 }
 
 cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int32_t *ids, const float *w,
                            const int32_t *off, const int32_t *poff, int64_t T, int k, int64_t H,
                            __nv_bfloat16 *out, cudaStream_t s)
 {
-    combine_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(y, inv, ids, w, off, poff, k, H, out);
+    const dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>((H + kCombineChunk - 1) / kCombineChunk));
+    combine_kernel<<<grid, 128, 0, s>>>(y, inv, ids, w, off, poff, k, H, out);
     return cudaGetLastError();
 }
 

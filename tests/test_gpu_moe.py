@@ -261,3 +261,33 @@ def test_prefill_sampled_tokens():
     # every routed row of the batch: inv matches the oracle's stable positions
     o, n = region(p, 5)
     np.testing.assert_array_equal(ws[o:o + n].cpu().numpy().view(np.int32), route["pos_padded"])
+
+
+def test_forward_timed_matches_forward_eager_and_in_graph(tiny):
+    """nvfp4_moe_forward_timed gives the same output as nvfp4_moe_forward and
+    records six increasing timestamps, also when captured into a CUDA graph."""
+    from nvfp4_moe_expert_topk_b200 import nvfp4_moe_forward_timed
+    p = tiny
+    cfg = p.cfg
+    T = p.x.shape[0]
+    inputs = p.device_inputs()
+    ref, ws = p.run(inputs)
+    for graph in (False, True):
+        ev = [torch.cuda.Event(enable_timing=True, external=graph) for _ in range(6)]
+        out = torch.full((T, cfg.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+        if graph:
+            for e in ev:
+                e.record()
+            torch.cuda.synchronize()
+            s = torch.cuda.Stream()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    nvfp4_moe_forward_timed(**inputs, out=out, workspace=ws, events=ev, stream=s)
+            g.replay()
+        else:
+            nvfp4_moe_forward_timed(**inputs, out=out, workspace=ws, events=ev)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+        times = [ev[0].elapsed_time(e) for e in ev]
+        assert all(b >= a for a, b in zip(times, times[1:])) and times[-1] > 0
