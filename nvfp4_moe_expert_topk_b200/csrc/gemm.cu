@@ -9,12 +9,12 @@
 // GEMM -> SiLU -> re-quantise -> L2 GEMM; with one group it is the plain
 // NVFP4 GEMM of page 1 "Phase 2").
 //
-// Block of 10 warps, one block per SM, persistent over the tile list:
+// Block of 14 warps, one block per SM, persistent over the tile list:
 //   warp 0    TMA producer: per k-tile (256 elements) the valid 32-row boxes
 //             (or one 128-row box) of A, the BN rows of B as 128-row boxes,
 //             and the matching 512-byte scale atoms by bulk copy, into a
 //             shared-memory ring guarded by mbarriers;
-//   warps 6-9 scale stagers, one per TMEM lane quarter: move each stage's
+//   warps 10-13 scale stagers, one per TMEM lane quarter: move each stage's
 //             E4M3 scales from shared memory into that stage's TMEM scale
 //             slot with tcgen05.st (the layout the MMA reads: lane l, column
 //             4*j + m holds the 4 scales of row 128*h + 32*m + l for k-block
@@ -24,8 +24,10 @@
 //   warp 1    allocates TMEM; one thread issues the 4 tcgen05.mma (K=64) of
 //             each k-tile; the block-scaled FP4 MMA costs about the same pipe
 //             time per instruction at N=128 as at N=256, so tiles are 256 wide;
-//   warps 2-5 epilogue: TMEM -> registers (each thread owns one row of the
-//             tile), release the accumulator to the MMA thread, then one of
+//   warps 2-9 epilogue, two per TMEM lane quarter (each owns one row of the
+//             tile and half of its columns): TMEM -> registers with one wait,
+//             release the accumulator to the MMA thread at once (the next
+//             tile's MMAs wait only for this drain), then one of
 //             EPI_SWIGLU_QUANT  h = SiLU(a_g*g) * (a_u*u), NVFP4-quantised
 //                               with the expert's inter_gs (L1),
 //             EPI_SWIGLU_AMAX   same h, max|h| per expert (warmup),
@@ -55,8 +57,9 @@ constexpr int kBKBytes = 128;                   // bytes of codes per row per k-
 constexpr int kTileBytes = 128 * kBKBytes;      // 16 KB: 128 rows of one k-tile
 constexpr int kSFAtom = 512;                    // 128 rows x 4 scales (64 elements)
 constexpr int kSFStage = 4 * kSFAtom;           // one 128-row block, 4 k-blocks
-constexpr int kThreads = 320;
-constexpr int kFirstSFWarp = 6;
+constexpr int kThreads = 448;
+constexpr int kEpiWarps = 8;                    // warps 2-9
+constexpr int kFirstSFWarp = 2 + kEpiWarps;     // warps 10-13
 constexpr uint32_t kTmemCols = 512;
 
 template <int BN>
@@ -159,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < kNumAcc; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], 4);
+            mbar_init(&acc_empty[b], kEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -346,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // -------------------------------------------------------- epilogue
         const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int hf = (warp - 2) >> 2;         // which half of the tile's columns this warp owns
         const int row = q * 32 + lane;          // row of the tile owned by this thread
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
         int acc = 0;
@@ -363,20 +367,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc * BN);
 
             if constexpr (EPI == EPI_SWIGLU_QUANT || EPI == EPI_SWIGLU_AMAX) {
+                // drain gate columns [64hf, 64hf+64) and the matching up columns in two rounds of
+                // 32 (one wait each), computing h as it arrives, then release the accumulator
                 const float a = p.a_gs[0];
                 const float alpha_g = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + 0]));
                 const float alpha_u = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + 1]));
-                // drain: h for the tile's 128 columns of this row, then give the accumulator back
-                float h[128];
+                float h[64];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t g[16], u[16];
-                    tc_ld_32x32b_x16(t_acc + c * 16, g);
-                    tc_ld_32x32b_x16(t_acc + 128 + c * 16, u);
+                for (int r = 0; r < 2; ++r) {
+                    uint32_t g[32], u[32];
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const uint32_t col = hf * 64 + r * 32 + c * 16;
+                        tc_ld_32x32b_x16(t_acc + col, *reinterpret_cast<uint32_t(*)[16]>(&g[16 * c]));
+                        tc_ld_32x32b_x16(t_acc + 128 + col, *reinterpret_cast<uint32_t(*)[16]>(&u[16 * c]));
+                    }
                     tc_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        h[c * 16 + i] = silu_mul(__uint_as_float(g[i]) * alpha_g, __uint_as_float(u[i]) * alpha_u);
+                    for (int i = 0; i < 32; ++i)
+                        h[r * 32 + i] = silu_mul(__uint_as_float(g[i]) * alpha_g, __uint_as_float(u[i]) * alpha_u);
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -385,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if constexpr (EPI == EPI_SWIGLU_AMAX) {
                     float amax = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < 128; ++i)
+                    for (int i = 0; i < 64; ++i)
                         amax = fmaxf(amax, fabsf(h[i]));
                     if (!valid)
                         amax = 0.0f;
@@ -396,49 +405,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                         atomicMax(p.amax_bits + ti.e, __float_as_uint(amax));
                 } else {
                     const float hgs = p.inter_gs[ti.e];
-                    uint32_t codes[16];
-                    uint32_t sfw[2] = {0, 0};
+                    uint32_t codes[8];
+                    uint32_t sfw = 0;
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         float blk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             blk[i] = h[c * 16 + i];
-                        const uint32_t s = quantize16(blk, hgs, codes[2 * c], codes[2 * c + 1]);
-                        sfw[c >> 2] |= s << (8 * (c & 3));
+                        sfw |= quantize16(blk, hgs, codes[2 * c], codes[2 * c + 1]) << (8 * c);
                     }
                     if (valid) {
-                        // 128 h columns: 64 bytes of codes and two 4-byte scale words (k-blocks 2nt, 2nt+1)
+                        // 64 h columns: 32 bytes of codes and one 4-byte scale word (k-block 2nt + hf)
                         uint4 *hrow = reinterpret_cast<uint4 *>(p.h_codes +
                                                                 static_cast<int64_t>(ti.row0 + row) * p.h_ld_bytes +
-                                                                ti.nt * 64);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            hrow[i] = make_uint4(codes[4 * i], codes[4 * i + 1], codes[4 * i + 2], codes[4 * i + 3]);
-                        uint8_t *sf = p.h_sf + static_cast<int64_t>(ti.row0 / kBM) * p.h_sf_block_stride +
-                                      static_cast<int64_t>(2 * ti.nt) * kSFAtom + lane * 16 + q * 4;
-                        *reinterpret_cast<uint32_t *>(sf) = sfw[0];
-                        *reinterpret_cast<uint32_t *>(sf + kSFAtom) = sfw[1];
+                                                                ti.nt * 64 + hf * 32);
+                        hrow[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                        hrow[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                        *reinterpret_cast<uint32_t *>(p.h_sf + static_cast<int64_t>(ti.row0 / kBM) * p.h_sf_block_stride +
+                                                      static_cast<int64_t>(2 * ti.nt + hf) * kSFAtom + lane * 16 +
+                                                      q * 4) = sfw;
                     }
                 }
             } else {
+                // drain columns [hf*BN/2, (hf+1)*BN/2) in rounds of 64 (one wait each),
+                // converting to bf16 as they arrive, then release the accumulator
+                constexpr int kCols = BN / 2;
+                constexpr int kRound = kCols < 64 ? kCols : 64;
                 const float a = p.a_gs[p.a_gs_per_expert ? ti.e : 0];
-                uint32_t o[BN / 2];
+                uint32_t o[kCols / 2];
 #pragma unroll
-                for (int c = 0; c < BN / 16; ++c) {
-                    uint32_t v[16];
-                    tc_ld_32x32b_x16(t_acc + c * 16, v);
+                for (int r = 0; r < kCols / kRound; ++r) {
+                    uint32_t v[kRound];
+#pragma unroll
+                    for (int c = 0; c < kRound / 16; ++c)
+                        tc_ld_32x32b_x16(t_acc + hf * kCols + r * kRound + c * 16,
+                                         *reinterpret_cast<uint32_t(*)[16]>(&v[16 * c]));
                     tc_wait_ld();
-                    const int col = ti.nt * BN + c * 16;
-                    int seg = 0;
 #pragma unroll
-                    for (int i = 0; i < 3; ++i)
-                        if (i < p.nseg - 1 && col >= p.seg_end[i])
-                            seg = i + 1;
-                    const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + seg]));
+                    for (int c = 0; c < kRound / 16; ++c) {
+                        const int col = ti.nt * BN + hf * kCols + r * kRound + c * 16;
+                        int seg = 0;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        o[c * 8 + i] = pack_bf16x2(__uint_as_float(v[2 * i]) * alpha, __uint_as_float(v[2 * i + 1]) * alpha);
+                        for (int i = 0; i < 3; ++i)
+                            if (i < p.nseg - 1 && col >= p.seg_end[i])
+                                seg = i + 1;
+                        const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + seg]));
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            o[(r * kRound + c * 16) / 2 + i] = pack_bf16x2(__uint_as_float(v[16 * c + 2 * i]) * alpha,
+                                                                           __uint_as_float(v[16 * c + 2 * i + 1]) * alpha);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -446,9 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive(&acc_empty[acc]);
                 if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(p.out + static_cast<int64_t>(ti.row0_out + row) * p.ldo +
-                                                           static_cast<int64_t>(ti.nt) * BN);
+                                                           static_cast<int64_t>(ti.nt) * BN + hf * kCols);
 #pragma unroll
-                    for (int i = 0; i < BN / 8; ++i)
+                    for (int i = 0; i < kCols / 8; ++i)
                         dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
                 }
             }
