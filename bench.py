@@ -164,10 +164,12 @@ def barrier(world):
 
 
 def max_over_ranks(world, v):
+    """Max of a per-rank scalar (a device time) over all ranks."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -330,6 +332,71 @@ def time_e2e(wl, steps, warmup, world):
     return ms, h2d, d2h
 
 
+# ---------------------------------------------------------------- MLA GEMMs
+def time_mla_gemms(dev, steps, warmup, peaks):
+    """The MLA projections as separate dense NVFP4 GEMMs at M=2048 (weights
+    quantised once; per step: activation global scale + quantisation + GEMM).
+    Device times from CUDA events; the GEMM alone is bracketed separately."""
+    from nvfp4_moe_expert_topk_b200 import (NVFP4_SCALES_MMA, nvfp4_gemm, nvfp4_quantize, nvfp4_scales_bytes)
+    res = {}
+    fp4_peak = peaks["bf16_tflops_sustained"] * BF16_TO_FP4_NOMINAL_RATIO
+    ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    stream = torch.cuda.current_stream()
+    for idx, (name, cfg) in enumerate(W.MLA_GEMMS.items()):
+        a, w = W.gemm_operands(cfg, idx, dev)
+        M, N, K = cfg.M, cfg.N, cfg.K
+        segs = list(cfg.seg_end)
+        w_codes = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+        w_sc = torch.empty(nvfp4_scales_bytes(N, K, NVFP4_SCALES_MMA), dtype=torch.uint8, device=dev)
+        w_gs = torch.empty(len(segs), dtype=torch.float32, device=dev)
+        start = 0
+        for i, end in enumerate(segs):
+            nvfp4_global_scale(w[start:end], w_gs[i:i + 1])
+            nvfp4_quantize(w[start:end], w_gs[i:i + 1], w_codes[start:end], w_sc[start * (K // 16):end * (K // 16)],
+                           NVFP4_SCALES_MMA)
+            start = end
+        del w
+        ad = a.to(dev)
+        a_gs = torch.empty(1, dtype=torch.float32, device=dev)
+        a_codes = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        a_sc = torch.empty(nvfp4_scales_bytes(M, K, NVFP4_SCALES_MMA), dtype=torch.uint8, device=dev)
+        out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            nvfp4_global_scale(ad, a_gs)
+            nvfp4_quantize(ad, a_gs, a_codes, a_sc, NVFP4_SCALES_MMA)
+            if ev is not None:
+                ev[1].record(stream)
+            nvfp4_gemm(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for e in evs:
+            step(e)
+        torch.cuda.synchronize()
+        step_ms = float(np.mean([e[0].elapsed_time(e[2]) for e in evs]))
+        gemm_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+        flops = 2.0 * M * N * K
+        gbytes = (M * K + N * K) * (0.5 + 1 / 16) + M * N * 2.0
+        ai = flops / gbytes
+        tflops = flops / (gemm_ms * 1e-3) / 1e12
+        gbs = gbytes / (gemm_ms * 1e-3) / 1e9
+        bound = "tensor" if ai >= ridge else "hbm"
+        res[name] = {"M": M, "N": N, "K": K, "ms_per_step": step_ms, "gemm_ms": gemm_ms, "tflops": tflops,
+                     "gbs": gbs, "arith_intensity": ai, "bound": bound,
+                     "frac": (tflops / fp4_peak) if bound == "tensor" else (gbs / peaks["hbm_gbs"]),
+                     "fp4_nominal_frac": tflops / FP4_NOMINAL_TFLOPS}
+        del ad, a_codes, a_sc, out, w_codes, w_sc
+        torch.cuda.empty_cache()
+    return res
+
+
 # ---------------------------------------------------------------- CPU oracle
 def oracle_sample(cfg, tokens, dev, inter_gs_dev):
     """Oracle inputs for a token sample of a workload: the sampled tokens'
@@ -423,6 +490,7 @@ def run_ours(args):
         if not torch.isfinite(wl.out.float()).all():
             raise RuntimeError(f"non-finite output in the {wl.cfg.name} run")
     e2e_ms, h2d, d2h = time_e2e(pre, steps, warmup, world)
+    mla = time_mla_gemms(dev, min(steps, 50), warmup, peaks)
 
     t_step = ms_pre / steps / 1e3
     tokens_s = world * pre.cfg.T / t_step
@@ -478,6 +546,7 @@ def run_ours(args):
         },
         "e2e": {"value": world * pre.cfg.T * steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / steps},
+        "mla_gemms": mla,
         "gpu_launches": KERNELS_PER_STEP * steps * 2,
         "clocks": clocks.summary(),
     }

@@ -94,3 +94,63 @@ def test_gemm_matches_oracle(M, N, K, segs):
     err = row_rel_l2(out, ref)
     assert err.max() <= 5e-3, err.max()
     assert cosine(out, ref) >= 0.99999
+
+
+@pytest.mark.parametrize("name", ["wqa_wkv", "q_b", "o_b"])
+def test_mla_projection_full_size(name):
+    """The MLA projections at M=2048 ("nvfp4-megamoe-kernel / CURRENT_BUG.md",
+    page 1 "Phase 2", option 1: one NVFP4 GEMM per projection; fused_wqa_wkv
+    with one global scale per half).  The device quantises activation and
+    weight through the library; both equal the oracle's quantisation bit for
+    bit; sampled output rows match the oracle GEMM."""
+    from nvfp4_moe_expert_topk_b200 import NVFP4_SCALES_MMA, nvfp4_global_scale, nvfp4_quantize, nvfp4_scales_bytes
+    from helpers import from_mma_layout
+    idx = list(W.MLA_GEMMS).index(name)
+    cfg = W.MLA_GEMMS[name]
+    a, w = W.gemm_operands(cfg, idx, DEV)
+    M, N, K = cfg.M, cfg.N, cfg.K
+    # device quantisation (activation: one global scale; weight: one per segment)
+    ad = a.to(DEV)
+    a_gs = torch.empty(1, dtype=torch.float32, device=DEV)
+    nvfp4_global_scale(ad, a_gs)
+    a_codes = torch.empty(M, K // 2, dtype=torch.uint8, device=DEV)
+    a_sc = torch.empty(nvfp4_scales_bytes(M, K, NVFP4_SCALES_MMA), dtype=torch.uint8, device=DEV)
+    nvfp4_quantize(ad, a_gs, a_codes, a_sc, NVFP4_SCALES_MMA)
+    w_codes = torch.empty(N, K // 2, dtype=torch.uint8, device=DEV)
+    w_sc = torch.empty(nvfp4_scales_bytes(N, K, NVFP4_SCALES_MMA), dtype=torch.uint8, device=DEV)
+    segs = list(cfg.seg_end)
+    w_gs = torch.empty(len(segs), dtype=torch.float32, device=DEV)
+    start = 0
+    for i, end in enumerate(segs):
+        nvfp4_global_scale(w[start:end], w_gs[i:i + 1])
+        nvfp4_quantize(w[start:end], w_gs[i:i + 1], w_codes[start:end],
+                       w_sc[start * (K // 16):end * (K // 16)], NVFP4_SCALES_MMA)
+        start = end
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    nvfp4_gemm(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out)
+    torch.cuda.synchronize()
+    # oracle quantisation of the same bf16 values
+    ab = W.bf16_bits(a)
+    oa_gs = O.global_scale_bf16(ab)
+    assert a_gs.item() == oa_gs
+    oac, oas = O.quantize_bf16(ab, oa_gs)
+    np.testing.assert_array_equal(a_codes.cpu().numpy(), oac)
+    np.testing.assert_array_equal(from_mma_layout(a_sc.cpu().numpy(), M, K), oas)
+    wb = W.bf16_bits(w)
+    owc, ows, owg = [], [], []
+    start = 0
+    for i, end in enumerate(segs):
+        gs = O.global_scale_bf16(wb[start:end])
+        assert w_gs[i].item() == gs
+        c, s_ = O.quantize_bf16(wb[start:end], gs)
+        owc.append(c), ows.append(s_), owg.append(gs)
+        start = end
+    owc, ows = np.concatenate(owc), np.concatenate(ows)
+    np.testing.assert_array_equal(w_codes.cpu().numpy(), owc)
+    # sampled rows: first, last, and random ones across the m-tiles
+    rows = np.unique(np.concatenate([[0, M - 1, 127, 128], np.random.default_rng(idx).choice(M, 4, replace=False)]))
+    ref = O.gemm(oac[rows], oas[rows], oa_gs, owc, ows, np.array(owg, np.float32), segs)
+    got = bf16_to_np(out[torch.from_numpy(rows).to(DEV)])
+    err = row_rel_l2(got, ref)
+    assert err.max() <= 5e-3, err.max()
+    assert cosine(got, ref) >= 0.99999
