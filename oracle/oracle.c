@@ -485,6 +485,47 @@ int oracle_moe_warmup_inter_gs(const oracle_moe_args *p_in, float *inter_gs_out)
     return bad;
 }
 
+/* ------------------------------------------------------------------ */
+/* Top-k router (the step before the path)                             */
+/* ------------------------------------------------------------------ */
+
+/* For each token: the k experts with the largest logits, in descending
+ * order, ties to the lower expert id (the router's scores -- softmax or
+ * sigmoid of the logits -- are increasing functions of the logit, so the
+ * same experts).  Weights (R9): scoring 0 = softmax renormalised over the
+ * selected experts, w_j = exp(l_j) / sum_i exp(l_i); scoring 1 = sigmoid
+ * renormalised, w_j = s_j / sum_i s_i.  Evaluated in fp64, stored fp32. */
+void oracle_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *ids, float *w)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; t++) {
+        const float *l = logits + t * E;
+        int32_t *id = ids + t * k;
+        for (int j = 0; j < k; j++) {
+            int best = -1;
+            for (int e = 0; e < E; e++) {
+                int taken = 0;
+                for (int i = 0; i < j; i++)
+                    if (id[i] == e)
+                        taken = 1;
+                if (taken)
+                    continue;
+                if (best < 0 || l[e] > l[best])   /* strict: the lower id wins a tie */
+                    best = e;
+            }
+            id[j] = best;
+        }
+        double sum = 0.0, v[32];
+        for (int j = 0; j < k; j++) {
+            double x = (double)l[id[j]];
+            v[j] = scoring == 0 ? exp(x - (double)l[id[0]]) : 1.0 / (1.0 + exp(-x));
+            sum += v[j];
+        }
+        for (int j = 0; j < k; j++)
+            w[t * k + j] = (float)(v[j] / sum);
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -15,6 +15,7 @@ Parity status of each entry point (what pins it lives in tests/test_oracle_*.py)
   gemm                           pinned (numpy matmul on dequantised operands)
   moe_forward                    pinned (per-token brute force, dense reduction)
   moe_warmup_inter_gs            pinned (brute-force amax of h)
+  topk                           pinned (numpy stable sort, torch softmax / sigmoid)
 """
 import ctypes
 import os
@@ -71,6 +72,7 @@ def lib():
         L.oracle_moe_forward.restype = ctypes.c_int
         L.oracle_moe_warmup_inter_gs.argtypes = [ctypes.POINTER(MoeArgs), P]
         L.oracle_moe_warmup_inter_gs.restype = ctypes.c_int
+        L.oracle_topk.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -242,3 +244,14 @@ def moe_warmup_inter_gs(x_bits, topk_ids, topk_weights, x_gs, w13_codes, w13_sca
     out = np.empty(E, np.float32)
     lib().oracle_moe_warmup_inter_gs(ctypes.byref(a), _ptr(out))
     return out
+
+
+def topk(logits: np.ndarray, k: int, scoring: str = "softmax"):
+    """(ids int32 [T, k], weights fp32 [T, k]) from router logits [T, E] fp32."""
+    l = _c(logits, np.float32)
+    T, E = l.shape
+    assert 1 <= k <= min(E, 32)
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    lib().oracle_topk(_ptr(l), T, E, k, {"softmax": 0, "sigmoid": 1}[scoring], _ptr(ids), _ptr(w))
+    return ids, w
