@@ -333,10 +333,149 @@ def time_e2e(wl, steps, warmup, world):
 
 
 # ---------------------------------------------------------------- MLA GEMMs
-def time_mla_gemms(dev, steps, warmup, peaks):
+def graph_time(fns, reps, warmup, flush=None):
+    """Per-call device times of a sequence of calls, issued back to back.
+    `reps` repetitions of [flush(); ev0; fns[0](); ev1; fns[1](); ...] are
+    captured into one CUDA graph (external event records, so the kernels run
+    without host gaps between them) and replayed once after a warm replay;
+    returns the mean milliseconds of each fns[j] over the repetitions.  With
+    `flush` (a write of a buffer larger than L2) every repetition starts
+    L2-cold; without it, repeated calls find their inputs in L2."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        for f in fns:
+            f()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(fns) + 1)] for _ in range(reps)]
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for row in ev:
+                if flush is not None:
+                    flush()
+                row[0].record()
+                for j, f in enumerate(fns):
+                    f()
+                    row[j + 1].record()
+    stream.wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    out = [float(np.mean([row[j].elapsed_time(row[j + 1]) for row in ev])) for j in range(len(fns))]
+    del g
+    return out
+
+
+class L2Flush:
+    """A 512 MB device buffer; calling the object overwrites it (4x the 126 MB L2)."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        self.i = 0
+
+    def __call__(self):
+        self.i = (self.i + 1) & 0xFF
+        self.buf.fill_(self.i)
+
+
+def time_router(cfg, dev, reps, warmup, flush):
+    """The device top-k router (logits [T, E] fp32 -> top-k ids and
+    renormalised sigmoid weights) on the batch's shape, one launch per call.
+    Hot: logits L2-resident (the router GEMM has just written them); cold:
+    after an L2 flush."""
+    from nvfp4_moe_expert_topk_b200 import NVFP4_SCORING_SIGMOID, nvfp4_moe_topk
+    logits = W.router_logits(cfg, dev)
+    ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
+
+    def call():
+        nvfp4_moe_topk(logits, cfg.k, ids, w, NVFP4_SCORING_SIGMOID)
+
+    hot, = graph_time([call], reps, warmup)
+    cold, = graph_time([call], reps, 0, flush)
+    nbytes = cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
+    return {"T": cfg.T, "E": cfg.E, "k": cfg.k, "scoring": "sigmoid", "us_per_call": round(hot * 1e3, 2),
+            "us_per_call_cold": round(cold * 1e3, 2), "GB_s": round(nbytes / (hot * 1e-3) / 1e9, 1),
+            "GB_s_cold": round(nbytes / (cold * 1e-3) / 1e9, 1), "bytes_per_call": nbytes, "launches": 1,
+            "timing": "CUDA graph of back-to-back calls; hot = logits in L2, cold = after a 512 MB L2 flush"}
+
+
+def time_variant_routing(wl, cfg, steps, warmup, world):
+    """The prefill step on the same weights and tokens with another routing
+    (pure Zipf: no expert forced empty), CUDA-graph timed like the headline."""
+    _, ids, w = W.batch(cfg)
+    saved = (wl.ids, wl.w)
+    wl.ids, wl.w = ids.to(wl.dev), w.to(wl.dev)
+    ms, stages = time_steps(wl, steps, warmup, world, graph=True, tag="variant")
+    wl.ids, wl.w = saved
+    counts = np.bincount(ids.numpy().reshape(-1), minlength=cfg.E)
+    t = ms / steps / 1e3
+    return {"workload": f"prefill_moe_E{cfg.E}_k{cfg.k}_T{cfg.T}_zipf{cfg.zipf_s}_pure",
+            "ms_per_step": ms / steps, "tokens_per_s": world * cfg.T / t,
+            "tflops": 2.0 * counts.sum() * 3 * cfg.H * cfg.I / t / 1e12,
+            "empty_experts": int((counts == 0).sum()), "max_rows_per_expert": int(counts.max()),
+            "m_tiles": int(np.ceil(counts / 128).sum()), "stage_ms": stages}
+
+
+def time_shared(dev, steps, warmup, flush):
+    """The shared-expert config (one expert, 256 tokens: 37 MB of weights,
+    which fit in L2): hot (back-to-back steps) and cold (L2 flushed before
+    every step), CUDA-graph timed."""
+    wl = Workload(W.MOE_CONFIGS["shared"], dev)
+    hot, = graph_time([wl.step], steps, warmup)
+    cold, = graph_time([wl.step], steps, 0, flush)
+    if nvfp4_moe_get_error(wl.ws) != 0:
+        raise RuntimeError("device error word after the shared-expert run")
+    b, f = wl.step_bytes(), wl.flops()
+    return {"workload": config_block(wl.cfg, 1)["workload"], "ms_hot": hot, "ms_cold": cold,
+            "GB_s_hot": b / (hot * 1e-3) / 1e9, "GB_s_cold": b / (cold * 1e-3) / 1e9,
+            "tflops_hot": f / (hot * 1e-3) / 1e12, "tflops_cold": f / (cold * 1e-3) / 1e12,
+            "algorithmic_bytes": b}
+
+
+def fp4_ceiling(dev, sms):
+    """Tensor-pipe ceiling of the FP4 MMA (nvfp4_fp4_mma_ceiling): one block
+    per SM issues k-tiles of four M=128 K=64 MMAs for ~20 ms (long enough to
+    reach the power-capped clock); TFLOP/s from CUDA events, cycles per MMA
+    from the blocks' own clocks."""
+    from nvfp4_moe_expert_topk_b200 import nvfp4_fp4_mma_ceiling
+    res = {}
+    for bn, iters in ((256, 50000), (128, 50000)):
+        cycles = torch.zeros(sms, dtype=torch.int64, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        nvfp4_fp4_mma_ceiling(bn, 2000, cycles, err)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        nvfp4_fp4_mma_ceiling(bn, iters, cycles, err)
+        b.record()
+        torch.cuda.synchronize()
+        if err.item() != 0 or (cycles < 0).any():
+            raise RuntimeError("FP4 ceiling probe: a bounded wait gave up")
+        ms = a.elapsed_time(b)
+        flops = sms * iters * 4 * 2.0 * 128 * bn * 64
+        cyc = cycles.double()
+        res[f"n{bn}"] = {"tflops": flops / (ms * 1e-3) / 1e12, "ms": ms,
+                         "cycles_per_mma": float(cyc.mean()) / (iters * 4),
+                         "cycles_per_mma_max": float(cyc.max()) / (iters * 4),
+                         "implied_sm_mhz": float(cyc.mean()) / (ms * 1e3)}
+    return res
+
+
+def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
     """The MLA projections as separate dense NVFP4 GEMMs at M=2048 (weights
     quantised once; per step: activation global scale + quantisation + GEMM).
-    Device times from CUDA events; the GEMM alone is bracketed separately."""
+    Device times from CUDA events inside a CUDA graph; the GEMM alone is
+    bracketed separately, hot (operands as the quantiser left them, weights
+    L2-resident where they fit) and cold (after a 512 MB L2 flush)."""
     from nvfp4_moe_expert_topk_b200 import (NVFP4_SCALES_MMA, nvfp4_gemm, nvfp4_quantize, nvfp4_scales_bytes)
     res = {}
     fp4_peak = peaks["bf16_tflops_sustained"] * BF16_TO_FP4_NOMINAL_RATIO
@@ -362,26 +501,16 @@ def time_mla_gemms(dev, steps, warmup, peaks):
         a_sc = torch.empty(nvfp4_scales_bytes(M, K, NVFP4_SCALES_MMA), dtype=torch.uint8, device=dev)
         out = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
 
-        def step(ev=None):
-            if ev is not None:
-                ev[0].record(stream)
+        def quant():
             nvfp4_global_scale(ad, a_gs)
             nvfp4_quantize(ad, a_gs, a_codes, a_sc, NVFP4_SCALES_MMA)
-            if ev is not None:
-                ev[1].record(stream)
-            nvfp4_gemm(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out)
-            if ev is not None:
-                ev[2].record(stream)
 
-        for _ in range(warmup):
-            step()
-        torch.cuda.synchronize()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-        for e in evs:
-            step(e)
-        torch.cuda.synchronize()
-        step_ms = float(np.mean([e[0].elapsed_time(e[2]) for e in evs]))
-        gemm_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+        def gemm():
+            nvfp4_gemm(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out)
+
+        quant_ms, gemm_ms = graph_time([quant, gemm], steps, warmup)
+        _, gemm_cold_ms = graph_time([quant, gemm], steps, 0, flush)
+        step_ms = quant_ms + gemm_ms
         flops = 2.0 * M * N * K
         gbytes = (M * K + N * K) * (0.5 + 1 / 16) + M * N * 2.0
         ai = flops / gbytes
@@ -389,9 +518,12 @@ def time_mla_gemms(dev, steps, warmup, peaks):
         gbs = gbytes / (gemm_ms * 1e-3) / 1e9
         bound = "tensor" if ai >= ridge else "hbm"
         res[name] = {"M": M, "N": N, "K": K, "ms_per_step": step_ms, "gemm_ms": gemm_ms, "tflops": tflops,
+                     "gemm_ms_cold": gemm_cold_ms, "tflops_cold": flops / (gemm_cold_ms * 1e-3) / 1e12,
                      "gbs": gbs, "arith_intensity": ai, "bound": bound,
                      "frac": (tflops / fp4_peak) if bound == "tensor" else (gbs / peaks["hbm_gbs"]),
                      "fp4_nominal_frac": tflops / FP4_NOMINAL_TFLOPS}
+        if ceiling_tflops:
+            res[name]["fp4_ceiling_frac"] = tflops / ceiling_tflops
         del ad, a_codes, a_sc, out, w_codes, w_sc
         torch.cuda.empty_cache()
     return res
@@ -490,7 +622,13 @@ def run_ours(args):
         if not torch.isfinite(wl.out.float()).all():
             raise RuntimeError(f"non-finite output in the {wl.cfg.name} run")
     e2e_ms, h2d, d2h = time_e2e(pre, steps, warmup, world)
-    mla = time_mla_gemms(dev, min(steps, 50), warmup, peaks)
+    flush = L2Flush(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ceiling = fp4_ceiling(dev, sms)
+    mla = time_mla_gemms(dev, min(steps, 50), warmup, peaks, flush, ceiling["n256"]["tflops"])
+    router = time_router(pre.cfg, dev, 50, warmup, flush)
+    pure = time_variant_routing(pre, W.MOE_CONFIGS["prefill_zipf_pure"], min(steps, 50), warmup, world)
+    shared = time_shared(dev, min(steps, 50), warmup, flush)
 
     t_step = ms_pre / steps / 1e3
     tokens_s = world * pre.cfg.T / t_step
@@ -524,7 +662,9 @@ def run_ours(args):
         "config": config_block(pre.cfg, world),
         "tflops": tflops,
         "fp4_peak_frac": {"of_nominal_9000": tflops / FP4_NOMINAL_TFLOPS,
-                          f"of_{peak_src}_bf16_sustained_x4": tflops / fp4_measured},
+                          f"of_{peak_src}_bf16_sustained_x4": tflops / fp4_measured,
+                          "of_measured_fp4_mma_ceiling": tflops / ceiling["n256"]["tflops"]},
+        "fp4_mma_ceiling": ceiling,
         "hbm_gbs_step": pre.step_bytes() / t_step / 1e9,
         "hbm_frac_step": pre.step_bytes() / t_step / 1e9 / hbm,
         "stage_ms": stages_pre,
@@ -547,6 +687,9 @@ def run_ours(args):
         "e2e": {"value": world * pre.cfg.T * steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / steps},
         "mla_gemms": mla,
+        "router": router,
+        "prefill_pure_zipf": pure,
+        "shared_expert": shared,
         "gpu_launches": KERNELS_PER_STEP * steps * 2,
         "clocks": clocks.summary(),
     }

@@ -201,6 +201,38 @@ int nvfp4_moe_forward_noalloc(const nvfp4_moe_args *args, void *stream);
  * `stream`. */
 int nvfp4_moe_get_error(void *workspace, int32_t *err_host, void *stream);
 
+/* Top-k router: the step that produces topk_ids / topk_weights for
+ * nvfp4_moe_forward (page 3 "Architecture Notes": every token is routed to
+ * 6 of 384 experts).  The pages name the routing but not the score function;
+ * this entry point takes router logits and offers both usual ones.
+ * logits [T, E] fp32 row-major (finite).  For each token the k experts with
+ * the largest logits, in descending order, ties to the lower expert id
+ * (softmax and sigmoid preserve order, so these are also the k largest
+ * scores).  topk_ids [T, k] int32.  topk_weights [T, k] fp32, renormalised
+ * over the selection:
+ *   NVFP4_SCORING_SOFTMAX  w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0)
+ *   NVFP4_SCORING_SIGMOID  w_j = sigmoid(l_j) / sum_i sigmoid(l_i)
+ * Ids are exact; weights are fp32 evaluations of these formulas (relative
+ * error a few units in the last place).  1 <= k <= min(E, 32), E <= 1024,
+ * T >= 0 (T = 0 launches nothing, and the pointers may then be NULL).
+ * Allocates nothing. */
+/* Tensor-core ceiling probe (measurement; the pages have no counterpart).
+ * Launches `ctas` blocks (one per SM when ctas <= the SM count), each
+ * issuing `iters` k-tiles of four block-scaled FP4 MMAs (M = 128, N = bn,
+ * K = 64, the GEMM engine's instruction) from one thread into one TMEM
+ * accumulator with operands already on chip: the rate the GEMMs cannot
+ * exceed.  FLOPs = ctas * iters * 4 * 2 * 128 * bn * 64.  cycles: device
+ * int64 [ctas], SM clock cycles from first issue to completion per block
+ * (-1 if the bounded completion wait gave up, which also writes
+ * NVFP4_ERR_TIMEOUT to *err when err is not NULL).  bn is 128 or 256;
+ * 1 <= iters <= 1 << 24; 1 <= ctas <= 65535. */
+int nvfp4_fp4_mma_ceiling(int bn, int iters, int ctas, int64_t *cycles, int32_t *err, void *stream);
+
+#define NVFP4_SCORING_SOFTMAX 0
+#define NVFP4_SCORING_SIGMOID 1
+int nvfp4_moe_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *topk_ids,
+                   float *topk_weights, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,7 +18,8 @@ __all__ = [
     "nvfp4_swizzle_scales", "nvfp4_gemm", "nvfp4_moe_workspace_size", "nvfp4_moe_forward",
     "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
-    "nvfp4_moe_get_error", "MoeArgs",
+    "nvfp4_moe_get_error", "nvfp4_moe_topk", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling",
+    "MoeArgs",
 ]
 
 NVFP4_SCALES_ROWMAJOR = 0
@@ -74,6 +75,8 @@ def lib():
         L.nvfp4_moe_workspace_region.argtypes = [i64, i32, i32, i64, i64, i32,
                                                  ctypes.POINTER(i64), ctypes.POINTER(i64)]
         L.nvfp4_moe_get_error.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
+        L.nvfp4_moe_topk.argtypes = [P, i64, i32, i32, i32, P, P, P]
+        L.nvfp4_fp4_mma_ceiling.argtypes = [i32, i32, i32, P, P, P]
         _lib = L
     return _lib
 
@@ -231,3 +234,26 @@ def nvfp4_moe_get_error(workspace, stream=None) -> int:
     _check(lib().nvfp4_moe_get_error(_dev(workspace, "workspace", torch.uint8), ctypes.byref(err), _stream(stream)),
            "nvfp4_moe_get_error")
     return err.value
+
+
+NVFP4_SCORING_SOFTMAX = 0
+NVFP4_SCORING_SIGMOID = 1
+
+
+def nvfp4_moe_topk(logits, k, topk_ids, topk_weights, scoring=NVFP4_SCORING_SOFTMAX, stream=None):
+    """Top-k router on the device: logits [T, E] fp32 -> topk_ids [T, k] int32,
+    topk_weights [T, k] fp32 (renormalised softmax or sigmoid of the selection)."""
+    T, E = logits.shape
+    _check(lib().nvfp4_moe_topk(_dev(logits, "logits", torch.float32), T, E, k, scoring,
+                                _dev(topk_ids, "topk_ids", torch.int32),
+                                _dev(topk_weights, "topk_weights", torch.float32), _stream(stream)),
+           "nvfp4_moe_topk")
+
+
+def nvfp4_fp4_mma_ceiling(bn, iters, cycles, err=None, stream=None):
+    """Tensor-core ceiling probe: cycles.numel() blocks each issue `iters`
+    k-tiles of four FP4 MMAs (M=128, N=bn, K=64); cycles (int64, device)
+    receives each block's issue-to-completion SM cycles."""
+    _check(lib().nvfp4_fp4_mma_ceiling(bn, iters, cycles.numel(), _dev(cycles, "cycles", torch.int64),
+                                       None if err is None else _dev(err, "err", torch.int32), _stream(stream)),
+           "nvfp4_fp4_mma_ceiling")

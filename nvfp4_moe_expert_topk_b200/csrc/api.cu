@@ -551,6 +551,36 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
                                     static_cast<cudaStream_t>(stream)));
 }
 
+int nvfp4_moe_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *topk_ids, float *topk_weights,
+                   void *stream)
+{
+    if (T < 0 || k < 1 || E < 1)
+        return NVFP4_ERR_INVALID_ARG;
+    if (T > 0 && (logits == nullptr || topk_ids == nullptr || topk_weights == nullptr))
+        return NVFP4_ERR_INVALID_ARG;
+    if (scoring != NVFP4_SCORING_SOFTMAX && scoring != NVFP4_SCORING_SIGMOID)
+        return NVFP4_ERR_INVALID_ARG;
+    if (E > 1024 || k > 32 || k > E || T * E >= (1LL << 40))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    int st = device_check(nullptr);
+    if (st != NVFP4_OK)
+        return st;
+    return cuda_status(launch_topk(logits, T, E, k, scoring, topk_ids, topk_weights, static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_fp4_mma_ceiling(int bn, int iters, int ctas, int64_t *cycles, int32_t *err, void *stream)
+{
+    if (cycles == nullptr || (bn != 128 && bn != 256) || iters < 1 || ctas < 1)
+        return NVFP4_ERR_INVALID_ARG;
+    if (iters > (1 << 24) || ctas > 65535)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    int st = device_check(nullptr);
+    if (st != NVFP4_OK)
+        return st;
+    return cuda_status(launch_mma_ceiling(bn, iters, ctas, reinterpret_cast<long long *>(cycles), err,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int nvfp4_moe_get_error(void *workspace, int32_t *err_host, void *stream)
 {
     if (workspace == nullptr || err_host == nullptr)

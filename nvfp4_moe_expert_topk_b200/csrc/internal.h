@@ -72,5 +72,8 @@ cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int
                            const int32_t *off, const int32_t *poff, int64_t T, int k, int64_t H,
                            __nv_bfloat16 *out, cudaStream_t s);
 cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float *inter_gs, cudaStream_t s);
+cudaError_t launch_mma_ceiling(int bn, int iters, int ctas, long long *cycles, int32_t *err, cudaStream_t s);
+cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *ids, float *weights,
+                        cudaStream_t s);
 
 } // namespace nvfp4

@@ -440,4 +440,106 @@ cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------ top-k router
+// One warp per token.  Every logit becomes a 64-bit key whose high word is
+// its fp32 value mapped to an unsigned integer of the same order (-0 folded
+// into +0) and whose low word is ~expert, so a larger key is a larger logit
+// and, between equal logits, the lower expert.  Lane l holds experts
+// l, l + 32, ...; k rounds of a warp max pick the winners in descending
+// order, each round retiring the winner's key to 0 (below every real key).
+constexpr int kTopkWarps = 8;
+
+__device__ __forceinline__ uint32_t order_bits(float x)
+{
+    const uint32_t u = __float_as_uint(x == 0.0f ? 0.0f : x);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float from_order_bits(uint32_t o)
+{
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
+
+template <int P>
+__global__ void __launch_bounds__(32 * kTopkWarps) topk_kernel(const float *__restrict__ logits, int64_t T, int E,
+                                                               int k, int scoring, int32_t *__restrict__ ids,
+                                                               float *__restrict__ weights)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * kTopkWarps + (threadIdx.x >> 5);
+    if (t >= T)
+        return;   // whole warp leaves together
+    const float *row = logits + t * E;
+    unsigned long long key[P];
+#pragma unroll
+    for (int i = 0; i < P; i++) {
+        const int e = lane + 32 * i;
+        key[i] = e < E ? (static_cast<unsigned long long>(order_bits(__ldg(row + e))) << 32) | (~static_cast<uint32_t>(e))
+                       : 0ull;
+    }
+    unsigned long long best = 0;
+#pragma unroll
+    for (int i = 0; i < P; i++)
+        best = key[i] > best ? key[i] : best;
+    float mine = 0.0f;   // lane j < k: logit of the j-th winner
+    int mine_id = 0;
+    for (int j = 0; j < k; j++) {
+        unsigned long long m = best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, m, o);
+            m = other > m ? other : m;
+        }
+        if (lane == j) {
+            mine = from_order_bits(static_cast<uint32_t>(m >> 32));
+            mine_id = static_cast<int>(~static_cast<uint32_t>(m));
+        }
+        if (best == m) {   // this lane owned the winner: retire it
+            best = 0;
+#pragma unroll
+            for (int i = 0; i < P; i++) {
+                key[i] = key[i] == m ? 0ull : key[i];
+                best = key[i] > best ? key[i] : best;
+            }
+        }
+    }
+    // Weights over the selection: softmax (shifted by the top logit) or
+    // sigmoid, then divided by their sum.
+    const float top = __shfl_sync(0xffffffffu, mine, 0);
+    float v = 0.0f;
+    if (lane < k)
+        v = scoring == 0 ? expf(mine - top) : __frcp_rn(1.0f + expf(-mine));
+    float sum = v;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane < k) {
+        ids[t * k + lane] = mine_id;
+        weights[t * k + lane] = __fdiv_rn(v, sum);
+    }
+}
+
+cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *ids, float *weights,
+                        cudaStream_t s)
+{
+    if (T == 0)
+        return cudaSuccess;
+    const unsigned grid = static_cast<unsigned>((T + kTopkWarps - 1) / kTopkWarps);
+    const int per_lane = (E + 31) / 32;
+#define NVFP4_TOPK_CASE(P)                                                                                       \
+    if (per_lane <= P) {                                                                                         \
+        topk_kernel<P><<<grid, 32 * kTopkWarps, 0, s>>>(logits, T, E, k, scoring, ids, weights);                 \
+        return cudaGetLastError();                                                                               \
+    }
+    NVFP4_TOPK_CASE(2)
+    NVFP4_TOPK_CASE(4)
+    NVFP4_TOPK_CASE(8)
+    NVFP4_TOPK_CASE(12)
+    NVFP4_TOPK_CASE(16)
+    NVFP4_TOPK_CASE(24)
+    NVFP4_TOPK_CASE(32)
+#undef NVFP4_TOPK_CASE
+    return cudaErrorInvalidValue;
+}
+
 } // namespace nvfp4

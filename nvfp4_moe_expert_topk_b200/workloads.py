@@ -27,6 +27,7 @@ SEED_X, SEED_X_WARMUP = 0, 1
 SEED_ROUTER, SEED_ROUTER_WARMUP = 4, 14
 SEED_OUTLIER, SEED_ZIPF_PERM = 5, 6
 SEED_W13, SEED_W2, SEED_MLA = 1000, 2000, 3000
+SEED_LOGITS = 7
 WEIGHT_STD = 0.02
 
 
@@ -50,6 +51,9 @@ MOE_CONFIGS = {
     "shared": MoeConfig("shared", E=1, k=1, T=256, H=7168, I=3072, routing="single", outliers=True, warmup_T=256),
     "decode": MoeConfig("decode", E=48, k=6, T=64, H=7168, I=3072, routing="sigmoid", outliers=False, warmup_T=64),
     "prefill": MoeConfig("prefill", E=384, k=6, T=4096, H=7168, I=3072, routing="zipf", outliers=True, warmup_T=16),
+    # the prefill batch with pure Zipf popularity (no expert forced empty)
+    "prefill_zipf_pure": MoeConfig("prefill_zipf_pure", E=384, k=6, T=4096, H=7168, I=3072, routing="zipf",
+                                   outliers=True, warmup_T=16, zipf_zero_tail=0),
     # prefill-shaped (64 routed rows per expert on average, Zipf-skewed) on one
     # expert-parallel slice: small enough to profile and to check in full
     "prefill_ep48": MoeConfig("prefill_ep48", E=48, k=6, T=512, H=7168, I=3072, routing="zipf", outliers=True,
@@ -167,3 +171,8 @@ def gemm_operands(cfg: GemmConfig, index: int, device="cpu"):
 def bf16_bits(t: torch.Tensor):
     """bf16 tensor -> numpy uint16 bit patterns (what the oracle takes)."""
     return t.contiguous().view(torch.int16).cpu().numpy().view("uint16")
+
+
+def router_logits(cfg: MoeConfig, device="cpu") -> torch.Tensor:
+    """Router logits [T, E] fp32 ~ N(0, 1), the input of the top-k router."""
+    return torch.randn(cfg.T, cfg.E, generator=_gen(SEED_LOGITS, device), device=device, dtype=torch.float32)

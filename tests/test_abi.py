@@ -31,7 +31,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ["nvfp4_quantize", "nvfp4_gemm", "nvfp4_moe_forward", "nvfp4_global_scale",
                  "nvfp4_swizzle_scales", "nvfp4_moe_workspace_size", "nvfp4_moe_get_error",
-                 "nvfp4_moe_route_debug", "nvfp4_moe_calibrate", "nvfp4_status_string"]:
+                 "nvfp4_moe_route_debug", "nvfp4_moe_calibrate", "nvfp4_status_string", "nvfp4_moe_topk",
+                 "nvfp4_moe_forward_noalloc", "nvfp4_moe_forward_timed"]:
         assert want in names
 
 
@@ -108,3 +109,23 @@ def test_moe_forward_checks(L):
     assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None) == -3
     a.w2_codes = None
     assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None) == -1
+
+
+def test_topk_checks(L):
+    P = ctypes.c_void_p
+    F = P(1 << 40)
+    assert L.nvfp4_moe_topk(None, 4, 48, 6, 0, F, F, None) == -1
+    assert L.nvfp4_moe_topk(F, -1, 48, 6, 0, F, F, None) == -1
+    assert L.nvfp4_moe_topk(F, 4, 48, 0, 0, F, F, None) == -1
+    assert L.nvfp4_moe_topk(F, 4, 48, 6, 2, F, F, None) == -1         # unknown scoring
+    assert L.nvfp4_moe_topk(F, 4, 1025, 6, 0, F, F, None) == -2      # E > 1024
+    assert L.nvfp4_moe_topk(F, 4, 48, 33, 0, F, F, None) == -2       # k > 32
+    assert L.nvfp4_moe_topk(F, 4, 4, 6, 1, F, F, None) == -2         # k > E
+
+
+def test_ceiling_checks(L):
+    F = ctypes.c_void_p(1 << 40)
+    assert L.nvfp4_fp4_mma_ceiling(256, 10, 148, None, None, None) == -1
+    assert L.nvfp4_fp4_mma_ceiling(192, 10, 148, F, None, None) == -1
+    assert L.nvfp4_fp4_mma_ceiling(256, 0, 148, F, None, None) == -1
+    assert L.nvfp4_fp4_mma_ceiling(256, (1 << 24) + 1, 148, F, None, None) == -2
