@@ -62,16 +62,22 @@ constexpr int kEpiWarps = 8;                    // warps 2-9
 constexpr int kFirstSFWarp = 2 + kEpiWarps;     // warps 10-13
 constexpr uint32_t kTmemCols = 512;
 
-template <int BN>
+// CG = 1: one CTA computes a 128 x BN tile.  CG = 2: a cluster of two CTAs
+// computes a 256 x 256 tile with pair MMAs; each CTA loads its own 128 A
+// rows and one 128-row half of B (so per CTA a k-tile fills 32 KB of codes
+// instead of 48 KB for the same MMA work) and holds the scales of all 256
+// B rows.
+template <int BN, int CG>
 struct Cfg {
     static constexpr int kHalves = BN / 128;                 // 128-row halves of the B tile
+    static constexpr int kBBoxes = CG == 2 ? 1 : kHalves;    // B boxes this CTA loads per k-tile
     static constexpr int kNumAcc = BN == 256 ? 1 : 2;        // TMEM accumulators
-    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kStages = CG == 2 ? 5 : (BN == 256 ? 4 : 6);
     static constexpr int kSFSlotCols = 16 + 16 * kHalves;    // A: 4 k-blocks x 4 cols; B: 4 x 4 per half
     static constexpr uint32_t kTmemSF = kNumAcc * BN;        // scale slots follow the accumulators
     static constexpr int kA = 0;
     static constexpr int kB = kA + kStages * kTileBytes;
-    static constexpr int kSFA = kB + kStages * kTileBytes * kHalves;
+    static constexpr int kSFA = kB + kStages * kTileBytes * kBBoxes;
     static constexpr int kSFB = kSFA + kStages * kSFStage;
     static constexpr int kBars = kSFB + kStages * kSFStage * kHalves;
     static constexpr int kBarCount = 3 * kStages + 2 * kNumAcc + 1;
@@ -79,15 +85,43 @@ struct Cfg {
     static constexpr int kSmem = kMisc + 16 + 1024;          // + tmem slot, abort flag, alignment slack
     static_assert(kTmemSF + kStages * kSFSlotCols <= kTmemCols, "TMEM budget");
     static_assert(kSmem <= 232448, "shared memory budget");
+    static_assert(CG == 1 || BN == 256, "pair tiles are 256 wide");
 };
 
 struct TileInfo {
     int e, row0, valid, row0_out, nt;
 };
 
-__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, int t, int m_tiles)
+// Tile t of the launch's tile space, as seen by CTA `rank` of its cluster.
+// CG = 1: m-tiles of 128 rows.  CG = 2: m-pairs; the even CTA takes the
+// pair's first m-tile and the odd CTA the second (valid = 0 when the expert
+// or matrix has no rows left for it).
+template <int CG>
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, int t, int m_units, uint32_t rank)
 {
     TileInfo ti;
+    if constexpr (CG == 2) {
+        if (p.mtiles != nullptr) {
+            const int mp = t / p.n_tiles;
+            ti.nt = t - mp * p.n_tiles;
+            const int2 pr = p.pairs[mp];
+            const int mt = rank == 0 ? pr.x : pr.y;
+            const int4 m = p.mtiles[mt >= 0 ? mt : pr.x];
+            ti.e = m.x;
+            ti.row0 = mt >= 0 ? m.y : m.y + kBM;
+            ti.valid = mt >= 0 ? m.z : 0;
+            ti.row0_out = mt >= 0 ? m.w : m.w + kBM;
+        } else {
+            const int nt = t / m_units;
+            const int mp = t - nt * m_units;
+            ti.nt = nt;
+            ti.e = 0;
+            ti.row0 = mp * 2 * kBM + static_cast<int>(rank) * kBM;
+            ti.valid = max(0, min(kBM, p.dense_M - ti.row0));
+            ti.row0_out = ti.row0;
+        }
+        return ti;
+    }
     if (p.mtiles != nullptr) {
         const int mt = t / p.n_tiles;
         ti.nt = t - mt * p.n_tiles;
@@ -97,8 +131,8 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, int t, int m_
         ti.valid = m.z;
         ti.row0_out = m.w;
     } else {
-        const int nt = t / m_tiles;
-        const int mt = t - nt * m_tiles;
+        const int nt = t / m_units;
+        const int mt = t - nt * m_units;
         ti.nt = nt;
         ti.e = 0;
         ti.row0 = mt * kBM;
@@ -127,15 +161,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int CG>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a32,
                       const __grid_constant__ CUtensorMap map_b, const GemmArgs p)
 {
-    using C = Cfg<BN>;
+    using C = Cfg<BN, CG>;
     constexpr int kStages = C::kStages;
     constexpr int kHalves = C::kHalves;
     constexpr int kNumAcc = C::kNumAcc;
+    constexpr bool kPair = CG == 2;
     static_assert(EPI == EPI_BF16 || BN == 256, "SwiGLU tiles are 128 gate + 128 up columns");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -154,15 +189,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ int never_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // pair tiles: the even CTA of the cluster issues the MMAs and owns the
+    // sf_ready / acc_empty barriers both CTAs arrive on
+    const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+    const int unit = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+    const int units = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&sf_ready[s], 4);
+            mbar_init(&sf_ready[s], 4 * CG);
         }
         for (int b = 0; b < kNumAcc; ++b) {
             mbar_init(&acc_full[b], 1);
-            mbar_init(&acc_empty[b], kEpiWarps);
+            mbar_init(&acc_empty[b], kEpiWarps * CG);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -173,17 +213,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&map_b);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
+        if constexpr (kPair) {
+            tmem_alloc_pair(tmem_slot, kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_slot, kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (kPair)
+        cluster_sync();             // both CTAs' barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // cluster addresses of the leader's sf_ready / acc_empty barriers
+    const uint32_t sf_ready_lead = kPair ? map_shared_to_cta(smem_u32(sf_ready), 0) : 0u;
+    const uint32_t acc_empty_lead = kPair ? map_shared_to_cta(smem_u32(acc_empty), 0) : 0u;
 
-    const int m_tiles = (p.mtiles != nullptr) ? *reinterpret_cast<volatile const int32_t *>(p.num_mtiles_dev)
-                                              : p.dense_m_tiles;
-    const int total = m_tiles * p.n_tiles;
+    const int m_units = (p.mtiles != nullptr)
+                            ? *reinterpret_cast<volatile const int32_t *>(kPair ? p.num_pairs_dev : p.num_mtiles_dev)
+                            : (kPair ? (p.dense_M + 2 * kBM - 1) / (2 * kBM) : p.dense_m_tiles);
+    const int total = m_units * p.n_tiles;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -191,12 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0, pend_mask = 0, pend_par = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-                const TileInfo ti = decode_tile(p, t, m_tiles);
+            for (int t = unit; t < total && ok; t += units) {
+                const TileInfo ti = decode_tile<CG>(p, t, m_units, rank);
                 const int64_t brow0 = ti.e * p.b_rows_per_expert + static_cast<int64_t>(ti.nt) * p.b_tile_rows;
                 const int64_t brow1 = brow0 + p.b_half_offset;
-                const int a_boxes = ti.valid >= kBM ? 0 : (ti.valid + 31) / 32;   // 0: one 128-row box
-                const uint32_t a_bytes = a_boxes == 0 ? kTileBytes : a_boxes * (kTileBytes / 4);
+                // A: nothing for an empty pair half, else one 128-row box or the valid 32-row boxes
+                const int a_boxes = ti.valid >= kBM ? 0 : (ti.valid + 31) / 32;
+                const uint32_t a_bytes = ti.valid == 0 ? 0u : (a_boxes == 0 ? kTileBytes : a_boxes * (kTileBytes / 4));
                 const uint8_t *sfa = p.sfa + static_cast<int64_t>(ti.row0 / kBM) * p.sfa_block_stride;
                 const uint8_t *sfb0 = p.sfb + (brow0 / 128) * p.sfb_block_stride;
                 const uint8_t *sfb1 = p.sfb + (brow1 / 128) * p.sfb_block_stride;
@@ -207,25 +259,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const int nkb = min(4, (p.K - kt * kBK) / 64);
                     const uint32_t sf_bytes = static_cast<uint32_t>(nkb * kSFAtom);
-                    mbar_arrive_expect_tx(&full[stage], a_bytes + kHalves * kTileBytes + sf_bytes * (1 + kHalves));
+                    mbar_arrive_expect_tx(&full[stage], a_bytes + C::kBBoxes * kTileBytes +
+                                                            sf_bytes * (kHalves + (ti.valid > 0 ? 1 : 0)));
                     uint8_t *a_dst = sA + stage * kTileBytes;
-                    if (a_boxes == 0) {
-                        tma_load_2d(a_dst, &map_a, kt * kBKBytes, ti.row0, &full[stage]);
+                    if (ti.valid > 0) {
+                        if (a_boxes == 0) {
+                            tma_load_2d(a_dst, &map_a, kt * kBKBytes, ti.row0, &full[stage]);
+                        } else {
+                            for (int i = 0; i < a_boxes; ++i)
+                                tma_load_2d(a_dst + i * (kTileBytes / 4), &map_a32, kt * kBKBytes, ti.row0 + 32 * i,
+                                            &full[stage]);
+                        }
+                        bulk_load(sSFA + stage * kSFStage, sfa + kt * kSFStage, sf_bytes, &full[stage]);
+                    }
+                    uint8_t *b_dst = sB + stage * C::kBBoxes * kTileBytes;
+                    uint8_t *sfb_dst = sSFB + stage * kHalves * kSFStage;
+                    if constexpr (kPair) {
+                        // this CTA's half of the B rows; the scales of both halves
+                        tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(rank == 0 ? brow0 : brow1),
+                                    &full[stage]);
                     } else {
-                        for (int i = 0; i < a_boxes; ++i)
-                            tma_load_2d(a_dst + i * (kTileBytes / 4), &map_a32, kt * kBKBytes, ti.row0 + 32 * i,
+                        tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
+                        if constexpr (kHalves == 2)
+                            tma_load_2d(b_dst + kTileBytes, &map_b, kt * kBKBytes, static_cast<int32_t>(brow1),
                                         &full[stage]);
                     }
-                    uint8_t *b_dst = sB + stage * kHalves * kTileBytes;
-                    uint8_t *sfb_dst = sSFB + stage * kHalves * kSFStage;
-                    tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
                     bulk_load(sfb_dst, sfb0 + kt * kSFStage, sf_bytes, &full[stage]);
-                    if constexpr (kHalves == 2) {
-                        tma_load_2d(b_dst + kTileBytes, &map_b, kt * kBKBytes, static_cast<int32_t>(brow1),
-                                    &full[stage]);
+                    if constexpr (kHalves == 2)
                         bulk_load(sfb_dst + kSFStage, sfb1 + kt * kSFStage, sf_bytes, &full[stage]);
-                    }
-                    bulk_load(sSFA + stage * kSFStage, sfa + kt * kSFStage, sf_bytes, &full[stage]);
                     pend_mask |= 1u << stage;
                     pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == kStages) {
@@ -245,12 +306,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 1) {
         // -------------------------------------------------------- MMA issuer
-        constexpr uint32_t idesc = idesc_nvf4(kBM, BN);
-        if (lane == 0) {
+        // (pair tiles: the even CTA's thread issues for both CTAs)
+        constexpr uint32_t idesc = idesc_nvf4(kBM * CG, BN);
+        if (lane == 0 && rank == 0) {
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int t = unit; t < total && ok; t += units) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
                     ok = false;
                     break;
@@ -258,19 +320,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * BN);
                 for (int kt = 0; kt < p.num_k_tiles; ++kt) {
-                    if (!mbar_wait(&sf_ready[stage], phase, abort_flag) || !mbar_wait(&full[stage], phase, abort_flag)) {
+                    // sf_ready completes only after every stager has seen its CTA's
+                    // full barrier complete (all of the stage's copies landed), so
+                    // one wait covers both the scales and the operand tiles
+                    if (!mbar_wait(&sf_ready[stage], phase, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int nkb = min(4, (p.K - kt * kBK) / 64);
                     const uint32_t a_addr = smem_u32(sA + stage * kTileBytes);
-                    const uint32_t b_addr = smem_u32(sB + stage * kHalves * kTileBytes);
+                    const uint32_t b_addr = smem_u32(sB + stage * C::kBBoxes * kTileBytes);
                     const uint32_t t_sfa = tmem + C::kTmemSF + static_cast<uint32_t>(stage * C::kSFSlotCols);
-                    for (int kb = 0; kb < nkb; ++kb)
-                        tc_mma_nvf4(d_tmem, sdesc_kmajor_sw128(a_addr + kb * 32), sdesc_kmajor_sw128(b_addr + kb * 32),
-                                    idesc, t_sfa + kb * 4, t_sfa + 16 + kb * 4 * kHalves, (kt | kb) != 0 ? 1u : 0u);
-                    tc_commit(&empty[stage]);
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        const uint64_t ad = sdesc_kmajor_sw128(a_addr + kb * 32);
+                        const uint64_t bd = sdesc_kmajor_sw128(b_addr + kb * 32);
+                        const uint32_t acc_flag = (kt | kb) != 0 ? 1u : 0u;
+                        if constexpr (kPair)
+                            tc_mma_nvf4_pair(d_tmem, ad, bd, idesc, t_sfa + kb * 4, t_sfa + 16 + kb * 4 * kHalves,
+                                             acc_flag);
+                        else
+                            tc_mma_nvf4(d_tmem, ad, bd, idesc, t_sfa + kb * 4, t_sfa + 16 + kb * 4 * kHalves, acc_flag);
+                    }
+                    if constexpr (kPair)
+                        tc_commit_pair(&empty[stage], 0x3);
+                    else
+                        tc_commit(&empty[stage]);
                     if (++stage == kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -278,7 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit(&acc_full[acc]);
+                if constexpr (kPair)
+                    tc_commit_pair(&acc_full[acc], 0x3);
+                else
+                    tc_commit(&acc_full[acc]);
                 if (++acc == kNumAcc) {
                     acc = 0;
                     acc_phase ^= 1u;
@@ -289,7 +367,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 record_error(p.err, NVFP4_ERR_TIMEOUT);
             }
             // all MMAs of this thread complete before TMEM is freed
-            tc_commit(drain);
+            if constexpr (kPair)
+                tc_commit_pair(drain, 0x1);
+            else
+                tc_commit(drain);
             mbar_wait(drain, 0, &never_abort);
         }
         __syncwarp();
@@ -300,7 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = unit; t < total && ok; t += units) {
+            // an empty pair half has no A scales: its rows get scale 0
+            const bool a_rows = !kPair || decode_tile<CG>(p, t, m_units, rank).valid > 0;
             for (int kt = 0; kt < p.num_k_tiles; ++kt) {
                 const bool got = mbar_wait(&full[stage], phase, abort_flag);
                 if (!__all_sync(0xffffffffu, got)) {
@@ -314,7 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t *src = sSFA + stage * kSFStage + lane * 16;
 #pragma unroll
                 for (int kb = 0; kb < 4; ++kb) {
-                    const uint4 v = kb < nkb ? *reinterpret_cast<const uint4 *>(src + kb * kSFAtom) : make_uint4(0, 0, 0, 0);
+                    const uint4 v = (kb < nkb && a_rows) ? *reinterpret_cast<const uint4 *>(src + kb * kSFAtom)
+                                                         : make_uint4(0, 0, 0, 0);
                     r[4 * kb] = v.x, r[4 * kb + 1] = v.y, r[4 * kb + 2] = v.z, r[4 * kb + 3] = v.w;
                 }
                 tc_st_32x32b_x16(t_slot, r);
@@ -334,8 +418,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&sf_ready[stage]);
+                if (lane == 0) {
+                    if constexpr (kPair)
+                        mbar_arrive_cluster(sf_ready_lead + stage * 8);
+                    else
+                        mbar_arrive(&sf_ready[stage]);
+                }
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1u;
@@ -354,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        for (int t = unit; t < total; t += units) {
             const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, got)) {
                 *abort_flag = 1;
@@ -362,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const TileInfo ti = decode_tile(p, t, m_tiles);
+            const TileInfo ti = decode_tile<CG>(p, t, m_units, rank);
             const bool valid = row < ti.valid;
             const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc * BN);
 
@@ -389,8 +477,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&acc_empty[acc]);
+                if (lane == 0) {
+                    if constexpr (kPair)
+                        mbar_arrive_cluster(acc_empty_lead + acc * 8);
+                    else
+                        mbar_arrive(&acc_empty[acc]);
+                }
                 if constexpr (EPI == EPI_SWIGLU_AMAX) {
                     float amax = 0.0f;
 #pragma unroll
@@ -459,8 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&acc_empty[acc]);
+                if (lane == 0) {
+                    if constexpr (kPair)
+                        mbar_arrive_cluster(acc_empty_lead + acc * 8);
+                    else
+                        mbar_arrive(&acc_empty[acc]);
+                }
                 if (valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(p.out + static_cast<int64_t>(ti.row0_out + row) * p.ldo +
                                                            static_cast<int64_t>(ti.nt) * BN + hf * kCols);
@@ -478,43 +574,109 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (kPair)
+        cluster_sync();             // no CTA leaves while the pair's MMAs or arrivals may touch it
     tc_fence_after();
     if (warp == 1) {
         __syncwarp();
-        tmem_dealloc(tmem, kTmemCols);
+        if constexpr (kPair)
+            tmem_dealloc_pair(tmem, kTmemCols);
+        else
+            tmem_dealloc(tmem, kTmemCols);
     }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, int CG>
 static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
                               const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    const int smem = Cfg<BN>::kSmem;
+    const int smem = Cfg<BN, CG>::kSmem;
     static int attr_done_device = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
     if (attr_done_device != dev) {
-        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, EPI, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess)
             return e;
         attr_done_device = dev;
     }
-    nvfp4_gemm_kernel<BN, EPI><<<grid, kThreads, smem, stream>>>(map_a, map_a32, map_b, args);
-    return cudaGetLastError();
+    if constexpr (CG == 1) {
+        nvfp4_gemm_kernel<BN, EPI, 1><<<grid, kThreads, smem, stream>>>(map_a, map_a32, map_b, args);
+        return cudaGetLastError();
+    } else {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, 2>, map_a, map_a32, map_b, args);
+    }
 }
 
-cudaError_t launch_gemm(int bn, int epi, const CUtensorMap &map_a, const CUtensorMap &map_a32,
+cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
                         const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    switch (epi) {
-    case EPI_SWIGLU_QUANT: return launch_one<256, EPI_SWIGLU_QUANT>(map_a, map_a32, map_b, args, grid, stream);
-    case EPI_SWIGLU_AMAX: return launch_one<256, EPI_SWIGLU_AMAX>(map_a, map_a32, map_b, args, grid, stream);
-    default:
-        return bn == 256 ? launch_one<256, EPI_BF16>(map_a, map_a32, map_b, args, grid, stream)
-                         : launch_one<128, EPI_BF16>(map_a, map_a32, map_b, args, grid, stream);
+    if (cg == 2) {
+        if (bn != 256 || grid % 2 != 0)
+            return cudaErrorInvalidValue;
+        switch (epi) {
+        case EPI_SWIGLU_QUANT: return launch_one<256, EPI_SWIGLU_QUANT, 2>(map_a, map_a32, map_b, args, grid, stream);
+        case EPI_SWIGLU_AMAX: return launch_one<256, EPI_SWIGLU_AMAX, 2>(map_a, map_a32, map_b, args, grid, stream);
+        default: return launch_one<256, EPI_BF16, 2>(map_a, map_a32, map_b, args, grid, stream);
+        }
     }
+    switch (epi) {
+    case EPI_SWIGLU_QUANT: return launch_one<256, EPI_SWIGLU_QUANT, 1>(map_a, map_a32, map_b, args, grid, stream);
+    case EPI_SWIGLU_AMAX: return launch_one<256, EPI_SWIGLU_AMAX, 1>(map_a, map_a32, map_b, args, grid, stream);
+    default:
+        return bn == 256 ? launch_one<256, EPI_BF16, 1>(map_a, map_a32, map_b, args, grid, stream)
+                         : launch_one<128, EPI_BF16, 1>(map_a, map_a32, map_b, args, grid, stream);
+    }
+}
+
+// Clusters of two GEMM CTAs that can be resident at once on the current
+// device (each CTA needs a whole SM's shared memory), cached per device.
+int gemm_pair_clusters(int num_sms)
+{
+    static int cached_device = -1, cached = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return num_sms / 2;
+    if (dev == cached_device)
+        return cached;
+    const int smem = Cfg<256, 2>::kSmem;
+    int n = 0;
+    if (cudaFuncSetAttribute(nvfp4_gemm_kernel<256, EPI_BF16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+        cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(num_sms));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<256, EPI_BF16, 2>, &cfg) != cudaSuccess)
+            n = 0;
+    }
+    (void)cudaGetLastError();
+    if (n <= 0 || n > num_sms / 2)
+        n = num_sms / 2;
+    cached_device = dev;
+    cached = n;
+    return n;
 }
 
 } // namespace nvfp4

@@ -22,6 +22,8 @@ struct GemmArgs {
     // tile space: grouped (m-tile table written on the device) or dense
     const int32_t *num_mtiles_dev;
     const int4 *mtiles;       // {expert, first padded row, valid rows, first output row}
+    const int32_t *num_pairs_dev;
+    const int2 *pairs;        // pair tiles: {first m-tile, second m-tile of the same expert or -1}
     int dense_m_tiles;
     int dense_M;
     int n_tiles;
@@ -51,12 +53,15 @@ struct GemmArgs {
 enum Epilogue { EPI_SWIGLU_QUANT = 0, EPI_BF16 = 1, EPI_SWIGLU_AMAX = 2 };
 
 // Launches the GEMM engine with 128 x bn tiles (bn 256, or 128 for EPI_BF16
-// when N is not a multiple of 256).  map_a / map_a32: 2-D uint8 tensor maps
-// over the A code matrix with boxes of 128 and 32 rows; map_b: over the B
-// code matrix with 128-row boxes; every box is 128 bytes wide with 128-byte
-// swizzle.
-cudaError_t launch_gemm(int bn, int epi, const CUtensorMap &map_a, const CUtensorMap &map_a32,
+// when N is not a multiple of 256), or with cg = 2 as clusters of two CTAs
+// computing 256 x 256 tiles with pair MMAs (bn 256, grid even).  map_a /
+// map_a32: 2-D uint8 tensor maps over the A code matrix with boxes of 128 and
+// 32 rows; map_b: over the B code matrix with 128-row boxes; every box is 128
+// bytes wide with 128-byte swizzle.
+cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
                         const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream);
+// Pair clusters that fit on the device at once (<= num_sms / 2).
+int gemm_pair_clusters(int num_sms);
 
 // Memory-bound kernels (kernels.cu).
 cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s);
@@ -67,7 +72,8 @@ cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, 
 cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64_t cols, uint8_t *out,
                            cudaStream_t s);
 cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
-                         int32_t *num_mtiles, int4 *mtiles, int32_t *inv, int32_t *err, cudaStream_t s);
+                         int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *inv,
+                         int32_t *err, cudaStream_t s);
 cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int32_t *ids, const float *w,
                            const int32_t *off, const int32_t *poff, int64_t T, int k, int64_t H,
                            __nv_bfloat16 *out, cudaStream_t s);

@@ -209,8 +209,10 @@ cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64
 //  1. per-warp histograms in shared memory;
 //  2. per expert: exclusive prefix over warps (so warp w starts after all
 //     earlier warps' slots of that expert) and the total count;
-//  3. exclusive scans over experts of the counts and of the 128-row m-tile
-//     counts -> unpadded offsets, padded offsets, the m-tile table;
+//  3. exclusive scans over experts of the counts, of the 128-row m-tile
+//     counts and of the m-tile pair counts -> unpadded offsets, padded
+//     offsets, the m-tile table and the pair table (consecutive m-tiles of
+//     one expert; the last of an odd count pairs with -1);
 //  4. each warp walks its range in order; lanes with equal ids find each
 //     other with match_any, so a slot's rank is the number of earlier slots
 //     of its expert: position = padded_offset[e] + rank (a stable counting
@@ -218,13 +220,14 @@ cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64
 __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__ ids, int R, int E,
                                                      int32_t *__restrict__ counts, int32_t *__restrict__ off,
                                                      int32_t *__restrict__ poff, int32_t *__restrict__ num_mtiles,
-                                                     int4 *__restrict__ mtiles, int32_t *__restrict__ inv,
+                                                     int4 *__restrict__ mtiles, int32_t *__restrict__ num_pairs,
+                                                     int2 *__restrict__ pairs, int32_t *__restrict__ inv,
                                                      int32_t *__restrict__ err)
 {
     extern __shared__ int32_t sm[];
     int32_t *wcnt = sm;                // [32][E]
     int32_t *poff_s = sm + 32 * E;     // [E]
-    __shared__ int32_t warp_sum_c[32], warp_sum_t[32];
+    __shared__ int32_t warp_sum_c[32], warp_sum_t[32], warp_sum_p[32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     for (int i = tid; i < 32 * E; i += blockDim.x)
@@ -246,7 +249,7 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
     __syncthreads();
 
     // 2 + 3: thread e owns expert e (E <= 1024)
-    int cnt = 0, tiles = 0;
+    int cnt = 0, tiles = 0, npair = 0;
     if (tid < E) {
         for (int w = 0; w < 32; ++w) {
             const int c = wcnt[w * E + tid];
@@ -254,40 +257,48 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
             cnt += c;
         }
         tiles = (cnt + 127) / 128;
+        npair = (tiles + 1) / 2;
     }
-    // block-wide exclusive scan of (cnt, tiles) over thread index
-    int ic = cnt, it = tiles;
+    // block-wide exclusive scan of (cnt, tiles, npair) over thread index
+    int ic = cnt, it = tiles, ip = npair;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int a = __shfl_up_sync(0xffffffffu, ic, o);
         const int b = __shfl_up_sync(0xffffffffu, it, o);
+        const int c = __shfl_up_sync(0xffffffffu, ip, o);
         if (lane >= o) {
             ic += a;
             it += b;
+            ip += c;
         }
     }
     if (lane == 31) {
         warp_sum_c[warp] = ic;
         warp_sum_t[warp] = it;
+        warp_sum_p[warp] = ip;
     }
     __syncthreads();
     if (warp == 0) {
-        int c = warp_sum_c[lane], t = warp_sum_t[lane];
+        int c = warp_sum_c[lane], t = warp_sum_t[lane], q = warp_sum_p[lane];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int a = __shfl_up_sync(0xffffffffu, c, o);
             const int b = __shfl_up_sync(0xffffffffu, t, o);
+            const int d = __shfl_up_sync(0xffffffffu, q, o);
             if (lane >= o) {
                 c += a;
                 t += b;
+                q += d;
             }
         }
         warp_sum_c[lane] = c;   // inclusive over warps
         warp_sum_t[lane] = t;
+        warp_sum_p[lane] = q;
     }
     __syncthreads();
     const int base_c = (warp > 0 ? warp_sum_c[warp - 1] : 0) + ic - cnt;   // exclusive
     const int base_t = (warp > 0 ? warp_sum_t[warp - 1] : 0) + it - tiles;
+    const int base_p = (warp > 0 ? warp_sum_p[warp - 1] : 0) + ip - npair;
     if (tid < E) {
         counts[tid] = cnt;
         off[tid] = base_c;
@@ -295,10 +306,13 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
         poff_s[tid] = base_t * 128;
         for (int i = 0; i < tiles; ++i)
             mtiles[base_t + i] = make_int4(tid, base_t * 128 + 128 * i, min(128, cnt - 128 * i), base_c + 128 * i);
+        for (int i = 0; i < npair; ++i)
+            pairs[base_p + i] = make_int2(base_t + 2 * i, 2 * i + 1 < tiles ? base_t + 2 * i + 1 : -1);
         if (tid == E - 1) {
             off[E] = base_c + cnt;
             poff[E] = (base_t + tiles) * 128;
             *num_mtiles = base_t + tiles;
+            *num_pairs = base_p + npair;
         }
     }
     __syncthreads();
@@ -324,7 +338,8 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
 }
 
 cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
-                         int32_t *num_mtiles, int4 *mtiles, int32_t *inv, int32_t *err, cudaStream_t s)
+                         int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *inv,
+                         int32_t *err, cudaStream_t s)
 {
     const size_t smem = sizeof(int32_t) * (33 * static_cast<size_t>(E));
     static bool attr_set = false;
@@ -334,7 +349,8 @@ cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, 
             return e;
         attr_set = true;
     }
-    route_kernel<<<1, 1024, smem, s>>>(ids, static_cast<int>(R), E, counts, off, poff, num_mtiles, mtiles, inv, err);
+    route_kernel<<<1, 1024, smem, s>>>(ids, static_cast<int>(R), E, counts, off, poff, num_mtiles, mtiles, num_pairs,
+                                       pairs, inv, err);
     return cudaGetLastError();
 }
 

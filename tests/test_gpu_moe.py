@@ -291,3 +291,25 @@ def test_forward_timed_matches_forward_eager_and_in_graph(tiny):
         assert torch.equal(out, ref)
         times = [ev[0].elapsed_time(e) for e in ev]
         assert all(b >= a for a, b in zip(times, times[1:])) and times[-1] > 0
+
+
+# 12 experts, top-3, 1024 tokens: 256 routed rows per expert on average (two
+# full m-tiles), so the grouped GEMMs run as pair tiles (clusters of two CTAs
+# on 256-row tiles).
+PAIRS = W.MoeConfig("pairs", E=12, k=3, T=1024, H=512, I=256, routing="zipf", outliers=True, warmup_T=256,
+                    zipf_zero_tail=2)
+
+
+def test_pair_tiles_end_to_end():
+    """Pair tiles: experts with an odd number of 128-row m-tiles (the second
+    CTA of the last pair has no rows), with one m-tile, with several, and
+    empty experts; the whole output against the oracle."""
+    p = Problem(PAIRS)
+    counts = np.bincount(p.ids.numpy().ravel(), minlength=PAIRS.E)
+    mt = (counts + 127) // 128
+    assert (mt % 2 == 1).any() and (mt >= 4).any() and (counts == 0).any()
+    assert PAIRS.T * PAIRS.k >= 256 * PAIRS.E
+    check_weights_bitexact(p, range(PAIRS.E))
+    out, ws = p.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    check_output(out, p.oracle())
