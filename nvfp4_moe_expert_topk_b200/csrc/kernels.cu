@@ -457,12 +457,12 @@ cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float
 }
 
 // ------------------------------------------------------------ top-k router
-// One warp per token.  Every logit becomes a 64-bit key whose high word is
-// its fp32 value mapped to an unsigned integer of the same order (-0 folded
-// into +0) and whose low word is ~expert, so a larger key is a larger logit
-// and, between equal logits, the lower expert.  Lane l holds experts
-// l, l + 32, ...; k rounds of a warp max pick the winners in descending
-// order, each round retiring the winner's key to 0 (below every real key).
+// One warp per token.  Every logit becomes a 32-bit key, its fp32 value
+// mapped to an unsigned integer of the same order (-0 folded into +0); lane l
+// holds experts l, l + 32, ... and keeps its largest key and, among equal
+// keys, its lowest expert.  Each of the k rounds takes two warp reductions
+// (redux.sync): the largest key, then the lowest expert holding it; the
+// owning lane retires that key (to 0, below every real key) and rescans.
 constexpr int kTopkWarps = 8;
 
 __device__ __forceinline__ uint32_t order_bits(float x)
@@ -486,36 +486,43 @@ __global__ void __launch_bounds__(32 * kTopkWarps) topk_kernel(const float *__re
     if (t >= T)
         return;   // whole warp leaves together
     const float *row = logits + t * E;
-    unsigned long long key[P];
+    uint32_t key[P];
 #pragma unroll
     for (int i = 0; i < P; i++) {
         const int e = lane + 32 * i;
-        key[i] = e < E ? (static_cast<unsigned long long>(order_bits(__ldg(row + e))) << 32) | (~static_cast<uint32_t>(e))
-                       : 0ull;
+        key[i] = e < E ? order_bits(__ldg(row + e)) : 0u;
     }
-    unsigned long long best = 0;
+    // this lane's best key and the lowest i holding it
+    uint32_t best = 0;
+    int best_i = 0;
 #pragma unroll
     for (int i = 0; i < P; i++)
-        best = key[i] > best ? key[i] : best;
+        if (key[i] > best) {
+            best = key[i];
+            best_i = i;
+        }
+    uint32_t alive = P >= 32 ? 0xffffffffu : (1u << P) - 1u;   // bit i: key[i] not yet taken
     float mine = 0.0f;   // lane j < k: logit of the j-th winner
     int mine_id = 0;
     for (int j = 0; j < k; j++) {
-        unsigned long long m = best;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xffffffffu, m, o);
-            m = other > m ? other : m;
-        }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, best);
+        const uint32_t cand = best == m ? static_cast<uint32_t>(lane + 32 * best_i) : 0xffffffffu;
+        const uint32_t w = __reduce_min_sync(0xffffffffu, cand);
         if (lane == j) {
-            mine = from_order_bits(static_cast<uint32_t>(m >> 32));
-            mine_id = static_cast<int>(~static_cast<uint32_t>(m));
+            mine = from_order_bits(m);
+            mine_id = static_cast<int>(w);
         }
-        if (best == m) {   // this lane owned the winner: retire it
+        if (lane == static_cast<int>(w & 31u)) {   // the winner was this lane's best: retire it, rescan
+            alive &= ~(1u << best_i);
             best = 0;
+            best_i = 0;
 #pragma unroll
             for (int i = 0; i < P; i++) {
-                key[i] = key[i] == m ? 0ull : key[i];
-                best = key[i] > best ? key[i] : best;
+                const uint32_t kv = ((alive >> i) & 1u) ? key[i] : 0u;
+                if (kv > best) {
+                    best = kv;
+                    best_i = i;
+                }
             }
         }
     }
