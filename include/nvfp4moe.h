@@ -196,6 +196,15 @@ int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, in
 #define NVFP4_NOALLOC_SCRATCH_BYTES (32u << 20)
 int nvfp4_moe_forward_noalloc(const nvfp4_moe_args *args, void *stream);
 
+/* Execution plan nvfp4_moe_forward uses for a shape (host only, no GPU
+ * work): *fused_l1_l2 = 1 when L1 and L2 run as one persistent launch (the
+ * L2 tiles of an m-tile start as soon as that m-tile's L1 tiles have written
+ * h; per-stage timing then reports L1 + L2 as one stage, between events 2
+ * and 3 of nvfp4_moe_forward_timed, and an empty stage between 3 and 4);
+ * *pair_tiles = 1 when the grouped GEMMs run on 256-row tiles computed by
+ * clusters of two CTAs.  Both are host outputs. */
+int nvfp4_moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int32_t *fused_l1_l2, int32_t *pair_tiles);
+
 /* Reads and clears the sticky device error word of a workspace (host
  * err_host receives NVFP4_OK or a device error code).  Synchronises
  * `stream`. */

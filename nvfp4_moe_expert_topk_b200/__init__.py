@@ -18,7 +18,7 @@ __all__ = [
     "nvfp4_swizzle_scales", "nvfp4_gemm", "nvfp4_moe_workspace_size", "nvfp4_moe_forward",
     "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
-    "nvfp4_moe_get_error", "nvfp4_moe_topk", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling",
+    "nvfp4_moe_get_error", "nvfp4_moe_topk", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan",
     "MoeArgs",
 ]
 
@@ -77,6 +77,8 @@ def lib():
         L.nvfp4_moe_get_error.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.nvfp4_moe_topk.argtypes = [P, i64, i32, i32, i32, P, P, P]
         L.nvfp4_fp4_mma_ceiling.argtypes = [i32, i32, i32, P, P, P]
+        L.nvfp4_moe_plan.argtypes = [i64, i32, i32, i64, i64, ctypes.POINTER(ctypes.c_int32),
+                                     ctypes.POINTER(ctypes.c_int32)]
         _lib = L
     return _lib
 
@@ -257,3 +259,10 @@ def nvfp4_fp4_mma_ceiling(bn, iters, cycles, err=None, stream=None):
     _check(lib().nvfp4_fp4_mma_ceiling(bn, iters, cycles.numel(), _dev(cycles, "cycles", torch.int64),
                                        None if err is None else _dev(err, "err", torch.int32), _stream(stream)),
            "nvfp4_fp4_mma_ceiling")
+
+
+def nvfp4_moe_plan(T, k, E, H, I):
+    """(fused_l1_l2, pair_tiles) booleans of the forward's execution plan."""
+    f, pt = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().nvfp4_moe_plan(T, k, E, H, I, ctypes.byref(f), ctypes.byref(pt)), "nvfp4_moe_plan")
+    return bool(f.value), bool(pt.value)

@@ -89,7 +89,7 @@ int64_t round_up(int64_t v, int64_t m)
 // ---------------------------------------------------------------- workspace
 struct Layout {
     int64_t mt_max = 0, rpad = 0;
-    int64_t counts = 0, off = 0, poff = 0, mtiles = 0, pairs = 0, inv = 0, amax = 0;
+    int64_t counts = 0, off = 0, poff = 0, mtiles = 0, pairs = 0, ready = 0, inv = 0, amax = 0;
     int64_t a_codes = 0, a_sf = 0, h_codes = 0, h_sf = 0, y = 0, total = 0;
 };
 
@@ -114,6 +114,7 @@ Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
     L.amax = take(4 * E);
     L.mtiles = take(16 * std::max<int64_t>(L.mt_max, 1));
     L.pairs = take(8 * std::max<int64_t>(L.mt_max, 1));
+    L.ready = take(4 * std::max<int64_t>(L.mt_max, 1));
     L.inv = take(4 * std::max<int64_t>(R, 1));
     L.a_codes = take(L.rpad * (H / 2));
     L.a_sf = take(L.rpad * (H / 16));
@@ -193,68 +194,128 @@ int gemm_grid(int cg, int64_t tiles, int num_sms)
     return static_cast<int>(std::min<int64_t>(std::max<int64_t>(tiles, 1), num_sms));
 }
 
-int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int l1_epi, void *const *events,
-              cudaStream_t s, int num_sms)
+// Maps and arguments of the grouped L1 GEMM (gate_up, SwiGLU epilogue).
+int l1_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, CUtensorMap *ma, CUtensorMap *ma32,
+             CUtensorMap *mb, GemmArgs *g)
 {
-    const int64_t T = a->T, H = a->H, I = a->I, R = T * a->k;
-    const int E = a->E, k = a->k;
-    int32_t *err = reinterpret_cast<int32_t *>(ws);
-    int32_t *num_mt = reinterpret_cast<int32_t *>(ws + 4);
-    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
-    int32_t *off = reinterpret_cast<int32_t *>(ws + L.off);
-    int32_t *poff = reinterpret_cast<int32_t *>(ws + L.poff);
-    int4 *mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
-    int32_t *num_pairs = reinterpret_cast<int32_t *>(ws + 8);
-    int2 *pairs = reinterpret_cast<int2 *>(ws + L.pairs);
-    int32_t *inv = reinterpret_cast<int32_t *>(ws + L.inv);
+    const int64_t H = a->H, I = a->I;
+    const int E = a->E;
+    int st = make_code_map(ma, ws + L.a_codes, L.rpad, H / 2, 128);
+    if (st == NVFP4_OK)
+        st = make_code_map(ma32, ws + L.a_codes, L.rpad, H / 2, 32);
+    if (st == NVFP4_OK)
+        st = make_code_map(mb, a->w13_codes, static_cast<int64_t>(E) * 2 * I, H / 2, 128);
+    if (st != NVFP4_OK)
+        return st;
+    *g = GemmArgs{};
+    g->sfa = ws + L.a_sf;
+    g->sfa_block_stride = (H / 64) * 512;
+    g->sfb = a->w13_scales;
+    g->sfb_block_stride = (H / 64) * 512;
+    g->K = static_cast<int>(H);
+    g->num_k_tiles = static_cast<int>((H + 255) / 256);
+    g->num_mtiles_dev = reinterpret_cast<int32_t *>(ws + 4);
+    g->mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
+    g->num_pairs_dev = reinterpret_cast<int32_t *>(ws + 8);
+    g->pairs = reinterpret_cast<int2 *>(ws + L.pairs);
+    g->ready = reinterpret_cast<int32_t *>(ws + L.ready);
+    g->n_tiles = static_cast<int>(I / 128);
+    g->b_rows_per_expert = 2 * I;
+    g->b_tile_rows = 128;
+    g->b_half_offset = static_cast<int>(I);
+    g->a_gs = a->x_gs;
+    g->a_gs_per_expert = 0;
+    g->b_gs = a->w13_gs;
+    g->b_gs_stride = 2;
+    g->nseg = 1;
+    g->inter_gs = a->inter_gs;
+    g->h_codes = ws + L.h_codes;
+    g->h_ld_bytes = I / 2;
+    g->h_sf = ws + L.h_sf;
+    g->h_sf_block_stride = (I / 64) * 512;
+    g->amax_bits = reinterpret_cast<unsigned int *>(ws + L.amax);
+    g->err = reinterpret_cast<int32_t *>(ws);
+    return NVFP4_OK;
+}
 
+// Maps and arguments of the grouped L2 GEMM (down, bf16 epilogue into y).
+int l2_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int bn, CUtensorMap *ma, CUtensorMap *ma32,
+             CUtensorMap *mb, GemmArgs *g)
+{
+    const int64_t H = a->H, I = a->I;
+    const int E = a->E;
+    int st = make_code_map(ma, ws + L.h_codes, L.rpad, I / 2, 128);
+    if (st == NVFP4_OK)
+        st = make_code_map(ma32, ws + L.h_codes, L.rpad, I / 2, 32);
+    if (st == NVFP4_OK)
+        st = make_code_map(mb, a->w2_codes, static_cast<int64_t>(E) * H, I / 2, 128);
+    if (st != NVFP4_OK)
+        return st;
+    *g = GemmArgs{};
+    g->sfa = ws + L.h_sf;
+    g->sfa_block_stride = (I / 64) * 512;
+    g->sfb = a->w2_scales;
+    g->sfb_block_stride = (I / 64) * 512;
+    g->K = static_cast<int>(I);
+    g->num_k_tiles = static_cast<int>((I + 255) / 256);
+    g->num_mtiles_dev = reinterpret_cast<int32_t *>(ws + 4);
+    g->mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
+    g->num_pairs_dev = reinterpret_cast<int32_t *>(ws + 8);
+    g->pairs = reinterpret_cast<int2 *>(ws + L.pairs);
+    g->ready = reinterpret_cast<int32_t *>(ws + L.ready);
+    g->n_tiles = static_cast<int>(H / bn);
+    g->b_rows_per_expert = H;
+    g->b_tile_rows = bn;
+    g->b_half_offset = 128;
+    g->a_gs = a->inter_gs;
+    g->a_gs_per_expert = 1;
+    g->b_gs = a->w2_gs;
+    g->b_gs_stride = 1;
+    g->nseg = 1;
+    g->seg_end[0] = static_cast<int>(H);
+    g->out = reinterpret_cast<__nv_bfloat16 *>(ws + L.y);
+    g->ldo = H;
+    g->err = reinterpret_cast<int32_t *>(ws);
+    return NVFP4_OK;
+}
+
+// Routing + quantise/permute (events 0-2 when timing).  Shared by forward and calibrate.
+int run_route_quant(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, void *const *events, cudaStream_t s)
+{
+    const int64_t T = a->T, H = a->H, R = T * a->k;
+    const int E = a->E, k = a->k;
+    int32_t *inv = reinterpret_cast<int32_t *>(ws + L.inv);
     if (mark(events, 0, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
-    cudaError_t e = launch_route(a->topk_ids, R, E, counts, off, poff, num_mt, mtiles, num_pairs, pairs, inv, err, s);
+    cudaError_t e = launch_route(a->topk_ids, R, E, reinterpret_cast<int32_t *>(ws + L.counts),
+                                 reinterpret_cast<int32_t *>(ws + L.off), reinterpret_cast<int32_t *>(ws + L.poff),
+                                 reinterpret_cast<int32_t *>(ws + 4), reinterpret_cast<int4 *>(ws + L.mtiles),
+                                 reinterpret_cast<int32_t *>(ws + 8), reinterpret_cast<int2 *>(ws + L.pairs),
+                                 reinterpret_cast<int32_t *>(ws + L.ready), inv, reinterpret_cast<int32_t *>(ws), s);
     if (e != cudaSuccess || mark(events, 1, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
     e = launch_quantize(reinterpret_cast<const __nv_bfloat16 *>(a->x), T, H, H, a->x_gs, ws + L.a_codes,
                         ws + L.a_sf, NVFP4_SCALES_MMA, inv, k, s);
     if (e != cudaSuccess || mark(events, 2, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
+    return NVFP4_OK;
+}
 
-    CUtensorMap ma, ma32, mb;
-    int st = make_code_map(&ma, ws + L.a_codes, L.rpad, H / 2, 128);
-    if (st == NVFP4_OK)
-        st = make_code_map(&ma32, ws + L.a_codes, L.rpad, H / 2, 32);
-    if (st == NVFP4_OK)
-        st = make_code_map(&mb, a->w13_codes, static_cast<int64_t>(E) * 2 * I, H / 2, 128);
-    if (st != NVFP4_OK)
-        return st;
-    GemmArgs g{};
-    g.sfa = ws + L.a_sf;
-    g.sfa_block_stride = (H / 64) * 512;
-    g.sfb = a->w13_scales;
-    g.sfb_block_stride = (H / 64) * 512;
-    g.K = static_cast<int>(H);
-    g.num_k_tiles = static_cast<int>((H + 255) / 256);
-    g.num_mtiles_dev = num_mt;
-    g.mtiles = mtiles;
-    g.num_pairs_dev = num_pairs;
-    g.pairs = pairs;
-    g.n_tiles = static_cast<int>(I / 128);
-    g.b_rows_per_expert = 2 * I;
-    g.b_tile_rows = 128;
-    g.b_half_offset = static_cast<int>(I);
-    g.a_gs = a->x_gs;
-    g.a_gs_per_expert = 0;
-    g.b_gs = a->w13_gs;
-    g.b_gs_stride = 2;
-    g.nseg = 1;
-    g.inter_gs = a->inter_gs;
-    g.h_codes = ws + L.h_codes;
-    g.h_ld_bytes = I / 2;
-    g.h_sf = ws + L.h_sf;
-    g.h_sf_block_stride = (I / 64) * 512;
-    g.amax_bits = reinterpret_cast<unsigned int *>(ws + L.amax);
-    g.err = err;
-    const int cg = moe_cg(R, E);
-    return cuda_status(launch_gemm(256, l1_epi, cg, ma, ma32, mb, g, gemm_grid(cg, 1LL << 30, num_sms), s));
+// The forward's execution plan: pair tiles for the grouped GEMMs, and
+// whether L1 and L2 run as one fused launch (1-CTA tiles, 256-wide L2 tiles).
+struct Plan {
+    int cg;
+    int l2_bn;
+    bool fused;
+};
+
+Plan moe_plan(int64_t T, int k, int E, int64_t H)
+{
+    Plan pl;
+    pl.cg = moe_cg(T * k, E);
+    pl.l2_bn = (H % 256 == 0) ? 256 : 128;
+    pl.fused = pl.cg == 1 && pl.l2_bn == 256;
+    return pl;
 }
 
 } // namespace
@@ -462,50 +523,33 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
         return NVFP4_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    st = run_front(a, ws, L, EPI_SWIGLU_QUANT, events, s, sms);
+    st = run_route_quant(a, ws, L, events, s);
     if (st != NVFP4_OK)
         return st;
-
-    const int64_t H = a->H, I = a->I;
-    const int E = a->E;
-    CUtensorMap ma2, ma2_32, mb2;
-    st = make_code_map(&ma2, ws + L.h_codes, L.rpad, I / 2, 128);
+    const Plan pl = moe_plan(a->T, a->k, a->E, a->H);
+    const int64_t H = a->H;
+    CUtensorMap ma1, ma1_32, mb1, ma2, ma2_32, mb2;
+    GemmArgs g1, g2;
+    st = l1_setup(a, ws, L, &ma1, &ma1_32, &mb1, &g1);
     if (st == NVFP4_OK)
-        st = make_code_map(&ma2_32, ws + L.h_codes, L.rpad, I / 2, 32);
-    if (st == NVFP4_OK)
-        st = make_code_map(&mb2, a->w2_codes, static_cast<int64_t>(E) * H, I / 2, 128);
+        st = l2_setup(a, ws, L, pl.l2_bn, &ma2, &ma2_32, &mb2, &g2);
     if (st != NVFP4_OK)
         return st;
-    const int bn = (H % 256 == 0) ? 256 : 128;
-    GemmArgs g{};
-    g.sfa = ws + L.h_sf;
-    g.sfa_block_stride = (I / 64) * 512;
-    g.sfb = a->w2_scales;
-    g.sfb_block_stride = (I / 64) * 512;
-    g.K = static_cast<int>(I);
-    g.num_k_tiles = static_cast<int>((I + 255) / 256);
-    g.num_mtiles_dev = reinterpret_cast<int32_t *>(ws + 4);
-    g.mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
-    g.num_pairs_dev = reinterpret_cast<int32_t *>(ws + 8);
-    g.pairs = reinterpret_cast<int2 *>(ws + L.pairs);
-    g.n_tiles = static_cast<int>(H / bn);
-    g.b_rows_per_expert = H;
-    g.b_tile_rows = bn;
-    g.b_half_offset = 128;
-    g.a_gs = a->inter_gs;
-    g.a_gs_per_expert = 1;
-    g.b_gs = a->w2_gs;
-    g.b_gs_stride = 1;
-    g.nseg = 1;
-    g.seg_end[0] = static_cast<int>(H);
-    g.out = reinterpret_cast<__nv_bfloat16 *>(ws + L.y);
-    g.ldo = H;
-    g.err = reinterpret_cast<int32_t *>(ws);
-    const int cg = bn == 256 ? moe_cg(a->T * a->k, E) : 1;
-    if (mark(events, 3, s) != NVFP4_OK ||
-        launch_gemm(bn, EPI_BF16, cg, ma2, ma2_32, mb2, g, gemm_grid(cg, 1LL << 30, sms), s) != cudaSuccess ||
-        mark(events, 4, s) != NVFP4_OK)
-        return NVFP4_ERR_CUDA;
+    if (pl.fused) {
+        // L1 and L2 in one launch: no stage boundary between events 3 and 4
+        if (launch_moe_fused(ma1, ma1_32, mb1, g1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
+            mark(events, 3, s) != NVFP4_OK || mark(events, 4, s) != NVFP4_OK)
+            return NVFP4_ERR_CUDA;
+    } else {
+        const int l2_cg = pl.l2_bn == 256 ? pl.cg : 1;
+        if (launch_gemm(256, EPI_SWIGLU_QUANT, pl.cg, ma1, ma1_32, mb1, g1, gemm_grid(pl.cg, 1LL << 30, sms), s) !=
+                cudaSuccess ||
+            mark(events, 3, s) != NVFP4_OK ||
+            launch_gemm(pl.l2_bn, EPI_BF16, l2_cg, ma2, ma2_32, mb2, g2, gemm_grid(l2_cg, 1LL << 30, sms), s) !=
+                cudaSuccess ||
+            mark(events, 4, s) != NVFP4_OK)
+            return NVFP4_ERR_CUDA;
+    }
 
     if (launch_combine(reinterpret_cast<const __nv_bfloat16 *>(ws + L.y),
                        reinterpret_cast<const int32_t *>(ws + L.inv), a->topk_ids, a->topk_weights,
@@ -513,6 +557,19 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
                        a->T, a->k, H, reinterpret_cast<__nv_bfloat16 *>(a->out), s) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return mark(events, 5, s);
+}
+
+int nvfp4_moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int32_t *fused_l1_l2, int32_t *pair_tiles)
+{
+    if (fused_l1_l2 == nullptr || pair_tiles == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    const int st = check_moe_shape(T, k, E, H, I);
+    if (st != NVFP4_OK)
+        return st;
+    const Plan pl = moe_plan(T, k, E, H);
+    *fused_l1_l2 = pl.fused ? 1 : 0;
+    *pair_tiles = pl.cg == 2 ? 1 : 0;
+    return NVFP4_OK;
 }
 
 int nvfp4_moe_forward(const nvfp4_moe_args *a, void *workspace, size_t ws_bytes, void *stream)
@@ -552,9 +609,17 @@ int nvfp4_moe_calibrate(const nvfp4_moe_args *a, float *inter_gs_out, void *work
     if (cudaMemsetAsync(ws + L.amax, 0, 4 * static_cast<size_t>(a->E), s) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     if (a->T > 0) {
-        st = run_front(a, ws, L, EPI_SWIGLU_AMAX, nullptr, s, sms);
+        st = run_route_quant(a, ws, L, nullptr, s);
         if (st != NVFP4_OK)
             return st;
+        CUtensorMap ma, ma32, mb;
+        GemmArgs g;
+        st = l1_setup(a, ws, L, &ma, &ma32, &mb, &g);
+        if (st != NVFP4_OK)
+            return st;
+        const int cg = moe_cg(a->T * a->k, a->E);
+        if (launch_gemm(256, EPI_SWIGLU_AMAX, cg, ma, ma32, mb, g, gemm_grid(cg, 1LL << 30, sms), s) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
     }
     return cuda_status(
         launch_finalize_inter_gs(reinterpret_cast<const unsigned int *>(ws + L.amax), a->E, inter_gs_out, s));
@@ -580,7 +645,8 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
     return cuda_status(launch_route(topk_ids, T * k, E, counts, reinterpret_cast<int32_t *>(ws + L.off),
                                     padded_offsets, reinterpret_cast<int32_t *>(ws + 4),
                                     reinterpret_cast<int4 *>(ws + L.mtiles), reinterpret_cast<int32_t *>(ws + 8),
-                                    reinterpret_cast<int2 *>(ws + L.pairs), inv, reinterpret_cast<int32_t *>(ws),
+                                    reinterpret_cast<int2 *>(ws + L.pairs), reinterpret_cast<int32_t *>(ws + L.ready),
+                                    inv, reinterpret_cast<int32_t *>(ws),
                                     static_cast<cudaStream_t>(stream)));
 }
 

@@ -90,16 +90,37 @@ struct Cfg {
 
 struct TileInfo {
     int e, row0, valid, row0_out, nt;
+    int mt;     // m-tile index in the grouped table
+    int ph;     // fused launch: 0 = L1 tile, 1 = L2 tile
 };
 
 // Tile t of the launch's tile space, as seen by CTA `rank` of its cluster.
 // CG = 1: m-tiles of 128 rows.  CG = 2: m-pairs; the even CTA takes the
 // pair's first m-tile and the odd CTA the second (valid = 0 when the expert
-// or matrix has no rows left for it).
-template <int CG>
-__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, int t, int m_units, uint32_t rank)
+// or matrix has no rows left for it).  FUSED: the L1 tiles of every m-tile
+// (p.n_tiles per m-tile), then the L2 tiles (p2.n_tiles per m-tile).
+template <int CG, int FUSED>
+__device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, const GemmArgs &p2, int t, int m_units,
+                                                uint32_t rank)
 {
     TileInfo ti;
+    ti.ph = 0;
+    ti.mt = 0;
+    if constexpr (FUSED) {
+        const int t1 = m_units * p.n_tiles;
+        ti.ph = t >= t1 ? 1 : 0;
+        const int n = ti.ph ? p2.n_tiles : p.n_tiles;
+        const int tt = ti.ph ? t - t1 : t;
+        const int mt = tt / n;
+        ti.nt = tt - mt * n;
+        ti.mt = mt;
+        const int4 m = p.mtiles[mt];
+        ti.e = m.x;
+        ti.row0 = m.y;
+        ti.valid = m.z;
+        ti.row0_out = m.w;
+        return ti;
+    }
     if constexpr (CG == 2) {
         if (p.mtiles != nullptr) {
             const int mp = t / p.n_tiles;
@@ -125,6 +146,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, int t, int m_
     if (p.mtiles != nullptr) {
         const int mt = t / p.n_tiles;
         ti.nt = t - mt * p.n_tiles;
+        ti.mt = mt;
         const int4 m = p.mtiles[mt];
         ti.e = m.x;
         ti.row0 = m.y;
@@ -161,12 +183,42 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int BN, int EPI, int CG>
+// Bounded wait (2 s) until the 32-bit counter reaches `target`; acquire at
+// GPU scope, then order this thread's later async-proxy reads (TMA) after it.
+__device__ __forceinline__ bool wait_counter(const int32_t *ctr, int target, volatile int *abort)
+{
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 0; i < kWaitLimitSpins; ++i) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+        if (v >= target) {
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            return true;
+        }
+        if ((i & 15u) == 15u && (*abort || global_timer_ns() - t0 > kWaitLimitNs))
+            return false;
+        __nanosleep(64);
+    }
+    return false;
+}
+
+// FUSED = 1 (grouped, CG = 1, BN = 256): one persistent launch runs the L1
+// tiles (arguments p, maps map_a / map_a32 / map_b, SwiGLU + re-quantisation
+// epilogue) and then the L2 tiles (p2, map_a2 / map_a2_32 / map_b2, bf16
+// epilogue).  Each L1 epilogue warp publishes its h rows by bumping the
+// m-tile's counter; the producer starts an L2 tile once all L1 tiles of its
+// m-tile have been published (a bounded wait).  Tiles are taken in order, so
+// every L1 tile a wait depends on belongs to a CTA that reaches it without
+// waiting itself; the launch is cooperative, so all CTAs are resident.
+template <int BN, int EPI, int CG, int FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a32,
-                      const __grid_constant__ CUtensorMap map_b, const GemmArgs p)
+                      const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_a2,
+                      const __grid_constant__ CUtensorMap map_a2_32, const __grid_constant__ CUtensorMap map_b2,
+                      const GemmArgs p, const GemmArgs p2)
 {
     using C = Cfg<BN, CG>;
+    static_assert(!FUSED || (CG == 1 && BN == 256 && EPI == EPI_SWIGLU_QUANT), "fused launch: L1 quant + L2 bf16");
     constexpr int kStages = C::kStages;
     constexpr int kHalves = C::kHalves;
     constexpr int kNumAcc = C::kNumAcc;
@@ -211,6 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&map_a);
         tma_prefetch_map(&map_a32);
         tma_prefetch_map(&map_b);
+        if (FUSED) {
+            tma_prefetch_map(&map_a2);
+            tma_prefetch_map(&map_a2_32);
+            tma_prefetch_map(&map_b2);
+        }
     }
     if (warp == 1) {
         if constexpr (kPair) {
@@ -234,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m_units = (p.mtiles != nullptr)
                             ? *reinterpret_cast<volatile const int32_t *>(kPair ? p.num_pairs_dev : p.num_mtiles_dev)
                             : (kPair ? (p.dense_M + 2 * kBM - 1) / (2 * kBM) : p.dense_m_tiles);
-    const int total = m_units * p.n_tiles;
+    const int total = m_units * (p.n_tiles + (FUSED ? p2.n_tiles : 0));
 
     if (warp == 0) {
         if (lane == 0) {
@@ -243,31 +300,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, pend_mask = 0, pend_par = 0;
             bool ok = true;
             for (int t = unit; t < total && ok; t += units) {
-                const TileInfo ti = decode_tile<CG>(p, t, m_units, rank);
-                const int64_t brow0 = ti.e * p.b_rows_per_expert + static_cast<int64_t>(ti.nt) * p.b_tile_rows;
-                const int64_t brow1 = brow0 + p.b_half_offset;
+                const TileInfo ti = decode_tile<CG, FUSED>(p, p2, t, m_units, rank);
+                const GemmArgs &q = (FUSED && ti.ph) ? p2 : p;
+                const CUtensorMap *ma = (FUSED && ti.ph) ? &map_a2 : &map_a;
+                const CUtensorMap *ma32 = (FUSED && ti.ph) ? &map_a2_32 : &map_a32;
+                const CUtensorMap *mb = (FUSED && ti.ph) ? &map_b2 : &map_b;
+                if (FUSED && ti.ph && !wait_counter(p2.ready + ti.mt, p.n_tiles * kEpiWarps, abort_flag)) {
+                    ok = false;     // this m-tile's h never got published
+                    break;
+                }
+                const int64_t brow0 = ti.e * q.b_rows_per_expert + static_cast<int64_t>(ti.nt) * q.b_tile_rows;
+                const int64_t brow1 = brow0 + q.b_half_offset;
                 // A: nothing for an empty pair half, else one 128-row box or the valid 32-row boxes
                 const int a_boxes = ti.valid >= kBM ? 0 : (ti.valid + 31) / 32;
                 const uint32_t a_bytes = ti.valid == 0 ? 0u : (a_boxes == 0 ? kTileBytes : a_boxes * (kTileBytes / 4));
-                const uint8_t *sfa = p.sfa + static_cast<int64_t>(ti.row0 / kBM) * p.sfa_block_stride;
-                const uint8_t *sfb0 = p.sfb + (brow0 / 128) * p.sfb_block_stride;
-                const uint8_t *sfb1 = p.sfb + (brow1 / 128) * p.sfb_block_stride;
-                for (int kt = 0; kt < p.num_k_tiles; ++kt) {
+                const uint8_t *sfa = q.sfa + static_cast<int64_t>(ti.row0 / kBM) * q.sfa_block_stride;
+                const uint8_t *sfb0 = q.sfb + (brow0 / 128) * q.sfb_block_stride;
+                const uint8_t *sfb1 = q.sfb + (brow1 / 128) * q.sfb_block_stride;
+                for (int kt = 0; kt < q.num_k_tiles; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const int nkb = min(4, (p.K - kt * kBK) / 64);
+                    const int nkb = min(4, (q.K - kt * kBK) / 64);
                     const uint32_t sf_bytes = static_cast<uint32_t>(nkb * kSFAtom);
                     mbar_arrive_expect_tx(&full[stage], a_bytes + C::kBBoxes * kTileBytes +
                                                             sf_bytes * (kHalves + (ti.valid > 0 ? 1 : 0)));
                     uint8_t *a_dst = sA + stage * kTileBytes;
                     if (ti.valid > 0) {
                         if (a_boxes == 0) {
-                            tma_load_2d(a_dst, &map_a, kt * kBKBytes, ti.row0, &full[stage]);
+                            tma_load_2d(a_dst, ma, kt * kBKBytes, ti.row0, &full[stage]);
                         } else {
                             for (int i = 0; i < a_boxes; ++i)
-                                tma_load_2d(a_dst + i * (kTileBytes / 4), &map_a32, kt * kBKBytes, ti.row0 + 32 * i,
+                                tma_load_2d(a_dst + i * (kTileBytes / 4), ma32, kt * kBKBytes, ti.row0 + 32 * i,
                                             &full[stage]);
                         }
                         bulk_load(sSFA + stage * kSFStage, sfa + kt * kSFStage, sf_bytes, &full[stage]);
@@ -276,12 +341,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *sfb_dst = sSFB + stage * kHalves * kSFStage;
                     if constexpr (kPair) {
                         // this CTA's half of the B rows; the scales of both halves
-                        tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(rank == 0 ? brow0 : brow1),
+                        tma_load_2d(b_dst, mb, kt * kBKBytes, static_cast<int32_t>(rank == 0 ? brow0 : brow1),
                                     &full[stage]);
                     } else {
-                        tma_load_2d(b_dst, &map_b, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
+                        tma_load_2d(b_dst, mb, kt * kBKBytes, static_cast<int32_t>(brow0), &full[stage]);
                         if constexpr (kHalves == 2)
-                            tma_load_2d(b_dst + kTileBytes, &map_b, kt * kBKBytes, static_cast<int32_t>(brow1),
+                            tma_load_2d(b_dst + kTileBytes, mb, kt * kBKBytes, static_cast<int32_t>(brow1),
                                         &full[stage]);
                     }
                     bulk_load(sfb_dst, sfb0 + kt * kSFStage, sf_bytes, &full[stage]);
@@ -319,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * BN);
-                for (int kt = 0; kt < p.num_k_tiles; ++kt) {
+                const GemmArgs &q = (FUSED && t >= m_units * p.n_tiles) ? p2 : p;
+                for (int kt = 0; kt < q.num_k_tiles; ++kt) {
                     // sf_ready completes only after every stager has seen its CTA's
                     // full barrier complete (all of the stage's copies landed), so
                     // one wait covers both the scales and the operand tiles
@@ -328,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const int nkb = min(4, (p.K - kt * kBK) / 64);
+                    const int nkb = min(4, (q.K - kt * kBK) / 64);
                     const uint32_t a_addr = smem_u32(sA + stage * kTileBytes);
                     const uint32_t b_addr = smem_u32(sB + stage * C::kBBoxes * kTileBytes);
                     const uint32_t t_sfa = tmem + C::kTmemSF + static_cast<uint32_t>(stage * C::kSFSlotCols);
@@ -383,14 +449,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int t = unit; t < total && ok; t += units) {
             // an empty pair half has no A scales: its rows get scale 0
-            const bool a_rows = !kPair || decode_tile<CG>(p, t, m_units, rank).valid > 0;
-            for (int kt = 0; kt < p.num_k_tiles; ++kt) {
+            const bool a_rows = !kPair || decode_tile<CG, FUSED>(p, p2, t, m_units, rank).valid > 0;
+            const GemmArgs &q = (FUSED && t >= m_units * p.n_tiles) ? p2 : p;
+            for (int kt = 0; kt < q.num_k_tiles; ++kt) {
                 const bool got = mbar_wait(&full[stage], phase, abort_flag);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
                     break;
                 }
-                const int nkb = min(4, (p.K - kt * kBK) / 64);
+                const int nkb = min(4, (q.K - kt * kBK) / 64);
                 const uint32_t t_slot = t_q + static_cast<uint32_t>(stage * C::kSFSlotCols);
                 // A: column 4*kb + m <- row `lane` of atom kb (the 4 scales of rows 32*m + lane)
                 uint32_t r[16];
@@ -450,16 +517,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const TileInfo ti = decode_tile<CG>(p, t, m_units, rank);
+            const TileInfo ti = decode_tile<CG, FUSED>(p, p2, t, m_units, rank);
+            const GemmArgs &ga = (FUSED && ti.ph) ? p2 : p;
             const bool valid = row < ti.valid;
             const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc * BN);
+            const bool swiglu_tile = FUSED ? ti.ph == 0 : EPI != EPI_BF16;
 
-            if constexpr (EPI == EPI_SWIGLU_QUANT || EPI == EPI_SWIGLU_AMAX) {
+            if (swiglu_tile && BN == 256) {
                 // drain gate columns [64hf, 64hf+64) and the matching up columns in two rounds of
                 // 32 (one wait each), computing h as it arrives, then release the accumulator
-                const float a = p.a_gs[0];
-                const float alpha_g = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + 0]));
-                const float alpha_u = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + 1]));
+                const float a = ga.a_gs[0];
+                const float alpha_g = __fdiv_rn(1.0f, __fmul_rn(a, ga.b_gs[ti.e * ga.b_gs_stride + 0]));
+                const float alpha_u = __fdiv_rn(1.0f, __fmul_rn(a, ga.b_gs[ti.e * ga.b_gs_stride + 1]));
                 float h[64];
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -494,9 +563,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int o = 16; o > 0; o >>= 1)
                         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                     if (lane == 0)
-                        atomicMax(p.amax_bits + ti.e, __float_as_uint(amax));
+                        atomicMax(ga.amax_bits + ti.e, __float_as_uint(amax));
                 } else {
-                    const float hgs = p.inter_gs[ti.e];
+                    const float hgs = ga.inter_gs[ti.e];
                     uint32_t codes[8];
                     uint32_t sfw = 0;
 #pragma unroll
@@ -509,14 +578,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (valid) {
                         // 64 h columns: 32 bytes of codes and one 4-byte scale word (k-block 2nt + hf)
-                        uint4 *hrow = reinterpret_cast<uint4 *>(p.h_codes +
-                                                                static_cast<int64_t>(ti.row0 + row) * p.h_ld_bytes +
+                        uint4 *hrow = reinterpret_cast<uint4 *>(ga.h_codes +
+                                                                static_cast<int64_t>(ti.row0 + row) * ga.h_ld_bytes +
                                                                 ti.nt * 64 + hf * 32);
                         hrow[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
                         hrow[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
-                        *reinterpret_cast<uint32_t *>(p.h_sf + static_cast<int64_t>(ti.row0 / kBM) * p.h_sf_block_stride +
+                        *reinterpret_cast<uint32_t *>(ga.h_sf + static_cast<int64_t>(ti.row0 / kBM) * ga.h_sf_block_stride +
                                                       static_cast<int64_t>(2 * ti.nt + hf) * kSFAtom + lane * 16 +
                                                       q * 4) = sfw;
+                    }
+                    if constexpr (FUSED) {
+                        // publish this warp's h rows to the L2 tiles of this m-tile
+                        __threadfence();
+                        __syncwarp();
+                        if (lane == 0) {
+                            __threadfence();
+                            atomicAdd(ga.ready + ti.mt, 1);
+                        }
                     }
                 }
             } else {
@@ -524,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // converting to bf16 as they arrive, then release the accumulator
                 constexpr int kCols = BN / 2;
                 constexpr int kRound = kCols < 64 ? kCols : 64;
-                const float a = p.a_gs[p.a_gs_per_expert ? ti.e : 0];
+                const float a = ga.a_gs[ga.a_gs_per_expert ? ti.e : 0];
                 uint32_t o[kCols / 2];
 #pragma unroll
                 for (int r = 0; r < kCols / kRound; ++r) {
@@ -540,9 +618,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         int seg = 0;
 #pragma unroll
                         for (int i = 0; i < 3; ++i)
-                            if (i < p.nseg - 1 && col >= p.seg_end[i])
+                            if (i < ga.nseg - 1 && col >= ga.seg_end[i])
                                 seg = i + 1;
-                        const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, p.b_gs[ti.e * p.b_gs_stride + seg]));
+                        const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, ga.b_gs[ti.e * ga.b_gs_stride + seg]));
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             o[(r * kRound + c * 16) / 2 + i] = pack_bf16x2(__uint_as_float(v[16 * c + 2 * i]) * alpha,
@@ -558,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive(&acc_empty[acc]);
                 }
                 if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + static_cast<int64_t>(ti.row0_out + row) * p.ldo +
+                    uint4 *dst = reinterpret_cast<uint4 *>(ga.out + static_cast<int64_t>(ti.row0_out + row) * ga.ldo +
                                                            static_cast<int64_t>(ti.nt) * BN + hf * kCols);
 #pragma unroll
                     for (int i = 0; i < kCols / 8; ++i)
@@ -586,9 +664,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int BN, int EPI, int CG>
+template <int BN, int EPI, int CG, int FUSED>
 static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
-                              const GemmArgs &args, int grid, cudaStream_t stream)
+                              const GemmArgs &args, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
+                              const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream)
 {
     const int smem = Cfg<BN, CG>::kSmem;
     static int attr_done_device = -1;
@@ -597,29 +676,41 @@ static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a
     if (e != cudaSuccess)
         return e;
     if (attr_done_device != dev) {
-        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, EPI, CG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, EPI, CG, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem);
         if (e != cudaSuccess)
             return e;
         attr_done_device = dev;
     }
-    if constexpr (CG == 1) {
-        nvfp4_gemm_kernel<BN, EPI, 1><<<grid, kThreads, smem, stream>>>(map_a, map_a32, map_b, args);
-        return cudaGetLastError();
-    } else {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(grid));
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    cfg.attrs = attr;
+    cfg.numAttrs = 0;
+    if constexpr (CG == 2) {
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, 2>, map_a, map_a32, map_b, args);
+    } else if constexpr (FUSED) {
+        // every CTA resident at once: L2 tiles wait for other CTAs' L1 tiles
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.numAttrs = 1;
     }
+    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, CG, FUSED>, map_a, map_a32, map_b, map_a2, map_a2_32,
+                              map_b2, args, args2);
+}
+
+template <int BN, int EPI, int CG>
+static cudaError_t launch_plain(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
+                                const GemmArgs &args, int grid, cudaStream_t stream)
+{
+    return launch_one<BN, EPI, CG, 0>(map_a, map_a32, map_b, args, map_a, map_a32, map_b, args, grid, stream);
 }
 
 cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
@@ -629,18 +720,28 @@ cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const
         if (bn != 256 || grid % 2 != 0)
             return cudaErrorInvalidValue;
         switch (epi) {
-        case EPI_SWIGLU_QUANT: return launch_one<256, EPI_SWIGLU_QUANT, 2>(map_a, map_a32, map_b, args, grid, stream);
-        case EPI_SWIGLU_AMAX: return launch_one<256, EPI_SWIGLU_AMAX, 2>(map_a, map_a32, map_b, args, grid, stream);
-        default: return launch_one<256, EPI_BF16, 2>(map_a, map_a32, map_b, args, grid, stream);
+        case EPI_SWIGLU_QUANT: return launch_plain<256, EPI_SWIGLU_QUANT, 2>(map_a, map_a32, map_b, args, grid, stream);
+        case EPI_SWIGLU_AMAX: return launch_plain<256, EPI_SWIGLU_AMAX, 2>(map_a, map_a32, map_b, args, grid, stream);
+        default: return launch_plain<256, EPI_BF16, 2>(map_a, map_a32, map_b, args, grid, stream);
         }
     }
     switch (epi) {
-    case EPI_SWIGLU_QUANT: return launch_one<256, EPI_SWIGLU_QUANT, 1>(map_a, map_a32, map_b, args, grid, stream);
-    case EPI_SWIGLU_AMAX: return launch_one<256, EPI_SWIGLU_AMAX, 1>(map_a, map_a32, map_b, args, grid, stream);
+    case EPI_SWIGLU_QUANT: return launch_plain<256, EPI_SWIGLU_QUANT, 1>(map_a, map_a32, map_b, args, grid, stream);
+    case EPI_SWIGLU_AMAX: return launch_plain<256, EPI_SWIGLU_AMAX, 1>(map_a, map_a32, map_b, args, grid, stream);
     default:
-        return bn == 256 ? launch_one<256, EPI_BF16, 1>(map_a, map_a32, map_b, args, grid, stream)
-                         : launch_one<128, EPI_BF16, 1>(map_a, map_a32, map_b, args, grid, stream);
+        return bn == 256 ? launch_plain<256, EPI_BF16, 1>(map_a, map_a32, map_b, args, grid, stream)
+                         : launch_plain<128, EPI_BF16, 1>(map_a, map_a32, map_b, args, grid, stream);
     }
+}
+
+cudaError_t launch_moe_fused(const CUtensorMap &map_a1, const CUtensorMap &map_a1_32, const CUtensorMap &map_b1,
+                             const GemmArgs &args1, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
+                             const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream)
+{
+    if (args1.mtiles == nullptr || args1.ready == nullptr || args2.ready != args1.ready)
+        return cudaErrorInvalidValue;
+    return launch_one<256, EPI_SWIGLU_QUANT, 1, 1>(map_a1, map_a1_32, map_b1, args1, map_a2, map_a2_32, map_b2, args2,
+                                                    grid, stream);
 }
 
 // Clusters of two GEMM CTAs that can be resident at once on the current
@@ -655,8 +756,8 @@ int gemm_pair_clusters(int num_sms)
         return cached;
     const int smem = Cfg<256, 2>::kSmem;
     int n = 0;
-    if (cudaFuncSetAttribute(nvfp4_gemm_kernel<256, EPI_BF16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
-        cudaSuccess) {
+    if (cudaFuncSetAttribute(nvfp4_gemm_kernel<256, EPI_BF16, 2, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(num_sms));
         cfg.blockDim = dim3(kThreads);
@@ -668,7 +769,7 @@ int gemm_pair_clusters(int num_sms)
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<256, EPI_BF16, 2>, &cfg) != cudaSuccess)
+        if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<256, EPI_BF16, 2, 0>, &cfg) != cudaSuccess)
             n = 0;
     }
     (void)cudaGetLastError();

@@ -24,6 +24,7 @@ struct GemmArgs {
     const int4 *mtiles;       // {expert, first padded row, valid rows, first output row}
     const int32_t *num_pairs_dev;
     const int2 *pairs;        // pair tiles: {first m-tile, second m-tile of the same expert or -1}
+    int32_t *ready;           // fused L1 -> L2 launch: per m-tile count of published L1 epilogue warps
     int dense_m_tiles;
     int dense_M;
     int n_tiles;
@@ -62,6 +63,13 @@ cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const
                         const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream);
 // Pair clusters that fit on the device at once (<= num_sms / 2).
 int gemm_pair_clusters(int num_sms);
+// One persistent cooperative launch of the grouped L1 (args1, maps *1, SwiGLU
+// + re-quantisation epilogue) and L2 (args2, maps *2, bf16 epilogue) tiles
+// over the same m-tile table; L2 tiles of an m-tile start once its L1 tiles
+// are published in args1.ready / args2.ready (zeroed by the routing kernel).
+cudaError_t launch_moe_fused(const CUtensorMap &map_a1, const CUtensorMap &map_a1_32, const CUtensorMap &map_b1,
+                             const GemmArgs &args1, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
+                             const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream);
 
 // Memory-bound kernels (kernels.cu).
 cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s);
@@ -72,8 +80,8 @@ cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, 
 cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64_t cols, uint8_t *out,
                            cudaStream_t s);
 cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
-                         int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *inv,
-                         int32_t *err, cudaStream_t s);
+                         int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *ready,
+                         int32_t *inv, int32_t *err, cudaStream_t s);
 cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int32_t *ids, const float *w,
                            const int32_t *off, const int32_t *poff, int64_t T, int k, int64_t H,
                            __nv_bfloat16 *out, cudaStream_t s);

@@ -221,7 +221,8 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
                                                      int32_t *__restrict__ counts, int32_t *__restrict__ off,
                                                      int32_t *__restrict__ poff, int32_t *__restrict__ num_mtiles,
                                                      int4 *__restrict__ mtiles, int32_t *__restrict__ num_pairs,
-                                                     int2 *__restrict__ pairs, int32_t *__restrict__ inv,
+                                                     int2 *__restrict__ pairs, int32_t *__restrict__ ready,
+                                                     int32_t *__restrict__ inv,
                                                      int32_t *__restrict__ err)
 {
     extern __shared__ int32_t sm[];
@@ -304,8 +305,11 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
         off[tid] = base_c;
         poff[tid] = base_t * 128;
         poff_s[tid] = base_t * 128;
-        for (int i = 0; i < tiles; ++i)
+        for (int i = 0; i < tiles; ++i) {
             mtiles[base_t + i] = make_int4(tid, base_t * 128 + 128 * i, min(128, cnt - 128 * i), base_c + 128 * i);
+            if (ready != nullptr)
+                ready[base_t + i] = 0;
+        }
         for (int i = 0; i < npair; ++i)
             pairs[base_p + i] = make_int2(base_t + 2 * i, 2 * i + 1 < tiles ? base_t + 2 * i + 1 : -1);
         if (tid == E - 1) {
@@ -338,8 +342,8 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
 }
 
 cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
-                         int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *inv,
-                         int32_t *err, cudaStream_t s)
+                         int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *ready,
+                         int32_t *inv, int32_t *err, cudaStream_t s)
 {
     const size_t smem = sizeof(int32_t) * (33 * static_cast<size_t>(E));
     static bool attr_set = false;
@@ -350,7 +354,7 @@ cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, 
         attr_set = true;
     }
     route_kernel<<<1, 1024, smem, s>>>(ids, static_cast<int>(R), E, counts, off, poff, num_mtiles, mtiles, num_pairs,
-                                       pairs, inv, err);
+                                       pairs, ready, inv, err);
     return cudaGetLastError();
 }
 

@@ -313,3 +313,16 @@ def test_pair_tiles_end_to_end():
     out, ws = p.run()
     assert nvfp4_moe_get_error(ws) == 0
     check_output(out, p.oracle())
+
+
+# H = 384: the L2 tiles are 128 wide, so L1 and L2 run as two launches.
+NARROW = W.MoeConfig("narrow", E=4, k=2, T=96, H=384, I=256, routing="softmax", outliers=False, warmup_T=64)
+
+
+def test_unfused_narrow_hidden():
+    from nvfp4_moe_expert_topk_b200 import nvfp4_moe_plan
+    assert nvfp4_moe_plan(NARROW.T, NARROW.k, NARROW.E, NARROW.H, NARROW.I) == (False, False)
+    p = Problem(NARROW)
+    out, ws = p.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    check_output(out, p.oracle())
