@@ -43,7 +43,7 @@ from nvfp4_moe_expert_topk_b200 import workloads as W  # noqa: E402
 FP4_NOMINAL_TFLOPS = 9000.0            # dense FP4, NVIDIA public B200 figure
 BF16_TO_FP4_NOMINAL_RATIO = 4.0        # 9 / 2.25 PFLOP/s dense
 STAGES = ["global_scale", "route", "quantize_permute", "l1_gate_up_swiglu_quant", "l2_down", "combine"]
-KERNELS_PER_STEP = 7                   # amax + finalize (global scale), route, quantise, L1, L2, combine
+FRONT_STAGE = "front"                  # global scale of the batch + routing + quantise/permute
 FUSED_STAGE = "l1_l2_fused"            # L1 and L2 as one launch (nvfp4_moe_plan)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 GEMM_SOURCES = ["gemm.cu", "ptx.cuh", "quant.cuh", "internal.h"]
@@ -203,24 +203,28 @@ class Workload:
         self.rows = int(counts.sum())
         self.nonempty = int((counts > 0).sum())
         self.fused, self.pair_tiles = nvfp4_moe_plan(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I)
-        self.launches_per_step = KERNELS_PER_STEP - (1 if self.fused else 0)
+        # global scale (amax + finalize), route, quantise, L1 + L2 (one launch or two), combine
+        self.launches_per_step = 6 if self.fused else 7
 
     def fold(self, per_stage):
-        """Per-stage figures keyed by the launches the plan runs: with the fused
-        plan, L1 and L2 are one launch (its time sits in the L1 slot of the
-        timed forward and the L2 slot is empty)."""
+        """Per-stage figures keyed by the stages the forward runs: the front
+        (global scale of the batch, routing, quantise+permute: four small
+        launches), the GEMMs (with the fused plan L1 and L2 are one launch,
+        whose time sits in the L1 slot of the timed forward, the L2 slot being
+        empty) and the combine."""
         d = dict(per_stage)
+        d[FRONT_STAGE] = d.pop("global_scale") + d.pop("route") + d.pop("quantize_permute")
         if self.fused:
             d[FUSED_STAGE] = d.pop("l1_gate_up_swiglu_quant") + d.pop("l2_down")
         return d
 
     def step(self, events=None):
-        nvfp4_global_scale(self.x, self.x_gs)
+        # x_gs = None: the forward computes this batch's global scale itself
         if events is None:
-            nvfp4_moe_forward(self.x, self.ids, self.w, self.x_gs, **self.weights.args(), inter_gs=self.inter_gs,
+            nvfp4_moe_forward(self.x, self.ids, self.w, None, **self.weights.args(), inter_gs=self.inter_gs,
                               out=self.out, workspace=self.ws)
         else:
-            nvfp4_moe_forward_timed(self.x, self.ids, self.w, self.x_gs, **self.weights.args(),
+            nvfp4_moe_forward_timed(self.x, self.ids, self.w, None, **self.weights.args(),
                                     inter_gs=self.inter_gs, out=self.out, workspace=self.ws, events=events)
 
     # algorithmic work (real rows only; weights of non-empty experts once)

@@ -120,7 +120,9 @@ typedef struct {
     int32_t E, k;
     const int32_t *topk_ids;      /* [T, k]; id < 0: slot skipped; id >= E: error word set, slot skipped */
     const float *topk_weights;    /* [T, k] fp32                                      */
-    const float *x_gs;            /* [1] global scale of x (nvfp4_global_scale, or warmup) */
+    const float *x_gs;            /* [1] global scale of x (nvfp4_global_scale, or warmup); NULL:
+                                     the call computes 2688 / max|x| of this batch itself (kept in
+                                     workspace region 8) */
     const uint8_t *w13_codes;     /* [E, 2I, H/2]: rows 0..I-1 gate, rows I..2I-1 up   */
     const uint8_t *w13_scales;    /* NVFP4_SCALES_MMA of [E*2I, H]                     */
     const float *w13_gs;          /* [E, 2]: global scale of (gate, up) of each expert */
@@ -139,15 +141,19 @@ size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
 /* out = sum_j topk_weights[t,j] * Expert_{ids[t,j]}(x[t]) with
  * Expert_e(x) = W2_e . q(SiLU(W13g_e . q(x)) * (W13u_e . q(x))), all GEMMs
  * in NVFP4 on the tensor cores, q() the NVFP4 quantiser (x with x_gs, h with
- * inter_gs[e]).  Launches route, quantise+permute, L1 (fused SiLU*up
- * re-quantise epilogue), L2 and combine on `stream`; no host sync, no
+ * inter_gs[e]).  Launches on `stream`: the global scale of x when x_gs is
+ * NULL (a 4-byte memset of the workspace and two kernels), routing,
+ * quantise+permute, L1 (fused SiLU*up re-quantise epilogue) and L2 (one fused
+ * launch or two, see nvfp4_moe_plan) and the combine; no host sync, no
  * allocation, so the call can be captured in a CUDA graph (make one eager
  * call per device first: it sets per-kernel attributes). */
 int nvfp4_moe_forward(const nvfp4_moe_args *args, void *workspace, size_t ws_bytes, void *stream);
 
-/* nvfp4_moe_forward with a CUDA event recorded on `stream` before each of
- * its five kernels (route, quantise+permute, L1, L2, combine) and after the
- * last: events = 6 cudaEvent_t handles created by the caller.  Otherwise
+/* nvfp4_moe_forward with CUDA events recorded on `stream` at its stage
+ * boundaries: events = 6 cudaEvent_t handles created by the caller, recorded
+ * before the global scale (x_gs NULL) and routing, before quantise+permute,
+ * before L1, after L1, after L2 (directly after L1's record when they are
+ * one launch) and after the combine.  Otherwise
  * identical; for per-stage timing.  While `stream` is being captured into a
  * CUDA graph the records become external event nodes, so the events can be
  * timed after each replay. */
@@ -173,7 +179,8 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
 /* Byte offset and size of a workspace region (for inspection and tests).
  * region: 0 A codes, 1 A scales (MMA layout), 2 h codes, 3 h scales
  * (MMA layout), 4 y (bf16 [T*k, H], rows in expert-major routing order),
- * 5 inv, 6 counts, 7 padded offsets. */
+ * 5 inv, 6 counts, 7 padded offsets, 8 the fp32 global scale of x computed
+ * by the last call made with x_gs = NULL. */
 int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, int region,
                                int64_t *offset, int64_t *bytes);
 

@@ -157,7 +157,7 @@ def _moe_args(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs, w2
     a.T, a.H, a.I, a.E, a.k = T, H, twoI // 2, E, topk_ids.shape[1]
     a.topk_ids = _dev(topk_ids, "topk_ids", torch.int32).value
     a.topk_weights = _dev(topk_weights, "topk_weights", torch.float32).value
-    a.x_gs = _dev(x_gs, "x_gs", torch.float32).value
+    a.x_gs = None if x_gs is None else _dev(x_gs, "x_gs", torch.float32).value   # None: from this batch
     a.w13_codes = _dev(w13_codes, "w13_codes", torch.uint8).value
     a.w13_scales = _dev(w13_scales, "w13_scales", torch.uint8).value
     a.w13_gs = _dev(w13_gs, "w13_gs", torch.float32).value

@@ -2,6 +2,8 @@
 // quantisation (plain and fused with the expert permutation), scale-layout
 // conversion, routing (histogram, prefix sums, stable permutation, m-tile
 // table) and the top-k weighted combine.
+#include <algorithm>
+
 #include "internal.h"
 #include "quant.cuh"
 
@@ -79,25 +81,21 @@ cudaError_t launch_finalize_gs(float *gs, cudaStream_t s)
 // row t.
 constexpr int kQuantChunk = 2048;
 
-__global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
-                                                            int64_t cols, int64_t ldx, const float *__restrict__ gs_ptr,
-                                                            uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
-                                                            int layout, const int32_t *__restrict__ inv, int k)
+// One (row, chunk) item by one whole warp (item < rows * chunks).
+__device__ __forceinline__ void quantize_item(const __nv_bfloat16 *__restrict__ x, int64_t cols, int64_t ldx,
+                                              float gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                                              int layout, const int32_t *__restrict__ inv, int k, int64_t item,
+                                              int lane)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t chunks = (cols + kQuantChunk - 1) / kQuantChunk;
-    const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + warp;
-    if (item >= rows * chunks)
-        return;
     const int64_t row = item / chunks;
     const int64_t c0 = (item - row * chunks) * kQuantChunk + static_cast<int64_t>(lane) * 64;
-    const float gs = __ldg(gs_ptr);
     int my_dst = -1;                         // lane j < k holds destination j
     int ndst = 1;
     if (inv != nullptr) {
         ndst = k;
         if (lane < k)
-            my_dst = __ldg(inv + row * k + lane);
+            my_dst = inv[row * k + lane];      // coherent load: the front kernel writes inv in the same launch
     }
     // lanes past the end of the row do no work but stay for the shuffles below
     const bool active = c0 < cols;
@@ -140,8 +138,10 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 
             reinterpret_cast<uint4 *>(crow)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
             reinterpret_cast<uint4 *>(crow)[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
         } else {
-            for (int b = 0; b < nb; ++b)
-                reinterpret_cast<uint2 *>(crow)[b] = make_uint2(cw[2 * b], cw[2 * b + 1]);
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (b < nb)
+                    reinterpret_cast<uint2 *>(crow)[b] = make_uint2(cw[2 * b], cw[2 * b + 1]);
         }
         if (layout == NVFP4_SCALES_MMA) {
             *reinterpret_cast<uint32_t *>(scales + mma_scale_offset(dst, c0 / 64, kb_per_block)) = sw;
@@ -154,6 +154,19 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 
                     srow[b] = static_cast<uint8_t>(sw >> (8 * b));
         }
     }
+}
+
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
+                                                            int64_t cols, int64_t ldx, const float *__restrict__ gs_ptr,
+                                                            uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                                                            int layout, const int32_t *__restrict__ inv, int k)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t chunks = (cols + kQuantChunk - 1) / kQuantChunk;
+    const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+    if (item >= rows * chunks)
+        return;
+    quantize_item(x, cols, ldx, __ldg(gs_ptr), codes, scales, layout, inv, k, item, lane);
 }
 
 cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs,
@@ -217,15 +230,14 @@ cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64
 //     other with match_any, so a slot's rank is the number of earlier slots
 //     of its expert: position = padded_offset[e] + rank (a stable counting
 //     sort, deterministic for a given input).
-__global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__ ids, int R, int E,
-                                                     int32_t *__restrict__ counts, int32_t *__restrict__ off,
-                                                     int32_t *__restrict__ poff, int32_t *__restrict__ num_mtiles,
-                                                     int4 *__restrict__ mtiles, int32_t *__restrict__ num_pairs,
-                                                     int2 *__restrict__ pairs, int32_t *__restrict__ ready,
-                                                     int32_t *__restrict__ inv,
-                                                     int32_t *__restrict__ err)
+// Executed by all 1024 threads of one block; sm: 33 * E int32 of shared memory.
+__device__ __forceinline__ void route_block(const int32_t *__restrict__ ids, int R, int E, int32_t *__restrict__ counts,
+                                            int32_t *__restrict__ off, int32_t *__restrict__ poff,
+                                            int32_t *__restrict__ num_mtiles, int4 *__restrict__ mtiles,
+                                            int32_t *__restrict__ num_pairs, int2 *__restrict__ pairs,
+                                            int32_t *__restrict__ ready, int32_t *__restrict__ inv,
+                                            int32_t *__restrict__ err, int32_t *sm)
 {
-    extern __shared__ int32_t sm[];
     int32_t *wcnt = sm;                // [32][E]
     int32_t *poff_s = sm + 32 * E;     // [E]
     __shared__ int32_t warp_sum_c[32], warp_sum_t[32], warp_sum_p[32];
@@ -341,18 +353,40 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
     }
 }
 
+__global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__ ids, int R, int E,
+                                                     int32_t *__restrict__ counts, int32_t *__restrict__ off,
+                                                     int32_t *__restrict__ poff, int32_t *__restrict__ num_mtiles,
+                                                     int4 *__restrict__ mtiles, int32_t *__restrict__ num_pairs,
+                                                     int2 *__restrict__ pairs, int32_t *__restrict__ ready,
+                                                     int32_t *__restrict__ inv, int32_t *__restrict__ err)
+{
+    extern __shared__ int32_t sm[];
+    route_block(ids, R, E, counts, off, poff, num_mtiles, mtiles, num_pairs, pairs, ready, inv, err, sm);
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+static cudaError_t allow_smem(K kernel, int bytes, int *done_device)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || *done_device == dev)
+        return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        *done_device = dev;
+    return e;
+}
+
 cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
                          int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *ready,
                          int32_t *inv, int32_t *err, cudaStream_t s)
 {
     const size_t smem = sizeof(int32_t) * (33 * static_cast<size_t>(E));
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 33 * 1024 * 4);
-        if (e != cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    static int attr_device = -1;
+    cudaError_t e = allow_smem(route_kernel, 33 * 1024 * 4, &attr_device);
+    if (e != cudaSuccess)
+        return e;
     route_kernel<<<1, 1024, smem, s>>>(ids, static_cast<int>(R), E, counts, off, poff, num_mtiles, mtiles, num_pairs,
                                        pairs, ready, inv, err);
     return cudaGetLastError();

@@ -326,3 +326,24 @@ def test_unfused_narrow_hidden():
     out, ws = p.run()
     assert nvfp4_moe_get_error(ws) == 0
     check_output(out, p.oracle())
+
+
+def test_forward_computes_batch_global_scale(tiny):
+    """x_gs = None: the forward computes 2688 / max|x| of the batch in its
+    front launch (kept in workspace region 8), equal bit for bit to the
+    oracle's global scale, and the output equals that of a call given the
+    same scale explicitly."""
+    p = tiny
+    inputs = p.device_inputs()
+    ref_out, ws = p.run(inputs)
+    cfg = p.cfg
+    T = p.x.shape[0]
+    inputs_none = dict(inputs, x_gs=None)
+    out = torch.full((T, cfg.H), float("nan"), dtype=torch.bfloat16, device=DEV)
+    nvfp4_moe_forward(**inputs_none, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert nvfp4_moe_get_error(ws) == 0
+    o, n = region(p, 8)
+    gs = ws[o:o + n].cpu().numpy().view(np.float32)[0]
+    assert gs == O.global_scale_bf16(W.bf16_bits(p.x)) == p.x_gs
+    assert torch.equal(out, ref_out)
