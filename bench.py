@@ -254,13 +254,31 @@ class Workload:
         return self.nonempty * 3 * c.H * c.I * fp4 + 2 * c.T * c.H * 2.0 + c.T * c.k * 8.0
 
 
+def _capture(fn):
+    """A CUDA graph of everything fn() issues (captured on a side stream)."""
+    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            fn()
+    stream.wait_stream(side)
+    g.replay()                          # upload + warm
+    torch.cuda.synchronize()
+    return g
+
+
 def time_steps(wl, steps, warmup, world, graph=True, tag="timed"):
     """Device time of `steps` steps: events on the launching stream, barrier +
-    synchronize on both sides, max over ranks; per-stage mean durations from
-    events recorded between the kernels of every step.  With graph=True the
-    `steps` steps (events included) are captured once into a CUDA graph and
-    the timed region is one replay of it -- the way a serving runtime issues
-    the block (the pages' runner is cudagraph-safe); otherwise eager launches."""
+    synchronize on both sides, max over ranks.  With graph=True the `steps`
+    steps are captured once into a CUDA graph and the timed region is one
+    replay of it -- the way a serving runtime issues the block (the pages'
+    runner is cudagraph-safe); otherwise eager launches.  Per-stage mean
+    durations come from a second run of the same steps with events recorded
+    between the forward's stages (in the graph case a second graph, so that
+    the event nodes, which also stop consecutive kernels from overlapping
+    their launch, stay out of the headline time)."""
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         wl.step()
@@ -271,22 +289,17 @@ def time_steps(wl, steps, warmup, world, graph=True, tag="timed"):
             e.record(stream)
     torch.cuda.synchronize()
 
-    def issue():
+    def issue_plain():
+        for _ in range(steps):
+            wl.step()
+
+    def issue_staged():
         for i in range(steps):
             ev[i][0].record()
             wl.step(events=ev[i][1:])
 
-    g = None
-    if graph:
-        side = torch.cuda.Stream()
-        side.wait_stream(stream)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(g, stream=side):
-                issue()
-        stream.wait_stream(side)
-        g.replay()                      # upload + warm
-        torch.cuda.synchronize()
+    g = _capture(issue_plain) if graph else None
+    g_staged = _capture(issue_staged) if graph else None
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -296,17 +309,22 @@ def time_steps(wl, steps, warmup, world, graph=True, tag="timed"):
     if g is not None:
         g.replay()
     else:
-        issue()
+        issue_plain()
     t1.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier(world)
     ms = t0.elapsed_time(t1)
+    if g_staged is not None:
+        g_staged.replay()
+    else:
+        issue_staged()
+    torch.cuda.synchronize()
     try:
         stage_ms = {name: float(np.mean([e[j].elapsed_time(e[j + 1]) for e in ev])) for j, name in enumerate(STAGES)}
     except Exception:                   # graph-recorded events not timeable here: time the stages eagerly
         stage_ms = None
-    del g
+    del g, g_staged
     if stage_ms is None:
         _, stage_ms = time_steps(wl, steps, 0, world, graph=False, tag="stages")
         return max_over_ranks(world, ms), stage_ms

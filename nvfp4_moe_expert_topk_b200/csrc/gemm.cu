@@ -287,6 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // cluster addresses of the leader's sf_ready / acc_empty barriers
     const uint32_t sf_ready_lead = kPair ? map_shared_to_cta(smem_u32(sf_ready), 0) : 0u;
     const uint32_t acc_empty_lead = kPair ? map_shared_to_cta(smem_u32(acc_empty), 0) : 0u;
+    // everything above overlaps the previous kernel's tail (dependent launch);
+    // from here on the tile table, the operands and the outputs are touched
+    pdl_wait();
 
     const int m_units = (p.mtiles != nullptr)
                             ? *reinterpret_cast<volatile const int32_t *>(kPair ? p.num_pairs_dev : p.num_mtiles_dev)
@@ -650,6 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    pdl_trigger();                  // the next kernel may start launching during the teardown
     tc_fence_before();
     __syncthreads();
     if constexpr (kPair)
@@ -687,20 +691,26 @@ static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cfg.attrs = attr;
     cfg.numAttrs = 0;
-    if constexpr (CG == 2) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.numAttrs = 1;
-    } else if constexpr (FUSED) {
+    if constexpr (FUSED) {
         // every CTA resident at once: L2 tiles wait for other CTAs' L1 tiles
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
-        cfg.numAttrs = 1;
+        attr[cfg.numAttrs].id = cudaLaunchAttributeCooperative;
+        attr[cfg.numAttrs].val.cooperative = 1;
+        ++cfg.numAttrs;
+    } else {
+        // the prologue (barriers, TMEM, tensor-map prefetch) overlaps the previous kernel
+        attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+        ++cfg.numAttrs;
+    }
+    if constexpr (CG == 2) {
+        attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+        attr[cfg.numAttrs].val.clusterDim.x = 2;
+        attr[cfg.numAttrs].val.clusterDim.y = 1;
+        attr[cfg.numAttrs].val.clusterDim.z = 1;
+        ++cfg.numAttrs;
     }
     return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, CG, FUSED>, map_a, map_a32, map_b, map_a2, map_a2_32,
                               map_b2, args, args2);

@@ -10,6 +10,25 @@
 
 namespace nvfp4 {
 
+// Launches `kernel` with programmatic stream serialization: it may begin
+// while the previous kernel on the stream finishes, and must call pdl_wait()
+// before touching anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Arguments of the persistent block-scaled FP4 GEMM engine (gemm.cu).
 struct GemmArgs {
     // scale factors, NVFP4_SCALES_MMA layout: one 128-row block = (K/64) atoms of 512 bytes

@@ -15,6 +15,8 @@ namespace nvfp4 {
 __global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t n,
                                                         unsigned int *__restrict__ out_bits)
 {
+    pdl_wait();
+    pdl_trigger();
     float m = 0.0f;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t nth = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -52,6 +54,8 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16 *__r
 // gs = 2688 / amax (fp32, round to nearest), 1 if amax == 0; in place.
 __global__ void finalize_gs_kernel(float *gs)
 {
+    pdl_wait();
+    pdl_trigger();
     const float a = __uint_as_float(*reinterpret_cast<unsigned int *>(gs));
     *gs = (a == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, a);
 }
@@ -63,14 +67,13 @@ cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, i
         blocks = 1;
     if (blocks > 8LL * num_sms)
         blocks = 8LL * num_sms;
-    amax_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, n, reinterpret_cast<unsigned int *>(gs_out));
-    return cudaGetLastError();
+    return launch_pdl(amax_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, n,
+                      reinterpret_cast<unsigned int *>(gs_out));
 }
 
 cudaError_t launch_finalize_gs(float *gs, cudaStream_t s)
 {
-    finalize_gs_kernel<<<1, 1, 0, s>>>(gs);
-    return cudaGetLastError();
+    return launch_pdl(finalize_gs_kernel, dim3(1), dim3(1), 0, s, gs);
 }
 
 // ------------------------------------------------------------ quantisation
@@ -161,6 +164,8 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 
                                                             uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
                                                             int layout, const int32_t *__restrict__ inv, int k)
 {
+    pdl_wait();
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t chunks = (cols + kQuantChunk - 1) / kQuantChunk;
     const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + warp;
@@ -174,9 +179,8 @@ cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, 
 {
     const int64_t items = rows * ((cols + kQuantChunk - 1) / kQuantChunk);
     const int64_t blocks = (items + 7) / 8;
-    quantize_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(x, rows, cols, ldx, gs, codes, scales, layout,
-                                                                     inv, k);
-    return cudaGetLastError();
+    return launch_pdl(quantize_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, rows, cols, ldx, gs,
+                      codes, scales, layout, inv, k);
 }
 
 // ------------------------------------------------------------ scale layout
@@ -361,6 +365,8 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
                                                      int32_t *__restrict__ inv, int32_t *__restrict__ err)
 {
     extern __shared__ int32_t sm[];
+    pdl_wait();
+    pdl_trigger();
     route_block(ids, R, E, counts, off, poff, num_mtiles, mtiles, num_pairs, pairs, ready, inv, err, sm);
 }
 
@@ -387,9 +393,8 @@ cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, 
     cudaError_t e = allow_smem(route_kernel, 33 * 1024 * 4, &attr_device);
     if (e != cudaSuccess)
         return e;
-    route_kernel<<<1, 1024, smem, s>>>(ids, static_cast<int>(R), E, counts, off, poff, num_mtiles, mtiles, num_pairs,
-                                       pairs, ready, inv, err);
-    return cudaGetLastError();
+    return launch_pdl(route_kernel, dim3(1), dim3(1024), smem, s, ids, static_cast<int>(R), E, counts, off, poff,
+                      num_mtiles, mtiles, num_pairs, pairs, ready, inv, err);
 }
 
 // ------------------------------------------------------------ combine
@@ -407,6 +412,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__res
 {
     __shared__ int64_t s_row[32];
     __shared__ float s_w[32];
+    pdl_wait();
+    pdl_trigger();
     const int64_t t = blockIdx.x;
     if (threadIdx.x < k) {
         const int64_t f = t * k + threadIdx.x;
@@ -454,8 +461,7 @@ cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int
                            __nv_bfloat16 *out, cudaStream_t s)
 {
     const dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>((H + kCombineChunk - 1) / kCombineChunk));
-    combine_kernel<<<grid, 128, 0, s>>>(y, inv, ids, w, off, poff, k, H, out);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, grid, dim3(128), 0, s, y, inv, ids, w, off, poff, k, H, out);
 }
 
 // ------------------------------------------------------------ warmup scales

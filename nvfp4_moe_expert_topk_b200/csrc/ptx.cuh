@@ -89,6 +89,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     return false;
 }
 
+// ---------------------------------------------------------------- dependent launches
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before its predecessor in the stream finishes;
+// pdl_wait() returns once the predecessor has completed and its memory is
+// visible (immediately for a kernel launched without the attribute).
+// pdl_trigger() lets the successor be scheduled once every CTA of this grid
+// has triggered or exited.
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_trigger()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- clusters
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {
