@@ -89,7 +89,7 @@ int64_t round_up(int64_t v, int64_t m)
 // ---------------------------------------------------------------- workspace
 struct Layout {
     int64_t mt_max = 0, rpad = 0;
-    int64_t counts = 0, off = 0, poff = 0, mtiles = 0, pairs = 0, ready = 0, inv = 0, amax = 0;
+    int64_t counts = 0, off = 0, poff = 0, mtiles = 0, pairs = 0, ready = 0, inv = 0, yrow = 0, amax = 0;
     int64_t a_codes = 0, a_sf = 0, h_codes = 0, h_sf = 0, y = 0, total = 0;
 };
 
@@ -116,6 +116,7 @@ Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
     L.pairs = take(8 * std::max<int64_t>(L.mt_max, 1));
     L.ready = take(4 * std::max<int64_t>(L.mt_max, 1));
     L.inv = take(4 * std::max<int64_t>(R, 1));
+    L.yrow = take(4 * std::max<int64_t>(R, 1));
     L.a_codes = take(L.rpad * (H / 2));
     L.a_sf = take(L.rpad * (H / 16));
     L.h_codes = take(L.rpad * (I / 2));
@@ -311,7 +312,8 @@ int run_route_quant(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, void 
                                  reinterpret_cast<int32_t *>(ws + L.off), reinterpret_cast<int32_t *>(ws + L.poff),
                                  reinterpret_cast<int32_t *>(ws + 4), reinterpret_cast<int4 *>(ws + L.mtiles),
                                  reinterpret_cast<int32_t *>(ws + 8), reinterpret_cast<int2 *>(ws + L.pairs),
-                                 reinterpret_cast<int32_t *>(ws + L.ready), inv, reinterpret_cast<int32_t *>(ws), s);
+                                 reinterpret_cast<int32_t *>(ws + L.ready), inv,
+                                 reinterpret_cast<int32_t *>(ws + L.yrow), reinterpret_cast<int32_t *>(ws), s);
     if (e != cudaSuccess || mark(events, 1, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
     e = launch_quantize(reinterpret_cast<const __nv_bfloat16 *>(a->x), T, H, H, x_gs_ptr(a, ws), ws + L.a_codes,
@@ -573,9 +575,8 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
     }
 
     if (launch_combine(reinterpret_cast<const __nv_bfloat16 *>(ws + L.y),
-                       reinterpret_cast<const int32_t *>(ws + L.inv), a->topk_ids, a->topk_weights,
-                       reinterpret_cast<const int32_t *>(ws + L.off), reinterpret_cast<const int32_t *>(ws + L.poff),
-                       a->T, a->k, H, reinterpret_cast<__nv_bfloat16 *>(a->out), s) != cudaSuccess)
+                       reinterpret_cast<const int32_t *>(ws + L.yrow), a->topk_weights, a->T, a->k, H,
+                       reinterpret_cast<__nv_bfloat16 *>(a->out), s) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     return mark(events, 5, s);
 }
@@ -667,7 +668,7 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
                                     padded_offsets, reinterpret_cast<int32_t *>(ws + 4),
                                     reinterpret_cast<int4 *>(ws + L.mtiles), reinterpret_cast<int32_t *>(ws + 8),
                                     reinterpret_cast<int2 *>(ws + L.pairs), reinterpret_cast<int32_t *>(ws + L.ready),
-                                    inv, reinterpret_cast<int32_t *>(ws),
+                                    inv, reinterpret_cast<int32_t *>(ws + L.yrow), reinterpret_cast<int32_t *>(ws),
                                     static_cast<cudaStream_t>(stream)));
 }
 

@@ -100,9 +100,8 @@ cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64
                            cudaStream_t s);
 cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
                          int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *ready,
-                         int32_t *inv, int32_t *err, cudaStream_t s);
-cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int32_t *ids, const float *w,
-                           const int32_t *off, const int32_t *poff, int64_t T, int k, int64_t H,
+                         int32_t *inv, int32_t *yrow, int32_t *err, cudaStream_t s);
+cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *yrow, const float *w, int64_t T, int k, int64_t H,
                            __nv_bfloat16 *out, cudaStream_t s);
 cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float *inter_gs, cudaStream_t s);
 cudaError_t launch_mma_ceiling(int bn, int iters, int ctas, long long *cycles, int32_t *err, cudaStream_t s);

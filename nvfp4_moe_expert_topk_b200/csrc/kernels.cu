@@ -24,13 +24,19 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16 *__r
     if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
         const int64_t n8 = n / 8;
         const uint4 *xv = reinterpret_cast<const uint4 *>(x);
-        for (int64_t i = tid; i < n8; i += nth) {
-            const uint4 v = __ldg(xv + i);
-            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+        for (int64_t i0 = tid; i0 < n8; i0 += 4 * nth) {
+            uint4 v[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = __bfloat1622float2(h[j]);
-                m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+            for (int u = 0; u < 4; ++u)     // four 16-byte loads in flight per thread
+                v[u] = i0 + u * nth < n8 ? __ldg(xv + i0 + u * nth) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __bfloat1622float2(h[j]);
+                    m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+                }
             }
         }
         start_scalar = n8 * 8;
@@ -108,12 +114,19 @@ __device__ __forceinline__ void quantize_item(const __nv_bfloat16 *__restrict__ 
     const int nb = nb_left < 4 ? static_cast<int>(nb_left) : 4;
     uint32_t cw[8];
     uint32_t sw = 0;
+    // all of this lane's loads first (up to 8 x 16 bytes in flight)
+    uint4 ld[8];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(xr + c0 + 16 * b);
+        ld[2 * b] = b < nb ? __ldg(src) : make_uint4(0, 0, 0, 0);
+        ld[2 * b + 1] = b < nb ? __ldg(src + 1) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
         cw[2 * b] = cw[2 * b + 1] = 0;
         if (b < nb) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(xr + c0 + 16 * b);
-            const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+            const uint4 v0 = ld[2 * b], v1 = ld[2 * b + 1];
             const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&v0);
             const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&v1);
             float f[16];
@@ -240,10 +253,11 @@ __device__ __forceinline__ void route_block(const int32_t *__restrict__ ids, int
                                             int32_t *__restrict__ num_mtiles, int4 *__restrict__ mtiles,
                                             int32_t *__restrict__ num_pairs, int2 *__restrict__ pairs,
                                             int32_t *__restrict__ ready, int32_t *__restrict__ inv,
-                                            int32_t *__restrict__ err, int32_t *sm)
+                                            int32_t *__restrict__ yrow, int32_t *__restrict__ err, int32_t *sm)
 {
     int32_t *wcnt = sm;                // [32][E]
     int32_t *poff_s = sm + 32 * E;     // [E]
+    int32_t *off_s = sm + 33 * E;      // [E]
     __shared__ int32_t warp_sum_c[32], warp_sum_t[32], warp_sum_p[32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -254,12 +268,19 @@ __device__ __forceinline__ void route_block(const int32_t *__restrict__ ids, int
     const int chunk = (R + 31) / 32;
     const int f0 = min(R, warp * chunk), f1 = min(R, f0 + chunk);
     int bad = 0;
-    for (int f = f0 + lane; f < f1; f += 32) {
-        const int e = __ldg(ids + f);
-        if (e >= E)
-            bad = 1;
-        else if (e >= 0)
-            atomicAdd(&wcnt[warp * E + e], 1);
+    for (int base = f0; base < f1; base += 4 * 32) {
+        const int fb = base + lane;
+        int ev[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)         // four loads in flight per lane
+            ev[u] = fb + 32 * u < f1 ? __ldg(ids + fb + 32 * u) : -1;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (ev[u] >= E)
+                bad = 1;
+            else if (ev[u] >= 0)
+                atomicAdd(&wcnt[warp * E + ev[u]], 1);
+        }
     }
     if (bad)
         atomicCAS(err, 0, NVFP4_ERR_BAD_EXPERT_ID);
@@ -321,6 +342,7 @@ __device__ __forceinline__ void route_block(const int32_t *__restrict__ ids, int
         off[tid] = base_c;
         poff[tid] = base_t * 128;
         poff_s[tid] = base_t * 128;
+        off_s[tid] = base_c;
         for (int i = 0; i < tiles; ++i) {
             mtiles[base_t + i] = make_int4(tid, base_t * 128 + 128 * i, min(128, cnt - 128 * i), base_c + 128 * i);
             if (ready != nullptr)
@@ -339,21 +361,32 @@ __device__ __forceinline__ void route_block(const int32_t *__restrict__ ids, int
 
     // 4: stable positions
     const unsigned lt_mask = (1u << lane) - 1u;
-    for (int base = f0; base < f1; base += 32) {
-        const int f = base + lane;
-        const bool act = f < f1;
-        const int e = act ? __ldg(ids + f) : -1;
-        const bool valid = act && e >= 0 && e < E;
-        const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
-        const int rank = __popc(peers & lt_mask);
-        if (valid)
-            inv[f] = poff_s[e] + wcnt[warp * E + e] + rank;
-        else if (act)
-            inv[f] = -1;
-        __syncwarp();
-        if (valid && rank == 0)
-            wcnt[warp * E + e] += __popc(peers);
-        __syncwarp();
+    for (int base0 = f0; base0 < f1; base0 += 4 * 32) {
+        int ev[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)         // load four groups, then walk them in order
+            ev[u] = base0 + 32 * u + lane < f1 ? __ldg(ids + base0 + 32 * u + lane) : -1;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int f = base0 + 32 * u + lane;
+            const bool act = f < f1;
+            const int e = ev[u];
+            const bool valid = act && e >= 0 && e < E;
+            const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
+            const int rank = __popc(peers & lt_mask);
+            if (valid) {
+                const int r = wcnt[warp * E + e] + rank;
+                inv[f] = poff_s[e] + r;
+                yrow[f] = off_s[e] + r;
+            } else if (act) {
+                inv[f] = -1;
+                yrow[f] = -1;
+            }
+            __syncwarp();
+            if (valid && rank == 0)
+                wcnt[warp * E + e] += __popc(peers);
+            __syncwarp();
+        }
     }
 }
 
@@ -362,12 +395,13 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
                                                      int32_t *__restrict__ poff, int32_t *__restrict__ num_mtiles,
                                                      int4 *__restrict__ mtiles, int32_t *__restrict__ num_pairs,
                                                      int2 *__restrict__ pairs, int32_t *__restrict__ ready,
-                                                     int32_t *__restrict__ inv, int32_t *__restrict__ err)
+                                                     int32_t *__restrict__ inv, int32_t *__restrict__ yrow,
+                                                     int32_t *__restrict__ err)
 {
     extern __shared__ int32_t sm[];
     pdl_wait();
     pdl_trigger();
-    route_block(ids, R, E, counts, off, poff, num_mtiles, mtiles, num_pairs, pairs, ready, inv, err, sm);
+    route_block(ids, R, E, counts, off, poff, num_mtiles, mtiles, num_pairs, pairs, ready, inv, yrow, err, sm);
 }
 
 // Raises a kernel's dynamic shared-memory limit once per device.
@@ -386,29 +420,29 @@ static cudaError_t allow_smem(K kernel, int bytes, int *done_device)
 
 cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
                          int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *ready,
-                         int32_t *inv, int32_t *err, cudaStream_t s)
+                         int32_t *inv, int32_t *yrow, int32_t *err, cudaStream_t s)
 {
-    const size_t smem = sizeof(int32_t) * (33 * static_cast<size_t>(E));
+    const size_t smem = sizeof(int32_t) * (34 * static_cast<size_t>(E));
     static int attr_device = -1;
-    cudaError_t e = allow_smem(route_kernel, 33 * 1024 * 4, &attr_device);
+    cudaError_t e = allow_smem(route_kernel, 34 * 1024 * 4, &attr_device);
     if (e != cudaSuccess)
         return e;
     return launch_pdl(route_kernel, dim3(1), dim3(1024), smem, s, ids, static_cast<int>(R), E, counts, off, poff,
-                      num_mtiles, mtiles, num_pairs, pairs, ready, inv, err);
+                      num_mtiles, mtiles, num_pairs, pairs, ready, inv, yrow, err);
 }
 
 // ------------------------------------------------------------ combine
-// out[t] = bf16( sum_{j ascending} w[t,j] * y[row(t,j)] ) in fp32, where
-// row(t,j) is the slot's row in the unpadded expert-major y buffer.  One
-// block per (token, 1024-column chunk), 8 bf16 (16 bytes) per thread.
-constexpr int kCombineChunk = 1024;
+// out[t] = bf16( sum_{j ascending} w[t,j] * y[yrow[t*k+j]] ) in fp32, where
+// yrow is the slot's row in the unpadded expert-major y buffer (-1: skipped).
+// One block per (token, 2048-column chunk); each thread owns 8 columns (16
+// bytes) and issues the loads of four slots before accumulating them in order.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineCols = 8 * kCombineThreads;
 
-__global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__restrict__ y,
-                                                      const int32_t *__restrict__ inv,
-                                                      const int32_t *__restrict__ ids, const float *__restrict__ w,
-                                                      const int32_t *__restrict__ off,
-                                                      const int32_t *__restrict__ poff, int k, int64_t H,
-                                                      __nv_bfloat16 *__restrict__ out)
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfloat16 *__restrict__ y,
+                                                                  const int32_t *__restrict__ yrow,
+                                                                  const float *__restrict__ w, int k, int64_t H,
+                                                                  __nv_bfloat16 *__restrict__ out)
 {
     __shared__ int64_t s_row[32];
     __shared__ float s_w[32];
@@ -417,51 +451,51 @@ __global__ void __launch_bounds__(128) combine_kernel(const __nv_bfloat16 *__res
     const int64_t t = blockIdx.x;
     if (threadIdx.x < k) {
         const int64_t f = t * k + threadIdx.x;
-        const int p = __ldg(inv + f);
-        int64_t row = -1;
-        if (p >= 0) {
-            const int e = __ldg(ids + f);
-            row = static_cast<int64_t>(p) - __ldg(poff + e) + __ldg(off + e);
-        }
-        s_row[threadIdx.x] = row;
-        s_w[threadIdx.x] = __ldg(w + f);
+        s_row[threadIdx.x] = yrow[f];
+        s_w[threadIdx.x] = w[f];
     }
     __syncthreads();
-    const int64_t c = static_cast<int64_t>(blockIdx.y) * kCombineChunk + static_cast<int64_t>(threadIdx.x) * 8;
-    if (c >= H)
-        return;
-    float acc[8];
+    const int64_t c = static_cast<int64_t>(blockIdx.y) * kCombineCols + static_cast<int64_t>(threadIdx.x) * 8;
+    if (c < H) {
+        float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-        acc[i] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        const int64_t row = s_row[j];
-        if (row < 0)
-            continue;
-        const float wj = s_w[j];
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + row * H + c));
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+        for (int i = 0; i < 8; ++i)
+            acc[i] = 0.0f;
+        for (int j0 = 0; j0 < k; j0 += 4) {
+            uint4 v[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(h[i]);
-            acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wj, f.x));
-            acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wj, f.y));
+            for (int u = 0; u < 4; ++u) {
+                const int64_t row = j0 + u < k ? s_row[j0 + u] : -1;
+                v[u] = row >= 0 ? __ldg(reinterpret_cast<const uint4 *>(y + row * H + c)) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (j0 + u >= k || s_row[j0 + u] < 0)
+                    continue;
+                const float wj = s_w[j0 + u];
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(h[i]);
+                    acc[2 * i] = __fadd_rn(acc[2 * i], __fmul_rn(wj, f.x));
+                    acc[2 * i + 1] = __fadd_rn(acc[2 * i + 1], __fmul_rn(wj, f.y));
+                }
+            }
         }
-    }
-    uint4 o;
-    __nv_bfloat162 *oh = reinterpret_cast<__nv_bfloat162 *>(&o);
+        uint4 o;
+        __nv_bfloat162 *oh = reinterpret_cast<__nv_bfloat162 *>(&o);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        oh[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-    *reinterpret_cast<uint4 *>(out + t * H + c) = o;
+        for (int i = 0; i < 4; ++i)
+            oh[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        *reinterpret_cast<uint4 *>(out + t * H + c) = o;
+    }
 }
 
-cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *inv, const int32_t *ids, const float *w,
-                           const int32_t *off, const int32_t *poff, int64_t T, int k, int64_t H,
+cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *yrow, const float *w, int64_t T, int k, int64_t H,
                            __nv_bfloat16 *out, cudaStream_t s)
 {
-    const dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>((H + kCombineChunk - 1) / kCombineChunk));
-    return launch_pdl(combine_kernel, grid, dim3(128), 0, s, y, inv, ids, w, off, poff, k, H, out);
+    const dim3 grid(static_cast<unsigned>(T), static_cast<unsigned>((H + kCombineCols - 1) / kCombineCols));
+    return launch_pdl(combine_kernel, grid, dim3(kCombineThreads), 0, s, y, yrow, w, k, H, out);
 }
 
 // ------------------------------------------------------------ warmup scales
