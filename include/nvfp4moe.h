@@ -74,6 +74,12 @@ const char *nvfp4_status_string(int status);
  * gs_out is also used as the reduction's scratch word.  n >= 1. */
 int nvfp4_global_scale(const uint16_t *x, int64_t n, float *gs_out, void *stream);
 
+/* max|x| of a bf16 tensor: x [n] bf16; amax_out: device float (also the
+ * reduction's scratch word).  n >= 1.  The global scale of a tensor split
+ * over several devices is 2688 / (max over the devices of this value), as
+ * for one tensor. */
+int nvfp4_amax(const uint16_t *x, int64_t n, float *amax_out, void *stream);
+
 /* Bytes needed for the scales of a [rows, cols] NVFP4 tensor in a layout. */
 int64_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int scale_layout);
 

@@ -18,7 +18,7 @@ __all__ = [
     "nvfp4_swizzle_scales", "nvfp4_gemm", "nvfp4_moe_workspace_size", "nvfp4_moe_forward",
     "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
-    "nvfp4_moe_get_error", "nvfp4_moe_topk", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan",
+    "nvfp4_moe_get_error", "nvfp4_moe_topk", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax",
     "MoeArgs",
 ]
 
@@ -76,6 +76,7 @@ def lib():
                                                  ctypes.POINTER(i64), ctypes.POINTER(i64)]
         L.nvfp4_moe_get_error.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.nvfp4_moe_topk.argtypes = [P, i64, i32, i32, i32, P, P, P]
+        L.nvfp4_amax.argtypes = [P, i64, P, P]
         L.nvfp4_fp4_mma_ceiling.argtypes = [i32, i32, i32, P, P, P]
         L.nvfp4_moe_plan.argtypes = [i64, i32, i32, i64, i64, ctypes.POINTER(ctypes.c_int32),
                                      ctypes.POINTER(ctypes.c_int32)]
@@ -266,3 +267,9 @@ def nvfp4_moe_plan(T, k, E, H, I):
     f, pt = ctypes.c_int32(), ctypes.c_int32()
     _check(lib().nvfp4_moe_plan(T, k, E, H, I, ctypes.byref(f), ctypes.byref(pt)), "nvfp4_moe_plan")
     return bool(f.value), bool(pt.value)
+
+
+def nvfp4_amax(x, amax_out, stream=None):
+    """amax_out (device float [1]) = max|x| of a bf16 CUDA tensor."""
+    _check(lib().nvfp4_amax(_dev(x, "x", torch.bfloat16), x.numel(), _dev(amax_out, "amax_out", torch.float32),
+                            _stream(stream)), "nvfp4_amax")

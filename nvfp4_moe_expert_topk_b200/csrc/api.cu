@@ -376,6 +376,20 @@ int nvfp4_global_scale(const uint16_t *x, int64_t n, float *gs_out, void *stream
     return cuda_status(launch_finalize_gs(gs_out, s));
 }
 
+int nvfp4_amax(const uint16_t *x, int64_t n, float *amax_out, void *stream)
+{
+    if (x == nullptr || amax_out == nullptr || n < 1)
+        return NVFP4_ERR_INVALID_ARG;
+    int sms = 0;
+    int st = device_check(&sms);
+    if (st != NVFP4_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(amax_out, 0, sizeof(float), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    return cuda_status(launch_amax_bf16(reinterpret_cast<const __nv_bfloat16 *>(x), n, amax_out, sms, s));
+}
+
 int64_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int scale_layout)
 {
     if (rows < 0 || cols < 0 || cols % 16 != 0)

@@ -1,0 +1,101 @@
+"""Expert parallelism on two gloo ranks (CPU): each rank owns half of the
+experts and its own batch; the dispatch / per-rank experts / combine result
+equals the single-process oracle on the union batch with the union's global
+scale.  The per-rank expert computation here is the oracle (the library runs
+only on a GPU); the exchange logic is the product's (ep.py)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle as O
+from helpers import OracleWeights
+from nvfp4_moe_expert_topk_b200 import workloads as W
+from nvfp4_moe_expert_topk_b200.ep import ExpertParallelMoE, global_scale_from_amax
+
+CFG = W.MoeConfig("ep_tiny", E=8, k=2, T=48, H=256, I=128, routing="softmax", outliers=False, warmup_T=64)
+WORLD = 2
+
+
+def rank_batch(r, scenario):
+    x = W.activations(CFG.T + 8 * r, CFG.H, seed=100 + r)     # ranks hold different batch sizes
+    ids, w = W.routing(CFG, CFG.T + 8 * r, seed=200 + r)
+    if scenario == "one_sided":                                # every slot on rank 0's experts
+        ids = ids % (CFG.E // WORLD)
+    if scenario == "skips":
+        ids[::5, 1] = -1                                       # skipped slots travel as -1
+    return x, ids, w
+
+
+def inter_gs_all():
+    xw, idw, ww = W.batch(CFG, warmup=True)
+    ow = OracleWeights(CFG, range(CFG.E), "cpu")
+    xb = W.bf16_bits(xw)
+    _, inter = O.moe_forward(xb, idw.numpy(), ww.numpy(), O.global_scale_bf16(xb), **ow.oracle_kwargs(),
+                             inter_gs=None, intermediates=True)
+    amax = inter["h_amax"]
+    return np.array([O.global_scale_from_amax(a if a > 0 else amax.max()) for a in amax], np.float32)
+
+
+def worker(rank, port, scenario):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    try:
+        El = CFG.E // WORLD
+        local = list(range(rank * El, (rank + 1) * El))
+        ow = OracleWeights(CFG, local, "cpu")
+        igs = inter_gs_all()
+
+        def experts_fn(x, local_ids, w, gs):
+            out = O.moe_forward(W.bf16_bits(x), local_ids.numpy(), w.numpy(), gs, **ow.oracle_kwargs(),
+                                inter_gs=igs[local])
+            return torch.from_numpy(out)
+
+        ep = ExpertParallelMoE(CFG.E, amax_fn=lambda x: O.amax_bf16(W.bf16_bits(x)), experts_fn=experts_fn)
+        x, ids, w = rank_batch(rank, scenario)
+        got = ep.forward(x, ids, w, out_dtype=torch.float32).numpy()
+
+        # reference: one process, all experts, the union batch
+        xs, idss, ws = zip(*(rank_batch(r, scenario) for r in range(WORLD)))
+        xu, idu, wu = torch.cat(xs), torch.cat(idss), torch.cat(ws)
+        gs = global_scale_from_amax(max(O.amax_bf16(W.bf16_bits(xr)) for xr in xs))
+        assert gs == O.global_scale_bf16(W.bf16_bits(xu))
+        owa = OracleWeights(CFG, range(CFG.E), "cpu")
+        ref = O.moe_forward(W.bf16_bits(xu), idu.numpy(), wu.numpy(), gs, **owa.oracle_kwargs(), inter_gs=igs)
+        lo = sum(CFG.T + 8 * r for r in range(rank))
+        ref = ref[lo:lo + x.shape[0]]
+        scale = np.abs(ref).max()
+        np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6 * scale)
+    finally:
+        dist.destroy_process_group()
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("scenario", ["plain", "one_sided", "skips"])
+def test_expert_parallel_two_ranks(scenario):
+    mp.start_processes(worker, args=(free_port(), scenario), nprocs=WORLD, start_method="spawn")
+
+
+def test_plan_rewrites_ids_per_rank():
+    """The dispatch plan on its own: each destination gets exactly the tokens
+    with a slot there, ids rewritten to that rank's local range, -1 elsewhere."""
+    class Fake(ExpertParallelMoE):
+        def __init__(self):
+            self.world, self.rank, self.E, self.El = 4, 0, 16, 4
+    ids = torch.tensor([[0, 5], [15, 14], [-1, 3], [8, 9]])
+    tokens, local = Fake().plan(ids)
+    assert [t.tolist() for t in tokens] == [[0, 2], [0], [3], [1]]
+    assert local[0].tolist() == [[0, -1], [-1, 3]]
+    assert local[1].tolist() == [[-1, 1]]
+    assert local[2].tolist() == [[0, 1]]
+    assert local[3].tolist() == [[3, 2]]
