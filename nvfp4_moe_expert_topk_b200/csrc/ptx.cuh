@@ -1,6 +1,6 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA / bulk
-// copies, and the tcgen05 tensor-core family (TMEM alloc, scale-factor copy,
-// block-scaled FP4 MMA, TMEM loads).  Descriptor bit layouts follow the
+// copies, and the tcgen05 tensor-core family (TMEM alloc, block-scaled FP4
+// MMA, TMEM loads and stores).  Descriptor bit layouts follow the
 // public PTX ISA (shared-memory matrix descriptor, instruction descriptor for
 // kind::mxf4nvf4) as mirrored by the CUTLASS sm100 headers.
 #pragma once
@@ -164,7 +164,7 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
 }
 
 // Makes this thread's generic-proxy shared-memory writes visible to later
-// async-proxy reads (TMA stores, tcgen05.cp / tcgen05.mma operands).
+// async-proxy reads (TMA stores, tcgen05.mma operands).
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -236,13 +236,6 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar, uint16_t cta_mask)
             smem_u32(bar)),
         "h"(cta_mask)
         : "memory");
-}
-
-// Copies a 32-row x 16-byte block from shared memory into TMEM lanes 0-31 at
-// column taddr..taddr+3, replicated into the other three lane quarters.
-__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc)
-{
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // D[tmem] (+)= (A * sfA) x (B * sfB)^T, A/B E2M1 in shared memory, one E4M3
@@ -318,17 +311,6 @@ __device__ __forceinline__ uint64_t sdesc_kmajor_sw128(uint32_t saddr)
     d |= static_cast<uint64_t>(1024 >> 4) << 32;         // stride byte offset
     d |= static_cast<uint64_t>(1) << 46;                 // descriptor version
     d |= static_cast<uint64_t>(2) << 61;                 // SWIZZLE_128B
-    return d;
-}
-
-// Descriptor of a 32-row x 16-byte scale block for tcgen05.cp: no swizzle,
-// 8-row core matrices of 16-byte rows, 128 bytes apart.
-__device__ __forceinline__ uint64_t sdesc_scale_block(uint32_t saddr)
-{
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(128 >> 4) << 32;
-    d |= static_cast<uint64_t>(1) << 46;
     return d;
 }
 
