@@ -347,3 +347,35 @@ def test_forward_computes_batch_global_scale(tiny):
     gs = ws[o:o + n].cpu().numpy().view(np.float32)[0]
     assert gs == O.global_scale_bf16(W.bf16_bits(p.x)) == p.x_gs
     assert torch.equal(out, ref_out)
+
+
+EDGE = [
+    W.MoeConfig("one_token", E=8, k=2, T=1, H=256, I=128, routing="softmax", outliers=False, warmup_T=64),
+    W.MoeConfig("top32", E=64, k=32, T=16, H=256, I=128, routing="sigmoid", outliers=False, warmup_T=64),
+    W.MoeConfig("e1024", E=1024, k=4, T=24, H=256, I=128, routing="softmax", outliers=True, warmup_T=64),
+]
+
+
+@pytest.mark.parametrize("cfg", EDGE, ids=[c.name for c in EDGE])
+def test_edge_shapes_end_to_end(cfg):
+    """One token; the largest top-k (32); the largest expert count (1024,
+    most experts empty): the whole output against the oracle."""
+    p = Problem(cfg)
+    out, ws = p.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    check_output(out, p.oracle())
+
+
+def test_prefill_pure_zipf_sampled_tokens():
+    """The prefill batch with pure Zipf popularity (no empty expert, the
+    heaviest expert ~3100 rows): sampled tokens through the oracle."""
+    cfg = W.MOE_CONFIGS["prefill_zipf_pure"]
+    tokens = np.sort(np.random.default_rng(1).choice(cfg.T, 4, replace=False))
+    p = Problem(cfg, oracle_tokens=tokens)
+    route = O.route(p.ids.numpy(), cfg.E)
+    assert (route["counts"] == 0).sum() == 0
+    out, ws = p.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    ref = O.moe_forward(W.bf16_bits(p.x[tokens]), p.ow.remap_ids(p.ids.numpy()[tokens]), p.w.numpy()[tokens],
+                        p.x_gs, **p.ow.oracle_kwargs(), inter_gs=p.inter_gs[p.ow.experts])
+    check_output(out[torch.from_numpy(tokens).to(DEV)], ref)
