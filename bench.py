@@ -332,38 +332,70 @@ def time_steps(wl, steps, warmup, world, graph=True, tag="timed"):
 
 
 def time_e2e(wl, steps, warmup, world):
-    """Same step through the public API from pinned host buffers: H2D of x,
-    ids and weights, the step, D2H of the output, all inside the timed region."""
-    stream = torch.cuda.current_stream()
+    """The step through the public API from pinned host buffers, as a serving
+    loop issues it: every step copies its x, ids and weights host -> device,
+    runs nvfp4_moe_forward and copies its output device -> host, all inside
+    the timed region.  Copies run on their own streams into two alternating
+    device buffer sets, so step i+1's inputs upload and step i-1's output
+    downloads while step i computes; events order each buffer's reuse."""
+    dev = wl.x.device
+    compute = torch.cuda.Stream(dev)
+    up = torch.cuda.Stream(dev)
+    down = torch.cuda.Stream(dev)
     hx = wl.x_cpu.pin_memory()
     hids = wl.ids_cpu.pin_memory()
     hw = wl.w_cpu.pin_memory()
-    hout = torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True)
+    bufs = [dict(x=torch.empty_like(wl.x), ids=torch.empty_like(wl.ids), w=torch.empty_like(wl.w),
+                 out=torch.empty_like(wl.out)) for _ in range(2)]
+    houts = [torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True) for _ in range(2)]
+    n_all = warmup + steps
+    ev = [{k: torch.cuda.Event() for k in ("in", "done", "down")} for _ in range(n_all)]
 
-    def one():
-        wl.x.copy_(hx, non_blocking=True)
-        wl.ids.copy_(hids, non_blocking=True)
-        wl.w.copy_(hw, non_blocking=True)
-        wl.step()
-        hout.copy_(wl.out, non_blocking=True)
+    def issue(i):
+        b, e = bufs[i % 2], ev[i]
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(ev[i - 2]["done"])        # the forward two steps back has read this buffer set
+            b["x"].copy_(hx, non_blocking=True)
+            b["ids"].copy_(hids, non_blocking=True)
+            b["w"].copy_(hw, non_blocking=True)
+            e["in"].record(up)
+        with torch.cuda.stream(compute):
+            compute.wait_event(e["in"])
+            if i >= 2:
+                compute.wait_event(ev[i - 2]["down"])   # its output has left the device
+            nvfp4_moe_forward(b["x"], b["ids"], b["w"], None, **wl.weights.args(), inter_gs=wl.inter_gs,
+                              out=b["out"], workspace=wl.ws, stream=compute)
+            e["done"].record(compute)
+        with torch.cuda.stream(down):
+            down.wait_event(e["done"])
+            houts[i % 2].copy_(b["out"], non_blocking=True)
+            e["down"].record(down)
 
-    for _ in range(warmup):
-        one()
+    for i in range(warmup):
+        issue(i)
+    torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        one()
-    t1.record(stream)
+    t0.record(up)
+    compute.wait_event(t0)
+    down.wait_event(t0)
+    for i in range(warmup, n_all):
+        issue(i)
+    up.wait_stream(down)
+    up.wait_stream(compute)
+    t1.record(up)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(world, t0.elapsed_time(t1))
     h2d = hx.numel() * hx.element_size() + hids.numel() * 4 + hw.numel() * 4
-    d2h = hout.numel() * hout.element_size()
-    if not torch.isfinite(hout.float()).all():
+    d2h = houts[0].numel() * houts[0].element_size()
+    if not torch.isfinite(houts[(n_all - 1) % 2].float()).all():
         raise RuntimeError("non-finite output in the end-to-end run")
+    if not torch.equal(houts[(n_all - 1) % 2], bufs[(n_all - 1) % 2]["out"].cpu()):
+        raise RuntimeError("end-to-end output differs from the device result")
     return ms, h2d, d2h
 
 
