@@ -21,6 +21,7 @@ cores on a bounded sample of the same workload (rank 0 only).
 """
 import argparse
 import hashlib
+import re
 import json
 import os
 import subprocess
@@ -60,10 +61,15 @@ def load_peaks():
 
 
 def gemm_source_sha():
+    """Hash of the GEMM sources' code, comments and layout whitespace removed
+    (a comment edit does not invalidate the captured traffic)."""
     h = hashlib.sha256()
     for name in GEMM_SOURCES:
-        with open(os.path.join(ROOT, "nvfp4_moe_expert_topk_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "nvfp4_moe_expert_topk_b200", "csrc", name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -22,10 +22,11 @@
 //             stage's sf_ready barrier (copying scales through the tensor
 //             pipe with tcgen05.cp costs more pipe time than the MMAs);
 //   warp 1    allocates TMEM; one thread issues the 4 tcgen05.mma (K=64) of
-//             each k-tile; the block-scaled FP4 MMA costs about the same pipe
-//             time per instruction at N=128 as at N=256, so tiles are 256 wide;
+//             each k-tile once the stage's sf_ready barrier completes (which
+//             implies its operand copies landed); tiles are 256 wide, which
+//             halves the A bytes filled per FLOP against 128-wide tiles;
 //   warps 2-9 epilogue, two per TMEM lane quarter (each owns one row of the
-//             tile and half of its columns): TMEM -> registers with one wait,
+//             tile and half of its columns): TMEM -> registers in two waits,
 //             release the accumulator to the MMA thread at once (the next
 //             tile's MMAs wait only for this drain), then one of
 //             EPI_SWIGLU_QUANT  h = SiLU(a_g*g) * (a_u*u), NVFP4-quantised
@@ -41,7 +42,11 @@
 // m-tile table written on the device by the routing kernel (expert, first
 // padded row, valid rows, first output row), so the launch needs no host
 // sync and every expert's rows are covered by one tensor map over the padded
-// A buffer and one over all experts' stacked weights.
+// A buffer and one over all experts' stacked weights.  Two variants of the
+// same engine: pair tiles (CG = 2, clusters of two CTAs issuing
+// cta_group::2 MMAs on 256-row tiles) and the fused grouped launch
+// (FUSED = 1, every L1 tile then every L2 tile, L2 tiles gated per m-tile on
+// counters the L1 epilogues publish).  See the template's comment.
 //
 // Every mbarrier wait is bounded (ptx.cuh): on a timeout the block records
 // NVFP4_ERR_TIMEOUT in the error word, stops issuing, waits (bounded) for its
