@@ -209,6 +209,13 @@ int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, in
 #define NVFP4_NOALLOC_SCRATCH_BYTES (32u << 20)
 int nvfp4_moe_forward_noalloc(const nvfp4_moe_args *args, void *stream);
 
+/* Failure detection check (no counterpart on the pages): launches one
+ * thread that runs the fused launch's bounded device wait -- until the
+ * device int *flag >= target -- and, when the wait gives up (after 2 s),
+ * writes NVFP4_ERR_TIMEOUT into the device int *err if it is still 0.  No
+ * fault and no trap: the context stays usable.  flag, err: device pointers. */
+int nvfp4_debug_bounded_wait(const int32_t *flag, int32_t target, int32_t *err, void *stream);
+
 /* Execution plan nvfp4_moe_forward uses for a shape (host only, no GPU
  * work): *fused_l1_l2 = 1 when L1 and L2 run as one persistent launch (the
  * L2 tiles of an m-tile start as soon as that m-tile's L1 tiles have written

@@ -18,7 +18,7 @@ __all__ = [
     "nvfp4_swizzle_scales", "nvfp4_gemm", "nvfp4_moe_workspace_size", "nvfp4_moe_forward",
     "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
-    "nvfp4_moe_get_error", "nvfp4_moe_topk", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax",
+    "nvfp4_moe_get_error", "nvfp4_moe_topk", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax", "nvfp4_debug_bounded_wait",
     "MoeArgs",
 ]
 
@@ -77,6 +77,7 @@ def lib():
         L.nvfp4_moe_get_error.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.nvfp4_moe_topk.argtypes = [P, i64, i32, i32, i32, P, P, P]
         L.nvfp4_amax.argtypes = [P, i64, P, P]
+        L.nvfp4_debug_bounded_wait.argtypes = [P, i32, P, P]
         L.nvfp4_fp4_mma_ceiling.argtypes = [i32, i32, i32, P, P, P]
         L.nvfp4_moe_plan.argtypes = [i64, i32, i32, i64, i64, ctypes.POINTER(ctypes.c_int32),
                                      ctypes.POINTER(ctypes.c_int32)]
@@ -273,3 +274,11 @@ def nvfp4_amax(x, amax_out, stream=None):
     """amax_out (device float [1]) = max|x| of a bf16 CUDA tensor."""
     _check(lib().nvfp4_amax(_dev(x, "x", torch.bfloat16), x.numel(), _dev(amax_out, "amax_out", torch.float32),
                             _stream(stream)), "nvfp4_amax")
+
+
+def nvfp4_debug_bounded_wait(flag, target, err, stream=None):
+    """Runs the fused launch's bounded device wait on flag (int32 [1], device)
+    until flag >= target; err (int32 [1], device) receives NVFP4_ERR_TIMEOUT
+    if the wait gives up (after 2 s)."""
+    _check(lib().nvfp4_debug_bounded_wait(_dev(flag, "flag", torch.int32), target, _dev(err, "err", torch.int32),
+                                          _stream(stream)), "nvfp4_debug_bounded_wait")

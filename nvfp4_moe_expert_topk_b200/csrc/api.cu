@@ -595,6 +595,16 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
     return mark(events, 5, s);
 }
 
+int nvfp4_debug_bounded_wait(const int32_t *flag, int32_t target, int32_t *err, void *stream)
+{
+    if (flag == nullptr || err == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    int st = device_check(nullptr);
+    if (st != NVFP4_OK)
+        return st;
+    return cuda_status(launch_wait_probe(flag, target, err, static_cast<cudaStream_t>(stream)));
+}
+
 int nvfp4_moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int32_t *fused_l1_l2, int32_t *pair_tiles)
 {
     if (fused_l1_l2 == nullptr || pair_tiles == nullptr)

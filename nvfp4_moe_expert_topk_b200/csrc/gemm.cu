@@ -207,6 +207,24 @@ __device__ __forceinline__ bool wait_counter(const int32_t *ctr, int target, vol
     return false;
 }
 
+// The fused launch's counter wait on its own: one thread waits until *flag
+// >= target, or gives up after the bound and records NVFP4_ERR_TIMEOUT.
+__global__ void wait_probe_kernel(const int32_t *flag, int target, int32_t *err)
+{
+    __shared__ int no_abort;
+    if (threadIdx.x == 0) {
+        no_abort = 0;
+        if (!wait_counter(flag, target, &no_abort))
+            record_error(err, NVFP4_ERR_TIMEOUT);
+    }
+}
+
+cudaError_t launch_wait_probe(const int32_t *flag, int target, int32_t *err, cudaStream_t s)
+{
+    wait_probe_kernel<<<1, 32, 0, s>>>(flag, target, err);
+    return cudaGetLastError();
+}
+
 // FUSED = 1 (grouped, CG = 1, BN = 256): one persistent launch runs the L1
 // tiles (arguments p, maps map_a / map_a32 / map_b, SwiGLU + re-quantisation
 // epilogue) and then the L2 tiles (p2, map_a2 / map_a2_32 / map_b2, bf16

@@ -80,6 +80,8 @@ enum Epilogue { EPI_SWIGLU_QUANT = 0, EPI_BF16 = 1, EPI_SWIGLU_AMAX = 2 };
 // bytes wide with 128-byte swizzle.
 cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
                         const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream);
+// One bounded counter wait (the fused launch's) in a one-thread kernel.
+cudaError_t launch_wait_probe(const int32_t *flag, int target, int32_t *err, cudaStream_t s);
 // Pair clusters that fit on the device at once (<= num_sms / 2).
 int gemm_pair_clusters(int num_sms);
 // One persistent cooperative launch of the grouped L1 (args1, maps *1, SwiGLU

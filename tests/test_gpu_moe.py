@@ -379,3 +379,27 @@ def test_prefill_pure_zipf_sampled_tokens():
     ref = O.moe_forward(W.bf16_bits(p.x[tokens]), p.ow.remap_ids(p.ids.numpy()[tokens]), p.w.numpy()[tokens],
                         p.x_gs, **p.ow.oracle_kwargs(), inter_gs=p.inter_gs[p.ow.experts])
     check_output(out[torch.from_numpy(tokens).to(DEV)], ref)
+
+
+def test_bounded_wait_times_out_and_context_survives(tiny):
+    """Failure detection without a fault: the fused launch's device wait on a
+    counter that nothing raises gives up after its bound and reports
+    NVFP4_ERR_TIMEOUT; a satisfied wait reports nothing; the context is still
+    usable afterwards (a forward matches the oracle)."""
+    import time
+    from nvfp4_moe_expert_topk_b200 import nvfp4_debug_bounded_wait
+    flag = torch.zeros(1, dtype=torch.int32, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    t0 = time.perf_counter()
+    nvfp4_debug_bounded_wait(flag, 1, err)
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    assert err.item() == -7 and 1.5 < waited < 30.0
+    flag.fill_(3)
+    err.zero_()
+    nvfp4_debug_bounded_wait(flag, 3, err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    out, ws = tiny.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    check_output(out, tiny.oracle())
