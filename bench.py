@@ -497,11 +497,11 @@ def time_variant_routing(wl, cfg, steps, warmup, world):
             "m_tiles": int(np.ceil(counts / 128).sum()), "stage_ms": stages}
 
 
-def time_shared(dev, steps, warmup, flush):
-    """The shared-expert config (one expert, 256 tokens: 37 MB of weights,
-    which fit in L2): hot (back-to-back steps) and cold (L2 flushed before
-    every step), CUDA-graph timed."""
-    wl = Workload(W.MOE_CONFIGS["shared"], dev)
+def time_shared(dev, steps, warmup, flush, name="shared"):
+    """A config whose weights fit in L2 -- the shared expert (one expert, 256
+    tokens, 37 MB of weights) or the tiny MoE (0.4 MB): hot (back-to-back
+    steps) and cold (L2 flushed before every step), CUDA-graph timed."""
+    wl = Workload(W.MOE_CONFIGS[name], dev)
     hot, = graph_time([wl.step], steps, warmup)
     cold, = graph_time([wl.step], steps, 0, flush)
     if nvfp4_moe_get_error(wl.ws) != 0:
@@ -713,6 +713,7 @@ def run_ours(args):
     router = time_router(pre.cfg, dev, 50, warmup, flush)
     pure = time_variant_routing(pre, W.MOE_CONFIGS["prefill_zipf_pure"], min(steps, 50), warmup, world)
     shared = time_shared(dev, min(steps, 50), warmup, flush)
+    tiny = time_shared(dev, min(steps, 50), warmup, flush, name="tiny")
 
     t_step = ms_pre / steps / 1e3
     tokens_s = world * pre.cfg.T / t_step
@@ -774,6 +775,7 @@ def run_ours(args):
         "router": router,
         "prefill_pure_zipf": pure,
         "shared_expert": shared,
+        "tiny_moe": tiny,
         "gpu_launches": (pre.launches_per_step + dec.launches_per_step) * steps,
         "clocks": clocks.summary(),
     }
