@@ -549,7 +549,8 @@ def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
     Device times from CUDA events inside a CUDA graph; the GEMM alone is
     bracketed separately, hot (operands as the quantiser left them, weights
     L2-resident where they fit) and cold (after a 512 MB L2 flush)."""
-    from nvfp4_moe_expert_topk_b200 import (NVFP4_SCALES_MMA, nvfp4_gemm, nvfp4_quantize, nvfp4_scales_bytes)
+    from nvfp4_moe_expert_topk_b200 import (NVFP4_SCALES_MMA, nvfp4_gemm_workspace_size, nvfp4_gemm_ws,
+                                            nvfp4_quantize, nvfp4_scales_bytes)
     res = {}
     fp4_peak = peaks["bf16_tflops_sustained"] * BF16_TO_FP4_NOMINAL_RATIO
     ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -578,8 +579,11 @@ def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
             nvfp4_global_scale(ad, a_gs)
             nvfp4_quantize(ad, a_gs, a_codes, a_sc, NVFP4_SCALES_MMA)
 
+        nbytes = nvfp4_gemm_workspace_size(M, N, K)     # > 0: stream-K split over the SMs
+        gws = torch.zeros(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+
         def gemm():
-            nvfp4_gemm(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out)
+            nvfp4_gemm_ws(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out, gws)
 
         quant_ms, gemm_ms = graph_time([quant, gemm], steps, warmup)
         _, gemm_cold_ms = graph_time([quant, gemm], steps, 0, flush)
@@ -590,14 +594,15 @@ def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
         tflops = flops / (gemm_ms * 1e-3) / 1e12
         gbs = gbytes / (gemm_ms * 1e-3) / 1e9
         bound = "tensor" if ai >= ridge else "hbm"
-        res[name] = {"M": M, "N": N, "K": K, "ms_per_step": step_ms, "gemm_ms": gemm_ms, "tflops": tflops,
+        res[name] = {"M": M, "N": N, "K": K, "stream_k": bool(nbytes), "ms_per_step": step_ms, "gemm_ms": gemm_ms,
+                     "tflops": tflops,
                      "gemm_ms_cold": gemm_cold_ms, "tflops_cold": flops / (gemm_cold_ms * 1e-3) / 1e12,
                      "gbs": gbs, "arith_intensity": ai, "bound": bound,
                      "frac": (tflops / fp4_peak) if bound == "tensor" else (gbs / peaks["hbm_gbs"]),
                      "fp4_nominal_frac": tflops / FP4_NOMINAL_TFLOPS}
         if ceiling_tflops:
             res[name]["fp4_ceiling_frac"] = tflops / ceiling_tflops
-        del ad, a_codes, a_sc, out, w_codes, w_sc
+        del ad, a_codes, a_sc, out, w_codes, w_sc, gws
         torch.cuda.empty_cache()
     return res
 
