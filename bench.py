@@ -209,12 +209,12 @@ class Workload:
         self.rows = int(counts.sum())
         self.nonempty = int((counts > 0).sum())
         self.fused, self.pair_tiles = nvfp4_moe_plan(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I)
-        # global scale (amax + finalize), route, quantise, L1 + L2 (one launch or two), combine
-        self.launches_per_step = 6 if self.fused else 7
+        # global scale, route, quantise, L1 + L2 (one launch or two), combine
+        self.launches_per_step = 5 if self.fused else 6
 
     def fold(self, per_stage):
         """Per-stage figures keyed by the stages the forward runs: the front
-        (global scale of the batch, routing, quantise+permute: four small
+        (global scale of the batch, routing, quantise+permute: three small
         launches), the GEMMs (with the fused plan L1 and L2 are one launch,
         whose time sits in the L1 slot of the timed forward, the L2 slot being
         empty) and the combine."""

@@ -167,7 +167,7 @@ size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
  * Expert_e(x) = W2_e . q(SiLU(W13g_e . q(x)) * (W13u_e . q(x))), all GEMMs
  * in NVFP4 on the tensor cores, q() the NVFP4 quantiser (x with x_gs, h with
  * inter_gs[e]).  Launches on `stream`: the global scale of x when x_gs is
- * NULL (a 4-byte memset of the workspace and two kernels), routing,
+ * NULL (an 8-byte memset of the workspace and one kernel), routing,
  * quantise+permute, L1 (fused SiLU*up re-quantise epilogue) and L2 (one fused
  * launch or two, see nvfp4_moe_plan) and the combine; no host sync, no
  * allocation, so the call can be captured in a CUDA graph (make one eager

@@ -94,7 +94,8 @@ struct Layout {
 };
 
 // Header (256 B): int32 error word at 0, int32 m-tile count at 4, int32
-// m-tile pair count at 8, fp32 global scale of x computed from the batch at 12.
+// m-tile pair count at 8, fp32 global scale of x computed from the batch at
+// 12 and its completion ticket at 16.
 Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
 {
     Layout L;
@@ -302,10 +303,12 @@ int run_route_quant(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, void 
     if (mark(events, 0, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
     if (a->x_gs == nullptr) {
+        // the batch's global scale at ws + 12 (amax, then 2688 / amax by the
+        // last block to finish), its completion ticket at ws + 16
         float *gs = reinterpret_cast<float *>(ws + 12);
-        if (cudaMemsetAsync(gs, 0, sizeof(float), s) != cudaSuccess ||
-            launch_amax_bf16(reinterpret_cast<const __nv_bfloat16 *>(a->x), T * H, gs, num_sms, s) != cudaSuccess ||
-            launch_finalize_gs(gs, s) != cudaSuccess)
+        if (cudaMemsetAsync(gs, 0, 2 * sizeof(float), s) != cudaSuccess ||
+            launch_amax_bf16(reinterpret_cast<const __nv_bfloat16 *>(a->x), T * H, gs, num_sms, s,
+                             reinterpret_cast<unsigned int *>(ws + 16)) != cudaSuccess)
             return NVFP4_ERR_CUDA;
     }
     cudaError_t e = launch_route(a->topk_ids, R, E, reinterpret_cast<int32_t *>(ws + L.counts),

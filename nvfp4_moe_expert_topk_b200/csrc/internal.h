@@ -100,7 +100,9 @@ cudaError_t launch_moe_fused(const CUtensorMap &map_a1, const CUtensorMap &map_a
                              const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream);
 
 // Memory-bound kernels (kernels.cu).
-cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s);
+// ticket != nullptr (a zeroed counter): *gs_out ends as 2688 / amax, no finalize launch needed.
+cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s,
+                             unsigned int *ticket = nullptr);
 cudaError_t launch_finalize_gs(float *gs, cudaStream_t s);
 cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs,
                             uint8_t *codes, uint8_t *scales, int layout, const int32_t *inv, int k,

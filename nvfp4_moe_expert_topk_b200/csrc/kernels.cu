@@ -12,8 +12,11 @@ namespace nvfp4 {
 // ------------------------------------------------------------ global scale
 // amax of a bf16 tensor, accumulated into *out_bits (the float bit pattern;
 // non-negative floats order like their bits).  *out_bits must start at 0.
+// With a ticket (a zeroed counter), the last block to finish turns the
+// amax into the global scale in place: 2688 / amax (1 if amax = 0).
 __global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t n,
-                                                        unsigned int *__restrict__ out_bits)
+                                                        unsigned int *__restrict__ out_bits,
+                                                        unsigned int *__restrict__ ticket)
 {
     pdl_wait();
     pdl_trigger();
@@ -54,6 +57,14 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16 *__r
         for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
             m = fmaxf(m, wmax[w]);
         atomicMax(out_bits, __float_as_uint(m));
+        if (ticket != nullptr) {
+            __threadfence();
+            if (atomicAdd(ticket, 1u) == gridDim.x - 1) {     // every block's maximum is in
+                __threadfence();
+                const float a = __uint_as_float(atomicAdd(out_bits, 0u));
+                *reinterpret_cast<float *>(out_bits) = a == 0.0f ? 1.0f : __fdiv_rn(2688.0f, a);
+            }
+        }
     }
 }
 
@@ -66,7 +77,8 @@ __global__ void finalize_gs_kernel(float *gs)
     *gs = (a == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, a);
 }
 
-cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s)
+cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s,
+                             unsigned int *ticket)
 {
     int64_t blocks = (n / 8 + 255) / 256;
     if (blocks < 1)
@@ -74,7 +86,7 @@ cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, i
     if (blocks > 8LL * num_sms)
         blocks = 8LL * num_sms;
     return launch_pdl(amax_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, n,
-                      reinterpret_cast<unsigned int *>(gs_out));
+                      reinterpret_cast<unsigned int *>(gs_out), ticket);
 }
 
 cudaError_t launch_finalize_gs(float *gs, cudaStream_t s)
