@@ -293,7 +293,8 @@ int l2_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int bn, CUte
 // between 0 and 1, quantisation between 1 and 2).  Shared by forward and
 // calibrate.  (A single cooperative launch of all three, with a grid barrier
 // after the routing and the max|x| pass, measured 5 us slower on the 64-token
-// decode batch than these four small launches, and no faster on prefill.)
+// decode batch than separate launches, and no faster on prefill; so was one
+// launch of routing + quantisation in which every block routes all slots.)
 int run_route_quant(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, void *const *events, cudaStream_t s,
                     int num_sms)
 {
