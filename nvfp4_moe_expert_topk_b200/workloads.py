@@ -44,6 +44,10 @@ class MoeConfig:
     warmup_T: int           # tokens in the warmup batch that fixes inter_gs
     zipf_s: float = 1.1
     zipf_zero_tail: int = 16
+    # the last `shared` of the E experts are shared experts: every token runs
+    # them with weight 1 in its last `shared` of the k slots (the routed
+    # draw picks k - shared of the first E - shared experts)
+    shared: int = 0
 
 
 MOE_CONFIGS = {
@@ -58,6 +62,13 @@ MOE_CONFIGS = {
     # expert-parallel slice: small enough to profile and to check in full
     "prefill_ep48": MoeConfig("prefill_ep48", E=48, k=6, T=512, H=7168, I=3072, routing="zipf", outliers=True,
                               warmup_T=64, zipf_zero_tail=2),
+    # the decode batch with the shared expert folded in as a 49th group
+    # (page 1 "Phase 1": the shared expert is the routed chain with one
+    # expert and no routing; same H and I as a routed expert)
+    "decode_shared": MoeConfig("decode_shared", E=49, k=7, T=64, H=7168, I=3072, routing="sigmoid",
+                               outliers=False, warmup_T=64, shared=1),
+    "tiny_shared": MoeConfig("tiny_shared", E=9, k=3, T=64, H=256, I=128, routing="softmax", outliers=False,
+                             warmup_T=64, shared=1),
 }
 
 
@@ -115,10 +126,19 @@ def zipf_popularity(E: int, s: float, zero_tail: int) -> torch.Tensor:
 
 
 def routing(cfg: MoeConfig, T: Optional[int] = None, seed: int = SEED_ROUTER):
-    """Top-k expert ids [T, k] int32 (descending score) and weights [T, k] fp32."""
+    """Top-k expert ids [T, k] int32 (descending score) and weights [T, k] fp32;
+    with shared experts, the routed slots then one slot per shared expert
+    (id E - shared + i, weight 1)."""
     T = cfg.T if T is None else T
-    g = _gen(seed)
-    E, k = cfg.E, cfg.k
+    ids, w = _routed(cfg, T, _gen(seed), cfg.E - cfg.shared, cfg.k - cfg.shared)
+    if cfg.shared:
+        sid = torch.arange(cfg.E - cfg.shared, cfg.E, dtype=torch.int32).expand(T, cfg.shared)
+        ids = torch.cat([ids, sid], dim=1).contiguous()
+        w = torch.cat([w, torch.ones(T, cfg.shared, dtype=torch.float32)], dim=1).contiguous()
+    return ids, w
+
+
+def _routed(cfg: MoeConfig, T: int, g: torch.Generator, E: int, k: int):
     if cfg.routing == "single":
         return torch.zeros(T, 1, dtype=torch.int32), torch.ones(T, 1, dtype=torch.float32)
     if cfg.routing in ("softmax", "sigmoid"):

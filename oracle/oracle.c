@@ -47,6 +47,15 @@
  *   R8  Warmup: inter_gs[e] = 2688 / max|h| over expert e's warmup rows;
  *       an expert without warmup rows gets 2688 / (max over experts of that
  *       amax); if no expert has rows, 1.
+ *   R12 Router (page 3 "Architecture Notes" names top-6 of 384 but no score
+ *       function): the k largest logits, ties to the lower id, weights the
+ *       selected softmax terms or sigmoids renormalised to sum 1.
+ *   R13 Shared experts folded into the routed chain: rows get k + ns slots,
+ *       slot k + i = expert E + i with weight 1, summed with the routed slots
+ *       as in R7.
+ *   (R9, gate rows first, is stated with the chain above; R10, the packing,
+ *   under Layouts below; R11 concerns how the activation global scale is
+ *   obtained, which the oracle takes as an input.)
  *
  * Layouts (all row-major): codes [rows, cols/2] uint8, element 2i in the low
  * nibble of byte i, element 2i+1 in the high nibble; scales [rows, cols/16]
@@ -492,15 +501,20 @@ int oracle_moe_warmup_inter_gs(const oracle_moe_args *p_in, float *inter_gs_out)
 /* For each token: the k experts with the largest logits, in descending
  * order, ties to the lower expert id (the router's scores -- softmax or
  * sigmoid of the logits -- are increasing functions of the logit, so the
- * same experts).  Weights (R9): scoring 0 = softmax renormalised over the
+ * same experts).  Weights (R12): scoring 0 = softmax renormalised over the
  * selected experts, w_j = exp(l_j) / sum_i exp(l_i); scoring 1 = sigmoid
- * renormalised, w_j = s_j / sum_i s_i.  Evaluated in fp64, stored fp32. */
-void oracle_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *ids, float *w)
+ * renormalised, w_j = s_j / sum_i s_i.  Evaluated in fp64, stored fp32.
+ * R13: with ns shared experts (page 1 "Phase 1": a shared expert is the
+ * routed chain with one expert and no routing), rows hold k + ns slots and slot
+ * k + i is expert E + i with weight 1: every token runs every shared expert
+ * at full weight, as one more group of the routed chain. */
+void oracle_topk_shared(const float *logits, int64_t T, int E, int k, int scoring, int ns, int32_t *ids, float *w)
 {
+    const int ld = k + ns;
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; t++) {
         const float *l = logits + t * E;
-        int32_t *id = ids + t * k;
+        int32_t *id = ids + t * ld;
         for (int j = 0; j < k; j++) {
             int best = -1;
             for (int e = 0; e < E; e++) {
@@ -522,8 +536,17 @@ void oracle_topk(const float *logits, int64_t T, int E, int k, int scoring, int3
             sum += v[j];
         }
         for (int j = 0; j < k; j++)
-            w[t * k + j] = (float)(v[j] / sum);
+            w[t * ld + j] = (float)(v[j] / sum);
+        for (int i = 0; i < ns; i++) {
+            id[k + i] = E + i;
+            w[t * ld + k + i] = 1.0f;
+        }
     }
+}
+
+void oracle_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *ids, float *w)
+{
+    oracle_topk_shared(logits, T, E, k, scoring, 0, ids, w);
 }
 
 int oracle_num_threads(void)

@@ -15,7 +15,9 @@ Parity status of each entry point (what pins it lives in tests/test_oracle_*.py)
   gemm                           pinned (numpy matmul on dequantised operands)
   moe_forward                    pinned (per-token brute force, dense reduction)
   moe_warmup_inter_gs            pinned (brute-force amax of h)
-  topk                           pinned (numpy stable sort, torch softmax / sigmoid)
+  topk                           pinned (numpy stable sort, torch softmax / sigmoid;
+                                 shared slots: the folded chain equals the routed
+                                 chain plus the one-expert dense chain)
 """
 import ctypes
 import os
@@ -73,6 +75,7 @@ def lib():
         L.oracle_moe_warmup_inter_gs.argtypes = [ctypes.POINTER(MoeArgs), P]
         L.oracle_moe_warmup_inter_gs.restype = ctypes.c_int
         L.oracle_topk.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+        L.oracle_topk_shared.argtypes = [P, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
         L.oracle_num_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -246,12 +249,13 @@ def moe_warmup_inter_gs(x_bits, topk_ids, topk_weights, x_gs, w13_codes, w13_sca
     return out
 
 
-def topk(logits: np.ndarray, k: int, scoring: str = "softmax"):
-    """(ids int32 [T, k], weights fp32 [T, k]) from router logits [T, E] fp32."""
+def topk(logits: np.ndarray, k: int, scoring: str = "softmax", num_shared: int = 0):
+    """(ids int32 [T, k + num_shared], weights fp32 [T, k + num_shared]) from
+    router logits [T, E] fp32; slot k + i is shared expert E + i, weight 1."""
     l = _c(logits, np.float32)
     T, E = l.shape
-    assert 1 <= k <= min(E, 32)
-    ids = np.empty((T, k), np.int32)
-    w = np.empty((T, k), np.float32)
-    lib().oracle_topk(_ptr(l), T, E, k, {"softmax": 0, "sigmoid": 1}[scoring], _ptr(ids), _ptr(w))
+    assert 1 <= k <= min(E, 32) and 0 <= num_shared and k + num_shared <= 32
+    ids = np.empty((T, k + num_shared), np.int32)
+    w = np.empty((T, k + num_shared), np.float32)
+    lib().oracle_topk_shared(_ptr(l), T, E, k, {"softmax": 0, "sigmoid": 1}[scoring], num_shared, _ptr(ids), _ptr(w))
     return ids, w

@@ -175,6 +175,36 @@ def test_moe_single_expert_reduces_to_dense_chain():
     np.testing.assert_allclose(out, y, rtol=1e-6, atol=1e-7 * np.abs(y).max())
 
 
+def test_shared_expert_folded_equals_routed_plus_dense_chain():
+    """The shared expert folded in as one more group (reading R13: slot k is
+    expert E with weight 1, ids from the oracle router) gives the routed
+    chain's output plus the shared expert's dense chain (the one-expert
+    reduction pinned above), up to the fp32 rounding of the two partial sums."""
+    P, dims = _tiny_problem(E=5, k=2, T=10, seed=11)
+    E, k, T, H, I = dims
+    Er = E - 1                                            # routed experts 0..3, shared expert 4
+    logits = np.random.default_rng(4).normal(0, 1, (T, Er)).astype(np.float32)
+    ids, w = O.topk(logits, k, "softmax", num_shared=1)
+    assert (ids[:, :k] < Er).all() and (ids[:, k] == Er).all()
+    folded = dict(P, topk_ids=ids, topk_weights=w)
+    inter_gs = O.moe_warmup_inter_gs(**folded)
+    out = O.moe_forward(**folded, inter_gs=inter_gs)
+    routed = O.moe_forward(**dict(P, topk_ids=ids[:, :k].copy(), topk_weights=w[:, :k].copy()), inter_gs=inter_gs)
+    shared = O.moe_forward(**dict(P, topk_ids=ids[:, k:].copy(), topk_weights=w[:, k:].copy()), inter_gs=inter_gs)
+    np.testing.assert_allclose(out, routed.astype(np.float64) + shared, rtol=1e-6,
+                               atol=1e-7 * np.abs(out).max())
+    # the shared part is the dense chain of expert 4 on every token
+    xc, xs = O.quantize_bf16(P["x_bits"], P["x_gs"])
+    G = O.gemm(xc, xs, P["x_gs"], P["w13_codes"][Er], P["w13_scales"][Er], P["w13_gs"][Er], [I, 2 * I])
+    g, u = G[:, :I], G[:, I:]
+    h = (torch.nn.functional.silu(torch.from_numpy(g).double()) * torch.from_numpy(u).double()).float().numpy()
+    hc, hs = O.quantize_f32(h, inter_gs[Er])
+    y = O.gemm(hc, hs, inter_gs[Er], P["w2_codes"][Er], P["w2_scales"][Er], P["w2_gs"][Er:Er + 1])
+    np.testing.assert_allclose(shared, y, rtol=1e-6, atol=1e-7 * np.abs(y).max())
+    # and the shared expert's contribution is not negligible
+    assert np.abs(shared).max() > 0.1 * np.abs(routed).max()
+
+
 def test_moe_skipped_slots_contribute_nothing():
     P, dims = _tiny_problem(seed=7)
     inter_gs = O.moe_warmup_inter_gs(**P)

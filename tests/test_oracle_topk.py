@@ -35,3 +35,18 @@ def test_topk_equals_topk_of_scores():
         ids, _ = O.topk(logits, 6, scoring)
         _, ref = torch.topk(f(torch.from_numpy(logits)), 6, dim=1)
         np.testing.assert_array_equal(ids, ref.numpy())
+
+
+def test_shared_slots_follow_the_routed_ones():
+    """Shared-expert slots (reading R13): the routed slots are unchanged, then
+    slot k + i holds expert E + i with weight exactly 1."""
+    rng = np.random.default_rng(9)
+    logits = rng.normal(0, 1, (40, 48)).astype(np.float32)
+    for scoring in ("softmax", "sigmoid"):
+        ids, w = O.topk(logits, 6, scoring)
+        ids2, w2 = O.topk(logits, 6, scoring, num_shared=2)
+        assert ids2.shape == (40, 8) and w2.shape == (40, 8)
+        np.testing.assert_array_equal(ids2[:, :6], ids)
+        np.testing.assert_array_equal(w2[:, :6], w)
+        assert (ids2[:, 6] == 48).all() and (ids2[:, 7] == 49).all()
+        assert (w2[:, 6:] == 1.0).all()
