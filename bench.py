@@ -513,6 +513,34 @@ def time_shared(dev, steps, warmup, flush, name="shared"):
             "algorithmic_bytes": b}
 
 
+def time_shared_fold(dec, dev, steps, warmup):
+    """The decode batch plus the shared expert, two ways, CUDA-graph timed:
+    folded in as a 49th group of the routed launches (every token's slot 7
+    is the shared expert with weight 1, as nvfp4_moe_topk_shared writes it),
+    and run as its own one-group forward after the routed forward (two
+    chains, two outputs to add)."""
+    fold = Workload(W.MOE_CONFIGS["decode_shared"], dev)
+    c = dec.cfg
+    sep = Workload(W.MoeConfig("shared_T64", E=1, k=1, T=c.T, H=c.H, I=c.I, routing="single", outliers=False,
+                               warmup_T=c.T), dev)
+
+    def separate():
+        dec.step()
+        sep.step()
+
+    folded, = graph_time([fold.step], steps, warmup)
+    both, = graph_time([separate], steps, warmup)
+    for wl in (fold, sep):
+        if nvfp4_moe_get_error(wl.ws) != 0:
+            raise RuntimeError(f"device error word after the {wl.cfg.name} run")
+    b = fold.step_bytes()
+    return {"workload": config_block(fold.cfg, 1)["workload"], "ms_folded": folded,
+            "ms_separate": both, "GB_s_folded": b / (folded * 1e-3) / 1e9, "hbm_frac_folded": None,
+            "algorithmic_bytes": b, "launches_folded": fold.launches_per_step,
+            "launches_separate": dec.launches_per_step + sep.launches_per_step,
+            "timing": "CUDA graph of back-to-back steps; weights (1.8 GB) streamed from HBM every step"}
+
+
 def fp4_ceiling(dev, sms):
     """Tensor-pipe ceiling of the FP4 MMA (nvfp4_fp4_mma_ceiling): one block
     per SM issues k-tiles of four M=128 K=64 MMAs for ~20 ms (long enough to
@@ -719,6 +747,8 @@ def run_ours(args):
     pure = time_variant_routing(pre, W.MOE_CONFIGS["prefill_zipf_pure"], min(steps, 50), warmup, world)
     shared = time_shared(dev, min(steps, 50), warmup, flush)
     tiny = time_shared(dev, min(steps, 50), warmup, flush, name="tiny")
+    shared_fold = time_shared_fold(dec, dev, min(steps, 50), warmup)
+    shared_fold["hbm_frac_folded"] = shared_fold["GB_s_folded"] / peaks["hbm_gbs"]
 
     t_step = ms_pre / steps / 1e3
     tokens_s = world * pre.cfg.T / t_step
@@ -781,6 +811,7 @@ def run_ours(args):
         "prefill_pure_zipf": pure,
         "shared_expert": shared,
         "tiny_moe": tiny,
+        "decode_with_shared_expert": shared_fold,
         "gpu_launches": (pre.launches_per_step + dec.launches_per_step) * steps,
         "clocks": clocks.summary(),
     }

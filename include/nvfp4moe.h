@@ -281,6 +281,25 @@ int nvfp4_fp4_mma_ceiling(int bn, int iters, int ctas, int64_t *cycles, int32_t 
 int nvfp4_moe_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *topk_ids,
                    float *topk_weights, void *stream);
 
+/* The router with the shared experts folded in as extra groups.  Page 1
+ * "Phase 1" describes the shared expert as the routed chain with one expert
+ * and no routing (L1, SiLU, re-quantisation, L2, same stacked weights), so
+ * it can run as one more group of the routed launches.  Identical to
+ * nvfp4_moe_topk for the k routed slots, except that rows have
+ * k + num_shared slots: topk_ids / topk_weights are [T, k + num_shared],
+ * slot k + i holding expert id E + i with weight exactly 1.0f.  Fed to
+ * nvfp4_moe_forward with E + num_shared experts (the shared experts' NVFP4
+ * weights stored after the E routed ones, their inter_gs calibrated like
+ * any other expert's), the output is
+ *   out[t] = sum_j<k w[t,j] * Expert_{ids[t,j]}(x[t]) + sum_i Shared_i(x[t]),
+ * summed in fp32 in slot order and rounded once to bf16: the routed and
+ * shared contributions in one set of launches instead of two chains.
+ * 0 <= num_shared, k + num_shared <= 32, E + num_shared <= 1024; the other
+ * arguments and errors are nvfp4_moe_topk's (which is this call with
+ * num_shared = 0).  Allocates nothing. */
+int nvfp4_moe_topk_shared(const float *logits, int64_t T, int E, int k, int scoring, int num_shared,
+                          int32_t *topk_ids, float *topk_weights, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

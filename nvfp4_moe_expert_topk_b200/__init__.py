@@ -18,7 +18,7 @@ __all__ = [
     "nvfp4_swizzle_scales", "nvfp4_gemm", "nvfp4_moe_workspace_size", "nvfp4_moe_forward",
     "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
-    "nvfp4_moe_get_error", "nvfp4_moe_topk", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax", "nvfp4_debug_bounded_wait", "nvfp4_gemm_ws",
+    "nvfp4_moe_get_error", "nvfp4_moe_topk", "nvfp4_moe_topk_shared", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax", "nvfp4_debug_bounded_wait", "nvfp4_gemm_ws",
     "nvfp4_gemm_workspace_size",
     "MoeArgs",
 ]
@@ -77,6 +77,7 @@ def lib():
                                                  ctypes.POINTER(i64), ctypes.POINTER(i64)]
         L.nvfp4_moe_get_error.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.nvfp4_moe_topk.argtypes = [P, i64, i32, i32, i32, P, P, P]
+        L.nvfp4_moe_topk_shared.argtypes = [P, i64, i32, i32, i32, i32, P, P, P]
         L.nvfp4_amax.argtypes = [P, i64, P, P]
         L.nvfp4_debug_bounded_wait.argtypes = [P, i32, P, P]
         L.nvfp4_gemm_ws.argtypes = [P, P, P, i64, P, P, P, P, i32, i64, i64, P, i64, P, ctypes.c_size_t, P]
@@ -277,6 +278,20 @@ def nvfp4_moe_topk(logits, k, topk_ids, topk_weights, scoring=NVFP4_SCORING_SOFT
                                 _dev(topk_ids, "topk_ids", torch.int32),
                                 _dev(topk_weights, "topk_weights", torch.float32), _stream(stream)),
            "nvfp4_moe_topk")
+
+
+def nvfp4_moe_topk_shared(logits, k, num_shared, topk_ids, topk_weights, scoring=NVFP4_SCORING_SOFTMAX,
+                          stream=None):
+    """The router with shared experts folded in: logits [T, E] fp32 ->
+    topk_ids / topk_weights [T, k + num_shared], the k routed slots as
+    nvfp4_moe_topk writes them, then slot k + i = expert E + i, weight 1."""
+    T, E = logits.shape
+    if tuple(topk_ids.shape) != (T, k + num_shared) or tuple(topk_weights.shape) != (T, k + num_shared):
+        raise ValueError(f"topk_ids / topk_weights must be [{T}, {k + num_shared}]")
+    _check(lib().nvfp4_moe_topk_shared(_dev(logits, "logits", torch.float32), T, E, k, scoring, num_shared,
+                                       _dev(topk_ids, "topk_ids", torch.int32),
+                                       _dev(topk_weights, "topk_weights", torch.float32), _stream(stream)),
+           "nvfp4_moe_topk_shared")
 
 
 def nvfp4_fp4_mma_ceiling(bn, iters, cycles, err=None, stream=None):

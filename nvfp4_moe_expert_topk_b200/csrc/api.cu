@@ -786,21 +786,28 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
                                     static_cast<cudaStream_t>(stream)));
 }
 
-int nvfp4_moe_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *topk_ids, float *topk_weights,
-                   void *stream)
+int nvfp4_moe_topk_shared(const float *logits, int64_t T, int E, int k, int scoring, int num_shared,
+                          int32_t *topk_ids, float *topk_weights, void *stream)
 {
-    if (T < 0 || k < 1 || E < 1)
+    if (T < 0 || k < 1 || E < 1 || num_shared < 0)
         return NVFP4_ERR_INVALID_ARG;
     if (T > 0 && (logits == nullptr || topk_ids == nullptr || topk_weights == nullptr))
         return NVFP4_ERR_INVALID_ARG;
     if (scoring != NVFP4_SCORING_SOFTMAX && scoring != NVFP4_SCORING_SIGMOID)
         return NVFP4_ERR_INVALID_ARG;
-    if (E > 1024 || k > 32 || k > E || T * E >= (1LL << 40))
+    if (E > 1024 || k > E || k + num_shared > 32 || E + num_shared > 1024 || T * E >= (1LL << 40))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     int st = device_check(nullptr);
     if (st != NVFP4_OK)
         return st;
-    return cuda_status(launch_topk(logits, T, E, k, scoring, topk_ids, topk_weights, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_topk(logits, T, E, k, num_shared, scoring, topk_ids, topk_weights,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_moe_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *topk_ids, float *topk_weights,
+                   void *stream)
+{
+    return nvfp4_moe_topk_shared(logits, T, E, k, scoring, 0, topk_ids, topk_weights, stream);
 }
 
 int nvfp4_fp4_mma_ceiling(int bn, int iters, int ctas, int64_t *cycles, int32_t *err, void *stream)

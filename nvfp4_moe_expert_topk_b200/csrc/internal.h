@@ -116,7 +116,7 @@ cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *yrow, const fl
                            __nv_bfloat16 *out, cudaStream_t s);
 cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float *inter_gs, cudaStream_t s);
 cudaError_t launch_mma_ceiling(int bn, int iters, int ctas, long long *cycles, int32_t *err, cudaStream_t s);
-cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *ids, float *weights,
-                        cudaStream_t s);
+cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int ns, int scoring, int32_t *ids,
+                        float *weights, cudaStream_t s);
 
 } // namespace nvfp4

@@ -568,7 +568,7 @@ __device__ __forceinline__ float from_order_bits(uint32_t o)
 
 template <int P>
 __global__ void __launch_bounds__(32 * kTopkWarps) topk_kernel(const float *__restrict__ logits, int64_t T, int E,
-                                                               int k, int scoring, int32_t *__restrict__ ids,
+                                                               int k, int ns, int scoring, int32_t *__restrict__ ids,
                                                                float *__restrict__ weights)
 {
     const int lane = threadIdx.x & 31;
@@ -626,14 +626,21 @@ __global__ void __launch_bounds__(32 * kTopkWarps) topk_kernel(const float *__re
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    // Row stride k + ns: the routed slots, then one slot per shared expert
+    // (ids E .. E + ns - 1, weight 1), so that the forward runs the shared
+    // experts as extra groups of the same grouped GEMMs.
+    const int64_t ld = k + ns;
     if (lane < k) {
-        ids[t * k + lane] = mine_id;
-        weights[t * k + lane] = __fdiv_rn(v, sum);
+        ids[t * ld + lane] = mine_id;
+        weights[t * ld + lane] = __fdiv_rn(v, sum);
+    } else if (lane < ld) {
+        ids[t * ld + lane] = E + (lane - k);
+        weights[t * ld + lane] = 1.0f;
     }
 }
 
-cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *ids, float *weights,
-                        cudaStream_t s)
+cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int ns, int scoring, int32_t *ids,
+                        float *weights, cudaStream_t s)
 {
     if (T == 0)
         return cudaSuccess;
@@ -641,7 +648,7 @@ cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int scorin
     const int per_lane = (E + 31) / 32;
 #define NVFP4_TOPK_CASE(P)                                                                                       \
     if (per_lane <= P) {                                                                                         \
-        topk_kernel<P><<<grid, 32 * kTopkWarps, 0, s>>>(logits, T, E, k, scoring, ids, weights);                 \
+        topk_kernel<P><<<grid, 32 * kTopkWarps, 0, s>>>(logits, T, E, k, ns, scoring, ids, weights);             \
         return cudaGetLastError();                                                                               \
     }
     NVFP4_TOPK_CASE(2)

@@ -19,6 +19,13 @@ and holds its own batch of tokens.  One forward:
      again) and are summed there in fp32 in ascending rank order, then stored
      in x's dtype.
 
+Shared experts (the routed chain with one expert and no routing, page 1
+"Phase 1") are replicated on every rank.  Their slots arrive the way the
+router with shared experts writes them: ids E .. E + num_shared - 1 (weight 1).
+A token's shared slots are served on its own rank, as local experts
+El .. El + num_shared - 1 after the rank's routed ones, so the shared experts
+run as extra groups of the rank's local forward and add no traffic.
+
 The counts exchange reads the counts on the host, so a forward synchronises
 once with the device.  The per-rank compute is a pluggable callable; on a GPU
 it is the library's nvfp4_moe_forward (`LibraryExperts`).
@@ -43,10 +50,12 @@ class ExpertParallelMoE:
 
     amax_fn(x) -> float: max|x| of the local batch.
     experts_fn(x_recv, local_ids, weights, gs) -> [n, H]: the MoE block of
-    this rank's experts on received rows (local_ids < 0 are skipped slots)."""
+    this rank's experts on received rows (local_ids < 0 are skipped slots;
+    El .. El + num_shared - 1 are the shared experts).
+    num_experts counts the routed experts only."""
 
     def __init__(self, num_experts: int, amax_fn: Callable, experts_fn: Callable,
-                 group: Optional[dist.ProcessGroup] = None):
+                 group: Optional[dist.ProcessGroup] = None, num_shared: int = 0):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -55,6 +64,9 @@ class ExpertParallelMoE:
         self.E = num_experts
         self.El = num_experts // self.world
         self.first_expert = self.rank * self.El
+        if num_shared < 0:
+            raise ValueError("num_shared must be >= 0")
+        self.num_shared = num_shared
         self.amax_fn = amax_fn
         self.experts_fn = experts_fn
 
@@ -66,16 +78,20 @@ class ExpertParallelMoE:
 
     def plan(self, topk_ids: torch.Tensor):
         """For each destination rank d: the tokens with a slot on d (ascending)
-        and their ids rewritten to d's local expert ids (-1 elsewhere)."""
+        and their ids rewritten to d's local expert ids (-1 elsewhere).
+        Shared-expert slots (id >= E) stay on this rank, as local ids
+        El + (id - E)."""
         ids = topk_ids.to(torch.int64)
+        shared = ids >= self.E
         dest = torch.where(ids >= 0, ids // self.El, torch.full_like(ids, -1))
+        dest = torch.where(shared, torch.full_like(ids, self.rank), dest)
+        local_all = torch.where(shared, ids - self.E + self.El, ids - dest * self.El)
         tokens, local_ids = [], []
         for d in range(self.world):
             on_d = dest == d
             sel = torch.nonzero(on_d.any(dim=1), as_tuple=False).flatten()
             tokens.append(sel)
-            local_ids.append(torch.where(on_d[sel], ids[sel] - d * self.El,
-                                         torch.full_like(ids[sel], -1)).to(torch.int32))
+            local_ids.append(torch.where(on_d[sel], local_all[sel], torch.full_like(ids[sel], -1)).to(torch.int32))
         return tokens, local_ids
 
     def _exchange(self, send: torch.Tensor, send_counts, recv_counts) -> torch.Tensor:
@@ -87,6 +103,8 @@ class ExpertParallelMoE:
                 out_dtype: Optional[torch.dtype] = None) -> torch.Tensor:
         """out [T, H] in out_dtype (default x.dtype) for this rank's tokens."""
         T, H = x.shape
+        if topk_ids.numel() and int(topk_ids.max()) >= self.E + self.num_shared:
+            raise ValueError(f"expert id >= {self.E + self.num_shared} (routed + shared experts)")
         gs = self.batch_global_scale(x)
         tokens, local_ids = self.plan(topk_ids)
         send_counts = [int(t.numel()) for t in tokens]
@@ -112,8 +130,9 @@ class ExpertParallelMoE:
 
 class LibraryExperts:
     """experts_fn backed by the library on this rank's GPU: nvfp4_moe_forward
-    over the local experts' NVFP4 weights (a prep.MoeWeights of El experts)
-    and their warmup inter_gs; the workspace grows with the received rows."""
+    over the local experts' NVFP4 weights (a prep.MoeWeights of El experts,
+    then the shared experts) and their warmup inter_gs; the workspace grows
+    with the received rows."""
 
     def __init__(self, weights, inter_gs: torch.Tensor, top_k: int):
         self.weights = weights

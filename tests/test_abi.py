@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for want in ["nvfp4_quantize", "nvfp4_gemm", "nvfp4_moe_forward", "nvfp4_global_scale",
                  "nvfp4_swizzle_scales", "nvfp4_moe_workspace_size", "nvfp4_moe_get_error",
-                 "nvfp4_moe_route_debug", "nvfp4_moe_calibrate", "nvfp4_status_string", "nvfp4_moe_topk",
+                 "nvfp4_moe_route_debug", "nvfp4_moe_calibrate", "nvfp4_status_string", "nvfp4_moe_topk", "nvfp4_moe_topk_shared",
                  "nvfp4_moe_forward_noalloc", "nvfp4_moe_forward_timed"]:
         assert want in names
 
@@ -121,6 +121,12 @@ def test_topk_checks(L):
     assert L.nvfp4_moe_topk(F, 4, 1025, 6, 0, F, F, None) == -2      # E > 1024
     assert L.nvfp4_moe_topk(F, 4, 48, 33, 0, F, F, None) == -2       # k > 32
     assert L.nvfp4_moe_topk(F, 4, 4, 6, 1, F, F, None) == -2         # k > E
+    # the same checks with shared-expert slots, plus the slot and expert limits
+    assert L.nvfp4_moe_topk_shared(None, 4, 48, 6, 0, 1, F, F, None) == -1
+    assert L.nvfp4_moe_topk_shared(F, 4, 48, 6, 0, -1, F, F, None) == -1     # num_shared < 0
+    assert L.nvfp4_moe_topk_shared(F, 4, 48, 6, 3, 1, F, F, None) == -1      # unknown scoring
+    assert L.nvfp4_moe_topk_shared(F, 4, 48, 30, 0, 3, F, F, None) == -2     # k + num_shared > 32
+    assert L.nvfp4_moe_topk_shared(F, 4, 1020, 6, 0, 5, F, F, None) == -2    # E + num_shared > 1024
 
 
 def test_ceiling_checks(L):

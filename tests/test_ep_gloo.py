@@ -18,12 +18,19 @@ from nvfp4_moe_expert_topk_b200 import workloads as W
 from nvfp4_moe_expert_topk_b200.ep import ExpertParallelMoE, global_scale_from_amax
 
 CFG = W.MoeConfig("ep_tiny", E=8, k=2, T=48, H=256, I=128, routing="softmax", outliers=False, warmup_T=64)
+# the same routed experts plus one shared expert (global id 8, slot 2, weight 1)
+CFG_SHARED = W.MoeConfig("ep_tiny_shared", E=9, k=3, T=48, H=256, I=128, routing="softmax", outliers=False,
+                         warmup_T=64, shared=1)
 WORLD = 2
+
+
+def config(scenario):
+    return CFG_SHARED if scenario == "shared" else CFG
 
 
 def rank_batch(r, scenario):
     x = W.activations(CFG.T + 8 * r, CFG.H, seed=100 + r)     # ranks hold different batch sizes
-    ids, w = W.routing(CFG, CFG.T + 8 * r, seed=200 + r)
+    ids, w = W.routing(config(scenario), CFG.T + 8 * r, seed=200 + r)
     if scenario == "one_sided":                                # every slot on rank 0's experts
         ids = ids % (CFG.E // WORLD)
     if scenario == "skips":
@@ -31,9 +38,9 @@ def rank_batch(r, scenario):
     return x, ids, w
 
 
-def inter_gs_all():
-    xw, idw, ww = W.batch(CFG, warmup=True)
-    ow = OracleWeights(CFG, range(CFG.E), "cpu")
+def inter_gs_all(cfg):
+    xw, idw, ww = W.batch(cfg, warmup=True)
+    ow = OracleWeights(cfg, range(cfg.E), "cpu")
     xb = W.bf16_bits(xw)
     _, inter = O.moe_forward(xb, idw.numpy(), ww.numpy(), O.global_scale_bf16(xb), **ow.oracle_kwargs(),
                              inter_gs=None, intermediates=True)
@@ -46,17 +53,20 @@ def worker(rank, port, scenario):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=WORLD)
     try:
-        El = CFG.E // WORLD
-        local = list(range(rank * El, (rank + 1) * El))
-        ow = OracleWeights(CFG, local, "cpu")
-        igs = inter_gs_all()
+        cfg = config(scenario)
+        El = CFG.E // WORLD                                    # routed experts per rank
+        shared = list(range(CFG.E, cfg.E))                     # replicated on every rank
+        local = list(range(rank * El, (rank + 1) * El)) + shared
+        ow = OracleWeights(cfg, local, "cpu")
+        igs = inter_gs_all(cfg)
 
         def experts_fn(x, local_ids, w, gs):
             out = O.moe_forward(W.bf16_bits(x), local_ids.numpy(), w.numpy(), gs, **ow.oracle_kwargs(),
                                 inter_gs=igs[local])
             return torch.from_numpy(out)
 
-        ep = ExpertParallelMoE(CFG.E, amax_fn=lambda x: O.amax_bf16(W.bf16_bits(x)), experts_fn=experts_fn)
+        ep = ExpertParallelMoE(CFG.E, amax_fn=lambda x: O.amax_bf16(W.bf16_bits(x)), experts_fn=experts_fn,
+                               num_shared=len(shared))
         x, ids, w = rank_batch(rank, scenario)
         got = ep.forward(x, ids, w, out_dtype=torch.float32).numpy()
 
@@ -65,7 +75,7 @@ def worker(rank, port, scenario):
         xu, idu, wu = torch.cat(xs), torch.cat(idss), torch.cat(ws)
         gs = global_scale_from_amax(max(O.amax_bf16(W.bf16_bits(xr)) for xr in xs))
         assert gs == O.global_scale_bf16(W.bf16_bits(xu))
-        owa = OracleWeights(CFG, range(CFG.E), "cpu")
+        owa = OracleWeights(cfg, range(cfg.E), "cpu")
         ref = O.moe_forward(W.bf16_bits(xu), idu.numpy(), wu.numpy(), gs, **owa.oracle_kwargs(), inter_gs=igs)
         lo = sum(CFG.T + 8 * r for r in range(rank))
         ref = ref[lo:lo + x.shape[0]]
@@ -81,7 +91,7 @@ def free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("scenario", ["plain", "one_sided", "skips"])
+@pytest.mark.parametrize("scenario", ["plain", "one_sided", "skips", "shared"])
 def test_expert_parallel_two_ranks(scenario):
     mp.start_processes(worker, args=(free_port(), scenario), nprocs=WORLD, start_method="spawn")
 
@@ -99,3 +109,17 @@ def test_plan_rewrites_ids_per_rank():
     assert local[1].tolist() == [[-1, 1]]
     assert local[2].tolist() == [[0, 1]]
     assert local[3].tolist() == [[3, 2]]
+
+
+def test_plan_keeps_shared_slots_home():
+    """Shared-expert slots (ids >= E) are served on the token's own rank as
+    local ids El + (id - E); every token of the rank goes to itself."""
+    class Fake(ExpertParallelMoE):
+        def __init__(self, rank):
+            self.world, self.rank, self.E, self.El, self.num_shared = 4, rank, 16, 4, 2
+    ids = torch.tensor([[0, 5, 16, 17], [15, 14, 16, 17], [-1, 3, 16, -1]])
+    tokens, local = Fake(2).plan(ids)
+    assert [t.tolist() for t in tokens] == [[0, 2], [0], [0, 1, 2], [1]]
+    assert local[0].tolist() == [[0, -1, -1, -1], [-1, 3, -1, -1]]
+    assert local[2].tolist() == [[-1, -1, 4, 5], [-1, -1, 4, 5], [-1, -1, 4, -1]]
+    assert local[3].tolist() == [[3, 2, -1, -1]]

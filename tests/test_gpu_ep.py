@@ -16,7 +16,10 @@ from test_gpu_moe import Problem
 pytestmark = pytest.mark.gpu
 
 
-def test_expert_parallel_single_rank_matches_forward():
+@pytest.mark.parametrize("name", ["tiny", "tiny_shared"])
+def test_expert_parallel_single_rank_matches_forward(name):
+    """tiny_shared: 8 routed experts plus a shared one (slot 2, id 8, weight 1),
+    served on the token's own rank as local expert 8."""
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
@@ -24,14 +27,15 @@ def test_expert_parallel_single_rank_matches_forward():
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("nccl", rank=0, world_size=1)
     try:
-        cfg = W.MOE_CONFIGS["tiny"]
+        cfg = W.MOE_CONFIGS[name]
         p = Problem(cfg)
         inputs = p.device_inputs()
         ref = torch.empty(p.x.shape[0], cfg.H, dtype=torch.bfloat16, device="cuda")
         ws = torch.zeros_like(p.run(inputs)[1])
         nvfp4_moe_forward(**dict(inputs, x_gs=None), out=ref, workspace=ws)
         inter_gs = inputs["inter_gs"]
-        ep = ExpertParallelMoE(cfg.E, amax_fn=library_amax, experts_fn=LibraryExperts(p.dw, inter_gs, cfg.k))
+        ep = ExpertParallelMoE(cfg.E - cfg.shared, amax_fn=library_amax,
+                               experts_fn=LibraryExperts(p.dw, inter_gs, cfg.k), num_shared=cfg.shared)
         out = ep.forward(inputs["x"], inputs["topk_ids"], inputs["topk_weights"])
         torch.cuda.synchronize()
         assert torch.equal(out, ref)

@@ -233,7 +233,7 @@ def test_cuda_graph_replay_with_new_inputs(tiny):
     assert torch.equal(eager, out)
 
 
-@pytest.mark.parametrize("name", ["decode", "shared"])
+@pytest.mark.parametrize("name", ["decode", "shared", "decode_shared", "tiny_shared"])
 def test_full_size_configs(name):
     cfg = W.MOE_CONFIGS[name]
     p = Problem(cfg)

@@ -8,7 +8,8 @@ import pytest
 import torch
 
 import oracle as O
-from nvfp4_moe_expert_topk_b200 import NVFP4_SCORING_SIGMOID, NVFP4_SCORING_SOFTMAX, nvfp4_moe_topk
+from nvfp4_moe_expert_topk_b200 import (NVFP4_SCORING_SIGMOID, NVFP4_SCORING_SOFTMAX, nvfp4_moe_topk,
+                                        nvfp4_moe_topk_shared)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -81,5 +82,46 @@ def test_topk_feeds_forward():
     np.testing.assert_array_equal(ids, rid)
     np.testing.assert_allclose(w, rw, rtol=1e-5, atol=0)
     p.ids, p.w = torch.from_numpy(ids), torch.from_numpy(w)
+    out, _ = p.run()
+    check_output(out, p.oracle())
+
+
+@pytest.mark.parametrize("T,E,k,ns,scoring", [
+    (64, 48, 6, 1, "sigmoid"),    # the decode shard with the shared expert folded in
+    (300, 384, 6, 2, "softmax"),
+    (7, 40, 30, 2, "softmax"),    # k + num_shared = 32: every lane writes a slot
+    (5, 1023, 8, 1, "sigmoid"),   # E + num_shared = 1024
+])
+def test_topk_shared_matches_oracle(T, E, k, ns, scoring):
+    rng = np.random.default_rng(T + 7 * E)
+    logits = rng.normal(0, 1.5, (T, E)).astype(np.float32)
+    ids = torch.full((T, k + ns), -7, dtype=torch.int32, device=DEV)
+    w = torch.full((T, k + ns), float("nan"), dtype=torch.float32, device=DEV)
+    nvfp4_moe_topk_shared(torch.from_numpy(logits).to(DEV), k, ns, ids, w, SCORING[scoring])
+    torch.cuda.synchronize()
+    rid, rw = O.topk(logits, k, scoring, num_shared=ns)
+    np.testing.assert_array_equal(ids.cpu().numpy(), rid)
+    np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=1e-5, atol=0)
+    assert (w[:, k:] == 1.0).all()
+
+
+def test_topk_shared_feeds_forward():
+    """Router with the shared expert folded in drives the forward over the
+    routed experts plus the shared one: ids bit-exact against the oracle
+    router, the output against the oracle forward on them."""
+    from test_gpu_moe import Problem, check_output
+    from nvfp4_moe_expert_topk_b200 import workloads as W
+    cfg = W.MOE_CONFIGS["tiny_shared"]
+    p = Problem(cfg)
+    rng = np.random.default_rng(12)
+    T, Er, k = p.x.shape[0], cfg.E - cfg.shared, cfg.k - cfg.shared
+    logits = rng.normal(0, 1, (T, Er)).astype(np.float32)
+    ids = torch.empty((T, cfg.k), dtype=torch.int32, device=DEV)
+    w = torch.empty((T, cfg.k), dtype=torch.float32, device=DEV)
+    nvfp4_moe_topk_shared(torch.from_numpy(logits).to(DEV), k, cfg.shared, ids, w, NVFP4_SCORING_SOFTMAX)
+    torch.cuda.synchronize()
+    rid, rw = O.topk(logits, k, "softmax", num_shared=cfg.shared)
+    np.testing.assert_array_equal(ids.cpu().numpy(), rid)
+    p.ids, p.w = ids.cpu(), w.cpu()
     out, _ = p.run()
     check_output(out, p.oracle())
