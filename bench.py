@@ -513,16 +513,16 @@ def time_shared(dev, steps, warmup, flush, name="shared"):
             "algorithmic_bytes": b}
 
 
-def time_shared_fold(dec, dev, steps, warmup):
-    """The decode batch plus the shared expert, two ways, CUDA-graph timed:
-    folded in as a 49th group of the routed launches (every token's slot 7
-    is the shared expert with weight 1, as nvfp4_moe_topk_shared writes it),
-    and run as its own one-group forward after the routed forward (two
+def time_shared_fold(dec, fold_cfg, dev, steps, warmup, hbm_gbs):
+    """A routed batch plus the shared expert, two ways, CUDA-graph timed:
+    folded in as one more group of the routed launches (every token's last
+    slot is the shared expert with weight 1, as nvfp4_moe_topk_shared writes
+    it), and run as its own one-group forward after the routed forward (two
     chains, two outputs to add)."""
-    fold = Workload(W.MOE_CONFIGS["decode_shared"], dev)
+    fold = Workload(fold_cfg, dev)
     c = dec.cfg
-    sep = Workload(W.MoeConfig("shared_T64", E=1, k=1, T=c.T, H=c.H, I=c.I, routing="single", outliers=False,
-                               warmup_T=c.T), dev)
+    sep = Workload(W.MoeConfig(f"shared_T{c.T}", E=1, k=1, T=c.T, H=c.H, I=c.I, routing="single",
+                               outliers=c.outliers, warmup_T=min(c.T, 256)), dev)
 
     def separate():
         dec.step()
@@ -535,10 +535,11 @@ def time_shared_fold(dec, dev, steps, warmup):
             raise RuntimeError(f"device error word after the {wl.cfg.name} run")
     b = fold.step_bytes()
     return {"workload": config_block(fold.cfg, 1)["workload"], "ms_folded": folded,
-            "ms_separate": both, "GB_s_folded": b / (folded * 1e-3) / 1e9, "hbm_frac_folded": None,
+            "ms_separate": both, "GB_s_folded": b / (folded * 1e-3) / 1e9,
+            "hbm_frac_folded": b / (folded * 1e-3) / 1e9 / hbm_gbs,
             "algorithmic_bytes": b, "launches_folded": fold.launches_per_step,
             "launches_separate": dec.launches_per_step + sep.launches_per_step,
-            "timing": "CUDA graph of back-to-back steps; weights (1.8 GB) streamed from HBM every step"}
+            "timing": "CUDA graph of back-to-back steps; all weights streamed from HBM every step"}
 
 
 def fp4_ceiling(dev, sms):
@@ -747,8 +748,7 @@ def run_ours(args):
     pure = time_variant_routing(pre, W.MOE_CONFIGS["prefill_zipf_pure"], min(steps, 50), warmup, world)
     shared = time_shared(dev, min(steps, 50), warmup, flush)
     tiny = time_shared(dev, min(steps, 50), warmup, flush, name="tiny")
-    shared_fold = time_shared_fold(dec, dev, min(steps, 50), warmup)
-    shared_fold["hbm_frac_folded"] = shared_fold["GB_s_folded"] / peaks["hbm_gbs"]
+    shared_fold = time_shared_fold(dec, W.MOE_CONFIGS["decode_shared"], dev, min(steps, 50), warmup, peaks["hbm_gbs"])
 
     t_step = ms_pre / steps / 1e3
     tokens_s = world * pre.cfg.T / t_step
@@ -825,7 +825,22 @@ def run_ours(args):
 
 
 def run_single(name, world, rank, dev, peaks, peak_src, steps, warmup):
-    """One MoE workload alone (small cases for profiling: decode, prefill_ep48)."""
+    """One MoE workload alone (small cases for profiling: decode, prefill_ep48);
+    for decode_shared / prefill_shared, the shared expert folded in against
+    run as a second chain."""
+    if name.endswith("_shared"):
+        routed = Workload(W.MOE_CONFIGS[name[:-len("_shared")]], dev)
+        res = time_shared_fold(routed, W.MOE_CONFIGS[name], dev, steps, warmup, peaks["hbm_gbs"])
+        t = res["ms_folded"] / 1e3
+        line = {"metric": f"moe_{name}_tokens_per_s", "value": world * routed.cfg.T / t, "unit": "tokens/s",
+                "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": res["ms_folded"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+                "data": "synthetic", "config": config_block(W.MOE_CONFIGS[name], world),
+                "tokens_per_s_separate": world * routed.cfg.T / (res["ms_separate"] / 1e3), "shared_fold": res,
+                "gpu_launches": (res["launches_folded"] + res["launches_separate"]) * steps}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     dec = Workload(W.MOE_CONFIGS[name], dev)
     clocks = ClockSampler(dev)
     clocks.start()
@@ -913,7 +928,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA-graph replay")
-    ap.add_argument("--only", choices=["all", "decode", "prefill", "prefill_ep48", "shared", "tiny"], default="all",
+    ap.add_argument("--only", choices=["all", "decode", "prefill", "prefill_ep48", "shared", "tiny", "decode_shared",
+                                       "prefill_shared"], default="all",
                     help="one workload alone (small profiling cases)")
     args = ap.parse_args()
     if args.impl == "reference":

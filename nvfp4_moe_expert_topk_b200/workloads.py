@@ -67,6 +67,8 @@ MOE_CONFIGS = {
     # expert and no routing; same H and I as a routed expert)
     "decode_shared": MoeConfig("decode_shared", E=49, k=7, T=64, H=7168, I=3072, routing="sigmoid",
                                outliers=False, warmup_T=64, shared=1),
+    "prefill_shared": MoeConfig("prefill_shared", E=385, k=7, T=4096, H=7168, I=3072, routing="zipf",
+                                outliers=True, warmup_T=16, shared=1),
     "tiny_shared": MoeConfig("tiny_shared", E=9, k=3, T=64, H=256, I=128, routing="softmax", outliers=False,
                              warmup_T=64, shared=1),
 }

@@ -244,10 +244,12 @@ def test_full_size_configs(name):
     assert nvfp4_moe_get_error(ws) == 0
 
 
-def test_prefill_sampled_tokens():
+@pytest.mark.parametrize("name", ["prefill", "prefill_shared"])
+def test_prefill_sampled_tokens(name):
     """384 experts, Zipf-skewed routing with empty experts: the whole batch on
-    the GPU, sampled tokens through the oracle."""
-    cfg = W.MOE_CONFIGS["prefill"]
+    the GPU, sampled tokens through the oracle.  prefill_shared adds the shared
+    expert as a 385th group that every token reaches (32 m-tiles)."""
+    cfg = W.MOE_CONFIGS[name]
     tokens = np.sort(np.random.default_rng(0).choice(cfg.T, 6, replace=False))
     p = Problem(cfg, oracle_tokens=tokens)
     route = O.route(p.ids.numpy(), cfg.E)
