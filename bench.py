@@ -3,9 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one pass of the whole chain over one batch: the activation global
-scale (nvfp4_global_scale) and nvfp4_moe_forward (route, quantise+permute,
-L1 gate_up GEMM with fused SiLU*up re-quantisation, L2 down GEMM, combine).
+One step = one pass of the whole chain over one batch: nvfp4_moe_forward
+with no global scale given (the batch's activation global scale, route,
+quantise+permute, L1 gate_up GEMM with fused SiLU*up re-quantisation and L2
+down GEMM in one persistent launch, combine).
 Headline workload: the 384-expert prefill MoE (T=4096, top-6, H=7168,
 I=3072, Zipf-skewed routing with empty experts) -> tokens/s, TFLOP/s and the
 fraction of the FP4 peak; the 48-expert decode MoE (T=64) is measured in the
@@ -17,7 +18,8 @@ parallel over token batches, weights replicated, no collective on the data
 path); timing is the max over ranks; value = all ranks' tokens / that time.
 
 --impl reference times the CPU oracle (oracle/, plain C) on this host's
-cores on a bounded sample of the same workload (rank 0 only).
+cores on a bounded sample of the same workload (rank 0 only); nothing of the
+library runs on that path.
 """
 import argparse
 import hashlib
@@ -663,7 +665,7 @@ def oracle_sample(cfg, tokens, dev, inter_gs_dev):
         b2 = W.bf16_bits(W.expert_w2(cfg, e, dev))
         w2g[i] = O.global_scale_bf16(b2)
         w2c[i], w2s[i] = O.quantize_bf16(b2, w2g[i])
-    inter = inter_gs_dev.cpu().numpy()[experts]
+    inter = None if inter_gs_dev is None else inter_gs_dev.cpu().numpy()[experts]
     remap = np.vectorize(lambda e: lut[e])(sub_ids).astype(np.int32)
     return dict(x_bits=xb[tokens], topk_ids=remap, topk_weights=w.numpy()[tokens], x_gs=x_gs,
                 w13_codes=w13c, w13_scales=w13s, w13_gs=w13g, w2_codes=w2c, w2_scales=w2s, w2_gs=w2g,
@@ -881,12 +883,10 @@ def run_reference(args):
     cfg = W.MOE_CONFIGS["prefill"]
     steps, warmup = args.steps, max(3, args.warmup)
     tokens = np.sort(np.random.default_rng(321).choice(cfg.T, 4, replace=False))
-    # warmup inter_gs is the library's; it only sets the arithmetic's scale, not the work
-    if dev.type == "cuda":
-        inter_gs = _calibrated_inter_gs(cfg, dev)
-    else:
-        inter_gs = torch.full((cfg.E,), 1000.0)
-    sample = oracle_sample(cfg, tokens, dev, inter_gs)
+    # nothing of the library on this path: the sampled tokens are the oracle's
+    # own warmup batch for inter_gs (it sets the values, not the work)
+    sample = oracle_sample(cfg, tokens, dev, None)
+    sample["inter_gs"] = O.moe_warmup_inter_gs(**{key: v for key, v in sample.items() if key != "inter_gs"})
     k = cfg.k
     n_slots = len(tokens) * k
     for i in range(warmup):
@@ -904,20 +904,6 @@ def run_reference(args):
                                        f"cycling over the {n_slots} slots of {len(tokens)} tokens"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
-
-
-def _calibrated_inter_gs(cfg, dev):
-    wts = prep.MoeWeights.synthetic(cfg, dev)
-    xw, idw, ww = W.batch(cfg, warmup=True)
-    xw = xw.to(dev)
-    gs = torch.empty(1, dtype=torch.float32, device=dev)
-    nvfp4_global_scale(xw, gs)
-    ws = prep.workspace(cfg.warmup_T, cfg.k, cfg.E, cfg.H, cfg.I, dev)
-    out = torch.empty(cfg.E, dtype=torch.float32, device=dev)
-    nvfp4_moe_calibrate(xw, idw.to(dev), ww.to(dev), gs, **wts.args(), inter_gs_out=out, workspace=ws)
-    torch.cuda.synchronize()
-    del wts
-    return out.cpu()
 
 
 def main():
