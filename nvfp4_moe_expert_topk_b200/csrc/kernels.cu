@@ -553,6 +553,7 @@ cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float
 // keys, its lowest expert.  Each of the k rounds takes two warp reductions
 // (redux.sync): the largest key, then the lowest expert holding it; the
 // owning lane retires that key (to 0, below every real key) and rescans.
+// With ns shared experts, lanes k .. k + ns - 1 write the shared slots.
 constexpr int kTopkWarps = 8;
 
 __device__ __forceinline__ uint32_t order_bits(float x)
