@@ -1,0 +1,83 @@
+"""Host-side logic of bench.py (CPU only): the stage folding that turns the
+timed forward's six stage slots into the stages the plan runs, the committed
+traffic figures being used only for the GEMM sources they were taken on, and
+the workload description of the JSON line."""
+import os
+import shutil
+
+import pytest
+
+import bench
+from nvfp4_moe_expert_topk_b200 import workloads as W
+
+
+class _Plan:
+    """A Workload's plan without the device (fold() reads only `fused`)."""
+
+    def __init__(self, fused):
+        self.fused = fused
+
+
+STAGE_MS = {"global_scale": 0.01, "route": 0.02, "quantize_permute": 0.04,
+            "l1_gate_up_swiglu_quant": 2.0, "l2_down": 1.0, "combine": 0.07}
+
+
+def test_fold_fused_plan():
+    d = bench.Workload.fold(_Plan(True), STAGE_MS)
+    assert set(d) == {bench.FRONT_STAGE, bench.FUSED_STAGE, "combine"}
+    assert d[bench.FRONT_STAGE] == pytest.approx(0.07)
+    assert d[bench.FUSED_STAGE] == pytest.approx(3.0)
+    assert sum(d.values()) == pytest.approx(sum(STAGE_MS.values()))
+
+
+def test_fold_two_launch_plan():
+    d = bench.Workload.fold(_Plan(False), STAGE_MS)
+    assert set(d) == {bench.FRONT_STAGE, "l1_gate_up_swiglu_quant", "l2_down", "combine"}
+    assert d["l2_down"] == 1.0
+
+
+def _copy_tree(tmp_path):
+    root = tmp_path / "repo"
+    csrc = root / "nvfp4_moe_expert_topk_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name in bench.GEMM_SOURCES:
+        shutil.copy(os.path.join(bench.ROOT, "nvfp4_moe_expert_topk_b200", "csrc", name), csrc / name)
+    (root / "profiles").mkdir()
+    return root, csrc
+
+
+def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    root, csrc = _copy_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h0 = bench.gemm_source_sha()
+    assert h0 == bench.gemm_source_sha()
+    g = csrc / "gemm.cu"
+    text = g.read_text()
+    g.write_text("// a new comment line\n/* and a block\n   comment */\n" + text.replace("\n", "\n\n", 3))
+    assert bench.gemm_source_sha() == h0                  # comments and blank lines only
+    g.write_text(text.replace("kBM = 128", "kBM = 64", 1))
+    assert "kBM = 64" in g.read_text()
+    assert bench.gemm_source_sha() != h0                  # a code change
+
+
+def test_traffic_used_only_for_matching_sources(tmp_path, monkeypatch):
+    root, csrc = _copy_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    prof = root / "profiles" / "ncu_traffic.txt"
+    assert bench.ncu_traffic("l1_l2_fused", "decode") is None            # no summary
+    prof.write_text(f"# comment\nsource_sha: {bench.gemm_source_sha()}\n"
+                    "decode.l1_l2_fused.dram_bytes_per_launch: 1809793536\n")
+    assert bench.ncu_traffic("l1_l2_fused", "decode") == 1809793536.0
+    assert bench.ncu_traffic("l1_l2_fused", "prefill") is None           # not captured
+    prof.write_text("source_sha: 0123456789abcdef\ndecode.l1_l2_fused.dram_bytes_per_launch: 1\n")
+    assert bench.ncu_traffic("l1_l2_fused", "decode") is None            # taken on other sources
+
+
+def test_config_block_names_the_workload():
+    c = bench.config_block(W.MOE_CONFIGS["prefill"], 8)
+    assert c["workload"] == "prefill_moe_E384_k6_T4096_H7168_I3072_zipf1.1_16empty"
+    assert c["global_batch"] == 8 * 4096 and c["tokens_per_gpu"] == 4096
+    assert c["parallelism"].startswith("dp8")
+    c1 = bench.config_block(W.MOE_CONFIGS["decode_shared"], 1)
+    assert c1["workload"] == "decode_shared_moe_E49_k7_T64_H7168_I3072"
+    assert c1["parallelism"] == "replicas"
