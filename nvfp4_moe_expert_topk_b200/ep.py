@@ -72,7 +72,8 @@ class ExpertParallelMoE:
 
     # ------------------------------------------------------------ steps
     def batch_global_scale(self, x: torch.Tensor) -> np.float32:
-        t = torch.tensor([float(self.amax_fn(x))], dtype=torch.float32, device=x.device)
+        a = float(self.amax_fn(x)) if x.numel() else 0.0     # a rank without tokens adds nothing
+        t = torch.tensor([a], dtype=torch.float32, device=x.device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX, group=self.group)
         return global_scale_from_amax(t.item())
 
