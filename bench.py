@@ -22,6 +22,7 @@ cores on a bounded sample of the same workload (rank 0 only); nothing of the
 library runs on that path.
 """
 import argparse
+import contextlib
 import hashlib
 import re
 import json
@@ -94,61 +95,133 @@ def ncu_traffic(kernel, workload):
     return float(v) if v else None
 
 
-class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+class Clocks:
+    """SM clock, power draw and clock-event reasons, sampled from NVML every
+    5 ms by a background thread for the whole run (read-only queries: nothing
+    is set).  Each timed region records its host interval (the device work
+    inside it is bracketed by synchronisations), so every time reported
+    carries the median SM clock it ran at.  Falls back to one nvidia-smi
+    process sampling every 200 ms when NVML is unavailable."""
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4}
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device):
+    def __init__(self, device, period=0.005):
         self.device = device
-        self.proc = None
-        self.samples = []
+        self.period = period
+        self.samples = []               # (monotonic s, sm MHz, max MHz, power W, reason bits)
+        self.regions = {}
+        self.source = None
+        self._stop = None
+        self._thread = None
+        self._proc = None
 
-    def _id(self):
+    def _uuid(self):
         try:
             return "GPU-" + str(torch.cuda.get_device_properties(self.device).uuid)
         except Exception:
             return None
 
     def start(self):
-        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
-        gid = self._id()
-        if gid:
-            cmd[1:1] = ["-i", gid]
+        import threading
         try:
-            self.proc = subprocess.Popen(cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+            import pynvml as N
+            N.nvmlInit()
+            uid = self._uuid()
+            h = N.nvmlDeviceGetHandleByUUID(uid) if uid else N.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+            mx = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+        except Exception:
+            return self._start_smi()
+        self.source = "nvml"
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((time.monotonic(), float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)), mx,
+                                         N.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                         int(N.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+
+    def _start_smi(self):
+        self.source = "nvidia-smi"
+        self._file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200"]
+        uid = self._uuid()
+        if uid:
+            cmd[1:1] = ["-i", uid]
+        self._t0 = time.monotonic()
+        try:
+            self._proc = subprocess.Popen(cmd, stdout=self._file, stderr=subprocess.DEVNULL)
         except OSError:
-            self.proc = None
+            self._proc = None
 
     def stop(self):
-        if self.proc is None:
-            return
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.file.seek(0)
-        for line in self.file.read().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append(parts)
-        self.file.close()
-        os.unlink(self.file.name)
-        self.proc = None
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+            self._thread = None
+        if self._proc is not None:
+            time.sleep(0.25)
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+            self._file.seek(0)
+            rows = [[p.strip() for p in line.split(",")] for line in self._file.read().splitlines()]
+            self._file.close()
+            os.unlink(self._file.name)
+            names = list(self.REASONS)
+            for i, r in enumerate(r for r in rows if len(r) >= 9):
+                try:
+                    bits = sum(self.REASONS[names[j]] for j in range(4) if r[5 + j].lower() == "active")
+                    # no per-sample timestamps: spread the samples 200 ms apart from the start
+                    self.samples.append((self._t0 + 0.2 * i, float(r[1]), float(r[2]), float(r[3]), bits))
+                except ValueError:
+                    pass
+            self._proc = None
 
-    def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
-        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[5 + i].lower() == "active"})
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+    @contextlib.contextmanager
+    def region(self, name):
+        t0 = time.monotonic()
+        try:
+            yield
+        finally:
+            self.regions[name] = (t0, time.monotonic())
+
+    def summary(self, names=None):
+        """Median SM MHz, max MHz, median power and the clock-event reasons
+        seen over the samples inside the named regions (all regions if None)."""
+        spans = [self.regions[n] for n in (names or list(self.regions)) if n in self.regions]
+        sel = [smp for smp in self.samples if any(a <= smp[0] <= b for a, b in spans)]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples in the region"], "samples": 0,
+                    "source": self.source}
+        bits = 0
+        for smp in sel:
+            bits |= smp[4]
+        return {"sm_mhz": float(np.median([smp[1] for smp in sel])), "sm_max_mhz": max(smp[2] for smp in sel),
+                "power_w": round(float(np.median([smp[3] for smp in sel])), 1),
+                "reasons": sorted(n for n, b in self.REASONS.items() if bits & b), "samples": len(sel),
+                "source": self.source}
+
+    def mhz(self, name):
+        return self.summary([name])["sm_mhz"]
+
+
+CLOCKS = None                           # the run's Clocks, started in run_ours / run_single
+
+
+def clock_region(name):
+    return CLOCKS.region(name) if CLOCKS is not None else contextlib.nullcontext()
 
 
 def dist_setup():
@@ -313,14 +386,15 @@ def time_steps(wl, steps, warmup, world, graph=True, tag="timed"):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     torch.cuda.nvtx.range_push(f"{tag}_{wl.cfg.name}")
-    t0.record(stream)
-    if g is not None:
-        g.replay()
-    else:
-        issue_plain()
-    t1.record(stream)
+    with clock_region(f"{tag}_{wl.cfg.name}"):
+        t0.record(stream)
+        if g is not None:
+            g.replay()
+        else:
+            issue_plain()
+        t1.record(stream)
+        torch.cuda.synchronize()
     torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
     barrier(world)
     ms = t0.elapsed_time(t1)
     if g_staged is not None:
@@ -387,15 +461,16 @@ def time_e2e(wl, steps, warmup, world):
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(up)
-    compute.wait_event(t0)
-    down.wait_event(t0)
-    for i in range(warmup, n_all):
-        issue(i)
-    up.wait_stream(down)
-    up.wait_stream(compute)
-    t1.record(up)
-    torch.cuda.synchronize()
+    with clock_region(f"e2e_{wl.cfg.name}"):
+        t0.record(up)
+        compute.wait_event(t0)
+        down.wait_event(t0)
+        for i in range(warmup, n_all):
+            issue(i)
+        up.wait_stream(down)
+        up.wait_stream(compute)
+        t1.record(up)
+        torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(world, t0.elapsed_time(t1))
     h2d = hx.numel() * hx.element_size() + hids.numel() * 4 + hw.numel() * 4
@@ -408,7 +483,7 @@ def time_e2e(wl, steps, warmup, world):
 
 
 # ---------------------------------------------------------------- MLA GEMMs
-def graph_time(fns, reps, warmup, flush=None):
+def graph_time(fns, reps, warmup, flush=None, region=None):
     """Per-call device times of a sequence of calls, issued back to back.
     `reps` repetitions of [flush(); ev0; fns[0](); ev1; fns[1](); ...] are
     captured into one CUDA graph (external event records, so the kernels run
@@ -441,8 +516,9 @@ def graph_time(fns, reps, warmup, flush=None):
     stream.wait_stream(side)
     g.replay()
     torch.cuda.synchronize()
-    g.replay()
-    torch.cuda.synchronize()
+    with clock_region(region) if region else contextlib.nullcontext():
+        g.replay()
+        torch.cuda.synchronize()
     out = [float(np.mean([row[j].elapsed_time(row[j + 1]) for row in ev])) for j in range(len(fns))]
     del g
     return out
@@ -473,13 +549,13 @@ def time_router(cfg, dev, reps, warmup, flush):
     def call():
         nvfp4_moe_topk(logits, cfg.k, ids, w, NVFP4_SCORING_SIGMOID)
 
-    hot, = graph_time([call], reps, warmup)
-    cold, = graph_time([call], reps, 0, flush)
+    hot, = graph_time([call], reps, warmup, region="router_hot")
+    cold, = graph_time([call], reps, 0, flush, region="router_cold")
     nbytes = cfg.T * cfg.E * 4 + cfg.T * cfg.k * 8
     return {"T": cfg.T, "E": cfg.E, "k": cfg.k, "scoring": "sigmoid", "us_per_call": round(hot * 1e3, 2),
             "us_per_call_cold": round(cold * 1e3, 2), "GB_s": round(nbytes / (hot * 1e-3) / 1e9, 1),
             "GB_s_cold": round(nbytes / (cold * 1e-3) / 1e9, 1), "bytes_per_call": nbytes, "launches": 1,
-            "timing": "CUDA graph of back-to-back calls; hot = logits in L2, cold = after a 512 MB L2 flush"}
+            "sm_mhz": CLOCKS.mhz("router_hot") if CLOCKS else None}
 
 
 def time_variant_routing(wl, cfg, steps, warmup, world):
@@ -496,7 +572,8 @@ def time_variant_routing(wl, cfg, steps, warmup, world):
             "ms_per_step": ms / steps, "tokens_per_s": world * cfg.T / t,
             "tflops": 2.0 * counts.sum() * 3 * cfg.H * cfg.I / t / 1e12,
             "empty_experts": int((counts == 0).sum()), "max_rows_per_expert": int(counts.max()),
-            "m_tiles": int(np.ceil(counts / 128).sum()), "stage_ms": stages}
+            "m_tiles": int(np.ceil(counts / 128).sum()), "stage_ms": stages,
+            "sm_mhz": CLOCKS.mhz(f"variant_{wl.cfg.name}") if CLOCKS else None}
 
 
 def time_shared(dev, steps, warmup, flush, name="shared"):
@@ -504,15 +581,15 @@ def time_shared(dev, steps, warmup, flush, name="shared"):
     tokens, 37 MB of weights) or the tiny MoE (0.4 MB): hot (back-to-back
     steps) and cold (L2 flushed before every step), CUDA-graph timed."""
     wl = Workload(W.MOE_CONFIGS[name], dev)
-    hot, = graph_time([wl.step], steps, warmup)
-    cold, = graph_time([wl.step], steps, 0, flush)
+    hot, = graph_time([wl.step], steps, warmup, region=f"{name}_hot")
+    cold, = graph_time([wl.step], steps, 0, flush, region=f"{name}_cold")
     if nvfp4_moe_get_error(wl.ws) != 0:
         raise RuntimeError("device error word after the shared-expert run")
     b, f = wl.step_bytes(), wl.flops()
     return {"workload": config_block(wl.cfg, 1)["workload"], "ms_hot": hot, "ms_cold": cold,
             "GB_s_hot": b / (hot * 1e-3) / 1e9, "GB_s_cold": b / (cold * 1e-3) / 1e9,
             "tflops_hot": f / (hot * 1e-3) / 1e12, "tflops_cold": f / (cold * 1e-3) / 1e12,
-            "algorithmic_bytes": b}
+            "sm_mhz": CLOCKS.mhz(f"{name}_hot") if CLOCKS else None}
 
 
 def time_shared_fold(dec, fold_cfg, dev, steps, warmup, hbm_gbs):
@@ -530,8 +607,8 @@ def time_shared_fold(dec, fold_cfg, dev, steps, warmup, hbm_gbs):
         dec.step()
         sep.step()
 
-    folded, = graph_time([fold.step], steps, warmup)
-    both, = graph_time([separate], steps, warmup)
+    folded, = graph_time([fold.step], steps, warmup, region=f"{fold_cfg.name}_folded")
+    both, = graph_time([separate], steps, warmup, region=f"{fold_cfg.name}_separate")
     for wl in (fold, sep):
         if nvfp4_moe_get_error(wl.ws) != 0:
             raise RuntimeError(f"device error word after the {wl.cfg.name} run")
@@ -541,7 +618,7 @@ def time_shared_fold(dec, fold_cfg, dev, steps, warmup, hbm_gbs):
             "hbm_frac_folded": b / (folded * 1e-3) / 1e9 / hbm_gbs,
             "algorithmic_bytes": b, "launches_folded": fold.launches_per_step,
             "launches_separate": dec.launches_per_step + sep.launches_per_step,
-            "timing": "CUDA graph of back-to-back steps; all weights streamed from HBM every step"}
+            "sm_mhz": CLOCKS.mhz(f"{fold_cfg.name}_folded") if CLOCKS else None}
 
 
 def fp4_ceiling(dev, sms):
@@ -558,10 +635,11 @@ def fp4_ceiling(dev, sms):
         torch.cuda.synchronize()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        nvfp4_fp4_mma_ceiling(bn, iters, cycles, err)
-        b.record()
-        torch.cuda.synchronize()
+        with clock_region(f"fp4_ceiling_n{bn}"):
+            a.record()
+            nvfp4_fp4_mma_ceiling(bn, iters, cycles, err)
+            b.record()
+            torch.cuda.synchronize()
         if err.item() != 0 or (cycles < 0).any():
             raise RuntimeError("FP4 ceiling probe: a bounded wait gave up")
         ms = a.elapsed_time(b)
@@ -570,7 +648,8 @@ def fp4_ceiling(dev, sms):
         res[f"n{bn}"] = {"tflops": flops / (ms * 1e-3) / 1e12, "ms": ms,
                          "cycles_per_mma": float(cyc.mean()) / (iters * 4),
                          "cycles_per_mma_max": float(cyc.max()) / (iters * 4),
-                         "implied_sm_mhz": float(cyc.mean()) / (ms * 1e3)}
+                         "implied_sm_mhz": float(cyc.mean()) / (ms * 1e3),
+                         "sm_mhz": CLOCKS.mhz(f"fp4_ceiling_n{bn}") if CLOCKS else None}
     return res
 
 
@@ -616,8 +695,8 @@ def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
         def gemm():
             nvfp4_gemm_ws(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out, gws)
 
-        quant_ms, gemm_ms = graph_time([quant, gemm], steps, warmup)
-        _, gemm_cold_ms = graph_time([quant, gemm], steps, 0, flush)
+        quant_ms, gemm_ms = graph_time([quant, gemm], steps, warmup, region=f"mla_{name}")
+        _, gemm_cold_ms = graph_time([quant, gemm], steps, 0, flush, region=f"mla_{name}_cold")
         step_ms = quant_ms + gemm_ms
         flops = 2.0 * M * N * K
         gbytes = (M * K + N * K) * (0.5 + 1 / 16) + M * N * 2.0
@@ -630,7 +709,8 @@ def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
                      "gemm_ms_cold": gemm_cold_ms, "tflops_cold": flops / (gemm_cold_ms * 1e-3) / 1e12,
                      "gbs": gbs, "arith_intensity": ai, "bound": bound,
                      "frac": (tflops / fp4_peak) if bound == "tensor" else (gbs / peaks["hbm_gbs"]),
-                     "fp4_nominal_frac": tflops / FP4_NOMINAL_TFLOPS}
+                     "fp4_nominal_frac": tflops / FP4_NOMINAL_TFLOPS,
+                     "sm_mhz": CLOCKS.mhz(f"mla_{name}") if CLOCKS else None}
         if ceiling_tflops:
             res[name]["fp4_ceiling_frac"] = tflops / ceiling_tflops
         del ad, a_codes, a_sc, out, w_codes, w_sc, gws
@@ -716,23 +796,52 @@ def config_block(cfg, world):
             "parallelism": "replicas" if world == 1 else f"dp{world} replicas (no data-path collective)"}
 
 
+def compact(obj, digits=4):
+    """Floats rounded to `digits` significant digits, recursively (keeps the
+    one-line record short)."""
+    if isinstance(obj, float):
+        return float(f"{obj:.{digits}g}")
+    if isinstance(obj, dict):
+        return {k: compact(v, digits) for k, v in obj.items()}
+    if isinstance(obj, (list, tuple)):
+        return [compact(v, digits) for v in obj]
+    return obj
+
+
+def timed(ms, region):
+    """A device time with the median SM clock of its region and their
+    product (time x clock: comparable across runs at different clocks)."""
+    mhz = CLOCKS.mhz(region) if CLOCKS else None
+    return {"ms": ms, "sm_mhz": mhz, "ms_x_ghz": ms * mhz / 1e3 if mhz else None}
+
+
 def run_ours(args):
+    global CLOCKS
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
     steps, warmup = args.steps, max(3, args.warmup)
+    CLOCKS = Clocks(dev)
+    CLOCKS.start()
+    try:
+        if args.only != "all":
+            return run_single(args.only, world, rank, dev, peaks, peak_src, steps, warmup)
+        return _run_all(args, world, rank, dev, peaks, peak_src, steps, warmup)
+    finally:
+        CLOCKS.stop()
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
 
-    if args.only != "all":
-        return run_single(args.only, world, rank, dev, peaks, peak_src, steps, warmup)
+
+def _run_all(args, world, rank, dev, peaks, peak_src, steps, warmup):
     pre = Workload(W.MOE_CONFIGS["prefill"], dev)
     dec = Workload(W.MOE_CONFIGS["decode"], dev)
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(dev)
-    clocks.start()
+    mode = "eager" if args.eager else "timed"
     ms_pre, stages_pre = time_steps(pre, steps, warmup, world, graph=not args.eager)
     ms_dec, stages_dec = time_steps(dec, steps, warmup, world, graph=not args.eager)
-    clocks.stop()
     ms_pre_eager, _ = time_steps(pre, steps, warmup, world, graph=False, tag="eager")
     ms_dec_eager, _ = time_steps(dec, steps, warmup, world, graph=False, tag="eager")
     for wl in (pre, dec):
@@ -767,6 +876,8 @@ def run_ours(args):
     dec_gbs = dec.step_bytes() / t_dec / 1e9
     dec_kb = dec.fold(dec.kernel_bytes())
     dec_dom = max(stages_dec, key=lambda s: stages_dec[s])
+    dec_ach = dec_kb[dec_dom] / (stages_dec[dec_dom] / 1e3) / 1e9
+    r_pre, r_dec = f"{mode}_{pre.cfg.name}", f"{mode}_{dec.cfg.name}"
 
     line = {
         "metric": "moe_prefill_tokens_per_s",
@@ -786,44 +897,45 @@ def run_ours(args):
         "fp4_peak_frac": {"of_nominal_9000": tflops / FP4_NOMINAL_TFLOPS,
                           f"of_{peak_src}_bf16_sustained_x4": tflops / fp4_measured,
                           "of_measured_fp4_mma_ceiling": tflops / ceiling["n256"]["tflops"]},
-        "fp4_mma_ceiling": ceiling,
         "hbm_gbs_step": pre.step_bytes() / t_step / 1e9,
         "hbm_frac_step": pre.step_bytes() / t_step / 1e9 / hbm,
         "stage_ms": stages_pre,
         "launch": "eager" if args.eager else "cuda_graph",
-        "eager_ms_per_step": ms_pre_eager / steps,
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "peak_source": f"{peak_src} hbm_gbs",
                      "algorithmic_bytes": kb[dominant], "traffic": traffic},
-        "decode": {
-            "workload": config_block(dec.cfg, world)["workload"],
-            "metric": "moe_decode_GB_per_s", "value": dec_gbs, "unit": "GB/s", "ms_per_step": ms_dec / steps,
-            "hbm_frac": dec_gbs / hbm, "tokens_per_s": world * dec.cfg.T / t_dec,
-            "eager_ms_per_step": ms_dec_eager / steps,
-            "algorithmic_bytes_per_step": dec.step_bytes(), "stage_ms": stages_dec,
-            "roofline": {"bound": "hbm", "kernel": dec_dom,
-                         "achieved": dec_kb[dec_dom] / (stages_dec[dec_dom] / 1e3) / 1e9, "peak": hbm,
-                         "unit": "GB/s", "frac": dec_kb[dec_dom] / (stages_dec[dec_dom] / 1e3) / 1e9 / hbm,
-                         "traffic": ncu_traffic(dec_dom, "decode")},
-        },
         "e2e": {"value": world * pre.cfg.T * steps / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / steps},
+        "gpu_launches": (pre.launches_per_step + dec.launches_per_step) * steps,
+        "clocks": CLOCKS.summary([r_pre]),
+        # every timed region with the median SM clock it ran at (time x clock compares runs)
+        "timings": {"prefill": timed(ms_pre / steps, r_pre), "prefill_eager": timed(ms_pre_eager / steps,
+                                                                                   f"eager_{pre.cfg.name}"),
+                    "e2e_prefill": timed(e2e_ms / steps, f"e2e_{pre.cfg.name}"),
+                    "decode": timed(ms_dec / steps, r_dec),
+                    "decode_eager": timed(ms_dec_eager / steps, f"eager_{dec.cfg.name}")},
+        "fp4_mma_ceiling": ceiling,
         "mla_gemms": mla,
         "router": router,
         "prefill_pure_zipf": pure,
         "shared_expert": shared,
         "tiny_moe": tiny,
         "decode_with_shared_expert": shared_fold,
-        "gpu_launches": (pre.launches_per_step + dec.launches_per_step) * steps,
-        "clocks": clocks.summary(),
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(pre.cfg, dev, pre.inter_gs)
+    # last, so that a record keeping only the end of the line still holds it
+    line["decode"] = {
+        "workload": config_block(dec.cfg, world)["workload"],
+        "metric": "moe_decode_GB_per_s", "value": dec_gbs, "unit": "GB/s", "ms_per_step": ms_dec / steps,
+        "hbm_frac": dec_gbs / hbm, "tokens_per_s": world * dec.cfg.T / t_dec,
+        "eager_ms_per_step": ms_dec_eager / steps, "algorithmic_bytes_per_step": dec.step_bytes(),
+        "stage_ms": stages_dec, "clocks": CLOCKS.summary([r_dec]),
+        "roofline": {"bound": "hbm", "kernel": dec_dom, "achieved": dec_ach, "peak": hbm, "unit": "GB/s",
+                     "frac": dec_ach / hbm, "traffic": ncu_traffic(dec_dom, "decode")},
+    }
     if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+        print(json.dumps(compact(line)), flush=True)
 
 
 def run_single(name, world, rank, dev, peaks, peak_src, steps, warmup):
@@ -844,10 +956,7 @@ def run_single(name, world, rank, dev, peaks, peak_src, steps, warmup):
             print(json.dumps(line), flush=True)
         return
     dec = Workload(W.MOE_CONFIGS[name], dev)
-    clocks = ClockSampler(dev)
-    clocks.start()
     ms_dec, stages = time_steps(dec, steps, warmup, world, graph=False)
-    clocks.stop()
     err = nvfp4_moe_get_error(dec.ws)
     if err != 0:
         raise RuntimeError(f"device error word {err}")
@@ -863,7 +972,7 @@ def run_single(name, world, rank, dev, peaks, peak_src, steps, warmup):
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
                          "algorithmic_bytes": kb[dom], "traffic": ncu_traffic(dom, name)},
-            "gpu_launches": dec.launches_per_step * steps, "clocks": clocks.summary()}
+            "gpu_launches": dec.launches_per_step * steps, "clocks": CLOCKS.summary([f"timed_{name}"])}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -158,9 +158,12 @@ typedef struct {
     uint16_t *out;                /* [T, H] bf16 output                                */
 } nvfp4_moe_args;
 
-/* Workspace bytes nvfp4_moe_forward / nvfp4_moe_calibrate need.  The
- * workspace is caller-owned device memory; zero it once after allocation
- * (it holds the sticky device error word). */
+/* Workspace bytes nvfp4_moe_forward / nvfp4_moe_calibrate need (page 1
+ * "Phase 1": a cudagraph-safe runner works on pre-allocated buffers, so the
+ * caller allocates this once and every call reuses it).  The workspace is
+ * caller-owned device memory; zero it once after allocation (it holds the
+ * sticky device error word).  Host only; 0 for a shape outside the
+ * constraints of nvfp4_moe_forward. */
 size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
 
 /* out = sum_j topk_weights[t,j] * Expert_{ids[t,j]}(x[t]) with
@@ -174,7 +177,8 @@ size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
  * call per device first: it sets per-kernel attributes). */
 int nvfp4_moe_forward(const nvfp4_moe_args *args, void *workspace, size_t ws_bytes, void *stream);
 
-/* nvfp4_moe_forward with CUDA events recorded on `stream` at its stage
+/* Measurement hook, not a step of the method: nvfp4_moe_forward with CUDA
+ * events recorded on `stream` at its stage
  * boundaries: events = 6 cudaEvent_t handles created by the caller, recorded
  * before the global scale (x_gs NULL) and routing, before quantise+permute,
  * before L1, after L1, after L2 (directly after L1's record when they are
@@ -193,7 +197,9 @@ int nvfp4_moe_forward_timed(const nvfp4_moe_args *args, void *workspace, size_t 
 int nvfp4_moe_calibrate(const nvfp4_moe_args *args, float *inter_gs_out, void *workspace,
                         size_t ws_bytes, void *stream);
 
-/* Routing step alone, for inspection: counts [E], padded_offsets [E+1]
+/* The routing step alone (page 3 "Architecture Notes": each token's top-6
+ * expert ids decide which expert's grouped-GEMM segment its row joins), for
+ * inspection and tests: counts [E], padded_offsets [E+1]
  * (expert segments padded to 128 rows), inv [T*k] (padded row of each slot,
  * -1 if skipped).  Slot f = t*k + j of expert e lands at
  * padded_offsets[e] + #{f' < f : ids[f'] == e} (a stable counting sort). */
@@ -201,7 +207,8 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
                           int32_t *padded_offsets, int32_t *inv, void *workspace, size_t ws_bytes,
                           void *stream);
 
-/* Byte offset and size of a workspace region (for inspection and tests).
+/* Byte offset and size of a workspace region (build helper for inspection
+ * and tests, no passage on the pages; host only).
  * region: 0 A codes, 1 A scales (MMA layout), 2 h codes, 3 h scales
  * (MMA layout), 4 y (bf16 [T*k, H], rows in expert-major routing order),
  * 5 inv, 6 counts, 7 padded offsets, 8 the fp32 global scale of x computed
@@ -210,25 +217,34 @@ int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, in
                                int64_t *offset, int64_t *bytes);
 
 /* nvfp4_moe_forward without a caller-supplied workspace, for callers that
- * cannot allocate device memory: code running while a CUDA graph is being
- * captured (cudaMalloc cannot be captured), plug-ins whose host framework
- * owns all device memory and forbids side allocations, and latency-critical
- * paths that cannot take cudaMalloc's implicit synchronisation.  The pages
- * have no counterpart of this entry point; it is a deployment convenience.
- * Scratch: one static device array of NVFP4_NOALLOC_SCRATCH_BYTES (32 MiB)
- * that every device using this entry point holds until the process exits;
- * shapes whose nvfp4_moe_workspace_size() exceeds it return
- * NVFP4_ERR_WORKSPACE_TOO_SMALL without launching.  The call allocates
- * nothing.  Its first call on a device looks up the array's device address
- * with that device current; make that first call before any stream capture.
- * All calls on a device share the array (it keeps the last call's contents,
- * and each call clears its error word), so calls that overlap on the GPU
- * race: serialise them (one stream, or events).  Device-side errors (a top-k
- * id >= E) skip the slot as in nvfp4_moe_forward but cannot be read back. */
+ * cannot allocate device memory: a plug-in inside a host framework that owns
+ * all device memory through its own pool and forbids side allocations, a
+ * serving loop that cannot take cudaMalloc's implicit device-wide
+ * synchronisation on its latency path, an embedded deployment whose memory
+ * budget is fixed at start-up.  The pages have no counterpart of this entry
+ * point; it is a deployment convenience.
+ * Scratch: one static device array of NVFP4_NOALLOC_SCRATCH_BYTES (32 MiB).
+ * With lazy module loading (the CUDA 12 default) a device holds it from the
+ * first call of this entry point on that device; with
+ * CUDA_MODULE_LOADING=EAGER every device the process initialises holds it;
+ * in both cases until the process exits.  Shapes whose
+ * nvfp4_moe_workspace_size() exceeds it return
+ * NVFP4_ERR_WORKSPACE_TOO_SMALL; like every other argument error, that is
+ * reported before any device work is queued.  The call allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library routine).  Its first
+ * call on a device looks up the array's device address with that device
+ * current (cudaGetSymbolAddress) and caches it: make that first call before
+ * any stream capture, and do not use this entry point across a
+ * cudaDeviceReset.  All calls on a device share the array (it keeps the last
+ * call's contents; each call clears the error word, and the forward rewrites
+ * every other word it reads), so calls that overlap on the GPU race:
+ * serialise them (one stream, or events).  Device-side errors (a top-k id
+ * >= E) skip the slot as in nvfp4_moe_forward but cannot be read back. */
 #define NVFP4_NOALLOC_SCRATCH_BYTES (32u << 20)
 int nvfp4_moe_forward_noalloc(const nvfp4_moe_args *args, void *stream);
 
-/* Failure detection check (no counterpart on the pages): launches one
+/* Test hook for failure detection, not a step of the method (no
+ * counterpart on the pages): launches one
  * thread that runs the fused launch's bounded device wait -- until the
  * device int *flag >= target -- and, when the wait gives up (after 2 s),
  * writes NVFP4_ERR_TIMEOUT into the device int *err if it is still 0.  No
@@ -244,10 +260,26 @@ int nvfp4_debug_bounded_wait(const int32_t *flag, int32_t target, int32_t *err, 
  * clusters of two CTAs.  Both are host outputs. */
 int nvfp4_moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int32_t *fused_l1_l2, int32_t *pair_tiles);
 
-/* Reads and clears the sticky device error word of a workspace (host
- * err_host receives NVFP4_OK or a device error code).  Synchronises
+/* Reads and clears the sticky device error word of a workspace (build
+ * helper: the pages' NaN hunt, page 3 "Root Cause Investigation", checked
+ * every stage for bad values by hand; here the kernels record a top-k id
+ * >= E or a bounded wait that gave up in this word).  Host err_host receives
+ * NVFP4_OK or a device error code.  The only call that synchronises
  * `stream`. */
 int nvfp4_moe_get_error(void *workspace, int32_t *err_host, void *stream);
+
+/* Measurement hook, not a step of the method (the pages have no
+ * counterpart): tensor-core ceiling probe.
+ * Launches `ctas` blocks (one per SM when ctas <= the SM count), each
+ * issuing `iters` k-tiles of four block-scaled FP4 MMAs (M = 128, N = bn,
+ * K = 64, the GEMM engine's instruction) from one thread into one TMEM
+ * accumulator with operands already on chip: the rate the GEMMs cannot
+ * exceed.  FLOPs = ctas * iters * 4 * 2 * 128 * bn * 64.  cycles: device
+ * int64 [ctas], SM clock cycles from first issue to completion per block
+ * (-1 if the bounded completion wait gave up, which also writes
+ * NVFP4_ERR_TIMEOUT to *err when err is not NULL).  bn is 128 or 256;
+ * 1 <= iters <= 1 << 24; 1 <= ctas <= 65535. */
+int nvfp4_fp4_mma_ceiling(int bn, int iters, int ctas, int64_t *cycles, int32_t *err, void *stream);
 
 /* Top-k router: the step that produces topk_ids / topk_weights for
  * nvfp4_moe_forward (page 3 "Architecture Notes": every token is routed to
@@ -264,18 +296,6 @@ int nvfp4_moe_get_error(void *workspace, int32_t *err_host, void *stream);
  * error a few units in the last place).  1 <= k <= min(E, 32), E <= 1024,
  * T >= 0 (T = 0 launches nothing, and the pointers may then be NULL).
  * Allocates nothing. */
-/* Tensor-core ceiling probe (measurement; the pages have no counterpart).
- * Launches `ctas` blocks (one per SM when ctas <= the SM count), each
- * issuing `iters` k-tiles of four block-scaled FP4 MMAs (M = 128, N = bn,
- * K = 64, the GEMM engine's instruction) from one thread into one TMEM
- * accumulator with operands already on chip: the rate the GEMMs cannot
- * exceed.  FLOPs = ctas * iters * 4 * 2 * 128 * bn * 64.  cycles: device
- * int64 [ctas], SM clock cycles from first issue to completion per block
- * (-1 if the bounded completion wait gave up, which also writes
- * NVFP4_ERR_TIMEOUT to *err when err is not NULL).  bn is 128 or 256;
- * 1 <= iters <= 1 << 24; 1 <= ctas <= 65535. */
-int nvfp4_fp4_mma_ceiling(int bn, int iters, int ctas, int64_t *cycles, int32_t *err, void *stream);
-
 #define NVFP4_SCORING_SOFTMAX 0
 #define NVFP4_SCORING_SIGMOID 1
 int nvfp4_moe_topk(const float *logits, int64_t T, int E, int k, int scoring, int32_t *topk_ids,

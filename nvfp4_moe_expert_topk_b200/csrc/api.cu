@@ -346,6 +346,11 @@ Plan moe_plan(int64_t T, int k, int E, int64_t H)
 
 } // namespace
 
+int nvfp4::moe_args_status(const nvfp4_moe_args *args, bool need_out)
+{
+    return check_moe_args(args, need_out);
+}
+
 extern "C" {
 
 const char *nvfp4_status_string(int status)

@@ -51,6 +51,8 @@
 // Every mbarrier wait is bounded (ptx.cuh): on a timeout the block records
 // NVFP4_ERR_TIMEOUT in the error word, stops issuing, waits (bounded) for its
 // copies and MMAs in flight, frees its TMEM and returns.
+#include <mutex>
+
 #include "internal.h"
 #include "quant.cuh"
 
@@ -875,18 +877,11 @@ static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a
                               const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream)
 {
     const int smem = Cfg<BN, CG>::kSmem;
-    static int attr_done_device = -1;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static unsigned long long attr_done = 0;     // one bit per device
+    const cudaError_t e =
+        ensure_smem_limit(reinterpret_cast<const void *>(nvfp4_gemm_kernel<BN, EPI, CG, FUSED, SK>), smem, &attr_done);
     if (e != cudaSuccess)
         return e;
-    if (attr_done_device != dev) {
-        e = cudaFuncSetAttribute(nvfp4_gemm_kernel<BN, EPI, CG, FUSED, SK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 smem);
-        if (e != cudaSuccess)
-            return e;
-        attr_done_device = dev;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kThreads);
@@ -971,12 +966,15 @@ cudaError_t launch_moe_fused(const CUtensorMap &map_a1, const CUtensorMap &map_a
 // device (each CTA needs a whole SM's shared memory), cached per device.
 int gemm_pair_clusters(int num_sms)
 {
-    static int cached_device = -1, cached = 0;
+    constexpr int kMaxDev = 64;
+    static int cached[kMaxDev];             // 0: not yet queried on that device
+    static std::mutex mu;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return num_sms / 2;
-    if (dev == cached_device)
-        return cached;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < kMaxDev && cached[dev] > 0)
+        return cached[dev];
     const int smem = Cfg<256, 2>::kSmem;
     int n = 0;
     if (cudaFuncSetAttribute(nvfp4_gemm_kernel<256, EPI_BF16, 2, 0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -998,8 +996,8 @@ int gemm_pair_clusters(int num_sms)
     (void)cudaGetLastError();
     if (n <= 0 || n > num_sms / 2)
         n = num_sms / 2;
-    cached_device = dev;
-    cached = n;
+    if (dev >= 0 && dev < kMaxDev)
+        cached[dev] = n;
     return n;
 }
 

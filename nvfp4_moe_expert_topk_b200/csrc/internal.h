@@ -29,6 +29,16 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per (kernel, device): *done_mask keeps one bit per device id
+// below 64 (larger ids set the attribute on every call).  Safe to call from
+// several host threads driving different devices.
+cudaError_t ensure_smem_limit(const void *kernel, int bytes, unsigned long long *done_mask);
+
+// Host-side checks of nvfp4_moe_forward's arguments (shapes, null pointers,
+// 16-byte alignment), as a status code; no device work (api.cu).
+int moe_args_status(const nvfp4_moe_args *args, bool need_out);
+
 // Arguments of the persistent block-scaled FP4 GEMM engine (gemm.cu).
 struct GemmArgs {
     // scale factors, NVFP4_SCALES_MMA layout: one 128-row block = (K/64) atoms of 512 bytes

@@ -3,6 +3,7 @@
 // conversion, routing (histogram, prefix sums, stable permutation, m-tile
 // table) and the top-k weighted combine.
 #include <algorithm>
+#include <mutex>
 
 #include "internal.h"
 #include "quant.cuh"
@@ -416,17 +417,20 @@ __global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__
     route_block(ids, R, E, counts, off, poff, num_mtiles, mtiles, num_pairs, pairs, ready, inv, yrow, err, sm);
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device.
-template <typename K>
-static cudaError_t allow_smem(K kernel, int bytes, int *done_device)
+cudaError_t ensure_smem_limit(const void *kernel, int bytes, unsigned long long *done_mask)
 {
+    static std::mutex mu;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || *done_device == dev)
+    if (e != cudaSuccess)
         return e;
+    const unsigned long long bit = dev < 64 ? 1ull << dev : 0ull;
+    std::lock_guard<std::mutex> lock(mu);
+    if (bit != 0 && (*done_mask & bit) != 0)
+        return cudaSuccess;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess)
-        *done_device = dev;
+        *done_mask |= bit;
     return e;
 }
 
@@ -435,8 +439,8 @@ cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, 
                          int32_t *inv, int32_t *yrow, int32_t *err, cudaStream_t s)
 {
     const size_t smem = sizeof(int32_t) * (34 * static_cast<size_t>(E));
-    static int attr_device = -1;
-    cudaError_t e = allow_smem(route_kernel, 34 * 1024 * 4, &attr_device);
+    static unsigned long long attr_done = 0;
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(route_kernel), 34 * 1024 * 4, &attr_done);
     if (e != cudaSuccess)
         return e;
     return launch_pdl(route_kernel, dim3(1), dim3(1024), smem, s, ids, static_cast<int>(R), E, counts, off, poff,

@@ -91,6 +91,7 @@ def test_argument_checks_before_any_launch(L):
                         None) == -1                                                     # segment end % 32
     assert L.nvfp4_gemm(fake, fake, fake, 8, fake, fake, fake, cseg, 1, 256, 128, fake, 100, None) == -1   # ldo < N
     assert L.nvfp4_moe_forward(None, fake, 1 << 30, None) == -1
+    assert L.nvfp4_moe_forward_noalloc(None, None) == -1
     assert L.nvfp4_moe_get_error(None, None, None) == -1
 
 
@@ -107,8 +108,13 @@ def test_moe_forward_checks(L):
     a.I = 3072
     a.w2_codes = F + 8
     assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None) == -3
+    assert L.nvfp4_moe_forward_noalloc(ctypes.byref(a), None) == -3    # checked before the scratch is touched
     a.w2_codes = None
     assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None) == -1
+    assert L.nvfp4_moe_forward_noalloc(ctypes.byref(a), None) == -1
+    a.w2_codes = F
+    a.out = None
+    assert L.nvfp4_moe_forward_noalloc(ctypes.byref(a), None) == -1
 
 
 def test_topk_checks(L):

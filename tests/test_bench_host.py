@@ -81,3 +81,21 @@ def test_config_block_names_the_workload():
     c1 = bench.config_block(W.MOE_CONFIGS["decode_shared"], 1)
     assert c1["workload"] == "decode_shared_moe_E49_k7_T64_H7168_I3072"
     assert c1["parallelism"] == "replicas"
+
+
+def test_clock_regions_summarise_only_their_samples():
+    c = bench.Clocks(device=None)
+    c.source = "test"
+    cap, hw = bench.Clocks.REASONS["sw_power_cap"], bench.Clocks.REASONS["hw_slowdown"]
+    # (monotonic s, SM MHz, max MHz, power W, reason bits)
+    c.samples = [(1.0, 1965.0, 1965.0, 400.0, 0), (2.0, 1400.0, 1965.0, 990.0, cap),
+                 (2.1, 1420.0, 1965.0, 995.0, cap), (3.0, 1000.0, 1965.0, 500.0, hw)]
+    c.regions = {"a": (1.5, 2.5), "b": (2.9, 3.1), "empty": (5.0, 6.0)}
+    a = c.summary(["a"])
+    assert a["sm_mhz"] == 1410.0 and a["samples"] == 2 and a["reasons"] == ["sw_power_cap"]
+    assert c.summary(["b"])["reasons"] == ["hw_slowdown"]
+    assert c.summary(["empty"])["samples"] == 0 and c.mhz("empty") is None
+    both = c.summary()
+    assert both["samples"] == 3 and both["sm_max_mhz"] == 1965.0
+    t = bench.compact({"x": 3.14159265, "y": [2.718281828], "z": "s", "n": 7})
+    assert t == {"x": 3.142, "y": [2.718], "z": "s", "n": 7}

@@ -105,23 +105,22 @@ def tiny():
     return Problem(W.MOE_CONFIGS["tiny"])
 
 
-def test_tiny_end_to_end_and_intermediates(tiny):
-    p = tiny
+def check_intermediates(p, ws, inter):
+    """Inside the forward's workspace: inv and counts equal the oracle's
+    routing; x's codes and scales at every slot's padded row are bit-exact;
+    h codes (which depend on fp32 accumulation order) >= 99 % identical with
+    every mismatch an adjacent code; the oracle's L2 GEMM fed the GPU's own h
+    matches the GPU's y within 5e-3 per row."""
     cfg = p.cfg
     T, k, H, I = p.x.shape[0], cfg.k, cfg.H, cfg.I
-    check_weights_bitexact(p, range(cfg.E))
-    out, ws = p.run()
-    ref, inter = p.oracle(intermediates=True)
-    check_output(out, ref)
-    assert nvfp4_moe_get_error(ws) == 0
     wsn = ws.cpu().numpy()
-
     route = O.route(p.ids.numpy(), cfg.E)
     o, n = region(p, 5)
     inv = wsn[o:o + n].view(np.int32)
     np.testing.assert_array_equal(inv, route["pos_padded"])
     o, n = region(p, 6)
     np.testing.assert_array_equal(wsn[o:o + n].view(np.int32), route["counts"])
+    live = inv >= 0
 
     # x codes / scales at every slot's padded row: bit-exact
     xc, xs = O.quantize_bf16(W.bf16_bits(p.x), p.x_gs)
@@ -130,34 +129,49 @@ def test_tiny_end_to_end_and_intermediates(tiny):
     o, n = region(p, 1)
     a_sc = from_mma_layout(wsn[o:o + n], a_codes.shape[0], H)
     tok = np.arange(T * k) // k
-    np.testing.assert_array_equal(a_codes[inv], xc[tok])
-    np.testing.assert_array_equal(a_sc[inv], xs[tok])
+    np.testing.assert_array_equal(a_codes[inv[live]], xc[tok[live]])
+    np.testing.assert_array_equal(a_sc[inv[live]], xs[tok[live]])
 
     # h codes: fp32 accumulation order may move a value across a rounding edge
     o, n = region(p, 2)
-    h_codes = wsn[o:o + n].reshape(-1, I // 2)[inv]
+    h_codes = wsn[o:o + n].reshape(-1, I // 2)[inv[live]]
     o, n = region(p, 3)
-    h_sc = from_mma_layout(wsn[o:o + n], a_codes.shape[0], I)[inv]
-    ref_q = np.stack([inter["h_codes"] & 15, inter["h_codes"] >> 4], -1).reshape(T * k, I)
-    got_q = np.stack([h_codes & 15, h_codes >> 4], -1).reshape(T * k, I)
+    h_sc = from_mma_layout(wsn[o:o + n], a_codes.shape[0], I)[inv[live]]
+    ref_codes = inter["h_codes"][live]
+    ref_q = np.stack([ref_codes & 15, ref_codes >> 4], -1).reshape(-1, I)
+    got_q = np.stack([h_codes & 15, h_codes >> 4], -1).reshape(-1, I)
     same = got_q == ref_q
     assert same.mean() >= 0.99, same.mean()
     mag = lambda c: np.where(c & 8, -(c & 7).astype(int), (c & 7).astype(int))
     assert np.all(np.abs(mag(got_q) - mag(ref_q))[~same] <= 1)
-    assert (h_sc == inter["h_scales"]).mean() >= 0.99
+    assert (h_sc == inter["h_scales"][live]).mean() >= 0.99
 
     # staged: oracle L2 on the GPU's own h, per expert, against the GPU's y
     o, n = region(p, 4)
     y = wsn[o:o + n].view(np.uint16).reshape(T * k, H)
     y = (y.astype(np.uint32) << 16).view(np.float32)
-    yrow = route["offsets"][p.ids.numpy().reshape(-1)] + route["rank"]
+    flat = p.ids.numpy().reshape(-1)
+    yrow = np.where(live, route["offsets"][np.clip(flat, 0, cfg.E - 1)] + route["rank"], -1)
+    live_idx = np.nonzero(live)[0]
     for e in range(cfg.E):
-        sl = np.nonzero(p.ids.numpy().reshape(-1) == e)[0]
-        if sl.size == 0:
+        sel = np.nonzero(flat[live_idx] == e)[0]          # positions among the live slots
+        if sel.size == 0:
             continue
-        ye = O.gemm(h_codes[sl], h_sc[sl], p.inter_gs[e], p.ow.w2_codes[e], p.ow.w2_scales[e], p.ow.w2_gs[e:e + 1])
-        err = row_rel_l2(y[yrow[sl]], ye)
+        j = p.ow.experts.index(e)
+        ye = O.gemm(h_codes[sel], h_sc[sel], p.inter_gs[e], p.ow.w2_codes[j], p.ow.w2_scales[j],
+                    p.ow.w2_gs[j:j + 1])
+        err = row_rel_l2(y[yrow[live_idx[sel]]], ye)
         assert err.max() <= 5e-3, (e, err.max())
+
+
+def test_tiny_end_to_end_and_intermediates(tiny):
+    p = tiny
+    check_weights_bitexact(p, range(p.cfg.E))
+    out, ws = p.run()
+    ref, inter = p.oracle(intermediates=True)
+    check_output(out, ref)
+    assert nvfp4_moe_get_error(ws) == 0
+    check_intermediates(p, ws, inter)
 
 
 def test_tiny_with_skipped_slots(tiny):
@@ -239,18 +253,63 @@ def test_full_size_configs(name):
     p = Problem(cfg)
     check_weights_bitexact(p, [0, cfg.E - 1])
     out, ws = p.run()
-    ref = p.oracle()
+    ref, inter = p.oracle(intermediates=True)
     check_output(out, ref)
     assert nvfp4_moe_get_error(ws) == 0
+    if name == "decode":            # the full-size epilogue's h codes and the staged L2 as well
+        check_intermediates(p, ws, inter)
+
+
+def test_prefill_ep48_full_output():
+    """Prefill-shaped routing on one expert-parallel slice (48 experts, top-6,
+    T = 512, Zipf-skewed with 2 empty experts, heavy experts of several
+    128-row m-tiles next to experts of a few rows): every output row against
+    the oracle, and the intermediates inside the workspace."""
+    cfg = W.MOE_CONFIGS["prefill_ep48"]
+    p = Problem(cfg)
+    counts = np.bincount(p.ids.numpy().ravel(), minlength=cfg.E)
+    assert (counts == 0).sum() >= 2 and counts.max() > 256 and ((counts > 0) & (counts <= 32)).any()
+    out, ws = p.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    ref, inter = p.oracle(intermediates=True)
+    check_output(out, ref)
+    check_intermediates(p, ws, inter)
+
+
+def boundary_tokens(ids, E, k):
+    """Tokens whose routed slots land where a full-size launch does something
+    special: the heaviest expert's first row, the rows on both sides of its
+    first 128-row and 256-row boundaries, a row of a middle m-tile and the
+    last row of its last (partial) m-tile; the second heaviest expert's first
+    row of its second m-tile and its last row; the first row of the expert
+    with the fewest rows (one or two)."""
+    flat = ids.reshape(-1)
+    counts = np.bincount(flat[flat >= 0], minlength=E)
+    order = np.argsort(-counts, kind="stable")
+
+    def tok(e, r):
+        return int(np.nonzero(flat == e)[0][min(r, counts[e] - 1)]) // k
+
+    e0, e1 = int(order[0]), int(order[1])
+    c0 = int(counts[e0])
+    mid = ((c0 + 127) // 128 // 2) * 128 + 5
+    picks = [tok(e0, r) for r in (0, 127, 128, 255, 256, mid, c0 - 1)]
+    picks += [tok(e1, 128), tok(e1, int(counts[e1]) - 1)]
+    emin = int(np.where(counts > 0, counts, np.iinfo(np.int64).max).argmin())
+    picks.append(tok(emin, 0))
+    return sorted(set(picks))
 
 
 @pytest.mark.parametrize("name", ["prefill", "prefill_shared"])
 def test_prefill_sampled_tokens(name):
     """384 experts, Zipf-skewed routing with empty experts: the whole batch on
-    the GPU, sampled tokens through the oracle.  prefill_shared adds the shared
+    the GPU; through the oracle, the tokens at the launch's boundaries
+    (boundary_tokens) and four random ones.  prefill_shared adds the shared
     expert as a 385th group that every token reaches (32 m-tiles)."""
     cfg = W.MOE_CONFIGS[name]
-    tokens = np.sort(np.random.default_rng(0).choice(cfg.T, 6, replace=False))
+    ids = W.batch(cfg)[1].numpy()
+    targeted = boundary_tokens(ids, cfg.E, cfg.k)
+    tokens = np.unique(np.concatenate([targeted, np.random.default_rng(0).choice(cfg.T, 4, replace=False)]))
     p = Problem(cfg, oracle_tokens=tokens)
     route = O.route(p.ids.numpy(), cfg.E)
     assert (route["counts"] == 0).sum() >= 16                  # some experts are empty
@@ -370,12 +429,15 @@ def test_edge_shapes_end_to_end(cfg):
 
 def test_prefill_pure_zipf_sampled_tokens():
     """The prefill batch with pure Zipf popularity (no empty expert, the
-    heaviest expert ~3100 rows): sampled tokens through the oracle."""
+    heaviest expert ~3100 rows, one expert of a single row): the boundary
+    tokens and two random ones through the oracle."""
     cfg = W.MOE_CONFIGS["prefill_zipf_pure"]
-    tokens = np.sort(np.random.default_rng(1).choice(cfg.T, 4, replace=False))
+    ids = W.batch(cfg)[1].numpy()
+    targeted = boundary_tokens(ids, cfg.E, cfg.k)
+    tokens = np.unique(np.concatenate([targeted, np.random.default_rng(1).choice(cfg.T, 2, replace=False)]))
     p = Problem(cfg, oracle_tokens=tokens)
     route = O.route(p.ids.numpy(), cfg.E)
-    assert (route["counts"] == 0).sum() == 0
+    assert (route["counts"] == 0).sum() == 0 and (route["counts"] == 1).sum() >= 1
     out, ws = p.run()
     assert nvfp4_moe_get_error(ws) == 0
     ref = O.moe_forward(W.bf16_bits(p.x[tokens]), p.ow.remap_ids(p.ids.numpy()[tokens]), p.w.numpy()[tokens],
