@@ -49,6 +49,8 @@ BF16_TO_FP4_NOMINAL_RATIO = 4.0        # 9 / 2.25 PFLOP/s dense
 STAGES = ["global_scale", "route", "quantize_permute", "l1_gate_up_swiglu_quant", "l2_down", "combine"]
 FRONT_STAGE = "front"                  # global scale of the batch + routing + quantise/permute
 FUSED_STAGE = "l1_l2_fused"            # L1 and L2 as one launch (nvfp4_moe_plan)
+PAIRS_STAGE = "pairs_l1_l2"            # pair mode 1: the heavy experts' pair-tile L1 and L2 launches
+LIGHT_STAGE = "l1_l2_fused_light"      # pair mode 1: the fused 1-CTA launch over the other m-tiles
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 GEMM_SOURCES = ["gemm.cu", "ptx.cuh", "quant.cuh", "internal.h"]
 
@@ -280,24 +282,14 @@ class Workload:
         nvfp4_moe_calibrate(xw, idw.to(dev), ww.to(dev), gsw, **self.weights.args(), inter_gs_out=self.inter_gs,
                             workspace=wsw)
         del wsw
-        counts = np.bincount(ids.numpy().reshape(-1), minlength=cfg.E)
-        self.rows = int(counts.sum())
-        self.nonempty = int((counts > 0).sum())
-        self.fused, self.pair_tiles = nvfp4_moe_plan(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I)
-        # global scale, route, quantise, L1 + L2 (one launch or two), combine
-        self.launches_per_step = 5 if self.fused else 6
+        self.counts = np.bincount(ids.numpy().reshape(-1), minlength=cfg.E)
+        self.rows = int(self.counts.sum())
+        self.nonempty = int((self.counts > 0).sum())
+        self.fused, self.pair_mode = nvfp4_moe_plan(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I)
+        self.launches_per_step = launches_per_step(self.fused, self.pair_mode)
 
     def fold(self, per_stage):
-        """Per-stage figures keyed by the stages the forward runs: the front
-        (global scale of the batch, routing, quantise+permute: three small
-        launches), the GEMMs (with the fused plan L1 and L2 are one launch,
-        whose time sits in the L1 slot of the timed forward, the L2 slot being
-        empty) and the combine."""
-        d = dict(per_stage)
-        d[FRONT_STAGE] = d.pop("global_scale") + d.pop("route") + d.pop("quantize_permute")
-        if self.fused:
-            d[FUSED_STAGE] = d.pop("l1_gate_up_swiglu_quant") + d.pop("l2_down")
-        return d
+        return fold_stages(per_stage, self.fused, self.pair_mode)
 
     def step(self, events=None):
         # x_gs = None: the forward computes this batch's global scale itself
@@ -314,25 +306,86 @@ class Workload:
         return 2.0 * self.rows * 3 * c.H * c.I
 
     def kernel_bytes(self):
-        c = self.cfg
-        fp4 = 0.5 + 1.0 / 16                # code + scale bytes per element
-        R, T, H, I, k = self.rows, c.T, c.H, c.I, c.k
-        w13 = self.nonempty * 2 * I * H * fp4
-        w2 = self.nonempty * H * I * fp4
-        return {
-            "global_scale": T * H * 2.0,
-            "route": T * k * 4.0 * 2 + c.E * 16.0,
-            "quantize_permute": T * H * 2.0 + R * H * fp4 + T * k * 4.0,
-            "l1_gate_up_swiglu_quant": w13 + R * H * fp4 + R * I * fp4,
-            "l2_down": w2 + R * I * fp4 + R * H * 2.0,
-            "combine": R * H * 2.0 + T * H * 2.0 + T * k * 12.0,
-        }
+        """Algorithmic bytes of each stage the plan runs (stage_bytes)."""
+        return stage_bytes(self.cfg, self.counts, self.fused, self.pair_mode)
 
     def step_bytes(self):
         """Algorithmic bytes of one step: non-empty experts' weights + x in + out + ids/weights."""
         c = self.cfg
         fp4 = 0.5 + 1.0 / 16
         return self.nonempty * 3 * c.H * c.I * fp4 + 2 * c.T * c.H * 2.0 + c.T * c.k * 8.0
+
+
+FP4_BYTES = 0.5 + 1.0 / 16             # NVFP4 code + scale bytes per element
+
+
+def launches_per_step(fused, pair_mode):
+    """Launches of one forward: the front, the GEMMs, the combine."""
+    gemm = {0: 1 if fused else 2, 1: 2 + (1 if fused else 2), 2: 2}[pair_mode]
+    return 2 + gemm
+
+
+def fold_stages(per_stage, fused, pair_mode):
+    """The timed forward's six stage slots (nvfp4_moe_forward_timed) keyed by
+    what the plan runs there: the front (one launch: global scale, routing,
+    quantise + permute) and then
+      pair mode 0, fused   the fused 1-CTA L1 + L2 launch;
+      pair mode 1          the heavy experts' pair L1 + L2 launches, then the
+                           fused 1-CTA launch over the other m-tiles;
+      otherwise            L1, then L2;
+    and the combine."""
+    d = dict(per_stage)
+    d[FRONT_STAGE] = d.pop("global_scale") + d.pop("route") + d.pop("quantize_permute")
+    if pair_mode == 1:
+        d[PAIRS_STAGE] = d.pop("l1_gate_up_swiglu_quant")
+        d[LIGHT_STAGE] = d.pop("l2_down")
+    elif fused and pair_mode == 0:
+        d[FUSED_STAGE] = d.pop("l1_gate_up_swiglu_quant") + d.pop("l2_down")
+    return d
+
+
+def tile_split(counts, pair_mode):
+    """Per expert: (rows on pair tiles, rows on 1-CTA tiles), the rule the
+    routing applies (pair mode 1: the full m-tile pairs of experts with two or
+    more 128-row m-tiles; 2: everything)."""
+    tiles = (counts + 127) // 128
+    if pair_mode == 2:
+        npair = (tiles + 1) // 2
+    elif pair_mode == 1:
+        npair = np.where(tiles >= 2, tiles // 2, 0)
+    else:
+        npair = np.zeros_like(tiles)
+    pair_rows = np.minimum(counts, 256 * npair)
+    return pair_rows, counts - pair_rows
+
+
+def stage_bytes(cfg, counts, fused, pair_mode):
+    """Algorithmic bytes per stage: each launch reads the weights of the
+    experts it touches once, its activation rows once and writes its outputs
+    once (real rows only; workspace traffic beyond that is implementation's)."""
+    T, H, I, k, E = cfg.T, cfg.H, cfg.I, cfg.k, cfg.E
+    R = int(counts.sum())
+
+    def gemm(rows_e):
+        n_exp = int((rows_e > 0).sum())
+        r = int(rows_e.sum())
+        l1 = n_exp * 2 * I * H * FP4_BYTES + r * H * FP4_BYTES + r * I * FP4_BYTES
+        l2 = n_exp * H * I * FP4_BYTES + r * I * FP4_BYTES + r * H * 2.0
+        return l1, l2
+
+    d = {FRONT_STAGE: T * H * 2.0 + R * H * FP4_BYTES + T * k * 4.0 * 3 + E * 16.0,
+         "combine": R * H * 2.0 + T * H * 2.0 + T * k * 12.0}
+    pair_rows, light_rows = tile_split(counts, pair_mode)
+    if pair_mode == 1:
+        d[PAIRS_STAGE] = sum(gemm(pair_rows))
+        d[LIGHT_STAGE] = sum(gemm(light_rows))
+    else:
+        l1, l2 = gemm(counts)
+        if fused and pair_mode == 0:
+            d[FUSED_STAGE] = l1 + l2
+        else:
+            d["l1_gate_up_swiglu_quant"], d["l2_down"] = l1, l2
+    return d
 
 
 def _capture(fn):
@@ -865,7 +918,7 @@ def _run_all(args, world, rank, dev, peaks, peak_src, steps, warmup):
     tokens_s = world * pre.cfg.T / t_step
     tflops = pre.flops() / t_step / 1e12
     fp4_measured = peaks["bf16_tflops_sustained"] * BF16_TO_FP4_NOMINAL_RATIO
-    kb = pre.fold(pre.kernel_bytes())
+    kb = pre.kernel_bytes()
     dominant = max(stages_pre, key=lambda s: stages_pre[s])
     dom_ms = stages_pre[dominant]
     achieved = kb[dominant] / (dom_ms / 1e3) / 1e9
@@ -874,7 +927,7 @@ def _run_all(args, world, rank, dev, peaks, peak_src, steps, warmup):
 
     t_dec = ms_dec / steps / 1e3
     dec_gbs = dec.step_bytes() / t_dec / 1e9
-    dec_kb = dec.fold(dec.kernel_bytes())
+    dec_kb = dec.kernel_bytes()
     dec_dom = max(stages_dec, key=lambda s: stages_dec[s])
     dec_ach = dec_kb[dec_dom] / (stages_dec[dec_dom] / 1e3) / 1e9
     r_pre, r_dec = f"{mode}_{pre.cfg.name}", f"{mode}_{dec.cfg.name}"
@@ -962,7 +1015,7 @@ def run_single(name, world, rank, dev, peaks, peak_src, steps, warmup):
         raise RuntimeError(f"device error word {err}")
     t = ms_dec / steps / 1e3
     gbs = dec.step_bytes() / t / 1e9
-    kb = dec.fold(dec.kernel_bytes())
+    kb = dec.kernel_bytes()
     dom = max(stages, key=lambda s: stages[s])
     achieved = kb[dom] / (stages[dom] / 1e3) / 1e9
     line = {"metric": f"moe_{name}_GB_per_s", "value": gbs, "unit": "GB/s", "n_gpus": world, "steps": steps,

@@ -169,21 +169,21 @@ size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
 /* out = sum_j topk_weights[t,j] * Expert_{ids[t,j]}(x[t]) with
  * Expert_e(x) = W2_e . q(SiLU(W13g_e . q(x)) * (W13u_e . q(x))), all GEMMs
  * in NVFP4 on the tensor cores, q() the NVFP4 quantiser (x with x_gs, h with
- * inter_gs[e]).  Launches on `stream`: the global scale of x when x_gs is
- * NULL (an 8-byte memset of the workspace and one kernel), routing,
- * quantise+permute, L1 (fused SiLU*up re-quantise epilogue) and L2 (one fused
- * launch or two, see nvfp4_moe_plan) and the combine; no host sync, no
+ * inter_gs[e]).  Launches on `stream`: the front (one kernel: the global
+ * scale of x when x_gs is NULL, routing, quantise+permute), L1 (fused
+ * SiLU*up re-quantise epilogue) and L2 (one to three launches, see
+ * nvfp4_moe_plan) and the combine; no memset, no host sync, no
  * allocation, so the call can be captured in a CUDA graph (make one eager
  * call per device first: it sets per-kernel attributes). */
 int nvfp4_moe_forward(const nvfp4_moe_args *args, void *workspace, size_t ws_bytes, void *stream);
 
 /* Measurement hook, not a step of the method: nvfp4_moe_forward with CUDA
- * events recorded on `stream` at its stage
- * boundaries: events = 6 cudaEvent_t handles created by the caller, recorded
- * before the global scale (x_gs NULL) and routing, before quantise+permute,
- * before L1, after L1, after L2 (directly after L1's record when they are
- * one launch) and after the combine.  Otherwise
- * identical; for per-stage timing.  While `stream` is being captured into a
+ * events recorded on `stream` at its stage boundaries: events = 6
+ * cudaEvent_t handles created by the caller; event 0 before the front
+ * launch, 1 and 2 after it, 3 and 4 after the first and the second GEMM
+ * stage of the plan (nvfp4_moe_plan says which launches each holds; a stage
+ * may be empty) and 5 after the combine.  Otherwise identical; for
+ * per-stage timing.  While `stream` is being captured into a
  * CUDA graph the records become external event nodes, so the events can be
  * timed after each replay. */
 int nvfp4_moe_forward_timed(const nvfp4_moe_args *args, void *workspace, size_t ws_bytes, void *stream,
@@ -212,7 +212,12 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
  * region: 0 A codes, 1 A scales (MMA layout), 2 h codes, 3 h scales
  * (MMA layout), 4 y (bf16 [T*k, H], rows in expert-major routing order),
  * 5 inv, 6 counts, 7 padded offsets, 8 the fp32 global scale of x computed
- * by the last call made with x_gs = NULL. */
+ * by the last call made with x_gs = NULL, 9 the m-tile table (int32 x 4 per
+ * m-tile: expert, first padded row, rows, first y row), 10 the pair table
+ * (int32 x 2 per pair: first m-tile, second m-tile or -1), 11 the light list
+ * (int32 m-tile indices run on 1-CTA tiles), 12 the 256-byte header (int32
+ * error word at byte 0, m-tile count at 4, pair count at 8, light count at
+ * 24). */
 int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, int region,
                                int64_t *offset, int64_t *bytes);
 
@@ -252,12 +257,24 @@ int nvfp4_moe_forward_noalloc(const nvfp4_moe_args *args, void *stream);
 int nvfp4_debug_bounded_wait(const int32_t *flag, int32_t target, int32_t *err, void *stream);
 
 /* Execution plan nvfp4_moe_forward uses for a shape (host only, no GPU
- * work): *fused_l1_l2 = 1 when L1 and L2 run as one persistent launch (the
- * L2 tiles of an m-tile start as soon as that m-tile's L1 tiles have written
- * h; per-stage timing then reports L1 + L2 as one stage, between events 2
- * and 3 of nvfp4_moe_forward_timed, and an empty stage between 3 and 4);
- * *pair_tiles = 1 when the grouped GEMMs run on 256-row tiles computed by
- * clusters of two CTAs.  Both are host outputs. */
+ * work; page 3 "Architecture Notes": a persistent grouped GEMM over skewed
+ * expert loads).  Each expert's routed rows form 128-row m-tiles.
+ * *pair_tiles (the pair mode):
+ *   0  every m-tile runs on 1-CTA tiles (128 x 256);
+ *   1  batches of >= 2048 routed rows: an expert with two or more m-tiles
+ *      runs its consecutive full pairs of m-tiles on pair tiles (256 x 256,
+ *      a cluster of two CTAs sharing each weight tile), in an L1 launch and
+ *      an L2 launch of their own; its odd last m-tile and every other expert
+ *      run on 1-CTA tiles;
+ *   2  experts average two full m-tiles or more (T*k >= 256*E): every m-tile
+ *      on pair tiles (an odd last m-tile with an empty partner).
+ * *fused_l1_l2 = 1 when the 1-CTA tiles run L1 and L2 in one persistent
+ * launch (the L2 tiles of an m-tile start as soon as that m-tile's L1 tiles
+ * have written h).  Stages between the events of nvfp4_moe_forward_timed:
+ * 0-1 the front launch (1-2 empty); then pair mode 0 fused: 2-3 the fused
+ * launch (3-4 empty); pair mode 1: 2-3 the pair L1 and L2 launches, 3-4 the
+ * fused 1-CTA launch; otherwise 2-3 L1, 3-4 L2; 4-5 the combine.  Both
+ * outputs are host ints. */
 int nvfp4_moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int32_t *fused_l1_l2, int32_t *pair_tiles);
 
 /* Reads and clears the sticky device error word of a workspace (build

@@ -304,10 +304,11 @@ def nvfp4_fp4_mma_ceiling(bn, iters, cycles, err=None, stream=None):
 
 
 def nvfp4_moe_plan(T, k, E, H, I):
-    """(fused_l1_l2, pair_tiles) booleans of the forward's execution plan."""
+    """(fused_l1_l2: bool, pair_mode: 0 | 1 | 2) of the forward's execution
+    plan (see nvfp4_moe_plan in include/nvfp4moe.h)."""
     f, pt = ctypes.c_int32(), ctypes.c_int32()
     _check(lib().nvfp4_moe_plan(T, k, E, H, I, ctypes.byref(f), ctypes.byref(pt)), "nvfp4_moe_plan")
-    return bool(f.value), bool(pt.value)
+    return bool(f.value), int(pt.value)
 
 
 def nvfp4_amax(x, amax_out, stream=None):

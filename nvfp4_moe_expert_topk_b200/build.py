@@ -11,7 +11,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libnvfp4moe.so")
-SOURCES = ["api.cu", "kernels.cu", "gemm.cu", "noalloc.cu", "ceiling.cu"]
+SOURCES = ["api.cu", "front.cu", "kernels.cu", "gemm.cu", "noalloc.cu", "ceiling.cu"]
 HEADERS = ["internal.h", "ptx.cuh", "quant.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

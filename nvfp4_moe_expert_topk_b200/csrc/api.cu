@@ -89,13 +89,16 @@ int64_t round_up(int64_t v, int64_t m)
 // ---------------------------------------------------------------- workspace
 struct Layout {
     int64_t mt_max = 0, rpad = 0;
-    int64_t counts = 0, off = 0, poff = 0, mtiles = 0, pairs = 0, ready = 0, inv = 0, yrow = 0, amax = 0;
+    int64_t counts = 0, off = 0, poff = 0, mtiles = 0, pairs = 0, light = 0, ready = 0, inv = 0, yrow = 0, amax = 0;
+    int64_t blk_hist = 0, blk_amax = 0;
     int64_t a_codes = 0, a_sf = 0, h_codes = 0, h_sf = 0, y = 0, total = 0;
 };
 
 // Header (256 B): int32 error word at 0, int32 m-tile count at 4, int32
 // m-tile pair count at 8, fp32 global scale of x computed from the batch at
-// 12 and its completion ticket at 16.
+// 12, the front launch's grid ticket at 20, int32 light m-tile count at 24.
+constexpr int kHdrNumMtiles = 4, kHdrNumPairs = 8, kHdrGs = 12, kHdrTicket = 20, kHdrNumLight = 24;
+
 Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
 {
     Layout L;
@@ -115,9 +118,12 @@ Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
     L.amax = take(4 * E);
     L.mtiles = take(16 * std::max<int64_t>(L.mt_max, 1));
     L.pairs = take(8 * std::max<int64_t>(L.mt_max, 1));
+    L.light = take(4 * std::max<int64_t>(L.mt_max, 1));
     L.ready = take(4 * std::max<int64_t>(L.mt_max, 1));
     L.inv = take(4 * std::max<int64_t>(R, 1));
     L.yrow = take(4 * std::max<int64_t>(R, 1));
+    L.blk_hist = take(4LL * kFrontMaxBlocks * ((E + 3) & ~3));
+    L.blk_amax = take(4LL * kFrontMaxBlocks);
     L.a_codes = take(L.rpad * (H / 2));
     L.a_sf = take(L.rpad * (H / 16));
     L.h_codes = take(L.rpad * (I / 2));
@@ -189,6 +195,11 @@ int moe_cg(int64_t R, int E)
     return R >= 256LL * E ? 2 : 1;
 }
 
+// Batches of at least this many routed rows put the pairs of full m-tiles of
+// experts with two or more m-tiles on pair tiles (pair mode 1): the pair
+// launches cost a few microseconds even when no expert is that heavy.
+constexpr int64_t kSplitMinRows = 2048;
+
 int gemm_grid(int cg, int64_t tiles, int num_sms)
 {
     if (cg == 2)
@@ -200,7 +211,7 @@ int gemm_grid(int cg, int64_t tiles, int num_sms)
 // kernel computes from the batch into the workspace header.
 const float *x_gs_ptr(const nvfp4_moe_args *a, uint8_t *ws)
 {
-    return a->x_gs != nullptr ? a->x_gs : reinterpret_cast<const float *>(ws + 12);
+    return a->x_gs != nullptr ? a->x_gs : reinterpret_cast<const float *>(ws + kHdrGs);
 }
 
 // Maps and arguments of the grouped L1 GEMM (gate_up, SwiGLU epilogue).
@@ -223,10 +234,12 @@ int l1_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, CUtensorMap 
     g->sfb_block_stride = (H / 64) * 512;
     g->K = static_cast<int>(H);
     g->num_k_tiles = static_cast<int>((H + 255) / 256);
-    g->num_mtiles_dev = reinterpret_cast<int32_t *>(ws + 4);
+    g->num_mtiles_dev = reinterpret_cast<int32_t *>(ws + kHdrNumMtiles);
     g->mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
-    g->num_pairs_dev = reinterpret_cast<int32_t *>(ws + 8);
+    g->num_pairs_dev = reinterpret_cast<int32_t *>(ws + kHdrNumPairs);
     g->pairs = reinterpret_cast<int2 *>(ws + L.pairs);
+    g->num_light_dev = reinterpret_cast<int32_t *>(ws + kHdrNumLight);
+    g->light = reinterpret_cast<int32_t *>(ws + L.light);
     g->ready = reinterpret_cast<int32_t *>(ws + L.ready);
     g->n_tiles = static_cast<int>(I / 128);
     g->b_rows_per_expert = 2 * I;
@@ -267,10 +280,12 @@ int l2_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int bn, CUte
     g->sfb_block_stride = (I / 64) * 512;
     g->K = static_cast<int>(I);
     g->num_k_tiles = static_cast<int>((I + 255) / 256);
-    g->num_mtiles_dev = reinterpret_cast<int32_t *>(ws + 4);
+    g->num_mtiles_dev = reinterpret_cast<int32_t *>(ws + kHdrNumMtiles);
     g->mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
-    g->num_pairs_dev = reinterpret_cast<int32_t *>(ws + 8);
+    g->num_pairs_dev = reinterpret_cast<int32_t *>(ws + kHdrNumPairs);
     g->pairs = reinterpret_cast<int2 *>(ws + L.pairs);
+    g->num_light_dev = reinterpret_cast<int32_t *>(ws + kHdrNumLight);
+    g->light = reinterpret_cast<int32_t *>(ws + L.light);
     g->ready = reinterpret_cast<int32_t *>(ws + L.ready);
     g->n_tiles = static_cast<int>(H / bn);
     g->b_rows_per_expert = H;
@@ -288,49 +303,66 @@ int l2_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int bn, CUte
     return NVFP4_OK;
 }
 
-// Global scale of x (when the caller passes none), routing and
-// quantise/permute (events 0-2 when timing: the global scale and routing
-// between 0 and 1, quantisation between 1 and 2).  Shared by forward and
-// calibrate.  (A single cooperative launch of all three, with a grid barrier
-// after the routing and the max|x| pass, measured 5 us slower on the 64-token
-// decode batch than separate launches, and no faster on prefill; so was one
-// launch of routing + quantisation in which every block routes all slots.)
-int run_route_quant(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, void *const *events, cudaStream_t s,
-                    int num_sms)
+// The front of the forward in one launch (front.cu): the global scale of x
+// when the caller passes none, routing and tile tables for `pair_mode`, and
+// quantise/permute; x == nullptr: routing only.  Events 0-2 when timing
+// (0 before it, 1 and 2 after it).  (Earlier designs ran the global scale,
+// the routing and the quantisation as three launches, the routing in one
+// block; one launch with a grid-wide ticket between the histograms and the
+// positions reads x once from HBM and once from L2.)
+FrontArgs front_args(const nvfp4_moe_args *a, const int32_t *ids, int64_t T, int k, int E, uint8_t *ws,
+                     const Layout &L, int pair_mode)
 {
-    const int64_t T = a->T, H = a->H, R = T * a->k;
-    const int E = a->E, k = a->k;
-    int32_t *inv = reinterpret_cast<int32_t *>(ws + L.inv);
+    FrontArgs f{};
+    f.x = a != nullptr ? reinterpret_cast<const __nv_bfloat16 *>(a->x) : nullptr;
+    f.ids = ids;
+    f.T = T;
+    f.H = a != nullptr ? a->H : 128;
+    f.E = E;
+    f.k = k;
+    f.x_gs = a != nullptr ? a->x_gs : nullptr;
+    f.gs_out = reinterpret_cast<float *>(ws + kHdrGs);
+    f.pair_mode = pair_mode;
+    f.counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    f.off = reinterpret_cast<int32_t *>(ws + L.off);
+    f.poff = reinterpret_cast<int32_t *>(ws + L.poff);
+    f.num_mtiles = reinterpret_cast<int32_t *>(ws + kHdrNumMtiles);
+    f.mtiles = reinterpret_cast<int4 *>(ws + L.mtiles);
+    f.num_pairs = reinterpret_cast<int32_t *>(ws + kHdrNumPairs);
+    f.pairs = reinterpret_cast<int2 *>(ws + L.pairs);
+    f.num_light = reinterpret_cast<int32_t *>(ws + kHdrNumLight);
+    f.light = reinterpret_cast<int32_t *>(ws + L.light);
+    f.ready = reinterpret_cast<int32_t *>(ws + L.ready);
+    f.inv = reinterpret_cast<int32_t *>(ws + L.inv);
+    f.yrow = reinterpret_cast<int32_t *>(ws + L.yrow);
+    f.err = reinterpret_cast<int32_t *>(ws);
+    f.a_codes = ws + L.a_codes;
+    f.a_sf = ws + L.a_sf;
+    f.blk_hist = reinterpret_cast<int32_t *>(ws + L.blk_hist);
+    f.blk_amax = reinterpret_cast<float *>(ws + L.blk_amax);
+    f.ticket = reinterpret_cast<unsigned int *>(ws + kHdrTicket);
+    return f;
+}
+
+int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int pair_mode, void *const *events,
+              cudaStream_t s, int num_sms)
+{
     if (mark(events, 0, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
-    if (a->x_gs == nullptr) {
-        // the batch's global scale at ws + 12 (amax, then 2688 / amax by the
-        // last block to finish), its completion ticket at ws + 16
-        float *gs = reinterpret_cast<float *>(ws + 12);
-        if (cudaMemsetAsync(gs, 0, 2 * sizeof(float), s) != cudaSuccess ||
-            launch_amax_bf16(reinterpret_cast<const __nv_bfloat16 *>(a->x), T * H, gs, num_sms, s,
-                             reinterpret_cast<unsigned int *>(ws + 16)) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-    }
-    cudaError_t e = launch_route(a->topk_ids, R, E, reinterpret_cast<int32_t *>(ws + L.counts),
-                                 reinterpret_cast<int32_t *>(ws + L.off), reinterpret_cast<int32_t *>(ws + L.poff),
-                                 reinterpret_cast<int32_t *>(ws + 4), reinterpret_cast<int4 *>(ws + L.mtiles),
-                                 reinterpret_cast<int32_t *>(ws + 8), reinterpret_cast<int2 *>(ws + L.pairs),
-                                 reinterpret_cast<int32_t *>(ws + L.ready), inv,
-                                 reinterpret_cast<int32_t *>(ws + L.yrow), reinterpret_cast<int32_t *>(ws), s);
-    if (e != cudaSuccess || mark(events, 1, s) != NVFP4_OK)
-        return NVFP4_ERR_CUDA;
-    e = launch_quantize(reinterpret_cast<const __nv_bfloat16 *>(a->x), T, H, H, x_gs_ptr(a, ws), ws + L.a_codes,
-                        ws + L.a_sf, NVFP4_SCALES_MMA, inv, k, s);
-    if (e != cudaSuccess || mark(events, 2, s) != NVFP4_OK)
+    if (launch_front(front_args(a, a->topk_ids, a->T, a->k, a->E, ws, L, pair_mode), num_sms, s) != cudaSuccess ||
+        mark(events, 1, s) != NVFP4_OK || mark(events, 2, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
 }
 
 // The forward's execution plan: pair tiles for the grouped GEMMs, and
 // whether L1 and L2 run as one fused launch (1-CTA tiles, 256-wide L2 tiles).
+// pair_mode: 0 every m-tile a 1-CTA tile; 1 the heavy experts' full m-tile
+// pairs on pair tiles (two launches: L1, L2) and the rest on 1-CTA tiles;
+// 2 every m-tile on pair tiles.  fused: the 1-CTA tiles run L1 and L2 in one
+// persistent launch (256-wide L2 tiles).
 struct Plan {
-    int cg;
+    int pair_mode;
     int l2_bn;
     bool fused;
 };
@@ -338,9 +370,15 @@ struct Plan {
 Plan moe_plan(int64_t T, int k, int E, int64_t H)
 {
     Plan pl;
-    pl.cg = moe_cg(T * k, E);
+    const int64_t R = T * k;
     pl.l2_bn = (H % 256 == 0) ? 256 : 128;
-    pl.fused = pl.cg == 1 && pl.l2_bn == 256;
+    if (pl.l2_bn == 256 && moe_cg(R, E) == 2)
+        pl.pair_mode = 2;
+    else if (pl.l2_bn == 256 && R >= kSplitMinRows && E > 1)
+        pl.pair_mode = 1;
+    else
+        pl.pair_mode = 0;
+    pl.fused = pl.pair_mode != 2 && pl.l2_bn == 256;
     return pl;
 }
 
@@ -432,7 +470,7 @@ int nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ldx, c
     if (rows == 0)
         return NVFP4_OK;
     return cuda_status(launch_quantize(reinterpret_cast<const __nv_bfloat16 *>(x), rows, cols, ldx, gs, codes, scales,
-                                       scale_layout, nullptr, 1, static_cast<cudaStream_t>(stream)));
+                                       scale_layout, static_cast<cudaStream_t>(stream)));
 }
 
 int nvfp4_swizzle_scales(const uint8_t *in, int64_t batch, int64_t rows, int64_t cols, uint8_t *out, void *stream)
@@ -628,7 +666,11 @@ int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, in
     case 5: *offset = L.inv; *bytes = R * 4; break;
     case 6: *offset = L.counts; *bytes = 4LL * E; break;
     case 7: *offset = L.poff; *bytes = 4LL * (E + 1); break;
-    case 8: *offset = 12; *bytes = 4; break;
+    case 8: *offset = kHdrGs; *bytes = 4; break;
+    case 9: *offset = L.mtiles; *bytes = 16 * std::max<int64_t>(L.mt_max, 1); break;
+    case 10: *offset = L.pairs; *bytes = 8 * std::max<int64_t>(L.mt_max, 1); break;
+    case 11: *offset = L.light; *bytes = 4 * std::max<int64_t>(L.mt_max, 1); break;
+    case 12: *offset = 0; *bytes = 256; break;
     default: return NVFP4_ERR_INVALID_ARG;
     }
     return NVFP4_OK;
@@ -655,10 +697,10 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
         return NVFP4_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    st = run_route_quant(a, ws, L, events, s, sms);
+    const Plan pl = moe_plan(a->T, a->k, a->E, a->H);
+    st = run_front(a, ws, L, pl.pair_mode, events, s, sms);
     if (st != NVFP4_OK)
         return st;
-    const Plan pl = moe_plan(a->T, a->k, a->E, a->H);
     const int64_t H = a->H;
     CUtensorMap ma1, ma1_32, mb1, ma2, ma2_32, mb2;
     GemmArgs g1, g2;
@@ -667,20 +709,35 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
         st = l2_setup(a, ws, L, pl.l2_bn, &ma2, &ma2_32, &mb2, &g2);
     if (st != NVFP4_OK)
         return st;
-    if (pl.fused) {
-        // L1 and L2 in one launch: no stage boundary between events 3 and 4
-        if (launch_moe_fused(ma1, ma1_32, mb1, g1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
-            mark(events, 3, s) != NVFP4_OK || mark(events, 4, s) != NVFP4_OK)
+    // the pair tiles (heavy experts' m-tile pairs, or every m-tile): L1
+    // launch, then L2 launch; each reads its tile count from the workspace
+    const int pair_grid = gemm_grid(2, 1LL << 30, sms);
+    if (pl.pair_mode != 0) {
+        if (launch_gemm(256, EPI_SWIGLU_QUANT, 2, ma1, ma1_32, mb1, g1, pair_grid, s) != cudaSuccess)
             return NVFP4_ERR_CUDA;
-    } else {
-        const int l2_cg = pl.l2_bn == 256 ? pl.cg : 1;
-        if (launch_gemm(256, EPI_SWIGLU_QUANT, pl.cg, ma1, ma1_32, mb1, g1, gemm_grid(pl.cg, 1LL << 30, sms), s) !=
-                cudaSuccess ||
-            mark(events, 3, s) != NVFP4_OK ||
-            launch_gemm(pl.l2_bn, EPI_BF16, l2_cg, ma2, ma2_32, mb2, g2, gemm_grid(l2_cg, 1LL << 30, sms), s) !=
-                cudaSuccess ||
-            mark(events, 4, s) != NVFP4_OK)
+        if (pl.pair_mode == 2 && mark(events, 3, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
+        if (launch_gemm(256, EPI_BF16, 2, ma2, ma2_32, mb2, g2, pair_grid, s) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        if (mark(events, pl.pair_mode == 2 ? 4 : 3, s) != NVFP4_OK)
+            return NVFP4_ERR_CUDA;
+    }
+    // the 1-CTA tiles (the light list): L1 and L2 in one persistent launch,
+    // or two launches when the L2 tiles are 128 wide
+    if (pl.pair_mode != 2) {
+        if (pl.fused) {
+            if (launch_moe_fused(ma1, ma1_32, mb1, g1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
+                (pl.pair_mode == 0 && mark(events, 3, s) != NVFP4_OK) || mark(events, 4, s) != NVFP4_OK)
+                return NVFP4_ERR_CUDA;
+        } else {
+            if (launch_gemm(256, EPI_SWIGLU_QUANT, 1, ma1, ma1_32, mb1, g1, gemm_grid(1, 1LL << 30, sms), s) !=
+                    cudaSuccess ||
+                mark(events, 3, s) != NVFP4_OK ||
+                launch_gemm(pl.l2_bn, EPI_BF16, 1, ma2, ma2_32, mb2, g2, gemm_grid(1, 1LL << 30, sms), s) !=
+                    cudaSuccess ||
+                mark(events, 4, s) != NVFP4_OK)
+                return NVFP4_ERR_CUDA;
+        }
     }
 
     if (launch_combine(reinterpret_cast<const __nv_bfloat16 *>(ws + L.y),
@@ -709,7 +766,7 @@ int nvfp4_moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int32_t *fused
         return st;
     const Plan pl = moe_plan(T, k, E, H);
     *fused_l1_l2 = pl.fused ? 1 : 0;
-    *pair_tiles = pl.cg == 2 ? 1 : 0;
+    *pair_tiles = pl.pair_mode;
     return NVFP4_OK;
 }
 
@@ -750,7 +807,10 @@ int nvfp4_moe_calibrate(const nvfp4_moe_args *a, float *inter_gs_out, void *work
     if (cudaMemsetAsync(ws + L.amax, 0, 4 * static_cast<size_t>(a->E), s) != cudaSuccess)
         return NVFP4_ERR_CUDA;
     if (a->T > 0) {
-        st = run_route_quant(a, ws, L, nullptr, s, sms);
+        // every m-tile on one kind of tile: all pairs when experts average two
+        // full m-tiles, else all 1-CTA tiles (the warmup epilogue runs once)
+        const int cg = moe_cg(a->T * a->k, a->E);
+        st = run_front(a, ws, L, cg == 2 ? 2 : 0, nullptr, s, sms);
         if (st != NVFP4_OK)
             return st;
         CUtensorMap ma, ma32, mb;
@@ -758,7 +818,6 @@ int nvfp4_moe_calibrate(const nvfp4_moe_args *a, float *inter_gs_out, void *work
         st = l1_setup(a, ws, L, &ma, &ma32, &mb, &g);
         if (st != NVFP4_OK)
             return st;
-        const int cg = moe_cg(a->T * a->k, a->E);
         if (launch_gemm(256, EPI_SWIGLU_AMAX, cg, ma, ma32, mb, g, gemm_grid(cg, 1LL << 30, sms), s) != cudaSuccess)
             return NVFP4_ERR_CUDA;
     }
@@ -779,16 +838,17 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
     const Layout L = ws_layout(T, k, E, 128, 128);
     if (ws_bytes < static_cast<size_t>(L.total))
         return NVFP4_ERR_WORKSPACE_TOO_SMALL;
-    int st = device_check(nullptr);
+    int st = NVFP4_OK;
+    int sms = 0;
+    st = device_check(&sms);
     if (st != NVFP4_OK)
         return st;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    return cuda_status(launch_route(topk_ids, T * k, E, counts, reinterpret_cast<int32_t *>(ws + L.off),
-                                    padded_offsets, reinterpret_cast<int32_t *>(ws + 4),
-                                    reinterpret_cast<int4 *>(ws + L.mtiles), reinterpret_cast<int32_t *>(ws + 8),
-                                    reinterpret_cast<int2 *>(ws + L.pairs), reinterpret_cast<int32_t *>(ws + L.ready),
-                                    inv, reinterpret_cast<int32_t *>(ws + L.yrow), reinterpret_cast<int32_t *>(ws),
-                                    static_cast<cudaStream_t>(stream)));
+    FrontArgs f = front_args(nullptr, topk_ids, T, k, E, ws, L, 0);
+    f.counts = counts;
+    f.poff = padded_offsets;
+    f.inv = inv;
+    return cuda_status(launch_front(f, sms, static_cast<cudaStream_t>(stream)));
 }
 
 int nvfp4_moe_topk_shared(const float *logits, int64_t T, int E, int k, int scoring, int num_shared,

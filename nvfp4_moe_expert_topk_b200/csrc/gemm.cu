@@ -118,8 +118,9 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, const GemmArg
         ti.ph = t >= t1 ? 1 : 0;
         const int n = ti.ph ? p2.n_tiles : p.n_tiles;
         const int tt = ti.ph ? t - t1 : t;
-        const int mt = tt / n;
-        ti.nt = tt - mt * n;
+        const int li = tt / n;
+        ti.nt = tt - li * n;
+        const int mt = p.light[li];
         ti.mt = mt;
         const int4 m = p.mtiles[mt];
         ti.e = m.x;
@@ -151,8 +152,9 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, const GemmArg
         return ti;
     }
     if (p.mtiles != nullptr) {
-        const int mt = t / p.n_tiles;
-        ti.nt = t - mt * p.n_tiles;
+        const int li = t / p.n_tiles;
+        ti.nt = t - li * p.n_tiles;
+        const int mt = p.light[li];
         ti.mt = mt;
         const int4 m = p.mtiles[mt];
         ti.e = m.x;
@@ -366,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_wait();
 
     const int m_units = (p.mtiles != nullptr)
-                            ? *reinterpret_cast<volatile const int32_t *>(kPair ? p.num_pairs_dev : p.num_mtiles_dev)
+                            ? *reinterpret_cast<volatile const int32_t *>(kPair ? p.num_pairs_dev : p.num_light_dev)
                             : (kPair ? (p.dense_M + 2 * kBM - 1) / (2 * kBM) : p.dense_m_tiles);
     const int total = m_units * (p.n_tiles + (FUSED ? p2.n_tiles : 0));
 

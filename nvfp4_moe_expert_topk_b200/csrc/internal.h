@@ -53,6 +53,8 @@ struct GemmArgs {
     const int4 *mtiles;       // {expert, first padded row, valid rows, first output row}
     const int32_t *num_pairs_dev;
     const int2 *pairs;        // pair tiles: {first m-tile, second m-tile of the same expert or -1}
+    const int32_t *num_light_dev;
+    const int32_t *light;     // 1-CTA tiles: the m-tiles not covered by pairs, by index into mtiles
     int32_t *ready;           // fused L1 -> L2 launch: per m-tile count of published L1 epilogue warps
     float *sk_partials;       // stream-K: one slot of 128 x 256 fp32 per CTA
     int32_t *sk_flags;        // stream-K: per (tile, CTA of the pair) count of published partial warps
@@ -109,19 +111,45 @@ cudaError_t launch_moe_fused(const CUtensorMap &map_a1, const CUtensorMap &map_a
                              const GemmArgs &args1, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
                              const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream);
 
+// The forward's front in one launch (front.cu): the batch's global scale of
+// x (x_gs == nullptr), routing and the tile tables, quantise + permute (x ==
+// nullptr: routing only).  pair_mode 0: every m-tile is a 1-CTA ("light")
+// tile; 1: experts with two or more m-tiles give their consecutive full
+// pairs to the pair list and only the odd last m-tile to the light list;
+// 2: every m-tile in a pair (the odd last one with an empty partner).
+constexpr int kFrontMaxBlocks = 256;
+struct FrontArgs {
+    const __nv_bfloat16 *x;
+    const int32_t *ids;
+    int64_t T, H;
+    int E, k;
+    const float *x_gs;
+    float *gs_out;
+    int pair_mode;
+    int32_t *counts, *off, *poff;
+    int32_t *num_mtiles;
+    int4 *mtiles;
+    int32_t *num_pairs;
+    int2 *pairs;
+    int32_t *num_light;
+    int32_t *light;
+    int32_t *ready;           // may be null
+    int32_t *inv, *yrow;
+    int32_t *err;
+    uint8_t *a_codes, *a_sf;  // MMA scale layout
+    int32_t *blk_hist;        // [kFrontMaxBlocks][(E + 3) & ~3]
+    float *blk_amax;          // [kFrontMaxBlocks]
+    unsigned int *ticket;     // zeroed once with the workspace
+};
+cudaError_t launch_front(const FrontArgs &args, int num_sms, cudaStream_t s);
+
 // Memory-bound kernels (kernels.cu).
-// ticket != nullptr (a zeroed counter): *gs_out ends as 2688 / amax, no finalize launch needed.
-cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s,
-                             unsigned int *ticket = nullptr);
+cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s);
 cudaError_t launch_finalize_gs(float *gs, cudaStream_t s);
 cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs,
-                            uint8_t *codes, uint8_t *scales, int layout, const int32_t *inv, int k,
-                            cudaStream_t s);
+                            uint8_t *codes, uint8_t *scales, int layout, cudaStream_t s);
 cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64_t cols, uint8_t *out,
                            cudaStream_t s);
-cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
-                         int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *ready,
-                         int32_t *inv, int32_t *yrow, int32_t *err, cudaStream_t s);
 cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *yrow, const float *w, int64_t T, int k, int64_t H,
                            __nv_bfloat16 *out, cudaStream_t s);
 cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float *inter_gs, cudaStream_t s);

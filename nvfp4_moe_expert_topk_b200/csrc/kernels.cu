@@ -1,7 +1,7 @@
-// kernels.cu -- the memory-bound steps of the chain: global scale, activation
-// quantisation (plain and fused with the expert permutation), scale-layout
-// conversion, routing (histogram, prefix sums, stable permutation, m-tile
-// table) and the top-k weighted combine.
+// kernels.cu -- memory-bound kernels: global scale and max|x| of a tensor,
+// plain NVFP4 quantisation, scale-layout conversion, the top-k weighted
+// combine, the warmup scales and the top-k router.  (The forward's front --
+// global scale, routing, quantise + permute -- is one launch, in front.cu.)
 #include <algorithm>
 #include <mutex>
 
@@ -13,11 +13,8 @@ namespace nvfp4 {
 // ------------------------------------------------------------ global scale
 // amax of a bf16 tensor, accumulated into *out_bits (the float bit pattern;
 // non-negative floats order like their bits).  *out_bits must start at 0.
-// With a ticket (a zeroed counter), the last block to finish turns the
-// amax into the global scale in place: 2688 / amax (1 if amax = 0).
 __global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16 *__restrict__ x, int64_t n,
-                                                        unsigned int *__restrict__ out_bits,
-                                                        unsigned int *__restrict__ ticket)
+                                                        unsigned int *__restrict__ out_bits)
 {
     pdl_wait();
     pdl_trigger();
@@ -58,14 +55,6 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const __nv_bfloat16 *__r
         for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
             m = fmaxf(m, wmax[w]);
         atomicMax(out_bits, __float_as_uint(m));
-        if (ticket != nullptr) {
-            __threadfence();
-            if (atomicAdd(ticket, 1u) == gridDim.x - 1) {     // every block's maximum is in
-                __threadfence();
-                const float a = __uint_as_float(atomicAdd(out_bits, 0u));
-                *reinterpret_cast<float *>(out_bits) = a == 0.0f ? 1.0f : __fdiv_rn(2688.0f, a);
-            }
-        }
     }
 }
 
@@ -78,8 +67,7 @@ __global__ void finalize_gs_kernel(float *gs)
     *gs = (a == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, a);
 }
 
-cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s,
-                             unsigned int *ticket)
+cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, int num_sms, cudaStream_t s)
 {
     int64_t blocks = (n / 8 + 255) / 256;
     if (blocks < 1)
@@ -87,7 +75,7 @@ cudaError_t launch_amax_bf16(const __nv_bfloat16 *x, int64_t n, float *gs_out, i
     if (blocks > 8LL * num_sms)
         blocks = 8LL * num_sms;
     return launch_pdl(amax_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, n,
-                      reinterpret_cast<unsigned int *>(gs_out), ticket);
+                      reinterpret_cast<unsigned int *>(gs_out));
 }
 
 cudaError_t launch_finalize_gs(float *gs, cudaStream_t s)
@@ -96,30 +84,19 @@ cudaError_t launch_finalize_gs(float *gs, cudaStream_t s)
 }
 
 // ------------------------------------------------------------ quantisation
-// One warp per (source row, 2048-column chunk); each lane handles 64
-// consecutive elements (4 blocks).  With inv != nullptr the row is token t of
-// a routed batch and its codes and scales are written to each padded
-// destination row inv[t*k + j] >= 0 (the expert permutation); otherwise to
-// row t.
+// One warp per (row, 2048-column chunk); each lane handles 64 consecutive
+// elements (4 blocks).  (The forward's quantisation of x, fused with the
+// expert permutation, is in front.cu.)
 constexpr int kQuantChunk = 2048;
 
 // One (row, chunk) item by one whole warp (item < rows * chunks).
 __device__ __forceinline__ void quantize_item(const __nv_bfloat16 *__restrict__ x, int64_t cols, int64_t ldx,
                                               float gs, uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
-                                              int layout, const int32_t *__restrict__ inv, int k, int64_t item,
-                                              int lane)
+                                              int layout, int64_t item, int lane)
 {
     const int64_t chunks = (cols + kQuantChunk - 1) / kQuantChunk;
     const int64_t row = item / chunks;
     const int64_t c0 = (item - row * chunks) * kQuantChunk + static_cast<int64_t>(lane) * 64;
-    int my_dst = -1;                         // lane j < k holds destination j
-    int ndst = 1;
-    if (inv != nullptr) {
-        ndst = k;
-        if (lane < k)
-            my_dst = inv[row * k + lane];      // coherent load: the front kernel writes inv in the same launch
-    }
-    // lanes past the end of the row do no work but stay for the shuffles below
     const bool active = c0 < cols;
     const int64_t kb_per_block = cols / 64;
     const __nv_bfloat16 *xr = x + row * ldx;
@@ -156,12 +133,8 @@ __device__ __forceinline__ void quantize_item(const __nv_bfloat16 *__restrict__ 
             sw |= sb << (8 * b);
         }
     }
-    for (int d = 0; d < ndst; ++d) {
-        int64_t dst = row;
-        if (inv != nullptr)
-            dst = __shfl_sync(0xffffffffu, my_dst, d);
-        if (!active || dst < 0)
-            continue;
+    if (active) {
+        const int64_t dst = row;
         uint8_t *crow = codes + dst * (cols / 2) + c0 / 2;
         if (nb == 4) {
             reinterpret_cast<uint4 *>(crow)[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
@@ -188,7 +161,7 @@ __device__ __forceinline__ void quantize_item(const __nv_bfloat16 *__restrict__ 
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
                                                             int64_t cols, int64_t ldx, const float *__restrict__ gs_ptr,
                                                             uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
-                                                            int layout, const int32_t *__restrict__ inv, int k)
+                                                            int layout)
 {
     pdl_wait();
     pdl_trigger();
@@ -197,16 +170,16 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const __nv_bfloat16 
     const int64_t item = static_cast<int64_t>(blockIdx.x) * 8 + warp;
     if (item >= rows * chunks)
         return;
-    quantize_item(x, cols, ldx, __ldg(gs_ptr), codes, scales, layout, inv, k, item, lane);
+    quantize_item(x, cols, ldx, __ldg(gs_ptr), codes, scales, layout, item, lane);
 }
 
 cudaError_t launch_quantize(const __nv_bfloat16 *x, int64_t rows, int64_t cols, int64_t ldx, const float *gs,
-                            uint8_t *codes, uint8_t *scales, int layout, const int32_t *inv, int k, cudaStream_t s)
+                            uint8_t *codes, uint8_t *scales, int layout, cudaStream_t s)
 {
     const int64_t items = rows * ((cols + kQuantChunk - 1) / kQuantChunk);
     const int64_t blocks = (items + 7) / 8;
     return launch_pdl(quantize_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, x, rows, cols, ldx, gs,
-                      codes, scales, layout, inv, k);
+                      codes, scales, layout);
 }
 
 // ------------------------------------------------------------ scale layout
@@ -246,177 +219,7 @@ cudaError_t launch_swizzle(const uint8_t *in, int64_t batch, int64_t rows, int64
     return cudaGetLastError();
 }
 
-// ------------------------------------------------------------ routing
-// One block of 1024 threads.  Warp w owns the contiguous slot range
-// [w*chunk, (w+1)*chunk) of the flattened ids (slot f = t*k + j):
-//  1. per-warp histograms in shared memory;
-//  2. per expert: exclusive prefix over warps (so warp w starts after all
-//     earlier warps' slots of that expert) and the total count;
-//  3. exclusive scans over experts of the counts, of the 128-row m-tile
-//     counts and of the m-tile pair counts -> unpadded offsets, padded
-//     offsets, the m-tile table and the pair table (consecutive m-tiles of
-//     one expert; the last of an odd count pairs with -1);
-//  4. each warp walks its range in order; lanes with equal ids find each
-//     other with match_any, so a slot's rank is the number of earlier slots
-//     of its expert: position = padded_offset[e] + rank (a stable counting
-//     sort, deterministic for a given input).
-// Executed by all 1024 threads of one block; sm: 33 * E int32 of shared memory.
-__device__ __forceinline__ void route_block(const int32_t *__restrict__ ids, int R, int E, int32_t *__restrict__ counts,
-                                            int32_t *__restrict__ off, int32_t *__restrict__ poff,
-                                            int32_t *__restrict__ num_mtiles, int4 *__restrict__ mtiles,
-                                            int32_t *__restrict__ num_pairs, int2 *__restrict__ pairs,
-                                            int32_t *__restrict__ ready, int32_t *__restrict__ inv,
-                                            int32_t *__restrict__ yrow, int32_t *__restrict__ err, int32_t *sm)
-{
-    int32_t *wcnt = sm;                // [32][E]
-    int32_t *poff_s = sm + 32 * E;     // [E]
-    int32_t *off_s = sm + 33 * E;      // [E]
-    __shared__ int32_t warp_sum_c[32], warp_sum_t[32], warp_sum_p[32];
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    for (int i = tid; i < 32 * E; i += blockDim.x)
-        wcnt[i] = 0;
-    __syncthreads();
-
-    const int chunk = (R + 31) / 32;
-    const int f0 = min(R, warp * chunk), f1 = min(R, f0 + chunk);
-    int bad = 0;
-    for (int base = f0; base < f1; base += 4 * 32) {
-        const int fb = base + lane;
-        int ev[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)         // four loads in flight per lane
-            ev[u] = fb + 32 * u < f1 ? __ldg(ids + fb + 32 * u) : -1;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (ev[u] >= E)
-                bad = 1;
-            else if (ev[u] >= 0)
-                atomicAdd(&wcnt[warp * E + ev[u]], 1);
-        }
-    }
-    if (bad)
-        atomicCAS(err, 0, NVFP4_ERR_BAD_EXPERT_ID);
-    __syncthreads();
-
-    // 2 + 3: thread e owns expert e (E <= 1024)
-    int cnt = 0, tiles = 0, npair = 0;
-    if (tid < E) {
-        for (int w = 0; w < 32; ++w) {
-            const int c = wcnt[w * E + tid];
-            wcnt[w * E + tid] = cnt;
-            cnt += c;
-        }
-        tiles = (cnt + 127) / 128;
-        npair = (tiles + 1) / 2;
-    }
-    // block-wide exclusive scan of (cnt, tiles, npair) over thread index
-    int ic = cnt, it = tiles, ip = npair;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int a = __shfl_up_sync(0xffffffffu, ic, o);
-        const int b = __shfl_up_sync(0xffffffffu, it, o);
-        const int c = __shfl_up_sync(0xffffffffu, ip, o);
-        if (lane >= o) {
-            ic += a;
-            it += b;
-            ip += c;
-        }
-    }
-    if (lane == 31) {
-        warp_sum_c[warp] = ic;
-        warp_sum_t[warp] = it;
-        warp_sum_p[warp] = ip;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int c = warp_sum_c[lane], t = warp_sum_t[lane], q = warp_sum_p[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int a = __shfl_up_sync(0xffffffffu, c, o);
-            const int b = __shfl_up_sync(0xffffffffu, t, o);
-            const int d = __shfl_up_sync(0xffffffffu, q, o);
-            if (lane >= o) {
-                c += a;
-                t += b;
-                q += d;
-            }
-        }
-        warp_sum_c[lane] = c;   // inclusive over warps
-        warp_sum_t[lane] = t;
-        warp_sum_p[lane] = q;
-    }
-    __syncthreads();
-    const int base_c = (warp > 0 ? warp_sum_c[warp - 1] : 0) + ic - cnt;   // exclusive
-    const int base_t = (warp > 0 ? warp_sum_t[warp - 1] : 0) + it - tiles;
-    const int base_p = (warp > 0 ? warp_sum_p[warp - 1] : 0) + ip - npair;
-    if (tid < E) {
-        counts[tid] = cnt;
-        off[tid] = base_c;
-        poff[tid] = base_t * 128;
-        poff_s[tid] = base_t * 128;
-        off_s[tid] = base_c;
-        for (int i = 0; i < tiles; ++i) {
-            mtiles[base_t + i] = make_int4(tid, base_t * 128 + 128 * i, min(128, cnt - 128 * i), base_c + 128 * i);
-            if (ready != nullptr)
-                ready[base_t + i] = 0;
-        }
-        for (int i = 0; i < npair; ++i)
-            pairs[base_p + i] = make_int2(base_t + 2 * i, 2 * i + 1 < tiles ? base_t + 2 * i + 1 : -1);
-        if (tid == E - 1) {
-            off[E] = base_c + cnt;
-            poff[E] = (base_t + tiles) * 128;
-            *num_mtiles = base_t + tiles;
-            *num_pairs = base_p + npair;
-        }
-    }
-    __syncthreads();
-
-    // 4: stable positions
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int base0 = f0; base0 < f1; base0 += 4 * 32) {
-        int ev[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)         // load four groups, then walk them in order
-            ev[u] = base0 + 32 * u + lane < f1 ? __ldg(ids + base0 + 32 * u + lane) : -1;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int f = base0 + 32 * u + lane;
-            const bool act = f < f1;
-            const int e = ev[u];
-            const bool valid = act && e >= 0 && e < E;
-            const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1);
-            const int rank = __popc(peers & lt_mask);
-            if (valid) {
-                const int r = wcnt[warp * E + e] + rank;
-                inv[f] = poff_s[e] + r;
-                yrow[f] = off_s[e] + r;
-            } else if (act) {
-                inv[f] = -1;
-                yrow[f] = -1;
-            }
-            __syncwarp();
-            if (valid && rank == 0)
-                wcnt[warp * E + e] += __popc(peers);
-            __syncwarp();
-        }
-    }
-}
-
-__global__ void __launch_bounds__(1024) route_kernel(const int32_t *__restrict__ ids, int R, int E,
-                                                     int32_t *__restrict__ counts, int32_t *__restrict__ off,
-                                                     int32_t *__restrict__ poff, int32_t *__restrict__ num_mtiles,
-                                                     int4 *__restrict__ mtiles, int32_t *__restrict__ num_pairs,
-                                                     int2 *__restrict__ pairs, int32_t *__restrict__ ready,
-                                                     int32_t *__restrict__ inv, int32_t *__restrict__ yrow,
-                                                     int32_t *__restrict__ err)
-{
-    extern __shared__ int32_t sm[];
-    pdl_wait();
-    pdl_trigger();
-    route_block(ids, R, E, counts, off, poff, num_mtiles, mtiles, num_pairs, pairs, ready, inv, yrow, err, sm);
-}
-
+// ------------------------------------------------------------ kernel attributes
 cudaError_t ensure_smem_limit(const void *kernel, int bytes, unsigned long long *done_mask)
 {
     static std::mutex mu;
@@ -432,19 +235,6 @@ cudaError_t ensure_smem_limit(const void *kernel, int bytes, unsigned long long 
     if (e == cudaSuccess)
         *done_mask |= bit;
     return e;
-}
-
-cudaError_t launch_route(const int32_t *ids, int64_t R, int E, int32_t *counts, int32_t *off, int32_t *poff,
-                         int32_t *num_mtiles, int4 *mtiles, int32_t *num_pairs, int2 *pairs, int32_t *ready,
-                         int32_t *inv, int32_t *yrow, int32_t *err, cudaStream_t s)
-{
-    const size_t smem = sizeof(int32_t) * (34 * static_cast<size_t>(E));
-    static unsigned long long attr_done = 0;
-    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(route_kernel), 34 * 1024 * 4, &attr_done);
-    if (e != cudaSuccess)
-        return e;
-    return launch_pdl(route_kernel, dim3(1), dim3(1024), smem, s, ids, static_cast<int>(R), E, counts, off, poff,
-                      num_mtiles, mtiles, num_pairs, pairs, ready, inv, yrow, err);
 }
 
 // ------------------------------------------------------------ combine

@@ -145,10 +145,11 @@ def test_ceiling_checks(L):
 
 def test_moe_plan(L):
     from nvfp4_moe_expert_topk_b200 import nvfp4_moe_plan
-    assert nvfp4_moe_plan(64, 6, 48, 7168, 3072) == (True, False)       # decode: fused, 1-CTA tiles
-    assert nvfp4_moe_plan(4096, 6, 384, 7168, 3072) == (True, False)    # prefill
-    assert nvfp4_moe_plan(256, 1, 1, 7168, 3072) == (False, True)       # shared expert: pair tiles
-    assert nvfp4_moe_plan(64, 2, 4, 384, 256) == (False, False)         # H % 256 != 0: 128-wide L2 tiles
+    assert nvfp4_moe_plan(64, 6, 48, 7168, 3072) == (True, 0)       # decode: fused, 1-CTA tiles
+    assert nvfp4_moe_plan(4096, 6, 384, 7168, 3072) == (True, 1)    # prefill: heavy experts' pairs + fused rest
+    assert nvfp4_moe_plan(512, 6, 48, 7168, 3072) == (True, 1)      # the 48-expert prefill slice
+    assert nvfp4_moe_plan(256, 1, 1, 7168, 3072) == (False, 2)      # shared expert: every m-tile on pairs
+    assert nvfp4_moe_plan(64, 2, 4, 384, 256) == (False, 0)         # H % 256 != 0: 128-wide L2 tiles
     import ctypes
     f = ctypes.c_int32()
     assert L.nvfp4_moe_plan(64, 6, 48, 7000, 3072, ctypes.byref(f), ctypes.byref(f)) == -2

@@ -12,10 +12,11 @@ from nvfp4_moe_expert_topk_b200 import workloads as W
 
 
 class _Plan:
-    """A Workload's plan without the device (fold() reads only `fused`)."""
+    """A Workload's plan without the device (fold() reads only the plan)."""
 
-    def __init__(self, fused):
+    def __init__(self, fused, pair_mode=0):
         self.fused = fused
+        self.pair_mode = pair_mode
 
 
 STAGE_MS = {"global_scale": 0.01, "route": 0.02, "quantize_permute": 0.04,
@@ -34,6 +35,29 @@ def test_fold_two_launch_plan():
     d = bench.Workload.fold(_Plan(False), STAGE_MS)
     assert set(d) == {bench.FRONT_STAGE, "l1_gate_up_swiglu_quant", "l2_down", "combine"}
     assert d["l2_down"] == 1.0
+
+
+def test_fold_split_plan_and_its_bytes():
+    """Pair mode 1: the pair launches' slot and the fused light launch's slot;
+    their algorithmic bytes count each launch's experts once, so an expert
+    with an odd number of m-tiles is counted in both."""
+    import numpy as np
+    d = bench.Workload.fold(_Plan(True, 1), STAGE_MS)
+    assert set(d) == {bench.FRONT_STAGE, bench.PAIRS_STAGE, bench.LIGHT_STAGE, "combine"}
+    assert d[bench.PAIRS_STAGE] == 2.0 and d[bench.LIGHT_STAGE] == 1.0
+    cfg = W.MoeConfig("t", E=4, k=2, T=400, H=256, I=128, routing="softmax", outliers=False, warmup_T=8)
+    counts = np.array([300, 256, 44, 200])          # m-tiles 3, 2, 1, 2
+    pair_rows, light_rows = bench.tile_split(counts, 1)
+    assert list(pair_rows) == [256, 256, 0, 200] and list(light_rows) == [44, 0, 44, 0]
+    assert list(bench.tile_split(counts, 2)[0]) == [300, 256, 44, 200]
+    assert list(bench.tile_split(counts, 0)[1]) == [300, 256, 44, 200]
+    split = bench.stage_bytes(cfg, counts, True, 1)
+    whole = bench.stage_bytes(cfg, counts, True, 0)
+    w_expert = 3 * cfg.H * cfg.I * bench.FP4_BYTES
+    # the pairs and the light launch read expert 0's weights each; the rest once
+    assert split[bench.PAIRS_STAGE] + split[bench.LIGHT_STAGE] == pytest.approx(whole[bench.FUSED_STAGE] + w_expert)
+    assert bench.launches_per_step(True, 0) == 3 and bench.launches_per_step(True, 1) == 5
+    assert bench.launches_per_step(False, 2) == 4
 
 
 def _copy_tree(tmp_path):

@@ -110,8 +110,12 @@ def test_swizzle_kernel_matches_layout_definition():
 
 
 @pytest.mark.parametrize("E,T,k,seed", [(8, 64, 2, 0), (48, 64, 6, 1), (384, 4096, 6, 2), (5, 3, 2, 3),
-                                        (1, 256, 1, 4), (1024, 300, 8, 5)])
+                                        (1, 256, 1, 4), (1024, 300, 8, 5), (64, 20011, 8, 6), (3, 1, 3, 7),
+                                        (1024, 4099, 32, 8)])
 def test_route_bitexact(E, T, k, seed):
+    """Routing (one launch over min(T, SMs) blocks, each owning a contiguous
+    token range) against the oracle's stable counting sort: one token; T not
+    a multiple of the block count; ~1000 slots per block; 1024 experts."""
     rng = np.random.default_rng(seed)
     ids = rng.integers(0, E, (T, k)).astype(np.int32)
     if E == 384:                                  # skewed, with empty experts

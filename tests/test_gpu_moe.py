@@ -382,7 +382,7 @@ NARROW = W.MoeConfig("narrow", E=4, k=2, T=96, H=384, I=256, routing="softmax", 
 
 def test_unfused_narrow_hidden():
     from nvfp4_moe_expert_topk_b200 import nvfp4_moe_plan
-    assert nvfp4_moe_plan(NARROW.T, NARROW.k, NARROW.E, NARROW.H, NARROW.I) == (False, False)
+    assert nvfp4_moe_plan(NARROW.T, NARROW.k, NARROW.E, NARROW.H, NARROW.I) == (False, 0)
     p = Problem(NARROW)
     out, ws = p.run()
     assert nvfp4_moe_get_error(ws) == 0
@@ -467,3 +467,89 @@ def test_bounded_wait_times_out_and_context_survives(tiny):
     out, ws = tiny.run()
     assert nvfp4_moe_get_error(ws) == 0
     check_output(out, tiny.oracle())
+
+
+# 16 experts, top-4, 768 tokens, Zipf-skewed: 3072 routed rows, so the plan
+# puts the full m-tile pairs of experts with two or more m-tiles on pair
+# tiles (their own L1 and L2 launches) and the rest on the fused 1-CTA
+# launch.  m-tiles per expert: 6, 4, 3, 3, 2, 2, 2, 2, six of 1, two empty.
+SPLIT = W.MoeConfig("split", E=16, k=4, T=768, H=512, I=256, routing="zipf", outliers=True, warmup_T=128,
+                    zipf_zero_tail=2)
+
+
+def expected_tile_tables(counts, pair_mode):
+    """The tile tables the routing must write, from the plan's rule (include/
+    nvfp4moe.h, nvfp4_moe_plan): m-tiles in expert order, 128 rows each, the
+    last one partial; pairs of consecutive m-tiles; the light list."""
+    mtiles, pairs, light = [], [], []
+    row, yrow = 0, 0
+    for e, c in enumerate(counts):
+        tiles = (int(c) + 127) // 128
+        first = len(mtiles)
+        for i in range(tiles):
+            mtiles.append((e, row + 128 * i, min(128, int(c) - 128 * i), yrow + 128 * i))
+        if pair_mode == 1:
+            npair = tiles // 2 if tiles >= 2 else 0
+        elif pair_mode == 2:
+            npair = (tiles + 1) // 2
+        else:
+            npair = 0
+        for i in range(npair):
+            pairs.append((first + 2 * i, first + 2 * i + 1 if 2 * i + 1 < tiles else -1))
+        light += list(range(first + min(2 * npair, tiles), first + tiles))
+        row += 128 * tiles
+        yrow += int(c)
+    return np.array(mtiles, np.int32).reshape(-1, 4), np.array(pairs, np.int32).reshape(-1, 2), \
+        np.array(light, np.int32)
+
+
+def check_tile_tables(p, ws, pair_mode):
+    cfg = p.cfg
+    counts = np.bincount(p.ids.numpy().ravel()[p.ids.numpy().ravel() >= 0], minlength=cfg.E)
+    mt, pr, lt = expected_tile_tables(counts, pair_mode)
+    wsn = ws.cpu().numpy()
+    o, n = region(p, 12)
+    hdr = wsn[o:o + n].view(np.int32)
+    assert (hdr[1], hdr[2], hdr[6]) == (len(mt), len(pr), len(lt))
+    o, n = region(p, 9)
+    np.testing.assert_array_equal(wsn[o:o + n].view(np.int32).reshape(-1, 4)[:len(mt)], mt)
+    o, n = region(p, 10)
+    np.testing.assert_array_equal(wsn[o:o + n].view(np.int32).reshape(-1, 2)[:len(pr)], pr)
+    o, n = region(p, 11)
+    np.testing.assert_array_equal(wsn[o:o + n].view(np.int32)[:len(lt)], lt)
+
+
+def test_split_pair_and_light_tiles_end_to_end():
+    from nvfp4_moe_expert_topk_b200 import nvfp4_moe_plan
+    assert nvfp4_moe_plan(SPLIT.T, SPLIT.k, SPLIT.E, SPLIT.H, SPLIT.I) == (True, 1)
+    p = Problem(SPLIT)
+    counts = np.bincount(p.ids.numpy().ravel(), minlength=SPLIT.E)
+    mt = (counts + 127) // 128
+    assert ((mt >= 2) & (mt % 2 == 0)).any() and ((mt >= 3) & (mt % 2 == 1)).any() and (mt == 1).any()
+    out, ws = p.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    ref, inter = p.oracle(intermediates=True)
+    check_output(out, ref)
+    check_intermediates(p, ws, inter)
+    check_tile_tables(p, ws, 1)
+
+
+@pytest.mark.parametrize("name,mode", [("decode", 0), ("prefill_ep48", 1)])
+def test_tile_tables_of_full_size_routing(name, mode):
+    """The routing's tile tables on the decode batch (every m-tile light) and
+    on the 48-expert prefill slice (pairs for its heavy experts)."""
+    cfg = W.MOE_CONFIGS[name]
+    x, ids, w = W.batch(cfg)
+    p = Problem.__new__(Problem)               # routing only: no oracle weights needed
+    p.cfg, p.x, p.ids, p.w = cfg, x, ids, w
+    dw = prep.MoeWeights.synthetic(cfg, DEV)
+    ws = prep.workspace(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I, DEV)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=DEV)
+    nvfp4_moe_forward(x.to(DEV), ids.to(DEV), w.to(DEV), None, **dw.args(),
+                      inter_gs=torch.ones(cfg.E, device=DEV), out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert nvfp4_moe_get_error(ws) == 0
+    check_tile_tables(p, ws, mode)
+    route = O.route(ids.numpy(), cfg.E)
+    o, n = region(p, 5)
+    np.testing.assert_array_equal(ws[o:o + n].cpu().numpy().view(np.int32), route["pos_padded"])
