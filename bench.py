@@ -49,8 +49,7 @@ BF16_TO_FP4_NOMINAL_RATIO = 4.0        # 9 / 2.25 PFLOP/s dense
 STAGES = ["global_scale", "route", "quantize_permute", "l1_gate_up_swiglu_quant", "l2_down", "combine"]
 FRONT_STAGE = "front"                  # global scale of the batch + routing + quantise/permute
 FUSED_STAGE = "l1_l2_fused"            # L1 and L2 as one launch (nvfp4_moe_plan)
-PAIRS_STAGE = "pairs_l1_l2"            # pair mode 1: the heavy experts' pair-tile L1 and L2 launches
-LIGHT_STAGE = "l1_l2_fused_light"      # pair mode 1: the fused 1-CTA launch over the other m-tiles
+SPLIT_STAGE = "l1_l2_pairs_beside_light"   # pair mode 1: the fused pair launch and, beside it, the fused 1-CTA one
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 GEMM_SOURCES = ["gemm.cu", "ptx.cuh", "quant.cuh", "internal.h"]
 
@@ -321,7 +320,7 @@ FP4_BYTES = 0.5 + 1.0 / 16             # NVFP4 code + scale bytes per element
 
 def launches_per_step(fused, pair_mode):
     """Launches of one forward: the front, the GEMMs, the combine."""
-    gemm = {0: 1 if fused else 2, 1: 2 + (1 if fused else 2), 2: 2}[pair_mode]
+    gemm = {0: 1 if fused else 2, 1: 2, 2: 2}[pair_mode]
     return 2 + gemm
 
 
@@ -330,15 +329,15 @@ def fold_stages(per_stage, fused, pair_mode):
     what the plan runs there: the front (one launch: global scale, routing,
     quantise + permute) and then
       pair mode 0, fused   the fused 1-CTA L1 + L2 launch;
-      pair mode 1          the heavy experts' pair L1 + L2 launches, then the
-                           fused 1-CTA launch over the other m-tiles;
+      pair mode 1          the heavy experts' fused pair launch and, running
+                           beside it, the fused 1-CTA launch over the other
+                           m-tiles (one stage: they overlap);
       otherwise            L1, then L2;
     and the combine."""
     d = dict(per_stage)
     d[FRONT_STAGE] = d.pop("global_scale") + d.pop("route") + d.pop("quantize_permute")
     if pair_mode == 1:
-        d[PAIRS_STAGE] = d.pop("l1_gate_up_swiglu_quant")
-        d[LIGHT_STAGE] = d.pop("l2_down")
+        d[SPLIT_STAGE] = d.pop("l1_gate_up_swiglu_quant") + d.pop("l2_down")
     elif fused and pair_mode == 0:
         d[FUSED_STAGE] = d.pop("l1_gate_up_swiglu_quant") + d.pop("l2_down")
     return d
@@ -375,10 +374,8 @@ def stage_bytes(cfg, counts, fused, pair_mode):
 
     d = {FRONT_STAGE: T * H * 2.0 + R * H * FP4_BYTES + T * k * 4.0 * 3 + E * 16.0,
          "combine": R * H * 2.0 + T * H * 2.0 + T * k * 12.0}
-    pair_rows, light_rows = tile_split(counts, pair_mode)
     if pair_mode == 1:
-        d[PAIRS_STAGE] = sum(gemm(pair_rows))
-        d[LIGHT_STAGE] = sum(gemm(light_rows))
+        d[SPLIT_STAGE] = sum(gemm(counts))     # the two launches together read each expert once
     else:
         l1, l2 = gemm(counts)
         if fused and pair_mode == 0:

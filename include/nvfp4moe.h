@@ -177,6 +177,19 @@ size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
  * call per device first: it sets per-kernel attributes). */
 int nvfp4_moe_forward(const nvfp4_moe_args *args, void *workspace, size_t ws_bytes, void *stream);
 
+/* nvfp4_moe_forward on activations that are already NVFP4 -- for expert
+ * parallelism (page 1 "Config values": 48 of the 384 experts per rank), where
+ * a rank quantises its tokens once and sends 4-bit rows (H/2 + H/16 bytes
+ * each) to the ranks owning their experts.  x_codes [T, H/2] and x_scales
+ * [T, H/16] (NVFP4_SCALES_ROWMAJOR, as nvfp4_quantize writes them), both
+ * 16-byte aligned, quantised with the global scale args->x_gs (required);
+ * args->x is not read (may be NULL).  The front launch copies each row to its
+ * slots' padded rows instead of quantising it; everything else is
+ * nvfp4_moe_forward, so given the codes nvfp4_quantize makes from x with
+ * x_gs, the output equals nvfp4_moe_forward's on x with x_gs bit for bit. */
+int nvfp4_moe_forward_quantized(const nvfp4_moe_args *args, const uint8_t *x_codes, const uint8_t *x_scales,
+                                void *workspace, size_t ws_bytes, void *stream);
+
 /* Measurement hook, not a step of the method: nvfp4_moe_forward with CUDA
  * events recorded on `stream` at its stage boundaries: events = 6
  * cudaEvent_t handles created by the caller; event 0 before the front

@@ -16,7 +16,7 @@ __all__ = [
     "Nvfp4Error", "lib", "NVFP4_SCALES_ROWMAJOR", "NVFP4_SCALES_MMA",
     "nvfp4_status_string", "nvfp4_global_scale", "nvfp4_scales_bytes", "nvfp4_quantize",
     "nvfp4_swizzle_scales", "nvfp4_gemm", "nvfp4_moe_workspace_size", "nvfp4_moe_forward",
-    "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc",
+    "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc", "nvfp4_moe_forward_quantized",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
     "nvfp4_moe_get_error", "nvfp4_moe_topk", "nvfp4_moe_topk_shared", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax", "nvfp4_debug_bounded_wait", "nvfp4_gemm_ws",
     "nvfp4_gemm_workspace_size",
@@ -71,6 +71,7 @@ def lib():
         L.nvfp4_moe_forward_timed.argtypes = [ctypes.POINTER(MoeArgs), P, ctypes.c_size_t, P,
                                               ctypes.POINTER(ctypes.c_void_p)]
         L.nvfp4_moe_forward_noalloc.argtypes = [ctypes.POINTER(MoeArgs), P]
+        L.nvfp4_moe_forward_quantized.argtypes = [ctypes.POINTER(MoeArgs), P, P, P, ctypes.c_size_t, P]
         L.nvfp4_moe_calibrate.argtypes = [ctypes.POINTER(MoeArgs), P, P, ctypes.c_size_t, P]
         L.nvfp4_moe_route_debug.argtypes = [P, i64, i32, i32, P, P, P, P, ctypes.c_size_t, P]
         L.nvfp4_moe_workspace_region.argtypes = [i64, i32, i32, i64, i64, i32,
@@ -177,11 +178,11 @@ def nvfp4_moe_workspace_size(T, k, E, H, I):
 
 
 def _moe_args(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs, w2_codes, w2_scales, w2_gs,
-              inter_gs, out):
-    T, H = x.shape
+              inter_gs, out, x_shape=None):
+    T, H = x.shape if x is not None else x_shape
     E, twoI = w13_codes.shape[0], w13_codes.shape[1]
     a = MoeArgs()
-    a.x = _dev(x, "x", torch.bfloat16).value
+    a.x = None if x is None else _dev(x, "x", torch.bfloat16).value
     a.T, a.H, a.I, a.E, a.k = T, H, twoI // 2, E, topk_ids.shape[1]
     a.topk_ids = _dev(topk_ids, "topk_ids", torch.int32).value
     a.topk_weights = _dev(topk_weights, "topk_weights", torch.float32).value
@@ -204,6 +205,24 @@ def nvfp4_moe_forward(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w1
                   inter_gs, out)
     _check(lib().nvfp4_moe_forward(ctypes.byref(a), _dev(workspace, "workspace", torch.uint8), workspace.numel(),
                                    _stream(stream)), "nvfp4_moe_forward")
+
+
+def nvfp4_moe_forward_quantized(x_codes, x_scales, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs,
+                                w2_codes, w2_scales, w2_gs, inter_gs, out, workspace, stream=None):
+    """nvfp4_moe_forward on activations already in NVFP4: x_codes uint8
+    [T, H/2] and row-major x_scales uint8 [T, H/16] made with the global scale
+    x_gs (float32 [1], required)."""
+    if x_gs is None:
+        raise ValueError("x_gs (the global scale of the codes) is required")
+    T, H = x_codes.shape[0], x_codes.shape[1] * 2
+    if tuple(x_scales.shape) != (T, H // 16):
+        raise ValueError(f"x_scales must be [{T}, {H // 16}] (row-major), got {tuple(x_scales.shape)}")
+    a = _moe_args(None, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs, w2_codes, w2_scales, w2_gs,
+                  inter_gs, out, x_shape=(T, H))
+    _check(lib().nvfp4_moe_forward_quantized(ctypes.byref(a), _dev(x_codes, "x_codes", torch.uint8),
+                                             _dev(x_scales, "x_scales", torch.uint8),
+                                             _dev(workspace, "workspace", torch.uint8), workspace.numel(),
+                                             _stream(stream)), "nvfp4_moe_forward_quantized")
 
 
 def nvfp4_moe_forward_timed(x, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs, w2_codes,

@@ -96,8 +96,9 @@ struct Layout {
 
 // Header (256 B): int32 error word at 0, int32 m-tile count at 4, int32
 // m-tile pair count at 8, fp32 global scale of x computed from the batch at
-// 12, the front launch's grid ticket at 20, int32 light m-tile count at 24.
-constexpr int kHdrNumMtiles = 4, kHdrNumPairs = 8, kHdrGs = 12, kHdrTicket = 20, kHdrNumLight = 24;
+// 12, the front launch's grid ticket at 20, int32 light m-tile count at 24,
+// the fused 1-CTA launch's tile claim counter at 28.
+constexpr int kHdrNumMtiles = 4, kHdrNumPairs = 8, kHdrGs = 12, kHdrTicket = 20, kHdrNumLight = 24, kHdrClaim = 28;
 
 Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
 {
@@ -145,21 +146,23 @@ int check_moe_shape(int64_t T, int k, int E, int64_t H, int64_t I)
     return NVFP4_OK;
 }
 
-int check_moe_args(const nvfp4_moe_args *a, bool need_out)
+// need_x false: the activations come pre-quantised (x is not read, x_gs is
+// required instead).
+int check_moe_args(const nvfp4_moe_args *a, bool need_out, bool need_x = true)
 {
     if (a == nullptr)
         return NVFP4_ERR_INVALID_ARG;
     int st = check_moe_shape(a->T, a->k, a->E, a->H, a->I);
     if (st != NVFP4_OK)
         return st;
-    const void *ptrs[] = {a->x, a->topk_ids, a->topk_weights, a->w13_codes, a->w13_scales,
+    const void *ptrs[] = {need_x ? static_cast<const void *>(a->x) : static_cast<const void *>(a->x_gs), a->topk_ids, a->topk_weights, a->w13_codes, a->w13_scales,
                           a->w13_gs, a->w2_codes, a->w2_scales, a->w2_gs};
     for (const void *p : ptrs)
         if (p == nullptr)
             return NVFP4_ERR_INVALID_ARG;
     if (need_out && (a->out == nullptr || a->inter_gs == nullptr))
         return NVFP4_ERR_INVALID_ARG;
-    const void *al[] = {a->x, a->w13_codes, a->w13_scales, a->w2_codes, a->w2_scales};
+    const void *al[] = {need_x ? static_cast<const void *>(a->x) : static_cast<const void *>(a->w13_codes), a->w13_codes, a->w13_scales, a->w2_codes, a->w2_scales};
     for (const void *p : al)
         if (!aligned16(p))
             return NVFP4_ERR_MISALIGNED;
@@ -197,8 +200,14 @@ int moe_cg(int64_t R, int E)
 
 // Batches of at least this many routed rows put the pairs of full m-tiles of
 // experts with two or more m-tiles on pair tiles (pair mode 1): the pair
-// launches cost a few microseconds even when no expert is that heavy.
+// launch costs a few microseconds even when no expert is that heavy.
 constexpr int64_t kSplitMinRows = 2048;
+// Pair mode 1 runs the pair launch on this many clusters of two SMs beside
+// the 1-CTA launch, which starts on the other SMs and takes over the pair
+// launch's SMs when it ends.  The 1-CTA tiles stream the light experts'
+// weights from HBM; the pair tiles re-read the heavy experts' weights from
+// L2, so the two overlap instead of running one after the other.
+constexpr int kSplitPairClusters = 24;
 
 int gemm_grid(int cg, int64_t tiles, int num_sms)
 {
@@ -241,6 +250,7 @@ int l1_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, CUtensorMap 
     g->num_light_dev = reinterpret_cast<int32_t *>(ws + kHdrNumLight);
     g->light = reinterpret_cast<int32_t *>(ws + L.light);
     g->ready = reinterpret_cast<int32_t *>(ws + L.ready);
+    g->claim = reinterpret_cast<int32_t *>(ws + kHdrClaim);
     g->n_tiles = static_cast<int>(I / 128);
     g->b_rows_per_expert = 2 * I;
     g->b_tile_rows = 128;
@@ -333,6 +343,7 @@ FrontArgs front_args(const nvfp4_moe_args *a, const int32_t *ids, int64_t T, int
     f.num_light = reinterpret_cast<int32_t *>(ws + kHdrNumLight);
     f.light = reinterpret_cast<int32_t *>(ws + L.light);
     f.ready = reinterpret_cast<int32_t *>(ws + L.ready);
+    f.claim = reinterpret_cast<int32_t *>(ws + kHdrClaim);
     f.inv = reinterpret_cast<int32_t *>(ws + L.inv);
     f.yrow = reinterpret_cast<int32_t *>(ws + L.yrow);
     f.err = reinterpret_cast<int32_t *>(ws);
@@ -345,11 +356,17 @@ FrontArgs front_args(const nvfp4_moe_args *a, const int32_t *ids, int64_t T, int
 }
 
 int run_front(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, int pair_mode, void *const *events,
-              cudaStream_t s, int num_sms)
+              cudaStream_t s, int num_sms, const uint8_t *xq_codes = nullptr, const uint8_t *xq_scales = nullptr)
 {
     if (mark(events, 0, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
-    if (launch_front(front_args(a, a->topk_ids, a->T, a->k, a->E, ws, L, pair_mode), num_sms, s) != cudaSuccess ||
+    FrontArgs f = front_args(a, a->topk_ids, a->T, a->k, a->E, ws, L, pair_mode);
+    if (xq_codes != nullptr) {
+        f.x = nullptr;
+        f.xq_codes = xq_codes;
+        f.xq_scales = xq_scales;
+    }
+    if (launch_front(f, num_sms, s) != cudaSuccess ||
         mark(events, 1, s) != NVFP4_OK || mark(events, 2, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
     return NVFP4_OK;
@@ -677,11 +694,13 @@ int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, in
 }
 
 static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_bytes, void *stream,
-                            void *const *events)
+                            void *const *events, const uint8_t *xq_codes = nullptr, const uint8_t *xq_scales = nullptr)
 {
-    int st = check_moe_args(a, true);
+    int st = check_moe_args(a, true, xq_codes == nullptr);
     if (st != NVFP4_OK)
         return st;
+    if (xq_codes != nullptr && (!aligned16(xq_codes) || !aligned16(xq_scales)))
+        return NVFP4_ERR_MISALIGNED;
     if (workspace == nullptr)
         return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(workspace))
@@ -698,7 +717,7 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     const Plan pl = moe_plan(a->T, a->k, a->E, a->H);
-    st = run_front(a, ws, L, pl.pair_mode, events, s, sms);
+    st = run_front(a, ws, L, pl.pair_mode, events, s, sms, xq_codes, xq_scales);
     if (st != NVFP4_OK)
         return st;
     const int64_t H = a->H;
@@ -709,35 +728,43 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
         st = l2_setup(a, ws, L, pl.l2_bn, &ma2, &ma2_32, &mb2, &g2);
     if (st != NVFP4_OK)
         return st;
-    // the pair tiles (heavy experts' m-tile pairs, or every m-tile): L1
-    // launch, then L2 launch; each reads its tile count from the workspace
-    const int pair_grid = gemm_grid(2, 1LL << 30, sms);
-    if (pl.pair_mode != 0) {
-        if (launch_gemm(256, EPI_SWIGLU_QUANT, 2, ma1, ma1_32, mb1, g1, pair_grid, s) != cudaSuccess)
+    if (pl.pair_mode == 1) {
+        // the heavy experts' pairs (fused L1 -> L2, kSplitPairClusters
+        // clusters), and beside it the fused 1-CTA launch over the light list:
+        // the pair launch lets its dependent start at once; the 1-CTA launch
+        // reads only what the front wrote and waits for the pair launch at its
+        // end, so that the combine after it sees both
+        GemmArgs p1 = g1;
+        p1.pdl_trigger_early = 1;
+        const int pairs = std::min(kSplitPairClusters, gemm_pair_clusters(sms));
+        GemmArgs l1 = g1;
+        l1.pdl_wait_at_end = 1;
+        if (launch_moe_fused(2, ma1, ma1_32, mb1, p1, ma2, ma2_32, mb2, g2, 2 * pairs, s) != cudaSuccess ||
+            launch_moe_fused(1, ma1, ma1_32, mb1, l1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
+            mark(events, 3, s) != NVFP4_OK || mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
-        if (pl.pair_mode == 2 && mark(events, 3, s) != NVFP4_OK)
+    } else if (pl.pair_mode == 2) {
+        // every m-tile on pair tiles: L1 launch, then L2 launch
+        const int pair_grid = gemm_grid(2, 1LL << 30, sms);
+        if (launch_gemm(256, EPI_SWIGLU_QUANT, 2, ma1, ma1_32, mb1, g1, pair_grid, s) != cudaSuccess ||
+            mark(events, 3, s) != NVFP4_OK ||
+            launch_gemm(256, EPI_BF16, 2, ma2, ma2_32, mb2, g2, pair_grid, s) != cudaSuccess ||
+            mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
-        if (launch_gemm(256, EPI_BF16, 2, ma2, ma2_32, mb2, g2, pair_grid, s) != cudaSuccess)
+    } else if (pl.fused) {
+        // every m-tile on 1-CTA tiles, L1 and L2 in one launch
+        if (launch_moe_fused(1, ma1, ma1_32, mb1, g1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
+            mark(events, 3, s) != NVFP4_OK || mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
-        if (mark(events, pl.pair_mode == 2 ? 4 : 3, s) != NVFP4_OK)
+    } else {
+        // 128-wide L2 tiles: L1 launch, then L2 launch, 1-CTA tiles
+        if (launch_gemm(256, EPI_SWIGLU_QUANT, 1, ma1, ma1_32, mb1, g1, gemm_grid(1, 1LL << 30, sms), s) !=
+                cudaSuccess ||
+            mark(events, 3, s) != NVFP4_OK ||
+            launch_gemm(pl.l2_bn, EPI_BF16, 1, ma2, ma2_32, mb2, g2, gemm_grid(1, 1LL << 30, sms), s) !=
+                cudaSuccess ||
+            mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
-    }
-    // the 1-CTA tiles (the light list): L1 and L2 in one persistent launch,
-    // or two launches when the L2 tiles are 128 wide
-    if (pl.pair_mode != 2) {
-        if (pl.fused) {
-            if (launch_moe_fused(ma1, ma1_32, mb1, g1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
-                (pl.pair_mode == 0 && mark(events, 3, s) != NVFP4_OK) || mark(events, 4, s) != NVFP4_OK)
-                return NVFP4_ERR_CUDA;
-        } else {
-            if (launch_gemm(256, EPI_SWIGLU_QUANT, 1, ma1, ma1_32, mb1, g1, gemm_grid(1, 1LL << 30, sms), s) !=
-                    cudaSuccess ||
-                mark(events, 3, s) != NVFP4_OK ||
-                launch_gemm(pl.l2_bn, EPI_BF16, 1, ma2, ma2_32, mb2, g2, gemm_grid(1, 1LL << 30, sms), s) !=
-                    cudaSuccess ||
-                mark(events, 4, s) != NVFP4_OK)
-                return NVFP4_ERR_CUDA;
-        }
     }
 
     if (launch_combine(reinterpret_cast<const __nv_bfloat16 *>(ws + L.y),
@@ -773,6 +800,14 @@ int nvfp4_moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int32_t *fused
 int nvfp4_moe_forward(const nvfp4_moe_args *a, void *workspace, size_t ws_bytes, void *stream)
 {
     return moe_forward_impl(a, workspace, ws_bytes, stream, nullptr);
+}
+
+int nvfp4_moe_forward_quantized(const nvfp4_moe_args *a, const uint8_t *x_codes, const uint8_t *x_scales,
+                                void *workspace, size_t ws_bytes, void *stream)
+{
+    if (x_codes == nullptr || x_scales == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    return moe_forward_impl(a, workspace, ws_bytes, stream, nullptr, x_codes, x_scales);
 }
 
 int nvfp4_moe_forward_timed(const nvfp4_moe_args *a, void *workspace, size_t ws_bytes, void *stream,

@@ -329,6 +329,8 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
                     a.light[ex[3] + i] = ex[1] + (tiles - nlight) + i;
             }
             if (tid == 0) {
+                if (a.claim != nullptr)
+                    *a.claim = 0;
                 a.off[E] = total[0];
                 a.poff[E] = total[1] * 128;
                 *a.num_mtiles = total[1];
@@ -369,7 +371,8 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
             }
         }
     }
-    if (a.x == nullptr)
+    const bool pre_quantised = a.xq_codes != nullptr;
+    if (a.x == nullptr && !pre_quantised)
         return;
     __syncthreads();                            // this block's inv is written
 
@@ -390,28 +393,40 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
         int my_dst = -1;                          // lane j < k: destination row of slot j
         if (lane < k)
             my_dst = __ldcg(a.inv + static_cast<int64_t>(t) * k + lane);
-        uint4 ld[4];
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.x + static_cast<int64_t>(t) * H + col0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            ld[i] = active ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
-        uint32_t cw[4];
+        uint32_t cw[4] = {0u, 0u, 0u, 0u};
         uint32_t s2 = 0;
-#pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-            const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&ld[2 * blk]);
-            const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&ld[2 * blk + 1]);
-            float f[16];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 p = __bfloat1622float2(h0[j]);
-                const float2 q = __bfloat1622float2(h1[j]);
-                f[2 * j] = p.x;
-                f[2 * j + 1] = p.y;
-                f[8 + 2 * j] = q.x;
-                f[8 + 2 * j + 1] = q.y;
+        if (pre_quantised) {
+            // NVFP4 rows quantised elsewhere (e.g. before an expert-parallel
+            // dispatch): this lane's 16 bytes of codes and two scales
+            if (active) {
+                const uint4 c4 = __ldg(reinterpret_cast<const uint4 *>(a.xq_codes + static_cast<int64_t>(t) * (H / 2) +
+                                                                       col0 / 2));
+                cw[0] = c4.x, cw[1] = c4.y, cw[2] = c4.z, cw[3] = c4.w;
+                s2 = __ldg(reinterpret_cast<const unsigned short *>(a.xq_scales + static_cast<int64_t>(t) * (H / 16) +
+                                                                   col0 / 16));
             }
-            s2 |= quantize16(f, gs, cw[2 * blk], cw[2 * blk + 1]) << (8 * blk);
+        } else if (active) {
+            uint4 ld[4];
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.x + static_cast<int64_t>(t) * H + col0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                ld[i] = __ldg(src + i);
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk) {
+                const __nv_bfloat162 *h0 = reinterpret_cast<const __nv_bfloat162 *>(&ld[2 * blk]);
+                const __nv_bfloat162 *h1 = reinterpret_cast<const __nv_bfloat162 *>(&ld[2 * blk + 1]);
+                float f[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 p = __bfloat1622float2(h0[j]);
+                    const float2 q = __bfloat1622float2(h1[j]);
+                    f[2 * j] = p.x;
+                    f[2 * j + 1] = p.y;
+                    f[8 + 2 * j] = q.x;
+                    f[8 + 2 * j + 1] = q.y;
+                }
+                s2 |= quantize16(f, gs, cw[2 * blk], cw[2 * blk + 1]) << (8 * blk);
+            }
         }
         const uint32_t s_hi = __shfl_xor_sync(0xffffffffu, s2, 1);
         const uint32_t sword = s2 | (s_hi << 16);          // valid on even lanes

@@ -68,6 +68,7 @@ constexpr int kThreads = 448;
 constexpr int kEpiWarps = 8;                    // warps 2-9
 constexpr int kFirstSFWarp = 2 + kEpiWarps;     // warps 10-13
 constexpr uint32_t kTmemCols = 512;
+constexpr int kTileQ = 8;                       // dynamically claimed launch: queue of claimed tile indices
 
 // CG = 1: one CTA computes a 128 x BN tile.  CG = 2: a cluster of two CTAs
 // computes a 256 x 256 tile with pair MMAs; each CTA loads its own 128 A
@@ -87,9 +88,9 @@ struct Cfg {
     static constexpr int kSFA = kB + kStages * kTileBytes * kBBoxes;
     static constexpr int kSFB = kSFA + kStages * kSFStage;
     static constexpr int kBars = kSFB + kStages * kSFStage * kHalves;
-    static constexpr int kBarCount = 3 * kStages + 2 * kNumAcc + 1;
+    static constexpr int kBarCount = 3 * kStages + 2 * kNumAcc + 1 + 2 * kTileQ;
     static constexpr int kMisc = kBars + kBarCount * 8;
-    static constexpr int kSmem = kMisc + 16 + 1024;          // + tmem slot, abort flag, alignment slack
+    static constexpr int kSmem = kMisc + 16 + 4 * kTileQ + 1024;   // + tmem slot, abort flag, tile queue, slack
     static_assert(kTmemSF + kStages * kSFSlotCols <= kTmemCols, "TMEM budget");
     static_assert(kSmem <= 232448, "shared memory budget");
     static_assert(CG == 1 || BN == 256, "pair tiles are 256 wide");
@@ -114,19 +115,30 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, const GemmArg
     ti.ph = 0;
     ti.mt = 0;
     if constexpr (FUSED) {
+        // every L1 tile (m-unit-major), then every L2 tile; an m-unit is a
+        // light m-tile (CG = 1) or a pair of m-tiles (CG = 2); the tables are
+        // read from L2 (they were written by the front launch of this step)
         const int t1 = m_units * p.n_tiles;
         ti.ph = t >= t1 ? 1 : 0;
         const int n = ti.ph ? p2.n_tiles : p.n_tiles;
         const int tt = ti.ph ? t - t1 : t;
-        const int li = tt / n;
-        ti.nt = tt - li * n;
-        const int mt = p.light[li];
+        const int u = tt / n;
+        ti.nt = tt - u * n;
+        int mt, mt_any;
+        if constexpr (CG == 2) {
+            const int2 pr = __ldcg(p.pairs + u);
+            mt = rank == 0 ? pr.x : pr.y;
+            mt_any = mt >= 0 ? mt : pr.x;
+        } else {
+            mt = __ldcg(p.light + u);
+            mt_any = mt;
+        }
+        const int4 m = __ldcg(p.mtiles + mt_any);
         ti.mt = mt;
-        const int4 m = p.mtiles[mt];
         ti.e = m.x;
-        ti.row0 = m.y;
-        ti.valid = m.z;
-        ti.row0_out = m.w;
+        ti.row0 = mt >= 0 ? m.y : m.y + kBM;
+        ti.valid = mt >= 0 ? m.z : 0;
+        ti.row0_out = mt >= 0 ? m.w : m.w + kBM;
         return ti;
     }
     if constexpr (CG == 2) {
@@ -211,6 +223,29 @@ __device__ __forceinline__ bool wait_counter(const int32_t *ctr, int target, vol
     return false;
 }
 
+// Consumer side of the dynamically claimed launch's tile queue: the next
+// tile the producer claimed, read in claim order from shared memory.
+// Returns 1 with the tile in t, 0 at the end of the tiles, -1 when the wait
+// gave up.  warp_wide: every lane of the warp calls it and lane 0 releases
+// the slot after all lanes have read it; otherwise the calling thread does.
+__device__ __forceinline__ int dyn_next(uint64_t *q_full, uint64_t *q_empty, const int *tile_q, int &qi, int &t,
+                                        bool warp_wide, volatile int *abort)
+{
+    const int slot = qi % kTileQ;
+    bool got = mbar_wait(&q_full[slot], static_cast<uint32_t>(qi / kTileQ) & 1u, abort);
+    if (warp_wide)
+        got = __all_sync(0xffffffffu, got);
+    if (!got)
+        return -1;
+    t = *reinterpret_cast<const volatile int *>(tile_q + slot);
+    if (warp_wide)
+        __syncwarp();
+    if (!warp_wide || (threadIdx.x & 31) == 0)
+        mbar_arrive(&q_empty[slot]);
+    ++qi;
+    return t >= 0 ? 1 : 0;
+}
+
 // Work cursor of a CTA (or pair) over its tiles.  SK = 0: whole tiles
 // t = unit, unit + units, ...  SK = 1 (stream-K, dense GEMMs): the
 // linearised (tile, k-tile) iterations are split evenly over the units, and
@@ -293,7 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const GemmArgs p, const GemmArgs p2)
 {
     using C = Cfg<BN, CG>;
-    static_assert(!FUSED || (CG == 1 && BN == 256 && EPI == EPI_SWIGLU_QUANT), "fused launch: L1 quant + L2 bf16");
+    static_assert(!FUSED || (BN == 256 && EPI == EPI_SWIGLU_QUANT), "fused launch: L1 quant + L2 bf16");
+    // the fused 1-CTA launch claims its tiles one at a time (no residency
+    // requirement); everything else deals tiles round-robin
+    constexpr bool kDyn = FUSED && CG == 1;
     static_assert(!SK || (!FUSED && EPI == EPI_BF16 && BN == 256), "stream-K: dense bf16 GEMMs");
     constexpr int kStages = C::kStages;
     constexpr int kHalves = C::kHalves;
@@ -312,8 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *acc_full = sf_ready + kStages;
     uint64_t *acc_empty = acc_full + kNumAcc;
     uint64_t *drain = acc_empty + kNumAcc;
+    uint64_t *q_full = drain + 1;                // tile queue (kDyn): a claimed index is in the slot
+    uint64_t *q_empty = q_full + kTileQ;         //                    every role has read the slot
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kMisc + 4);
+    int *tile_q = reinterpret_cast<int *>(smem + C::kMisc + 16);
     __shared__ int never_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -333,6 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&acc_empty[b], kEpiWarps * CG);
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < kTileQ; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1 + 4 + kEpiWarps);   // MMA thread, stager warps, epilogue warps
+        }
         *abort_flag = 0;
         never_abort = 0;
         fence_mbar_init();
@@ -364,11 +409,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sf_ready_lead = kPair ? map_shared_to_cta(smem_u32(sf_ready), 0) : 0u;
     const uint32_t acc_empty_lead = kPair ? map_shared_to_cta(smem_u32(acc_empty), 0) : 0u;
     // everything above overlaps the previous kernel's tail (dependent launch);
-    // from here on the tile table, the operands and the outputs are touched
-    pdl_wait();
+    // from here on the tile table, the operands and the outputs are touched.
+    // A launch that runs beside its predecessor (pdl_wait_at_end: it reads
+    // nothing that kernel writes; its own inputs were complete before that
+    // kernel let it start) waits for the predecessor only at its end, so that
+    // the next kernel sees both; a launch that lets its successor run beside
+    // it triggers at once.
+    if (!p.pdl_wait_at_end)
+        pdl_wait();
+    if (p.pdl_trigger_early)
+        pdl_trigger();
 
     const int m_units = (p.mtiles != nullptr)
-                            ? *reinterpret_cast<volatile const int32_t *>(kPair ? p.num_pairs_dev : p.num_light_dev)
+                            ? __ldcg(kPair ? p.num_pairs_dev : p.num_light_dev)
                             : (kPair ? (p.dense_M + 2 * kBM - 1) / (2 * kBM) : p.dense_m_tiles);
     const int total = m_units * (p.n_tiles + (FUSED ? p2.n_tiles : 0));
 
@@ -379,14 +432,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, pend_mask = 0, pend_par = 0;
             bool ok = true;
             Cursor cur = cursor_init<SK>(unit, units, total, p.num_k_tiles);
-            int t, kb0, kb1;
-            while (ok && cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+            int t = 0, kb0 = 0, kb1 = -1, pq = 0;
+            while (ok) {
+                if constexpr (kDyn) {
+                    // claim the next tile just before loading it, and queue its index for the other roles
+                    const int slot = pq % kTileQ;
+                    if (pq >= kTileQ &&
+                        !mbar_wait(&q_empty[slot], static_cast<uint32_t>(pq / kTileQ - 1) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    int tc = atomicAdd(p.claim, 1);
+                    if (tc >= total)
+                        tc = -1;
+                    tile_q[slot] = tc;
+                    mbar_arrive(&q_full[slot]);
+                    ++pq;
+                    if (tc < 0)
+                        break;
+                    t = tc;
+                } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+                    break;
+                }
                 const TileInfo ti = decode_tile<CG, FUSED>(p, p2, t, m_units, rank);
                 const GemmArgs &q = (FUSED && ti.ph) ? p2 : p;
                 const CUtensorMap *ma = (FUSED && ti.ph) ? &map_a2 : &map_a;
                 const CUtensorMap *ma32 = (FUSED && ti.ph) ? &map_a2_32 : &map_a32;
                 const CUtensorMap *mb = (FUSED && ti.ph) ? &map_b2 : &map_b;
-                if (FUSED && ti.ph && !wait_counter(p2.ready + ti.mt, p.n_tiles * kEpiWarps, abort_flag)) {
+                if (FUSED && ti.ph && ti.valid > 0 &&
+                    !wait_counter(p2.ready + ti.mt, p.n_tiles * kEpiWarps, abort_flag)) {
                     ok = false;     // this m-tile's h never got published
                     break;
                 }
@@ -460,8 +534,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             Cursor cur = cursor_init<SK>(unit, units, total, p.num_k_tiles);
-            int t, kb0, kb1;
-            while (ok && cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+            int t = 0, kb0 = 0, kb1 = -1, qi = 0;
+            while (ok) {
+                if constexpr (kDyn) {
+                    const int r = dyn_next(q_full, q_empty, tile_q, qi, t, false, abort_flag);
+                    if (r < 0)
+                        ok = false;
+                    if (r <= 0)
+                        break;
+                } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+                    break;
+                }
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
                     ok = false;
                     break;
@@ -533,8 +616,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t phase = 0;
         bool ok = true;
         Cursor cur = cursor_init<SK>(unit, units, total, p.num_k_tiles);
-        int t, kb0, kb1;
-        while (ok && cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+        int t = 0, kb0 = 0, kb1 = -1, qi = 0;
+        while (ok) {
+            if constexpr (kDyn) {
+                const int r = dyn_next(q_full, q_empty, tile_q, qi, t, true, abort_flag);
+                if (r < 0)
+                    ok = false;
+                if (r <= 0)
+                    break;
+            } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+                break;
+            }
             // an empty pair half has no A scales: its rows get scale 0
             const bool a_rows = !kPair || decode_tile<CG, FUSED>(p, p2, t, m_units, rank).valid > 0;
             const GemmArgs &q = (FUSED && t >= m_units * p.n_tiles) ? p2 : p;
@@ -598,8 +690,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         Cursor cur = cursor_init<SK>(unit, units, total, p.num_k_tiles);
-        int t, kb0, kb1;
-        while (cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+        int t = 0, kb0 = 0, kb1 = -1, qi = 0;
+        while (true) {
+            if constexpr (kDyn) {
+                const int r = dyn_next(q_full, q_empty, tile_q, qi, t, true, abort_flag);
+                if (r < 0) {
+                    if (lane == 0) {
+                        *abort_flag = 1;
+                        record_error(p.err, NVFP4_ERR_TIMEOUT);
+                    }
+                }
+                if (r <= 0)
+                    break;
+            } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+                break;
+            }
             const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, got)) {
                 *abort_flag = 1;
@@ -616,9 +721,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (swiglu_tile && BN == 256) {
                 // drain gate columns [64hf, 64hf+64) and the matching up columns in two rounds of
                 // 32 (one wait each), computing h as it arrives, then release the accumulator
-                const float a = ga.a_gs[0];
-                const float alpha_g = __fdiv_rn(1.0f, __fmul_rn(a, ga.b_gs[ti.e * ga.b_gs_stride + 0]));
-                const float alpha_u = __fdiv_rn(1.0f, __fmul_rn(a, ga.b_gs[ti.e * ga.b_gs_stride + 1]));
+                const float a = __ldcg(ga.a_gs);
+                const float alpha_g = __fdiv_rn(1.0f, __fmul_rn(a, __ldcg(ga.b_gs + ti.e * ga.b_gs_stride + 0)));
+                const float alpha_u = __fdiv_rn(1.0f, __fmul_rn(a, __ldcg(ga.b_gs + ti.e * ga.b_gs_stride + 1)));
                 float h[64];
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -655,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0)
                         atomicMax(ga.amax_bits + ti.e, __float_as_uint(amax));
                 } else {
-                    const float hgs = ga.inter_gs[ti.e];
+                    const float hgs = __ldcg(ga.inter_gs + ti.e);
                     uint32_t codes[8];
                     uint32_t sfw = 0;
 #pragma unroll
@@ -677,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                       static_cast<int64_t>(2 * ti.nt + hf) * kSFAtom + lane * 16 +
                                                       q * 4) = sfw;
                     }
-                    if constexpr (FUSED) {
+                    if (FUSED && ti.valid > 0) {
                         // publish this warp's h rows to the L2 tiles of this m-tile
                         __threadfence();
                         __syncwarp();
@@ -809,7 +914,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!sk_segment) {
                 // drain columns [hf*BN/2, (hf+1)*BN/2) in rounds of 64 (one wait each),
                 // converting to bf16 as they arrive, then release the accumulator
-                const float a = ga.a_gs[ga.a_gs_per_expert ? ti.e : 0];
+                const float a = __ldcg(ga.a_gs + (ga.a_gs_per_expert ? ti.e : 0));
                 uint32_t o[kCols / 2];
 #pragma unroll
                 for (int r = 0; r < kCols / kRound; ++r) {
@@ -827,7 +932,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 3; ++i)
                             if (i < ga.nseg - 1 && col >= ga.seg_end[i])
                                 seg = i + 1;
-                        const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, ga.b_gs[ti.e * ga.b_gs_stride + seg]));
+                        const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, __ldcg(ga.b_gs + ti.e * ga.b_gs_stride + seg)));
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             o[(r * kRound + c * 16) / 2 + i] = pack_bf16x2(__uint_as_float(v[16 * c + 2 * i]) * alpha,
@@ -858,6 +963,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    if (p.pdl_wait_at_end)
+        pdl_wait();                 // the kernel this one ran beside has finished: the next sees both
     pdl_trigger();                  // the next kernel may start launching during the teardown
     tc_fence_before();
     __syncthreads();
@@ -892,17 +999,14 @@ static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a
     cudaLaunchAttribute attr[2];
     cfg.attrs = attr;
     cfg.numAttrs = 0;
-    if constexpr (FUSED) {
-        // every CTA resident at once: L2 tiles wait for other CTAs' L1 tiles
-        attr[cfg.numAttrs].id = cudaLaunchAttributeCooperative;
-        attr[cfg.numAttrs].val.cooperative = 1;
-        ++cfg.numAttrs;
-    } else {
-        // the prologue (barriers, TMEM, tensor-map prefetch) overlaps the previous kernel
-        attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
-        ++cfg.numAttrs;
-    }
+    // the prologue (barriers, TMEM, tensor-map prefetch) overlaps the previous
+    // kernel; a fused launch needs no cooperative launch: the 1-CTA one claims
+    // its tiles (a wait only ever depends on tiles claimed before, by running
+    // CTAs), and the pair one starts right after the front has finished, on an
+    // empty GPU, with no more clusters than fit at once
+    attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+    ++cfg.numAttrs;
     if constexpr (CG == 2) {
         attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
         attr[cfg.numAttrs].val.clusterDim.x = 2;
@@ -954,11 +1058,18 @@ cudaError_t launch_gemm_streamk(int cg, const CUtensorMap &map_a, const CUtensor
     return launch_one<256, EPI_BF16, 1, 0, 1>(map_a, map_a32, map_b, args, map_a, map_a32, map_b, args, grid, stream);
 }
 
-cudaError_t launch_moe_fused(const CUtensorMap &map_a1, const CUtensorMap &map_a1_32, const CUtensorMap &map_b1,
-                             const GemmArgs &args1, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
-                             const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream)
+cudaError_t launch_moe_fused(int cg, const CUtensorMap &map_a1, const CUtensorMap &map_a1_32,
+                             const CUtensorMap &map_b1, const GemmArgs &args1, const CUtensorMap &map_a2,
+                             const CUtensorMap &map_a2_32, const CUtensorMap &map_b2, const GemmArgs &args2, int grid,
+                             cudaStream_t stream)
 {
     if (args1.mtiles == nullptr || args1.ready == nullptr || args2.ready != args1.ready)
+        return cudaErrorInvalidValue;
+    if (cg == 2)
+        return grid % 2 != 0 ? cudaErrorInvalidValue
+                             : launch_one<256, EPI_SWIGLU_QUANT, 2, 1>(map_a1, map_a1_32, map_b1, args1, map_a2,
+                                                                        map_a2_32, map_b2, args2, grid, stream);
+    if (args1.claim == nullptr)
         return cudaErrorInvalidValue;
     return launch_one<256, EPI_SWIGLU_QUANT, 1, 1>(map_a1, map_a1_32, map_b1, args1, map_a2, map_a2_32, map_b2, args2,
                                                     grid, stream);

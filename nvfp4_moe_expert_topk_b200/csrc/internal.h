@@ -82,6 +82,14 @@ struct GemmArgs {
     __nv_bfloat16 *out;
     int64_t ldo;
     int32_t *err;             // device error word
+    // fused grouped launches: the 1-CTA launch claims its tiles one at a time
+    // from this counter (zeroed by the front launch); in pair mode 1 the pair
+    // launch lets its dependent start at once (pdl_trigger_early) and the
+    // 1-CTA launch, which runs beside it, waits for it only at its end
+    // (pdl_wait_at_end)
+    int32_t *claim;
+    int pdl_trigger_early;
+    int pdl_wait_at_end;
 };
 
 enum Epilogue { EPI_SWIGLU_QUANT = 0, EPI_BF16 = 1, EPI_SWIGLU_AMAX = 2 };
@@ -103,13 +111,18 @@ cudaError_t launch_gemm_streamk(int cg, const CUtensorMap &map_a, const CUtensor
 cudaError_t launch_wait_probe(const int32_t *flag, int target, int32_t *err, cudaStream_t s);
 // Pair clusters that fit on the device at once (<= num_sms / 2).
 int gemm_pair_clusters(int num_sms);
-// One persistent cooperative launch of the grouped L1 (args1, maps *1, SwiGLU
-// + re-quantisation epilogue) and L2 (args2, maps *2, bf16 epilogue) tiles
-// over the same m-tile table; L2 tiles of an m-tile start once its L1 tiles
-// are published in args1.ready / args2.ready (zeroed by the routing kernel).
-cudaError_t launch_moe_fused(const CUtensorMap &map_a1, const CUtensorMap &map_a1_32, const CUtensorMap &map_b1,
-                             const GemmArgs &args1, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
-                             const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream);
+// One persistent launch of the grouped L1 (args1, maps *1, SwiGLU +
+// re-quantisation epilogue) and L2 (args2, maps *2, bf16 epilogue) tiles:
+// every L1 tile, then every L2 tile; an L2 tile starts once its m-tile's L1
+// tiles are published in args1.ready / args2.ready (zeroed by the front).
+// cg = 1: the light list on 1-CTA tiles, tiles claimed one at a time from
+// args1.claim (no residency requirement: a tile waits only on tiles claimed
+// before it, whose CTAs are running); cg = 2: the pair list on pair tiles,
+// tiles dealt round-robin to the clusters (grid / 2 of them, all resident).
+cudaError_t launch_moe_fused(int cg, const CUtensorMap &map_a1, const CUtensorMap &map_a1_32,
+                             const CUtensorMap &map_b1, const GemmArgs &args1, const CUtensorMap &map_a2,
+                             const CUtensorMap &map_a2_32, const CUtensorMap &map_b2, const GemmArgs &args2, int grid,
+                             cudaStream_t stream);
 
 // The forward's front in one launch (front.cu): the batch's global scale of
 // x (x_gs == nullptr), routing and the tile tables, quantise + permute (x ==
@@ -134,9 +147,13 @@ struct FrontArgs {
     int32_t *num_light;
     int32_t *light;
     int32_t *ready;           // may be null
+    int32_t *claim;           // tile claim counter of the fused 1-CTA launch (zeroed here)
     int32_t *inv, *yrow;
     int32_t *err;
     uint8_t *a_codes, *a_sf;  // MMA scale layout
+    // activations already in NVFP4 (x == nullptr, x_gs given): codes [T, H/2]
+    // and row-major scales [T, H/16] that phase 3 only permutes
+    const uint8_t *xq_codes, *xq_scales;
     int32_t *blk_hist;        // [kFrontMaxBlocks][(E + 3) & ~3]
     float *blk_amax;          // [kFrontMaxBlocks]
     unsigned int *ticket;     // zeroed once with the workspace

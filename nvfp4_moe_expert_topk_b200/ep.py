@@ -12,7 +12,12 @@ and holds its own batch of tokens.  One forward:
      experts, with its k ids rewritten to that rank's local ids (-1 for the
      slots whose expert lives elsewhere: the forward's skipped-slot rule) and
      its k weights; row counts are exchanged first, then the rows, ids and
-     weights with uneven all-to-alls;
+     weights with uneven all-to-alls.  With a quantize_fn the rows travel as
+     NVFP4: each rank quantises its batch once with the global scale of step
+     1 and sends codes and row-major scales (H/2 + H/16 bytes a row, 4032 at
+     H = 7168, against 14336 for bf16); the receiving rank's forward only
+     permutes them (nvfp4_moe_forward_quantized), so the result is the one
+     of bf16 dispatch bit for bit;
   3. each rank runs the MoE block on the rows it received with its own
      experts: the weighted sum over the token's local slots;
   4. combine: the partial outputs go back to the token's rank (all-to-all
@@ -51,11 +56,16 @@ class ExpertParallelMoE:
     amax_fn(x) -> float: max|x| of the local batch.
     experts_fn(x_recv, local_ids, weights, gs) -> [n, H]: the MoE block of
     this rank's experts on received rows (local_ids < 0 are skipped slots;
-    El .. El + num_shared - 1 are the shared experts).
+    El .. El + num_shared - 1 are the shared experts); x_recv is a bf16
+    [n, H] tensor, or with a quantize_fn the pair (codes [n, H/2], scales
+    [n, H/16]) of NVFP4 rows made with global scale gs.
+    quantize_fn(x, gs) -> (codes, scales): NVFP4 quantisation of the local
+    batch with a given global scale (None: dispatch bf16 rows).
     num_experts counts the routed experts only."""
 
     def __init__(self, num_experts: int, amax_fn: Callable, experts_fn: Callable,
-                 group: Optional[dist.ProcessGroup] = None, num_shared: int = 0):
+                 group: Optional[dist.ProcessGroup] = None, num_shared: int = 0,
+                 quantize_fn: Optional[Callable] = None):
         self.group = group
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -69,6 +79,7 @@ class ExpertParallelMoE:
         self.num_shared = num_shared
         self.amax_fn = amax_fn
         self.experts_fn = experts_fn
+        self.quantize_fn = quantize_fn
 
     # ------------------------------------------------------------ steps
     def batch_global_scale(self, x: torch.Tensor) -> np.float32:
@@ -114,7 +125,12 @@ class ExpertParallelMoE:
         dist.all_to_all_single(rc, c, group=self.group)
         recv_counts = [int(v) for v in rc.tolist()]
         order = torch.cat(tokens)
-        recv_x = self._exchange(x[order], send_counts, recv_counts)
+        if self.quantize_fn is None:
+            recv_x = self._exchange(x[order], send_counts, recv_counts)
+        else:
+            codes, scales = self.quantize_fn(x, gs)
+            recv_x = (self._exchange(codes[order], send_counts, recv_counts),
+                      self._exchange(scales[order], send_counts, recv_counts))
         recv_ids = self._exchange(torch.cat(local_ids), send_counts, recv_counts)
         recv_w = self._exchange(topk_weights[order].to(torch.float32), send_counts, recv_counts)
         y = self.experts_fn(recv_x, recv_ids, recv_w, gs)
@@ -142,18 +158,25 @@ class LibraryExperts:
         self.ws = None
 
     def __call__(self, x, local_ids, weights, gs):
-        from . import nvfp4_moe_forward, nvfp4_moe_workspace_size
+        from . import nvfp4_moe_forward, nvfp4_moe_forward_quantized, nvfp4_moe_workspace_size
         w = self.weights
-        n = x.shape[0]
-        out = torch.empty((n, w.H), dtype=torch.bfloat16, device=x.device)
+        quantised = isinstance(x, tuple)
+        dev = x[0].device if quantised else x.device
+        n = x[0].shape[0] if quantised else x.shape[0]
+        out = torch.empty((n, w.H), dtype=torch.bfloat16, device=dev)
         if n == 0:
             return out
         need = nvfp4_moe_workspace_size(n, self.k, w.E, w.H, w.I)
         if self.ws is None or self.ws.numel() < need:
-            self.ws = torch.zeros(need, dtype=torch.uint8, device=x.device)
-        x_gs = torch.tensor([float(gs)], dtype=torch.float32, device=x.device)
-        nvfp4_moe_forward(x.contiguous(), local_ids.contiguous(), weights.contiguous(), x_gs, **w.args(),
-                          inter_gs=self.inter_gs, out=out, workspace=self.ws)
+            self.ws = torch.zeros(need, dtype=torch.uint8, device=dev)
+        x_gs = torch.tensor([float(gs)], dtype=torch.float32, device=dev)
+        if quantised:
+            nvfp4_moe_forward_quantized(x[0].contiguous(), x[1].contiguous(), local_ids.contiguous(),
+                                        weights.contiguous(), x_gs, **w.args(), inter_gs=self.inter_gs, out=out,
+                                        workspace=self.ws)
+        else:
+            nvfp4_moe_forward(x.contiguous(), local_ids.contiguous(), weights.contiguous(), x_gs, **w.args(),
+                              inter_gs=self.inter_gs, out=out, workspace=self.ws)
         return out
 
 
@@ -163,3 +186,17 @@ def library_amax(x: torch.Tensor) -> float:
     a = torch.empty(1, dtype=torch.float32, device=x.device)
     nvfp4_amax(x.contiguous(), a)
     return a.item()
+
+
+def library_quantize(x: torch.Tensor, gs) -> tuple:
+    """quantize_fn backed by the library (nvfp4_quantize, row-major scales):
+    codes uint8 [T, H/2] and scales uint8 [T, H/16] of a bf16 CUDA tensor
+    with the given global scale."""
+    from . import NVFP4_SCALES_ROWMAJOR, nvfp4_quantize
+    T, H = x.shape
+    codes = torch.empty((T, H // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((T, H // 16), dtype=torch.uint8, device=x.device)
+    if T:
+        g = torch.tensor([float(gs)], dtype=torch.float32, device=x.device)
+        nvfp4_quantize(x.contiguous(), g, codes, scales, NVFP4_SCALES_ROWMAJOR)
+    return codes, scales

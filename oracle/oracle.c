@@ -24,6 +24,9 @@
  *     back per token with the top-k weights (page 1, "Phase 3": final scatter).
  *   - Per-expert intermediate global scale fixed by a warmup pass (page 1,
  *     "Phase 1", "Warmup-based gs computation"; page 2 step table, row 8).
+ *   - Expert parallelism (page 1, "Config values": 48 of the 384 experts per
+ *     rank) may ship the activations already quantised; the chain then starts
+ *     from the given codes and scales instead of quantising x.
  *
  * Readings where the pages are silent (each one is also listed in the design
  * notes of the repository):
@@ -355,6 +358,10 @@ typedef struct {
     uint8_t *h_scales;             /* [R, I/16] slot order */
     float *y;                      /* [R, H]  slot order */
     float *h_amax;                 /* [E] max |h| over each expert's rows */
+    /* activations given already quantised (both non-NULL): x is not read and
+     * these codes [T, H/2] and scales [T, H/16] stand for quantise(x, x_gs) */
+    const uint8_t *x_codes;
+    const uint8_t *x_scales;
 } oracle_moe_args;
 
 /* The whole chain, expert by expert, over the stable routing order (R6):
@@ -377,10 +384,15 @@ int oracle_moe_forward(const oracle_moe_args *p)
         if (rank[f] >= 0)
             slot_of[offsets[p->topk_ids[f]] + rank[f]] = f;
 
-    /* quantised activations, one row per token */
-    uint8_t *xq = (uint8_t *)malloc((size_t)(T * H / 2));
-    uint8_t *xs = (uint8_t *)malloc((size_t)(T * H / 16));
-    oracle_quantize_bf16(p->x, T, H, H, p->x_gs, xq, xs);
+    /* quantised activations, one row per token (or the caller's) */
+    uint8_t *xq = (uint8_t *)malloc((size_t)(T * H / 2 > 0 ? T * H / 2 : 1));
+    uint8_t *xs = (uint8_t *)malloc((size_t)(T * H / 16 > 0 ? T * H / 16 : 1));
+    if (p->x_codes && p->x_scales) {
+        memcpy(xq, p->x_codes, (size_t)(T * H / 2));
+        memcpy(xs, p->x_scales, (size_t)(T * H / 16));
+    } else {
+        oracle_quantize_bf16(p->x, T, H, H, p->x_gs, xq, xs);
+    }
     float *xd = (float *)malloc(sizeof(float) * (size_t)(T * H));
     oracle_dequantize(xq, xs, T, H, p->x_gs, xd);
 

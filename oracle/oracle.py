@@ -40,6 +40,7 @@ class MoeArgs(ctypes.Structure):
         ("inter_gs", ctypes.c_void_p),
         ("out", ctypes.c_void_p), ("h", ctypes.c_void_p), ("h_codes", ctypes.c_void_p),
         ("h_scales", ctypes.c_void_p), ("y", ctypes.c_void_p), ("h_amax", ctypes.c_void_p),
+        ("x_codes", ctypes.c_void_p), ("x_scales", ctypes.c_void_p),
     ]
 
 
@@ -189,9 +190,15 @@ def gemm(a_codes, a_scales, a_gs, b_codes, b_scales, b_gs, seg_end=None) -> np.n
 
 
 def _moe_args(x_bits, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs,
-              w2_codes, w2_scales, w2_gs, inter_gs, keep):
-    x = _c(x_bits, np.uint16)
-    T, H = x.shape
+              w2_codes, w2_scales, w2_gs, inter_gs, keep, x_codes=None, x_scales=None):
+    if x_codes is not None:                 # activations given already quantised
+        xc, xsc = _c(x_codes, np.uint8), _c(x_scales, np.uint8)
+        T, H = xc.shape[0], xc.shape[1] * 2
+        keep.append((xc, xsc))
+        x = np.zeros((T, H), np.uint16)      # not read
+    else:
+        x = _c(x_bits, np.uint16)
+        T, H = x.shape
     ids = _c(topk_ids, np.int32)
     k = ids.shape[1]
     wts = _c(topk_weights, np.float32)
@@ -210,18 +217,22 @@ def _moe_args(x_bits, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_g
     a.w13_codes, a.w13_scales, a.w13_gs = _ptr(arrays["w13_codes"]), _ptr(arrays["w13_scales"]), _ptr(arrays["w13_gs"])
     a.w2_codes, a.w2_scales, a.w2_gs = _ptr(arrays["w2_codes"]), _ptr(arrays["w2_scales"]), _ptr(arrays["w2_gs"])
     a.inter_gs = _ptr(arrays["inter_gs"])
+    if x_codes is not None:
+        a.x_codes, a.x_scales = _ptr(xc), _ptr(xsc)
     return a, (T, H, I, E, k)
 
 
 def moe_forward(x_bits, topk_ids, topk_weights, x_gs, w13_codes, w13_scales, w13_gs,
-                w2_codes, w2_scales, w2_gs, inter_gs, intermediates=False):
+                w2_codes, w2_scales, w2_gs, inter_gs, intermediates=False, x_codes=None, x_scales=None):
     """Full chain.  Weights are given with canonical row-major scales:
     w13_codes [E, 2I, H/2], w13_scales [E, 2I, H/16], w2_codes [E, H, I/2],
-    w2_scales [E, H, I/16].  Returns out fp32 [T, H] (and, with
-    intermediates=True, a dict of h / h_codes / h_scales / y in slot order)."""
+    w2_scales [E, H, I/16].  With x_codes / x_scales ([T, H/2], [T, H/16])
+    the activations are taken as already quantised with x_gs (x_bits is
+    ignored).  Returns out fp32 [T, H] (and, with intermediates=True, a dict
+    of h / h_codes / h_scales / y in slot order)."""
     keep = []
     a, (T, H, I, E, k) = _moe_args(x_bits, topk_ids, topk_weights, x_gs, w13_codes, w13_scales,
-                                   w13_gs, w2_codes, w2_scales, w2_gs, inter_gs, keep)
+                                   w13_gs, w2_codes, w2_scales, w2_gs, inter_gs, keep, x_codes, x_scales)
     out = np.zeros((T, H), np.float32)
     a.out = _ptr(out)
     inter = None

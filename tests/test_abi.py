@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
     for want in ["nvfp4_quantize", "nvfp4_gemm", "nvfp4_moe_forward", "nvfp4_global_scale",
                  "nvfp4_swizzle_scales", "nvfp4_moe_workspace_size", "nvfp4_moe_get_error",
                  "nvfp4_moe_route_debug", "nvfp4_moe_calibrate", "nvfp4_status_string", "nvfp4_moe_topk", "nvfp4_moe_topk_shared",
-                 "nvfp4_moe_forward_noalloc", "nvfp4_moe_forward_timed"]:
+                 "nvfp4_moe_forward_noalloc", "nvfp4_moe_forward_timed", "nvfp4_moe_forward_quantized"]:
         assert want in names
 
 
@@ -115,6 +115,20 @@ def test_moe_forward_checks(L):
     a.w2_codes = F
     a.out = None
     assert L.nvfp4_moe_forward_noalloc(ctypes.byref(a), None) == -1
+    a.out = F
+    # pre-quantised activations: x may be NULL, x_gs and both code buffers are required
+    a.x = None
+    a.w2_codes = None
+    assert L.nvfp4_moe_forward_quantized(ctypes.byref(a), ctypes.c_void_p(F), ctypes.c_void_p(F),
+                                         ctypes.c_void_p(F), 1 << 40, None) == -1     # w2_codes NULL
+    a.w2_codes = F
+    assert L.nvfp4_moe_forward_quantized(ctypes.byref(a), None, ctypes.c_void_p(F), ctypes.c_void_p(F),
+                                         1 << 40, None) == -1
+    assert L.nvfp4_moe_forward_quantized(ctypes.byref(a), ctypes.c_void_p(F + 4), ctypes.c_void_p(F),
+                                         ctypes.c_void_p(F), 1 << 40, None) == -3
+    a.x_gs = None
+    assert L.nvfp4_moe_forward_quantized(ctypes.byref(a), ctypes.c_void_p(F), ctypes.c_void_p(F),
+                                         ctypes.c_void_p(F), 1 << 40, None) == -1
 
 
 def test_topk_checks(L):

@@ -25,11 +25,11 @@ WORLD = 2
 
 
 def config(scenario):
-    return CFG_SHARED if scenario == "shared" else CFG
+    return CFG_SHARED if scenario.endswith("shared") else CFG
 
 
 def rank_tokens(r, scenario):
-    if scenario == "empty_rank" and r == 1:
+    if scenario.endswith("empty_rank") and r == 1:
         return 0                                               # a rank with no tokens this step
     return CFG.T + 8 * r                                       # ranks hold different batch sizes
 
@@ -68,12 +68,21 @@ def worker(rank, port, scenario):
         igs = inter_gs_all(cfg)
 
         def experts_fn(x, local_ids, w, gs):
-            out = O.moe_forward(W.bf16_bits(x), local_ids.numpy(), w.numpy(), gs, **ow.oracle_kwargs(),
-                                inter_gs=igs[local])
+            if isinstance(x, tuple):                           # NVFP4 rows: codes, row-major scales
+                out = O.moe_forward(None, local_ids.numpy(), w.numpy(), gs, **ow.oracle_kwargs(),
+                                    inter_gs=igs[local], x_codes=x[0].numpy(), x_scales=x[1].numpy())
+            else:
+                out = O.moe_forward(W.bf16_bits(x), local_ids.numpy(), w.numpy(), gs, **ow.oracle_kwargs(),
+                                    inter_gs=igs[local])
             return torch.from_numpy(out)
 
+        def quantize_fn(x, gs):
+            c, sc = O.quantize_bf16(W.bf16_bits(x), gs) if x.shape[0] else \
+                (np.zeros((0, CFG.H // 2), np.uint8), np.zeros((0, CFG.H // 16), np.uint8))
+            return torch.from_numpy(np.ascontiguousarray(c)), torch.from_numpy(np.ascontiguousarray(sc))
+
         ep = ExpertParallelMoE(CFG.E, amax_fn=lambda x: O.amax_bf16(W.bf16_bits(x)), experts_fn=experts_fn,
-                               num_shared=len(shared))
+                               num_shared=len(shared), quantize_fn=quantize_fn if "nvfp4" in scenario else None)
         x, ids, w = rank_batch(rank, scenario)
         got = ep.forward(x, ids, w, out_dtype=torch.float32).numpy()
 
@@ -99,7 +108,8 @@ def free_port():
         return s.getsockname()[1]
 
 
-@pytest.mark.parametrize("scenario", ["plain", "one_sided", "skips", "shared", "empty_rank"])
+@pytest.mark.parametrize("scenario", ["plain", "one_sided", "skips", "shared", "empty_rank", "nvfp4",
+                                      "nvfp4_shared", "nvfp4_empty_rank"])
 def test_expert_parallel_two_ranks(scenario):
     mp.start_processes(worker, args=(free_port(), scenario), nprocs=WORLD, start_method="spawn")
 

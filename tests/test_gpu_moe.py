@@ -553,3 +553,30 @@ def test_tile_tables_of_full_size_routing(name, mode):
     route = O.route(ids.numpy(), cfg.E)
     o, n = region(p, 5)
     np.testing.assert_array_equal(ws[o:o + n].cpu().numpy().view(np.int32), route["pos_padded"])
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill_ep48"])
+def test_forward_on_prequantised_rows_equals_forward(name):
+    """nvfp4_moe_forward_quantized on the codes and row-major scales that
+    nvfp4_quantize makes from x with x_gs gives nvfp4_moe_forward's output on
+    x with x_gs bit for bit (the front only permutes the given rows)."""
+    from nvfp4_moe_expert_topk_b200 import NVFP4_SCALES_ROWMAJOR, nvfp4_moe_forward_quantized, nvfp4_quantize
+    cfg = W.MOE_CONFIGS[name]
+    x, ids, w = W.batch(cfg)
+    dw = prep.MoeWeights.synthetic(cfg, DEV)
+    xd, idd, wd = x.to(DEV), ids.to(DEV), w.to(DEV)
+    gs = torch.empty(1, dtype=torch.float32, device=DEV)
+    nvfp4_global_scale(xd, gs)
+    inter = torch.full((cfg.E,), 40.0, dtype=torch.float32, device=DEV)
+    ws = prep.workspace(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I, DEV)
+    ref = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=DEV)
+    nvfp4_moe_forward(xd, idd, wd, gs, **dw.args(), inter_gs=inter, out=ref, workspace=ws)
+    codes = torch.empty(cfg.T, cfg.H // 2, dtype=torch.uint8, device=DEV)
+    scales = torch.empty(cfg.T, cfg.H // 16, dtype=torch.uint8, device=DEV)
+    nvfp4_quantize(xd, gs, codes, scales, NVFP4_SCALES_ROWMAJOR)
+    out = torch.full_like(ref, float("nan"))
+    ws2 = prep.workspace(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I, DEV)
+    nvfp4_moe_forward_quantized(codes, scales, idd, wd, gs, **dw.args(), inter_gs=inter, out=out, workspace=ws2)
+    torch.cuda.synchronize()
+    assert nvfp4_moe_get_error(ws2) == 0
+    assert torch.isfinite(out.float()).all() and torch.equal(out, ref)

@@ -101,11 +101,15 @@ def _tiny_problem(E=4, k=2, T=12, H=64, I=32, seed=0):
     return P, (E, k, T, H, I)
 
 
-def _brute_force(P, inter_gs, dims):
+def _brute_force(P, inter_gs, dims, x_codes=None, x_scales=None):
     """Per token, per slot: dense expert MLP on dequantised operands (numpy
-    matmul, torch SiLU), re-quantised with the oracle's pinned quantiser."""
+    matmul, torch SiLU), re-quantised with the oracle's pinned quantiser.
+    With x_codes / x_scales, those stand for the quantised activations."""
     E, k, T, H, I = dims
-    xc, xs = O.quantize_bf16(P["x_bits"], P["x_gs"])
+    if x_codes is None:
+        xc, xs = O.quantize_bf16(P["x_bits"], P["x_gs"])
+    else:
+        xc, xs = x_codes, x_scales
     A = O.dequantize(xc, xs, P["x_gs"]).astype(np.float64)
     out = np.zeros((T, H))
     h_amax = np.zeros(E, np.float32)
@@ -230,3 +234,25 @@ def test_warmup_fallback_for_experts_without_rows():
     amax = inter["h_amax"]
     assert amax[1] == 0 and amax[3] == 0
     assert inter_gs[1] == inter_gs[3] == O.global_scale_from_amax(max(amax[0], amax[2]))
+
+
+def test_moe_forward_on_given_codes_equals_brute_force():
+    """Activations given already in NVFP4 (expert-parallel dispatch of 4-bit
+    rows): arbitrary codes and scales, not those of any bf16 x, go through
+    the same chain as the brute force built from them; with the codes of x
+    itself the output is the bf16 path's bit for bit."""
+    P, dims = _tiny_problem(seed=3)
+    E, k, T, H, I = dims
+    rng = np.random.default_rng(3)
+    xc = rng.integers(0, 256, (T, H // 2), dtype=np.uint8)
+    xs = rng.integers(0x28, 0x48, (T, H // 16), dtype=np.uint8)      # E4M3 scales 0.25 .. 4
+    Q = dict(P, x_gs=np.float32(3.0))
+    _, h_amax, _ = _brute_force(Q, None, dims, xc, xs)
+    inter_gs = np.array([O.global_scale_from_amax(a if a > 0 else h_amax.max()) for a in h_amax], np.float32)
+    out = O.moe_forward(**Q, inter_gs=inter_gs, x_codes=xc, x_scales=xs)
+    ref, _, _ = _brute_force(Q, inter_gs, dims, xc, xs)
+    np.testing.assert_allclose(out, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+    own_c, own_s = O.quantize_bf16(P["x_bits"], P["x_gs"])
+    inter_gs = O.moe_warmup_inter_gs(**P)
+    assert np.array_equal(O.moe_forward(**P, inter_gs=inter_gs, x_codes=own_c, x_scales=own_s),
+                          O.moe_forward(**P, inter_gs=inter_gs))
