@@ -1073,8 +1073,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA-graph replay")
-    ap.add_argument("--only", choices=["all", "decode", "prefill", "prefill_ep48", "shared", "tiny", "decode_shared",
-                                       "prefill_shared"], default="all",
+    ap.add_argument("--only", choices=["all", "decode", "prefill", "prefill_ep48", "prefill_front", "shared", "tiny",
+                                       "decode_shared", "prefill_shared"], default="all",
                     help="one workload alone (small profiling cases)")
     args = ap.parse_args()
     if args.impl == "reference":

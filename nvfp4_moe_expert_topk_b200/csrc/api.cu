@@ -202,12 +202,16 @@ int moe_cg(int64_t R, int E)
 // experts with two or more m-tiles on pair tiles (pair mode 1): the pair
 // launch costs a few microseconds even when no expert is that heavy.
 constexpr int64_t kSplitMinRows = 2048;
-// Pair mode 1 runs the pair launch on this many clusters of two SMs beside
-// the 1-CTA launch, which starts on the other SMs and takes over the pair
-// launch's SMs when it ends.  The 1-CTA tiles stream the light experts'
-// weights from HBM; the pair tiles re-read the heavy experts' weights from
-// L2, so the two overlap instead of running one after the other.
-constexpr int kSplitPairClusters = 24;
+// Pair mode 1 runs the pair launch on every cluster of two SMs that fits,
+// then the 1-CTA launch, whose CTAs take over each SM as soon as the pair
+// launch's CTA there has finished (the pair launch lets its dependent start
+// at once; the 1-CTA launch claims tiles, so CTAs that start late just take
+// fewer).  Measured on the B200 (prefill, CTA start / end stamps): running the
+// pair launch on fewer clusters beside the 1-CTA launch gains nothing -- with
+// both resident, the two compete for the same L2 -> shared-memory fill and the
+// pair of launches takes as long as one after the other (2.56 against 2.58 ms
+// with two streams; as a dependent launch the second kernel's resident CTAs
+// made no progress until the first kernel ended).
 
 int gemm_grid(int cg, int64_t tiles, int num_sms)
 {
@@ -729,14 +733,14 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
     if (st != NVFP4_OK)
         return st;
     if (pl.pair_mode == 1) {
-        // the heavy experts' pairs (fused L1 -> L2, kSplitPairClusters
-        // clusters), and beside it the fused 1-CTA launch over the light list:
-        // the pair launch lets its dependent start at once; the 1-CTA launch
-        // reads only what the front wrote and waits for the pair launch at its
-        // end, so that the combine after it sees both
+        // the heavy experts' pairs (fused L1 -> L2 on pair tiles), then the
+        // fused 1-CTA launch over the light list: the pair launch lets its
+        // dependent start at once, so 1-CTA CTAs move onto SMs as pair CTAs
+        // finish; the 1-CTA launch reads only what the front wrote and waits
+        // for the pair launch at its end, so that the combine sees both
         GemmArgs p1 = g1;
         p1.pdl_trigger_early = 1;
-        const int pairs = std::min(kSplitPairClusters, gemm_pair_clusters(sms));
+        const int pairs = gemm_pair_clusters(sms);
         GemmArgs l1 = g1;
         l1.pdl_wait_at_end = 1;
         if (launch_moe_fused(2, ma1, ma1_32, mb1, p1, ma2, ma2_32, mb2, g2, 2 * pairs, s) != cudaSuccess ||

@@ -62,6 +62,11 @@ MOE_CONFIGS = {
     # expert-parallel slice: small enough to profile and to check in full
     "prefill_ep48": MoeConfig("prefill_ep48", E=48, k=6, T=512, H=7168, I=3072, routing="zipf", outliers=True,
                               warmup_T=64, zipf_zero_tail=2),
+    # the prefill batch and routing with a 128-wide expert intermediate:
+    # the front (global scale, routing, quantise + permute of x) is exactly
+    # the prefill's, the weights are 1/24 of its (a small profiling case)
+    "prefill_front": MoeConfig("prefill_front", E=384, k=6, T=4096, H=7168, I=128, routing="zipf", outliers=True,
+                               warmup_T=16),
     # the decode batch with the shared expert folded in as a 49th group
     # (page 1 "Phase 1": the shared expert is the routed chain with one
     # expert and no routing; same H and I as a routed expert)
