@@ -49,7 +49,7 @@ BF16_TO_FP4_NOMINAL_RATIO = 4.0        # 9 / 2.25 PFLOP/s dense
 STAGES = ["global_scale", "route", "quantize_permute", "l1_gate_up_swiglu_quant", "l2_down", "combine"]
 FRONT_STAGE = "front"                  # global scale of the batch + routing + quantise/permute
 FUSED_STAGE = "l1_l2_fused"            # L1 and L2 as one launch (nvfp4_moe_plan)
-SPLIT_STAGE = "l1_l2_pairs_beside_light"   # pair mode 1: the fused pair launch and, beside it, the fused 1-CTA one
+SPLIT_STAGE = "l1_l2_pairs_then_light"     # pair mode 1: the fused pair launch, then the fused 1-CTA one
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 GEMM_SOURCES = ["gemm.cu", "ptx.cuh", "quant.cuh", "internal.h"]
 
@@ -329,9 +329,10 @@ def fold_stages(per_stage, fused, pair_mode):
     what the plan runs there: the front (one launch: global scale, routing,
     quantise + permute) and then
       pair mode 0, fused   the fused 1-CTA L1 + L2 launch;
-      pair mode 1          the heavy experts' fused pair launch and, running
-                           beside it, the fused 1-CTA launch over the other
-                           m-tiles (one stage: they overlap);
+      pair mode 1          the heavy experts' fused pair launch, then the
+                           fused 1-CTA launch over the other m-tiles, whose
+                           CTAs take over the SMs as the pair CTAs finish
+                           (one stage: no event between them);
       otherwise            L1, then L2;
     and the combine."""
     d = dict(per_stage)

@@ -38,6 +38,7 @@ constexpr int kFrontThreads = 1024;
 constexpr int kFrontWarps = kFrontThreads / 32;
 constexpr int kRouteWarps = 16;             // warps that own slot chunks (per-warp histograms)
 constexpr int kQuantCols = 1024;            // columns per quantisation item: 32 per lane
+constexpr int kIdsCache = 4096;             // a block's slot ids kept in shared memory between phases 1 and 2
 
 __device__ __forceinline__ int block_count(int64_t T, int b, int G)
 {
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
     int32_t *pre_s = tot_s + Epad;                    // [Epad] slots of e in earlier blocks
     int32_t *poff_s = pre_s + Epad;                   // [Epad] padded row offset of e
     int32_t *off_s = poff_s + Epad;                   // [Epad] row offset of e
+    int32_t *ids_s = off_s + Epad;                    // [kIdsCache] this block's slot ids (when they fit)
     __shared__ int scan_scratch[256];
     __shared__ float red[kFrontWarps];
     __shared__ int abort_s;
@@ -142,13 +144,13 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
         const int64_t n8 = static_cast<int64_t>(t1 - t0) * a.H / 8;     // H % 128 == 0
         const uint4 *xv = reinterpret_cast<const uint4 *>(a.x + static_cast<int64_t>(t0) * a.H);
         float m = 0.0f;
-        for (int64_t i0 = tid; i0 < n8; i0 += 4 * kFrontThreads) {
-            uint4 v[4];
+        for (int64_t i0 = tid; i0 < n8; i0 += 8 * kFrontThreads) {
+            uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)            // four 16-byte loads in flight per thread (64 KB per block)
+            for (int u = 0; u < 8; ++u)            // eight 16-byte loads in flight per thread (128 KB per block)
                 v[u] = i0 + u * kFrontThreads < n8 ? __ldg(xv + i0 + u * kFrontThreads) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v[u]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
     const int64_t chunk = (nslots + kRouteWarps - 1) / kRouteWarps;
     const int64_t c0 = f0 + (nslots < warp * chunk ? nslots : warp * chunk);
     const int64_t c1 = f0 + (nslots < (warp + 1) * chunk ? nslots : (warp + 1) * chunk);
+    const bool ids_cached = nslots <= kIdsCache;
     if (warp < kRouteWarps) {
         int bad = 0;
         for (int64_t base = c0; base < c1; base += 4 * 32) {
@@ -176,6 +179,8 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
                 ev[u] = base + lane + 32 * u < c1 ? __ldg(a.ids + base + lane + 32 * u) : -1;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
+                if (ids_cached && base + lane + 32 * u < c1)
+                    ids_s[base + lane + 32 * u - f0] = ev[u];
                 if (ev[u] >= E)
                     bad = 1;
                 else if (ev[u] >= 0)
@@ -227,18 +232,62 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
         return;
 
     // ------------------------------------------------ phase 2: scans, positions
+    // One pass over what the blocks published, every load issued before any
+    // result is used: the blocks' max|x| (one per thread) and their expert
+    // counts -- nq column blocks of 32 int4 (128 experts) and ng = 32 / nq
+    // row groups of warps; warp (g, q) sums block rows g, g + ng, ... of its
+    // column block, eight rows in flight, then adds its sums into shared
+    // memory.
     float gs = 1.0f;
+    float amax_part = 0.0f;
+    if (do_amax && tid < G)
+        amax_part = __ldcg(a.blk_amax + tid);
+    {
+        const int E4 = Epad / 4;
+        const int nq = (E4 + 31) / 32;
+        const int ng = kFrontWarps / nq;
+        const int q = warp / ng, g = warp - (warp / ng) * ng;
+        const int c4 = 32 * q + lane;
+        int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
+        if (q < nq && c4 < E4) {
+            for (int r0 = g; r0 < G; r0 += 8 * ng) {
+                int4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int r = r0 + u * ng;
+                    v[u] = r < G ? __ldcg(reinterpret_cast<const int4 *>(a.blk_hist + static_cast<int64_t>(r) * Epad) + c4)
+                                 : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    tot.x += v[u].x, tot.y += v[u].y, tot.z += v[u].z, tot.w += v[u].w;
+                    if (r0 + u * ng < b)
+                        pre.x += v[u].x, pre.y += v[u].y, pre.z += v[u].z, pre.w += v[u].w;
+                }
+            }
+            const int e = 4 * c4;
+            const int tv[4] = {tot.x, tot.y, tot.z, tot.w};
+            const int pv[4] = {pre.x, pre.y, pre.z, pre.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (tv[i])
+                    atomicAdd(&tot_s[e + i], tv[i]);
+                if (pv[i])
+                    atomicAdd(&pre_s[e + i], pv[i]);
+            }
+        }
+    }
     if (do_amax) {
-        float m = 0.0f;
-        for (int i = tid; i < G; i += kFrontThreads)
-            m = fmaxf(m, __ldcg(a.blk_amax + i));
+        float m = amax_part;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0)
             red[warp] = m;
-        __syncthreads();
-        m = red[0];
+    }
+    __syncthreads();
+    if (do_amax) {
+        float m = red[0];
         for (int w = 1; w < kFrontWarps; ++w)
             m = fmaxf(m, red[w]);
         gs = m == 0.0f ? 1.0f : __fdiv_rn(2688.0f, m);
@@ -247,50 +296,6 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
     } else if (a.x != nullptr) {
         gs = __ldg(a.x_gs);
     }
-    // totals and earlier-block counts: 8 row groups x 4 column quarters of
-    // warps; warp (g, q) reads block rows g, g + 8, ... over int4 columns
-    // [64 q, 64 q + 64) (two per lane), sums them in registers, then adds
-    // its sums into shared memory
-    {
-        const int E4 = Epad / 4;
-        const int g = warp & 7, q = warp >> 3;
-        int4 tot[2], pre[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-            tot[j] = pre[j] = make_int4(0, 0, 0, 0);
-        if (64 * q < E4) {
-#pragma unroll 4
-            for (int r = g; r < G; r += 8) {
-                const int4 *row = reinterpret_cast<const int4 *>(a.blk_hist + static_cast<int64_t>(r) * Epad);
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int c4 = 64 * q + lane + 32 * j;
-                    if (c4 < E4) {
-                        const int4 v = __ldcg(row + c4);
-                        tot[j].x += v.x, tot[j].y += v.y, tot[j].z += v.z, tot[j].w += v.w;
-                        if (r < b)
-                            pre[j].x += v.x, pre[j].y += v.y, pre[j].z += v.z, pre[j].w += v.w;
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int e = 4 * (64 * q + lane + 32 * j);
-            if (e < Epad) {
-                const int tv[4] = {tot[j].x, tot[j].y, tot[j].z, tot[j].w};
-                const int pv[4] = {pre[j].x, pre[j].y, pre[j].z, pre[j].w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if (tv[i])
-                        atomicAdd(&tot_s[e + i], tv[i]);
-                    if (pv[i])
-                        atomicAdd(&pre_s[e + i], pv[i]);
-                }
-            }
-        }
-    }
-    __syncthreads();
     // expert scans: thread e owns expert e (E <= 1024)
     {
         const int e = tid;
@@ -346,8 +351,10 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
         for (int64_t base = c0; base < c1; base += 4 * 32) {
             int ev[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                ev[u] = base + 32 * u + lane < c1 ? __ldg(a.ids + base + 32 * u + lane) : -1;
+            for (int u = 0; u < 4; ++u) {
+                const int64_t f = base + 32 * u + lane;
+                ev[u] = f < c1 ? (ids_cached ? ids_s[f - f0] : __ldg(a.ids + f)) : -1;
+            }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int64_t f = base + 32 * u + lane;
@@ -383,7 +390,6 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
     // into the 4-byte word of one 64-column group of the MMA scale layout.
     const int64_t H = a.H;
     const int nchunks = static_cast<int>((H + kQuantCols - 1) / kQuantCols);
-    const int64_t kbs = H / 64;
     const int items = (t1 - t0) * nchunks;
     for (int it = warp; it < items; it += kFrontWarps) {
         const int t = t0 + it / nchunks;
@@ -429,16 +435,15 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
             }
         }
         const uint32_t s_hi = __shfl_xor_sync(0xffffffffu, s2, 1);
-        const uint32_t sword = s2 | (s_hi << 16);          // valid on even lanes
-        const int64_t kb = (col0 >> 6);                      // 64-column group of this lane pair
+        const uint32_t sword = s2 | (s_hi << 16);          // valid on even lanes: 4 scales, 64 columns
         for (int d = 0; d < k; ++d) {
             const int dst = __shfl_sync(0xffffffffu, my_dst, d);
             if (!active || dst < 0)
                 continue;
             *reinterpret_cast<uint4 *>(a.a_codes + static_cast<int64_t>(dst) * (H / 2) + col0 / 2) =
                 make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            if ((lane & 1) == 0)
-                *reinterpret_cast<uint32_t *>(a.a_sf + mma_scale_offset(dst, kb, kbs)) = sword;
+            if ((lane & 1) == 0)        // row-major: the warp's 64 scale bytes of this chunk are contiguous
+                *reinterpret_cast<uint32_t *>(a.a_sf + static_cast<int64_t>(dst) * a.a_sf_ld + col0 / 16) = sword;
         }
     }
 }
@@ -446,7 +451,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
 size_t front_smem_bytes(int E)
 {
     const int Epad = (E + 3) & ~3;
-    return sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * E + 4 * static_cast<size_t>(Epad));
+    return sizeof(int32_t) * (static_cast<size_t>(kRouteWarps) * E + 4 * static_cast<size_t>(Epad) + kIdsCache);
 }
 
 int front_blocks(int64_t T, int num_sms)

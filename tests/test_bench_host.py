@@ -38,9 +38,9 @@ def test_fold_two_launch_plan():
 
 
 def test_fold_split_plan_and_its_bytes():
-    """Pair mode 1: the fused pair launch and the fused 1-CTA launch run side
-    by side, one stage; its algorithmic bytes read each expert once.  The
-    tile split follows the plan's rule."""
+    """Pair mode 1: the fused pair launch and the fused 1-CTA launch form one
+    stage; its algorithmic bytes read each expert once.  The tile split
+    follows the plan's rule."""
     import numpy as np
     d = bench.Workload.fold(_Plan(True, 1), STAGE_MS)
     assert set(d) == {bench.FRONT_STAGE, bench.SPLIT_STAGE, "combine"}

@@ -126,8 +126,8 @@ def check_intermediates(p, ws, inter):
     xc, xs = O.quantize_bf16(W.bf16_bits(p.x), p.x_gs)
     o, n = region(p, 0)
     a_codes = wsn[o:o + n].reshape(-1, H // 2)
-    o, n = region(p, 1)
-    a_sc = from_mma_layout(wsn[o:o + n], a_codes.shape[0], H)
+    o, n = region(p, 1)                             # row-major, row stride H/16 rounded up to 16 bytes
+    a_sc = wsn[o:o + n].reshape(a_codes.shape[0], -1)[:, :H // 16]
     tok = np.arange(T * k) // k
     np.testing.assert_array_equal(a_codes[inv[live]], xc[tok[live]])
     np.testing.assert_array_equal(a_sc[inv[live]], xs[tok[live]])
