@@ -222,8 +222,9 @@ int nvfp4_moe_route_debug(const int32_t *topk_ids, int64_t T, int k, int E, int3
 
 /* Byte offset and size of a workspace region (build helper for inspection
  * and tests, no passage on the pages; host only).
- * region: 0 A codes, 1 A scales (row-major [rows, H/16 rounded up to a
- * multiple of 16] bytes), 2 h codes, 3 h scales
+ * region: 0 A codes, 1 A scales (row blocks: for each 128-row block and
+ * each 256-column k-tile, 2 KB holding the row's 16 scale bytes of that
+ * k-tile at (row % 128) * 16), 2 h codes, 3 h scales
  * (MMA layout), 4 y (bf16 [T*k, H], rows in expert-major routing order),
  * 5 inv, 6 counts, 7 padded offsets, 8 the fp32 global scale of x computed
  * by the last call made with x_gs = NULL, 9 the m-tile table (int32 x 4 per

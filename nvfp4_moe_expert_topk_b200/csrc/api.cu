@@ -71,21 +71,6 @@ int make_code_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
-// 2-D uint8 tensor map over row-major scales [rows, cols_bytes] with row
-// stride ld (a multiple of 16), box 16 bytes (one 256-element k-tile) x
-// box_rows rows, no swizzle; bytes past a row's end read as zero.
-int make_sf_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols_bytes, int64_t ld, int box_rows)
-{
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols_bytes), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
-    cuuint32_t box[2] = {16, static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
-}
-
 bool aligned16(const void *p)
 {
     return (reinterpret_cast<uintptr_t>(p) & 15) == 0;
@@ -103,7 +88,7 @@ int64_t round_up(int64_t v, int64_t m)
 
 // ---------------------------------------------------------------- workspace
 struct Layout {
-    int64_t mt_max = 0, rpad = 0, sfa_ld = 0;
+    int64_t mt_max = 0, rpad = 0, sfa_block = 0;
     int64_t counts = 0, off = 0, poff = 0, mtiles = 0, pairs = 0, light = 0, ready = 0, inv = 0, yrow = 0, amax = 0;
     int64_t blk_hist = 0, blk_amax = 0;
     int64_t a_codes = 0, a_sf = 0, h_codes = 0, h_sf = 0, y = 0, total = 0;
@@ -122,7 +107,7 @@ Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
     const int64_t ne = std::min<int64_t>(E, R);
     L.mt_max = (R + 127 * ne) / 128;          // >= sum_e ceil(count_e / 128)
     L.rpad = 128 * L.mt_max;
-    L.sfa_ld = round_up(H / 16, 16);          // row-major x scales: row stride a multiple of 16 bytes
+    L.sfa_block = ((H + 255) / 256) * 2048;  // x scales in row blocks: per 128 rows, 2 KB per k-tile
     int64_t o = 256;
     auto take = [&](int64_t bytes) {
         const int64_t at = o;
@@ -142,7 +127,7 @@ Layout ws_layout(int64_t T, int k, int E, int64_t H, int64_t I)
     L.blk_hist = take(4LL * kFrontMaxBlocks * ((E + 3) & ~3));
     L.blk_amax = take(4LL * kFrontMaxBlocks);
     L.a_codes = take(L.rpad * (H / 2));
-    L.a_sf = take(L.rpad * L.sfa_ld);
+    L.a_sf = take((L.rpad / 128) * L.sfa_block);
     L.h_codes = take(L.rpad * (I / 2));
     L.h_sf = take(L.rpad * (I / 16));
     L.y = take(R * H * 2);
@@ -245,7 +230,7 @@ const float *x_gs_ptr(const nvfp4_moe_args *a, uint8_t *ws)
 
 // Maps and arguments of the grouped L1 GEMM (gate_up, SwiGLU epilogue).
 int l1_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, CUtensorMap *ma, CUtensorMap *ma32,
-             CUtensorMap *mb, CUtensorMap *msf, CUtensorMap *msf32, GemmArgs *g)
+             CUtensorMap *mb, GemmArgs *g)
 {
     const int64_t H = a->H, I = a->I;
     const int E = a->E;
@@ -253,16 +238,13 @@ int l1_setup(const nvfp4_moe_args *a, uint8_t *ws, const Layout &L, CUtensorMap 
     if (st == NVFP4_OK)
         st = make_code_map(ma32, ws + L.a_codes, L.rpad, H / 2, 32);
     if (st == NVFP4_OK)
-        st = make_sf_map(msf, ws + L.a_sf, L.rpad, H / 16, L.sfa_ld, 128);
-    if (st == NVFP4_OK)
-        st = make_sf_map(msf32, ws + L.a_sf, L.rpad, H / 16, L.sfa_ld, 32);
-    if (st == NVFP4_OK)
         st = make_code_map(mb, a->w13_codes, static_cast<int64_t>(E) * 2 * I, H / 2, 128);
     if (st != NVFP4_OK)
         return st;
     *g = GemmArgs{};
     g->sfa = ws + L.a_sf;
     g->sfa_rowmajor = 1;
+    g->sfa_block_stride = L.sfa_block;
     g->sfb = a->w13_scales;
     g->sfb_block_stride = (H / 64) * 512;
     g->K = static_cast<int>(H);
@@ -373,7 +355,6 @@ FrontArgs front_args(const nvfp4_moe_args *a, const int32_t *ids, int64_t T, int
     f.err = reinterpret_cast<int32_t *>(ws);
     f.a_codes = ws + L.a_codes;
     f.a_sf = ws + L.a_sf;
-    f.a_sf_ld = L.sfa_ld;
     f.blk_hist = reinterpret_cast<int32_t *>(ws + L.blk_hist);
     f.blk_amax = reinterpret_cast<float *>(ws + L.blk_amax);
     f.ticket = reinterpret_cast<unsigned int *>(ws + kHdrTicket);
@@ -649,7 +630,7 @@ int gemm_impl(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs
         return cuda_status(launch_gemm_streamk(d.cg, ma, ma32, mb, g, d.grid, s));
     }
     const int grid = gemm_grid(d.cg, d.tiles, sms);
-    return cuda_status(launch_gemm(d.bn, EPI_BF16, d.cg, ma, ma32, mb, ma, ma32, g, grid, s));
+    return cuda_status(launch_gemm(d.bn, EPI_BF16, d.cg, ma, ma32, mb, g, grid, s));
 }
 
 } // namespace
@@ -701,7 +682,7 @@ int nvfp4_moe_workspace_region(int64_t T, int k, int E, int64_t H, int64_t I, in
     const int64_t R = T * k;
     switch (region) {
     case 0: *offset = L.a_codes; *bytes = L.rpad * (H / 2); break;
-    case 1: *offset = L.a_sf; *bytes = L.rpad * L.sfa_ld; break;
+    case 1: *offset = L.a_sf; *bytes = (L.rpad / 128) * L.sfa_block; break;
     case 2: *offset = L.h_codes; *bytes = L.rpad * (I / 2); break;
     case 3: *offset = L.h_sf; *bytes = L.rpad * (I / 16); break;
     case 4: *offset = L.y; *bytes = R * H * 2; break;
@@ -746,9 +727,9 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
     if (st != NVFP4_OK)
         return st;
     const int64_t H = a->H;
-    CUtensorMap ma1, ma1_32, mb1, msf1, msf1_32, ma2, ma2_32, mb2;
+    CUtensorMap ma1, ma1_32, mb1, ma2, ma2_32, mb2;
     GemmArgs g1, g2;
-    st = l1_setup(a, ws, L, &ma1, &ma1_32, &mb1, &msf1, &msf1_32, &g1);
+    st = l1_setup(a, ws, L, &ma1, &ma1_32, &mb1, &g1);
     if (st == NVFP4_OK)
         st = l2_setup(a, ws, L, pl.l2_bn, &ma2, &ma2_32, &mb2, &g2);
     if (st != NVFP4_OK)
@@ -764,30 +745,30 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
         const int pairs = gemm_pair_clusters(sms);
         GemmArgs l1 = g1;
         l1.pdl_wait_at_end = 1;
-        if (launch_moe_fused(2, ma1, ma1_32, mb1, msf1, msf1_32, p1, ma2, ma2_32, mb2, g2, 2 * pairs, s) !=
+        if (launch_moe_fused(2, ma1, ma1_32, mb1, p1, ma2, ma2_32, mb2, g2, 2 * pairs, s) !=
                 cudaSuccess ||
-            launch_moe_fused(1, ma1, ma1_32, mb1, msf1, msf1_32, l1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
+            launch_moe_fused(1, ma1, ma1_32, mb1, l1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
             mark(events, 3, s) != NVFP4_OK || mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
     } else if (pl.pair_mode == 2) {
         // every m-tile on pair tiles: L1 launch, then L2 launch
         const int pair_grid = gemm_grid(2, 1LL << 30, sms);
-        if (launch_gemm(256, EPI_SWIGLU_QUANT, 2, ma1, ma1_32, mb1, msf1, msf1_32, g1, pair_grid, s) != cudaSuccess ||
+        if (launch_gemm(256, EPI_SWIGLU_QUANT, 2, ma1, ma1_32, mb1, g1, pair_grid, s) != cudaSuccess ||
             mark(events, 3, s) != NVFP4_OK ||
-            launch_gemm(256, EPI_BF16, 2, ma2, ma2_32, mb2, ma2, ma2_32, g2, pair_grid, s) != cudaSuccess ||
+            launch_gemm(256, EPI_BF16, 2, ma2, ma2_32, mb2, g2, pair_grid, s) != cudaSuccess ||
             mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
     } else if (pl.fused) {
         // every m-tile on 1-CTA tiles, L1 and L2 in one launch
-        if (launch_moe_fused(1, ma1, ma1_32, mb1, msf1, msf1_32, g1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
+        if (launch_moe_fused(1, ma1, ma1_32, mb1, g1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
             mark(events, 3, s) != NVFP4_OK || mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
     } else {
         // 128-wide L2 tiles: L1 launch, then L2 launch, 1-CTA tiles
-        if (launch_gemm(256, EPI_SWIGLU_QUANT, 1, ma1, ma1_32, mb1, msf1, msf1_32, g1, gemm_grid(1, 1LL << 30, sms), s) !=
+        if (launch_gemm(256, EPI_SWIGLU_QUANT, 1, ma1, ma1_32, mb1, g1, gemm_grid(1, 1LL << 30, sms), s) !=
                 cudaSuccess ||
             mark(events, 3, s) != NVFP4_OK ||
-            launch_gemm(pl.l2_bn, EPI_BF16, 1, ma2, ma2_32, mb2, ma2, ma2_32, g2, gemm_grid(1, 1LL << 30, sms), s) !=
+            launch_gemm(pl.l2_bn, EPI_BF16, 1, ma2, ma2_32, mb2, g2, gemm_grid(1, 1LL << 30, sms), s) !=
                 cudaSuccess ||
             mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
@@ -874,12 +855,12 @@ int nvfp4_moe_calibrate(const nvfp4_moe_args *a, float *inter_gs_out, void *work
         st = run_front(a, ws, L, cg == 2 ? 2 : 0, nullptr, s, sms);
         if (st != NVFP4_OK)
             return st;
-        CUtensorMap ma, ma32, mb, msf, msf32;
+        CUtensorMap ma, ma32, mb;
         GemmArgs g;
-        st = l1_setup(a, ws, L, &ma, &ma32, &mb, &msf, &msf32, &g);
+        st = l1_setup(a, ws, L, &ma, &ma32, &mb, &g);
         if (st != NVFP4_OK)
             return st;
-        if (launch_gemm(256, EPI_SWIGLU_AMAX, cg, ma, ma32, mb, msf, msf32, g, gemm_grid(cg, 1LL << 30, sms), s) !=
+        if (launch_gemm(256, EPI_SWIGLU_AMAX, cg, ma, ma32, mb, g, gemm_grid(cg, 1LL << 30, sms), s) !=
             cudaSuccess)
             return NVFP4_ERR_CUDA;
     }

@@ -390,6 +390,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
     // into the 4-byte word of one 64-column group of the MMA scale layout.
     const int64_t H = a.H;
     const int nchunks = static_cast<int>((H + kQuantCols - 1) / kQuantCols);
+    const int64_t nkt = (H + 255) / 256;        // k-tiles of 256 columns per row block
     const int items = (t1 - t0) * nchunks;
     for (int it = warp; it < items; it += kFrontWarps) {
         const int t = t0 + it / nchunks;
@@ -442,8 +443,11 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
                 continue;
             *reinterpret_cast<uint4 *>(a.a_codes + static_cast<int64_t>(dst) * (H / 2) + col0 / 2) =
                 make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            if ((lane & 1) == 0)        // row-major: the warp's 64 scale bytes of this chunk are contiguous
-                *reinterpret_cast<uint32_t *>(a.a_sf + static_cast<int64_t>(dst) * a.a_sf_ld + col0 / 16) = sword;
+            // row blocks: the row's 16 scale bytes of a k-tile are contiguous, so
+            // four lane pairs write one 16-byte piece per k-tile of the chunk
+            if ((lane & 1) == 0)
+                *reinterpret_cast<uint32_t *>(a.a_sf + ((static_cast<int64_t>(dst) >> 7) * nkt + (col0 >> 8)) * 2048 +
+                                              (dst & 127) * 16 + ((col0 & 255) >> 4)) = sword;
         }
     }
 }

@@ -323,8 +323,7 @@ cudaError_t launch_wait_probe(const int32_t *flag, int target, int32_t *err, cud
 template <int BN, int EPI, int CG, int FUSED, int SK>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a32,
-                      const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_sfa,
-                      const __grid_constant__ CUtensorMap map_sfa32, const __grid_constant__ CUtensorMap map_a2,
+                      const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_a2,
                       const __grid_constant__ CUtensorMap map_a2_32, const __grid_constant__ CUtensorMap map_b2,
                       const GemmArgs p, const GemmArgs p2)
 {
@@ -385,10 +384,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&map_a);
         tma_prefetch_map(&map_a32);
         tma_prefetch_map(&map_b);
-        if (p.sfa_rowmajor) {
-            tma_prefetch_map(&map_sfa);
-            tma_prefetch_map(&map_sfa32);
-        }
         if (FUSED) {
             tma_prefetch_map(&map_a2);
             tma_prefetch_map(&map_a2_32);
@@ -485,8 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const int nkb = min(4, (q.K - kt * kBK) / 64);
                     const uint32_t sf_bytes = static_cast<uint32_t>(nkb * kSFAtom);
-                    // A scales: the k-tile's 16 scale bytes of each loaded row (row-major;
-                    // a whole box, zero-filled past the row end), else nkb atoms
+                    // A scales: row blocks hold a k-tile's scales as 16 bytes per row, so a
+                    // partial m-tile copies only its 32-row groups; MMA atoms take nkb x 512
                     const uint32_t sfa_bytes =
                         ti.valid == 0 ? 0u
                                       : (q.sfa_rowmajor ? (a_boxes == 0 ? 128u * 16u : static_cast<uint32_t>(a_boxes) * 512u)
@@ -501,17 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tma_load_2d(a_dst + i * (kTileBytes / 4), ma32, kt * kBKBytes, ti.row0 + 32 * i,
                                             &full[stage]);
                         }
-                        if (q.sfa_rowmajor) {
-                            if (a_boxes == 0) {
-                                tma_load_2d(sSFA + stage * kSFStage, &map_sfa, kt * 16, ti.row0, &full[stage]);
-                            } else {
-                                for (int i = 0; i < a_boxes; ++i)
-                                    tma_load_2d(sSFA + stage * kSFStage + i * 512, &map_sfa32, kt * 16, ti.row0 + 32 * i,
-                                                &full[stage]);
-                            }
-                        } else {
-                            bulk_load(sSFA + stage * kSFStage, sfa + kt * kSFStage, sf_bytes, &full[stage]);
-                        }
+                        bulk_load(sSFA + stage * kSFStage, sfa + kt * kSFStage, sfa_bytes, &full[stage]);
                     }
                     uint8_t *b_dst = sB + stage * C::kBBoxes * kTileBytes;
                     uint8_t *sfb_dst = sSFB + stage * kHalves * kSFStage;
@@ -661,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t t_slot = t_q + static_cast<uint32_t>(stage * C::kSFSlotCols);
                 // A: column 4*kb + m <- the 4 scales of row 32*m + lane for k-block kb:
                 // row `lane` of atom kb (MMA layout), or word kb of row 32*m + lane
-                // (row-major, 16 bytes a row)
+                // (row blocks, 16 bytes a row)
                 uint32_t r[16];
                 const uint8_t *src = sSFA + stage * kSFStage + lane * 16;
                 if (q.sfa_rowmajor) {
@@ -1015,9 +1000,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int BN, int EPI, int CG, int FUSED, int SK = 0>
 static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
-                              const CUtensorMap &map_sfa, const CUtensorMap &map_sfa32, const GemmArgs &args,
-                              const CUtensorMap &map_a2, const CUtensorMap &map_a2_32, const CUtensorMap &map_b2,
-                              const GemmArgs &args2, int grid, cudaStream_t stream)
+                              const GemmArgs &args, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
+                              const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream)
 {
     const int smem = Cfg<BN, CG>::kSmem;
     static unsigned long long attr_done = 0;     // one bit per device
@@ -1048,25 +1032,21 @@ static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a
         attr[cfg.numAttrs].val.clusterDim.z = 1;
         ++cfg.numAttrs;
     }
-    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, CG, FUSED, SK>, map_a, map_a32, map_b, map_sfa,
-                              map_sfa32, map_a2, map_a2_32, map_b2, args, args2);
+    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, CG, FUSED, SK>, map_a, map_a32, map_b, map_a2,
+                              map_a2_32, map_b2, args, args2);
 }
 
 template <int BN, int EPI, int CG>
 static cudaError_t launch_plain(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
-                                const CUtensorMap &map_sfa, const CUtensorMap &map_sfa32, const GemmArgs &args,
-                                int grid, cudaStream_t stream)
+                                const GemmArgs &args, int grid, cudaStream_t stream)
 {
-    return launch_one<BN, EPI, CG, 0>(map_a, map_a32, map_b, map_sfa, map_sfa32, args, map_a, map_a32, map_b, args,
-                                      grid, stream);
+    return launch_one<BN, EPI, CG, 0>(map_a, map_a32, map_b, args, map_a, map_a32, map_b, args, grid, stream);
 }
 
 cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
-                        const CUtensorMap &map_b, const CUtensorMap &map_sfa, const CUtensorMap &map_sfa32,
-                        const GemmArgs &args, int grid, cudaStream_t stream)
+                        const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream)
 {
-#define NVFP4_PLAIN(BN_, EPI_, CG_)                                                                              \
-    launch_plain<BN_, EPI_, CG_>(map_a, map_a32, map_b, map_sfa, map_sfa32, args, grid, stream)
+#define NVFP4_PLAIN(BN_, EPI_, CG_) launch_plain<BN_, EPI_, CG_>(map_a, map_a32, map_b, args, grid, stream)
     if (cg == 2) {
         if (bn != 256 || grid % 2 != 0)
             return cudaErrorInvalidValue;
@@ -1089,31 +1069,28 @@ cudaError_t launch_gemm_streamk(int cg, const CUtensorMap &map_a, const CUtensor
 {
     if (args.mtiles != nullptr || args.sk_partials == nullptr || args.sk_flags == nullptr)
         return cudaErrorInvalidValue;
-    // dense A: scales in the MMA layout (the row-major maps are not read)
     if (cg == 2)
         return grid % 2 != 0 ? cudaErrorInvalidValue
-                             : launch_one<256, EPI_BF16, 2, 0, 1>(map_a, map_a32, map_b, map_a, map_a32, args, map_a,
-                                                                   map_a32, map_b, args, grid, stream);
-    return launch_one<256, EPI_BF16, 1, 0, 1>(map_a, map_a32, map_b, map_a, map_a32, args, map_a, map_a32, map_b, args,
-                                              grid, stream);
+                             : launch_one<256, EPI_BF16, 2, 0, 1>(map_a, map_a32, map_b, args, map_a, map_a32, map_b,
+                                                                   args, grid, stream);
+    return launch_one<256, EPI_BF16, 1, 0, 1>(map_a, map_a32, map_b, args, map_a, map_a32, map_b, args, grid, stream);
 }
 
 cudaError_t launch_moe_fused(int cg, const CUtensorMap &map_a1, const CUtensorMap &map_a1_32,
-                             const CUtensorMap &map_b1, const CUtensorMap &map_sfa1, const CUtensorMap &map_sfa1_32,
-                             const GemmArgs &args1, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
-                             const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream)
+                             const CUtensorMap &map_b1, const GemmArgs &args1, const CUtensorMap &map_a2,
+                             const CUtensorMap &map_a2_32, const CUtensorMap &map_b2, const GemmArgs &args2, int grid,
+                             cudaStream_t stream)
 {
     if (args1.mtiles == nullptr || args1.ready == nullptr || args2.ready != args1.ready)
         return cudaErrorInvalidValue;
     if (cg == 2)
         return grid % 2 != 0 ? cudaErrorInvalidValue
-                             : launch_one<256, EPI_SWIGLU_QUANT, 2, 1>(map_a1, map_a1_32, map_b1, map_sfa1, map_sfa1_32,
-                                                                        args1, map_a2, map_a2_32, map_b2, args2, grid,
-                                                                        stream);
+                             : launch_one<256, EPI_SWIGLU_QUANT, 2, 1>(map_a1, map_a1_32, map_b1, args1, map_a2,
+                                                                        map_a2_32, map_b2, args2, grid, stream);
     if (args1.claim == nullptr)
         return cudaErrorInvalidValue;
-    return launch_one<256, EPI_SWIGLU_QUANT, 1, 1>(map_a1, map_a1_32, map_b1, map_sfa1, map_sfa1_32, args1, map_a2,
-                                                    map_a2_32, map_b2, args2, grid, stream);
+    return launch_one<256, EPI_SWIGLU_QUANT, 1, 1>(map_a1, map_a1_32, map_b1, args1, map_a2, map_a2_32, map_b2, args2,
+                                                    grid, stream);
 }
 
 // Clusters of two GEMM CTAs that can be resident at once on the current

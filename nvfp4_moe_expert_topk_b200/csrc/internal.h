@@ -46,10 +46,11 @@ struct GemmArgs {
     int64_t sfa_block_stride;
     const uint8_t *sfb;
     int64_t sfb_block_stride;
-    // sfa_rowmajor: A's scales are row-major [rows, ld] bytes instead, loaded
-    // by 2-D TMA boxes of 16 bytes (one k-tile) x 128 or 32 rows (the map_sfa
-    // / map_sfa32 kernel arguments): the permuted activations of the grouped
-    // L1, whose rows the front writes one token at a time
+    // sfa_rowmajor: A's scales in row blocks instead: for each 128-row block
+    // and k-tile, 2 KB holding 16 bytes per row (its 16 scales of the k-tile)
+    // -- same addressing as the MMA atoms, row-major inside; a partial m-tile
+    // copies only its first 32-row groups.  The permuted activations of the
+    // grouped L1 use it (the front writes them one token row at a time).
     int sfa_rowmajor;
     int K;                    // reduction length in elements, multiple of 64
     int num_k_tiles;          // ceil(K / 256)
@@ -105,11 +106,8 @@ enum Epilogue { EPI_SWIGLU_QUANT = 0, EPI_BF16 = 1, EPI_SWIGLU_AMAX = 2 };
 // map_a32: 2-D uint8 tensor maps over the A code matrix with boxes of 128 and
 // 32 rows; map_b: over the B code matrix with 128-row boxes; every box is 128
 // bytes wide with 128-byte swizzle.
-// map_sfa / map_sfa32: row-major A-scale maps (boxes of 128 and 32 rows)
-// when args.sfa_rowmajor, else ignored.
 cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
-                        const CUtensorMap &map_b, const CUtensorMap &map_sfa, const CUtensorMap &map_sfa32,
-                        const GemmArgs &args, int grid, cudaStream_t stream);
+                        const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream);
 // Dense bf16 GEMM with stream-K work split (256-wide tiles; cg 1 or 2):
 // args.sk_partials holds grid slots of 128 x 256 fp32 and args.sk_flags
 // one zeroed int per (tile, CTA of the pair).
@@ -128,9 +126,9 @@ int gemm_pair_clusters(int num_sms);
 // before it, whose CTAs are running); cg = 2: the pair list on pair tiles,
 // tiles dealt round-robin to the clusters (grid / 2 of them, all resident).
 cudaError_t launch_moe_fused(int cg, const CUtensorMap &map_a1, const CUtensorMap &map_a1_32,
-                             const CUtensorMap &map_b1, const CUtensorMap &map_sfa1, const CUtensorMap &map_sfa1_32,
-                             const GemmArgs &args1, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
-                             const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream);
+                             const CUtensorMap &map_b1, const GemmArgs &args1, const CUtensorMap &map_a2,
+                             const CUtensorMap &map_a2_32, const CUtensorMap &map_b2, const GemmArgs &args2, int grid,
+                             cudaStream_t stream);
 
 // The forward's front in one launch (front.cu): the batch's global scale of
 // x (x_gs == nullptr), routing and the tile tables, quantise + permute (x ==
@@ -158,8 +156,7 @@ struct FrontArgs {
     int32_t *claim;           // tile claim counter of the fused 1-CTA launch (zeroed here)
     int32_t *inv, *yrow;
     int32_t *err;
-    uint8_t *a_codes, *a_sf;  // a_sf row-major [rows, a_sf_ld] bytes
-    int64_t a_sf_ld;
+    uint8_t *a_codes, *a_sf;  // a_sf in row blocks: [rows/128][H/256 k-tiles][128 rows][16 bytes]
     // activations already in NVFP4 (x == nullptr, x_gs given): codes [T, H/2]
     // and row-major scales [T, H/16] that phase 3 only permutes
     const uint8_t *xq_codes, *xq_scales;

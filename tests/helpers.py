@@ -34,6 +34,17 @@ def from_mma_layout(buf: np.ndarray, rows: int, cols: int) -> np.ndarray:
     return sc
 
 
+def from_rowblock_layout(buf: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    """Scales in row blocks -> row-major [rows, cols/16]: for each 128-row
+    block and 256-column k-tile, 2 KB holding 16 bytes per row, the row's
+    scale of 16-column block j at (row % 128) * 16 + j % 16 of k-tile j // 16
+    (the layout stated for workspace region 1 in include/nvfp4moe.h)."""
+    nkt = (cols + 255) // 256
+    r = np.arange(rows)[:, None]
+    j = np.arange(cols // 16)[None, :]
+    return buf[((r // 128) * nkt + j // 16) * 2048 + (r % 128) * 16 + j % 16]
+
+
 def row_rel_l2(gpu: np.ndarray, ref: np.ndarray) -> np.ndarray:
     gpu = gpu.astype(np.float64)
     ref = ref.astype(np.float64)

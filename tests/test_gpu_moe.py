@@ -10,7 +10,8 @@ import pytest
 import torch
 
 import oracle as O
-from helpers import OracleWeights, bf16_to_np, cosine, from_mma_layout, row_max_rel, row_rel_l2
+from helpers import (OracleWeights, bf16_to_np, cosine, from_mma_layout, from_rowblock_layout, row_max_rel,
+                     row_rel_l2)
 from nvfp4_moe_expert_topk_b200 import (nvfp4_global_scale, nvfp4_moe_calibrate, nvfp4_moe_forward,
                                         nvfp4_moe_get_error, nvfp4_moe_workspace_region)
 from nvfp4_moe_expert_topk_b200 import prep
@@ -126,8 +127,8 @@ def check_intermediates(p, ws, inter):
     xc, xs = O.quantize_bf16(W.bf16_bits(p.x), p.x_gs)
     o, n = region(p, 0)
     a_codes = wsn[o:o + n].reshape(-1, H // 2)
-    o, n = region(p, 1)                             # row-major, row stride H/16 rounded up to 16 bytes
-    a_sc = wsn[o:o + n].reshape(a_codes.shape[0], -1)[:, :H // 16]
+    o, n = region(p, 1)                             # row blocks (include/nvfp4moe.h, region 1)
+    a_sc = from_rowblock_layout(wsn[o:o + n], a_codes.shape[0], H)
     tok = np.arange(T * k) // k
     np.testing.assert_array_equal(a_codes[inv[live]], xc[tok[live]])
     np.testing.assert_array_equal(a_sc[inv[live]], xs[tok[live]])
