@@ -581,3 +581,43 @@ def test_forward_on_prequantised_rows_equals_forward(name):
     torch.cuda.synchronize()
     assert nvfp4_moe_get_error(ws2) == 0
     assert torch.isfinite(out.float()).all() and torch.equal(out, ref)
+
+
+def test_cuda_graph_replay_split_plan_with_new_inputs():
+    """Pair mode 1 captured in a CUDA graph (the pair launch triggering its
+    dependent early, the 1-CTA launch claiming tiles, the counters reset by
+    the front each step): replays with new x and new routing equal eager
+    calls bit for bit, and the oracle within the bar."""
+    from nvfp4_moe_expert_topk_b200 import nvfp4_moe_plan
+    cfg = SPLIT
+    assert nvfp4_moe_plan(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I) == (True, 1)
+    p = Problem(cfg)
+    inputs = p.device_inputs()
+    inputs["x_gs"] = None                       # the batch's global scale inside the graph as well
+    ws = prep.workspace(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I, DEV)
+    out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=DEV)
+    nvfp4_moe_forward(**inputs, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            nvfp4_moe_forward(**inputs, out=out, workspace=ws, stream=s)
+    for seed in (5, 6):
+        rng = torch.Generator().manual_seed(seed)
+        x2 = torch.randn(cfg.T, cfg.H, generator=rng).to(torch.bfloat16)
+        ids2 = W.routing(cfg, cfg.T, seed=300 + seed)[0]
+        inputs["x"].copy_(x2.to(DEV))
+        inputs["topk_ids"].copy_(ids2.to(DEV))
+        g.replay()
+        torch.cuda.synchronize()
+        assert nvfp4_moe_get_error(ws) == 0
+        eager = torch.empty_like(out)
+        ws2 = prep.workspace(cfg.T, cfg.k, cfg.E, cfg.H, cfg.I, DEV)
+        nvfp4_moe_forward(**inputs, out=eager, workspace=ws2)
+        torch.cuda.synchronize()
+        assert torch.equal(eager, out)
+        xb = W.bf16_bits(x2)
+        ref = O.moe_forward(xb, ids2.numpy(), p.w.numpy(), O.global_scale_bf16(xb), **p.ow.oracle_kwargs(),
+                            inter_gs=p.inter_gs)
+        check_output(out, ref)
