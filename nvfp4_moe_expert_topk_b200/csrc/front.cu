@@ -367,9 +367,13 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
                     const int r = pre_s[e] + wcnt[warp * E + e] + rank;
                     a.inv[f] = poff_s[e] + r;
                     a.yrow[f] = off_s[e] + r;
+                    if (ids_cached)             // the slot's id is read: keep its padded row there
+                        ids_s[f - f0] = poff_s[e] + r;
                 } else if (act) {
                     a.inv[f] = -1;
                     a.yrow[f] = -1;
+                    if (ids_cached)
+                        ids_s[f - f0] = -1;
                 }
                 __syncwarp();
                 if (valid && rank == 0)
@@ -399,7 +403,8 @@ __global__ void __launch_bounds__(kFrontThreads, 1) front_kernel(const FrontArgs
         const bool active = col0 < H;
         int my_dst = -1;                          // lane j < k: destination row of slot j
         if (lane < k)
-            my_dst = __ldcg(a.inv + static_cast<int64_t>(t) * k + lane);
+            my_dst = ids_cached ? ids_s[static_cast<int64_t>(t) * k + lane - f0]
+                                : __ldcg(a.inv + static_cast<int64_t>(t) * k + lane);
         uint32_t cw[4] = {0u, 0u, 0u, 0u};
         uint32_t s2 = 0;
         if (pre_quantised) {
