@@ -49,7 +49,8 @@ BF16_TO_FP4_NOMINAL_RATIO = 4.0        # 9 / 2.25 PFLOP/s dense
 STAGES = ["global_scale", "route", "quantize_permute", "l1_gate_up_swiglu_quant", "l2_down", "combine"]
 FRONT_STAGE = "front"                  # global scale of the batch + routing + quantise/permute
 FUSED_STAGE = "l1_l2_fused"            # L1 and L2 as one launch (nvfp4_moe_plan)
-SPLIT_STAGE = "l1_l2_pairs_then_light"     # pair mode 1: the fused pair launch, then the fused 1-CTA one
+PAIRS_STAGE = "l1_l2_fused_pairs"      # pair mode 1: the heavy experts' fused pair-tile launch
+LIGHT_STAGE = "l1_l2_fused_light"      # pair mode 1: the fused 1-CTA launch over the other m-tiles
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 GEMM_SOURCES = ["gemm.cu", "ptx.cuh", "quant.cuh", "internal.h"]
 
@@ -330,15 +331,18 @@ def fold_stages(per_stage, fused, pair_mode):
     quantise + permute) and then
       pair mode 0, fused   the fused 1-CTA L1 + L2 launch;
       pair mode 1          the heavy experts' fused pair launch, then the
-                           fused 1-CTA launch over the other m-tiles, whose
-                           CTAs take over the SMs as the pair CTAs finish
-                           (one stage: no event between them);
+                           fused 1-CTA launch over the other m-tiles (the
+                           staged run records an event between them, so each
+                           has its own stage; in the headline run, without
+                           events, the 1-CTA CTAs take over SMs as pair CTAs
+                           finish);
       otherwise            L1, then L2;
     and the combine."""
     d = dict(per_stage)
     d[FRONT_STAGE] = d.pop("global_scale") + d.pop("route") + d.pop("quantize_permute")
     if pair_mode == 1:
-        d[SPLIT_STAGE] = d.pop("l1_gate_up_swiglu_quant") + d.pop("l2_down")
+        d[PAIRS_STAGE] = d.pop("l1_gate_up_swiglu_quant")
+        d[LIGHT_STAGE] = d.pop("l2_down")
     elif fused and pair_mode == 0:
         d[FUSED_STAGE] = d.pop("l1_gate_up_swiglu_quant") + d.pop("l2_down")
     return d
@@ -375,8 +379,10 @@ def stage_bytes(cfg, counts, fused, pair_mode):
 
     d = {FRONT_STAGE: T * H * 2.0 + R * H * FP4_BYTES + T * k * 4.0 * 3 + E * 16.0,
          "combine": R * H * 2.0 + T * H * 2.0 + T * k * 12.0}
-    if pair_mode == 1:
-        d[SPLIT_STAGE] = sum(gemm(counts))     # the two launches together read each expert once
+    pair_rows, light_rows = tile_split(counts, pair_mode)
+    if pair_mode == 1:                          # each launch reads the experts it touches once
+        d[PAIRS_STAGE] = sum(gemm(pair_rows))
+        d[LIGHT_STAGE] = sum(gemm(light_rows))
     else:
         l1, l2 = gemm(counts)
         if fused and pair_mode == 0:

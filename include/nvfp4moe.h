@@ -162,8 +162,11 @@ typedef struct {
  * "Phase 1": a cudagraph-safe runner works on pre-allocated buffers, so the
  * caller allocates this once and every call reuses it).  The workspace is
  * caller-owned device memory; zero it once after allocation (it holds the
- * sticky device error word).  Host only; 0 for a shape outside the
- * constraints of nvfp4_moe_forward. */
+ * sticky device error word and the front launch's grid ticket, which every
+ * call leaves at a multiple of 1024; a workspace that was not zeroed makes
+ * the first call report NVFP4_ERR_TIMEOUT after 2 s and resets the ticket).
+ * Calls sharing a workspace must not overlap on the device.  Host only; 0
+ * for a shape outside the constraints of nvfp4_moe_forward. */
 size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
 
 /* out = sum_j topk_weights[t,j] * Expert_{ids[t,j]}(x[t]) with
@@ -287,8 +290,10 @@ int nvfp4_debug_bounded_wait(const int32_t *flag, int32_t target, int32_t *err, 
  * launch (the L2 tiles of an m-tile start as soon as that m-tile's L1 tiles
  * have written h).  Stages between the events of nvfp4_moe_forward_timed:
  * 0-1 the front launch (1-2 empty); then pair mode 0 fused: 2-3 the fused
- * launch (3-4 empty); pair mode 1: 2-3 the pair L1 and L2 launches, 3-4 the
- * fused 1-CTA launch; otherwise 2-3 L1, 3-4 L2; 4-5 the combine.  Both
+ * launch (3-4 empty); pair mode 1: 2-3 the fused pair launch, 3-4 the fused
+ * 1-CTA launch (with the event between them the 1-CTA launch starts only
+ * when the pair launch has ended; without events its CTAs take over SMs as
+ * pair CTAs finish); otherwise 2-3 L1, 3-4 L2; 4-5 the combine.  Both
  * outputs are host ints. */
 int nvfp4_moe_plan(int64_t T, int k, int E, int64_t H, int64_t I, int32_t *fused_l1_l2, int32_t *pair_tiles);
 

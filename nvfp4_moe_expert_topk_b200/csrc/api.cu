@@ -745,10 +745,12 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
         const int pairs = gemm_pair_clusters(sms);
         GemmArgs l1 = g1;
         l1.pdl_wait_at_end = 1;
-        if (launch_moe_fused(2, ma1, ma1_32, mb1, p1, ma2, ma2_32, mb2, g2, 2 * pairs, s) !=
-                cudaSuccess ||
+        // (timed: an event between the two launches separates their stages;
+        // the 1-CTA launch then starts after the pair launch has ended)
+        if (launch_moe_fused(2, ma1, ma1_32, mb1, p1, ma2, ma2_32, mb2, g2, 2 * pairs, s) != cudaSuccess ||
+            mark(events, 3, s) != NVFP4_OK ||
             launch_moe_fused(1, ma1, ma1_32, mb1, l1, ma2, ma2_32, mb2, g2, sms, s) != cudaSuccess ||
-            mark(events, 3, s) != NVFP4_OK || mark(events, 4, s) != NVFP4_OK)
+            mark(events, 4, s) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
     } else if (pl.pair_mode == 2) {
         // every m-tile on pair tiles: L1 launch, then L2 launch

@@ -38,13 +38,14 @@ def test_fold_two_launch_plan():
 
 
 def test_fold_split_plan_and_its_bytes():
-    """Pair mode 1: the fused pair launch and the fused 1-CTA launch form one
-    stage; its algorithmic bytes read each expert once.  The tile split
-    follows the plan's rule."""
+    """Pair mode 1: the fused pair launch and the fused 1-CTA launch are two
+    stages; each stage's algorithmic bytes read the experts it touches once
+    (an expert with an odd number of m-tiles is read by both).  The tile
+    split follows the plan's rule."""
     import numpy as np
     d = bench.Workload.fold(_Plan(True, 1), STAGE_MS)
-    assert set(d) == {bench.FRONT_STAGE, bench.SPLIT_STAGE, "combine"}
-    assert d[bench.SPLIT_STAGE] == pytest.approx(3.0)
+    assert set(d) == {bench.FRONT_STAGE, bench.PAIRS_STAGE, bench.LIGHT_STAGE, "combine"}
+    assert d[bench.PAIRS_STAGE] == 2.0 and d[bench.LIGHT_STAGE] == 1.0
     cfg = W.MoeConfig("t", E=4, k=2, T=400, H=256, I=128, routing="softmax", outliers=False, warmup_T=8)
     counts = np.array([300, 256, 44, 200])          # m-tiles 3, 2, 1, 2
     pair_rows, light_rows = bench.tile_split(counts, 1)
@@ -53,7 +54,9 @@ def test_fold_split_plan_and_its_bytes():
     assert list(bench.tile_split(counts, 0)[1]) == [300, 256, 44, 200]
     split = bench.stage_bytes(cfg, counts, True, 1)
     whole = bench.stage_bytes(cfg, counts, True, 0)
-    assert split[bench.SPLIT_STAGE] == pytest.approx(whole[bench.FUSED_STAGE])
+    w_expert = 3 * cfg.H * cfg.I * bench.FP4_BYTES
+    # the pairs and the light launch read expert 0's weights each; the rest once
+    assert split[bench.PAIRS_STAGE] + split[bench.LIGHT_STAGE] == pytest.approx(whole[bench.FUSED_STAGE] + w_expert)
     assert bench.launches_per_step(True, 0) == 3 and bench.launches_per_step(True, 1) == 4
     assert bench.launches_per_step(False, 2) == 4 and bench.launches_per_step(False, 0) == 4
 
