@@ -161,12 +161,13 @@ typedef struct {
 /* Workspace bytes nvfp4_moe_forward / nvfp4_moe_calibrate need (page 1
  * "Phase 1": a cudagraph-safe runner works on pre-allocated buffers, so the
  * caller allocates this once and every call reuses it).  The workspace is
- * caller-owned device memory; zero it once after allocation (it holds the
+ * caller-owned device memory; zero it once after allocation.  It holds the
  * sticky device error word and the front launch's grid ticket, which every
- * call leaves at a multiple of 1024; a workspace that was not zeroed makes
- * the first call report NVFP4_ERR_TIMEOUT after 2 s and resets the ticket).
- * Calls sharing a workspace must not overlap on the device.  Host only; 0
- * for a shape outside the constraints of nvfp4_moe_forward. */
+ * call leaves at a multiple of 1024 and which the launch's grid barrier
+ * relies on: in a workspace that was not zeroed the barrier may release
+ * blocks early (wrong routing) or time out (NVFP4_ERR_TIMEOUT).  Calls
+ * sharing a workspace must not overlap on the device.  Host only; 0 for a
+ * shape outside the constraints of nvfp4_moe_forward. */
 size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I);
 
 /* out = sum_j topk_weights[t,j] * Expert_{ids[t,j]}(x[t]) with

@@ -17,8 +17,9 @@
 //            amax and its per-expert counts, then arrives on a grid ticket;
 //   barrier  one arrival per block on a 32-bit ticket: every launch adds
 //            exactly 1024 in total (block 0 adds 1025 - G, the others 1), so
-//            the ticket is a multiple of 1024 between launches and a block
-//            waits until it reaches the next multiple -- nothing to reset;
+//            the ticket (zero in a fresh workspace) is a multiple of 1024
+//            between launches and a block waits until it reaches the next
+//            multiple -- nothing to reset between launches;
 //   phase 2  every block reads all blocks' counts (L2), forms per expert the
 //            total and the count of earlier blocks, scans the experts (row
 //            offsets, 128-row padded offsets, tile tables; block 0 writes the
