@@ -39,7 +39,7 @@
 // 16-element block of h is produced and quantised by one thread.
 //
 // The tile list is either dense (m-tiles of M, n-major) or grouped: an
-// m-tile table written on the device by the routing kernel (expert, first
+// m-tile table written on the device by the front launch (expert, first
 // padded row, valid rows, first output row), so the launch needs no host
 // sync and every expert's rows are covered by one tensor map over the padded
 // A buffer and one over all experts' stacked weights.  Two variants of the
@@ -312,14 +312,17 @@ cudaError_t launch_wait_probe(const int32_t *flag, int target, int32_t *err, cud
     return cudaGetLastError();
 }
 
-// FUSED = 1 (grouped, CG = 1, BN = 256): one persistent launch runs the L1
-// tiles (arguments p, maps map_a / map_a32 / map_b, SwiGLU + re-quantisation
+// FUSED = 1 (grouped, BN = 256): one persistent launch runs the L1 tiles
+// (arguments p, maps map_a / map_a32 / map_b, SwiGLU + re-quantisation
 // epilogue) and then the L2 tiles (p2, map_a2 / map_a2_32 / map_b2, bf16
 // epilogue).  Each L1 epilogue warp publishes its h rows by bumping the
 // m-tile's counter; the producer starts an L2 tile once all L1 tiles of its
-// m-tile have been published (a bounded wait).  Tiles are taken in order, so
-// every L1 tile a wait depends on belongs to a CTA that reaches it without
-// waiting itself; the launch is cooperative, so all CTAs are resident.
+// m-tile have been published (a bounded wait).  CG = 1 claims tiles one at a
+// time from a counter, so every tile a wait depends on was claimed earlier
+// by a running CTA that reaches it without waiting (no residency
+// requirement); CG = 2 deals tiles round-robin over clusters that are all
+// resident (the launch follows the front on an idle GPU, one cluster per SM
+// pair).
 template <int BN, int EPI, int CG, int FUSED, int SK>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a32,
