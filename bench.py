@@ -998,7 +998,21 @@ def _run_all(args, world, rank, dev, peaks, peak_src, steps, warmup):
 def run_single(name, world, rank, dev, peaks, peak_src, steps, warmup):
     """One MoE workload alone (small cases for profiling: decode, prefill_ep48);
     for decode_shared / prefill_shared, the shared expert folded in against
-    run as a second chain."""
+    run as a second chain; mla: the three dense MLA projection GEMMs alone
+    (per GEMM: `warmup` eager calls, then 2 x `steps` hot and 2 x `steps`
+    L2-cold calls from CUDA graphs)."""
+    if name == "mla":
+        res = time_mla_gemms(dev, steps, warmup, peaks, L2Flush(dev))
+        flops = sum(2.0 * v["M"] * v["N"] * v["K"] for v in res.values())
+        ms = sum(v["gemm_ms"] for v in res.values())
+        line = {"metric": "mla_gemm_TFLOP_per_s", "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+                "config": {"workload": "mla_projection_gemms_M2048", "l2": "hot; cold figures after a 512 MB flush"},
+                "mla_gemms": res, "clocks": CLOCKS.summary([f"mla_{k}" for k in res])}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return
     if name.endswith("_shared"):
         routed = Workload(W.MOE_CONFIGS[name[:-len("_shared")]], dev)
         res = time_shared_fold(routed, W.MOE_CONFIGS[name], dev, steps, warmup, peaks["hbm_gbs"])
@@ -1081,7 +1095,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA-graph replay")
     ap.add_argument("--only", choices=["all", "decode", "prefill", "prefill_ep48", "prefill_front", "shared", "tiny",
-                                       "decode_shared", "prefill_shared"], default="all",
+                                       "decode_shared", "prefill_shared", "mla"], default="all",
                     help="one workload alone (small profiling cases)")
     args = ap.parse_args()
     if args.impl == "reference":

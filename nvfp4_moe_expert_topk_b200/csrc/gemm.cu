@@ -185,6 +185,12 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, const GemmArg
     return ti;
 }
 
+// v[i] for a run-time i < 4 without indexing a register array
+__device__ __forceinline__ float pick4(const float (&v)[4], int i)
+{
+    return i == 0 ? v[0] : (i == 1 ? v[1] : (i == 2 ? v[2] : v[3]));
+}
+
 __device__ __forceinline__ void record_error(int32_t *err, int code)
 {
     if (err != nullptr)
@@ -726,6 +732,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
                 break;
             }
+            // the tile's coordinates and global scales are read while its MMAs
+            // run, so that the drain (which holds the accumulator) waits on no load:
+            // dequantisation factors 1 / (a_gs * b_gs) per B segment (SwiGLU
+            // tiles: gate, up) and the global scale of h
+            const TileInfo ti = decode_tile<CG, FUSED>(p, p2, t, m_units, rank);
+            const GemmArgs &ga = (FUSED && ti.ph) ? p2 : p;
+            const bool valid = row < ti.valid;
+            const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc * BN);
+            const bool swiglu_tile = FUSED ? ti.ph == 0 : EPI != EPI_BF16;
+            float alpha_seg[4];
+            {
+                const float a = __ldcg(ga.a_gs + (ga.a_gs_per_expert ? ti.e : 0));
+                const int n_seg = swiglu_tile ? 2 : ga.nseg;
+                float b[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    b[i] = i < n_seg ? __ldcg(ga.b_gs + ti.e * ga.b_gs_stride + i) : 1.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    alpha_seg[i] = __fdiv_rn(1.0f, __fmul_rn(a, b[i]));
+            }
+            const float h_gs = (EPI == EPI_SWIGLU_QUANT && swiglu_tile) ? __ldcg(ga.inter_gs + ti.e) : 0.0f;
             const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, got)) {
                 *abort_flag = 1;
@@ -733,18 +761,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const TileInfo ti = decode_tile<CG, FUSED>(p, p2, t, m_units, rank);
-            const GemmArgs &ga = (FUSED && ti.ph) ? p2 : p;
-            const bool valid = row < ti.valid;
-            const uint32_t t_acc = t_lane + static_cast<uint32_t>(acc * BN);
-            const bool swiglu_tile = FUSED ? ti.ph == 0 : EPI != EPI_BF16;
 
             if (swiglu_tile && BN == 256) {
                 // drain gate columns [64hf, 64hf+64) and the matching up columns in two rounds of
                 // 32 (one wait each), computing h as it arrives, then release the accumulator
-                const float a = __ldcg(ga.a_gs);
-                const float alpha_g = __fdiv_rn(1.0f, __fmul_rn(a, __ldcg(ga.b_gs + ti.e * ga.b_gs_stride + 0)));
-                const float alpha_u = __fdiv_rn(1.0f, __fmul_rn(a, __ldcg(ga.b_gs + ti.e * ga.b_gs_stride + 1)));
+                const float alpha_g = alpha_seg[0], alpha_u = alpha_seg[1];
                 float h[64];
 #pragma unroll
                 for (int r = 0; r < 2; ++r) {
@@ -781,7 +802,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0)
                         atomicMax(ga.amax_bits + ti.e, __float_as_uint(amax));
                 } else {
-                    const float hgs = __ldcg(ga.inter_gs + ti.e);
+                    const float hgs = h_gs;
                     uint32_t codes[8];
                     uint32_t sfw = 0;
 #pragma unroll
@@ -879,7 +900,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 *abort_flag = 1;
                                 record_error(p.err, NVFP4_ERR_TIMEOUT);
                             } else {
-                                const float a = ga.a_gs[0];
                                 uint4 *dst = reinterpret_cast<uint4 *>(
                                     ga.out + static_cast<int64_t>(ti.row0_out + row) * ga.ldo +
                                     static_cast<int64_t>(ti.nt) * BN + hf * kCols);
@@ -910,7 +930,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     for (int i = 0; i < 3; ++i)
                                         if (i < ga.nseg - 1 && col >= ga.seg_end[i])
                                             seg = i + 1;
-                                    const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, ga.b_gs[seg]));
+                                    const float alpha = pick4(alpha_seg, seg);
                                     uint32_t o[8];
 #pragma unroll
                                     for (int i = 0; i < 8; ++i)
@@ -935,7 +955,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!sk_segment) {
                 // drain columns [hf*BN/2, (hf+1)*BN/2) in rounds of 64 (one wait each),
                 // converting to bf16 as they arrive, then release the accumulator
-                const float a = __ldcg(ga.a_gs + (ga.a_gs_per_expert ? ti.e : 0));
                 uint32_t o[kCols / 2];
 #pragma unroll
                 for (int r = 0; r < kCols / kRound; ++r) {
@@ -953,7 +972,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 3; ++i)
                             if (i < ga.nseg - 1 && col >= ga.seg_end[i])
                                 seg = i + 1;
-                        const float alpha = __fdiv_rn(1.0f, __fmul_rn(a, __ldcg(ga.b_gs + ti.e * ga.b_gs_stride + seg)));
+                        const float alpha = pick4(alpha_seg, seg);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             o[(r * kRound + c * 16) / 2 + i] = pack_bf16x2(__uint_as_float(v[16 * c + 2 * i]) * alpha,
