@@ -71,6 +71,20 @@ int make_code_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// bf16 output [rows, ldo] for the staged epilogue stores: 32 x 32 boxes,
+// 64-byte swizzle (a box row is 64 bytes).
+int make_out_map(CUtensorMap *map, void *base, int64_t rows, int64_t cols, int64_t ldo)
+{
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldo * 2)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 bool aligned16(const void *p)
 {
     return (reinterpret_cast<uintptr_t>(p) & 15) == 0;
@@ -630,6 +644,15 @@ int gemm_impl(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs
         return cuda_status(launch_gemm_streamk(d.cg, ma, ma32, mb, g, d.grid, s));
     }
     const int grid = gemm_grid(d.cg, d.tiles, sms);
+    if (d.cg == 2) {
+        // pair tiles write out through shared memory and TMA stores (rows >= M are not written)
+        CUtensorMap mo;
+        st = make_out_map(&mo, out, M, N, ldo);
+        if (st != NVFP4_OK)
+            return st;
+        g.out_tma = 1;
+        return cuda_status(launch_gemm(d.bn, EPI_BF16, d.cg, ma, ma32, mb, g, grid, s, &mo));
+    }
     return cuda_status(launch_gemm(d.bn, EPI_BF16, d.cg, ma, ma32, mb, g, grid, s));
 }
 

@@ -87,13 +87,19 @@ struct Cfg {
     static constexpr int kB = kA + kStages * kTileBytes;
     static constexpr int kSFA = kB + kStages * kTileBytes * kBBoxes;
     static constexpr int kSFB = kSFA + kStages * kSFStage;
-    static constexpr int kBars = kSFB + kStages * kSFStage * kHalves;
+    // pair tiles with a bf16 epilogue may store through shared memory: per
+    // epilogue warp two buffers of 32 rows x 32 bf16 columns
+    static constexpr bool kOutStage = CG == 2;
+    static constexpr int kOutBuf = 32 * 32 * 2;
+    static constexpr int kOut = kSFB + kStages * kSFStage * kHalves;
+    static constexpr int kBars = kOut + (kOutStage ? kEpiWarps * 2 * kOutBuf : 0);
     static constexpr int kBarCount = 3 * kStages + 2 * kNumAcc + 1 + 2 * kTileQ;
     static constexpr int kMisc = kBars + kBarCount * 8;
     static constexpr int kSmem = kMisc + 16 + 4 * kTileQ + 1024;   // + tmem slot, abort flag, tile queue, slack
     static_assert(kTmemSF + kStages * kSFSlotCols <= kTmemCols, "TMEM budget");
     static_assert(kSmem <= 232448, "shared memory budget");
     static_assert(CG == 1 || BN == 256, "pair tiles are 256 wide");
+    static_assert(kOut % 1024 == 0, "staging buffers on the 64-byte swizzle's 512-byte period");
 };
 
 struct TileInfo {
@@ -334,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a32,
                       const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_a2,
                       const __grid_constant__ CUtensorMap map_a2_32, const __grid_constant__ CUtensorMap map_b2,
-                      const GemmArgs p, const GemmArgs p2)
+                      const __grid_constant__ CUtensorMap map_out, const GemmArgs p, const GemmArgs p2)
 {
     using C = Cfg<BN, CG>;
     static_assert(!FUSED || (BN == 256 && EPI == EPI_SWIGLU_QUANT), "fused launch: L1 quant + L2 bf16");
@@ -353,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sB = smem + C::kB;
     uint8_t *sSFA = smem + C::kSFA;
     uint8_t *sSFB = smem + C::kSFB;
+    uint8_t *sOut = smem + C::kOut;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBars);
     uint64_t *empty = full + kStages;
     uint64_t *sf_ready = empty + kStages;
@@ -398,6 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_map(&map_a2_32);
             tma_prefetch_map(&map_b2);
         }
+        if (C::kOutStage && p.out_tma)
+            tma_prefetch_map(&map_out);
     }
     if (warp == 1) {
         if constexpr (kPair) {
@@ -987,7 +996,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                     else
                         mbar_arrive(&acc_empty[acc]);
                 }
-                if (valid) {
+                bool staged = false;
+                if constexpr (C::kOutStage && kCols == 128) {
+                    if (ga.out_tma) {
+                        // four boxes of 32 rows x 32 columns through this warp's two
+                        // buffers, written out by TMA stores (whole 64-byte row pieces
+                        // instead of one 16-byte piece per row per store instruction);
+                        // a row's 16-byte chunk c sits at c ^ ((row >> 1) & 3), the
+                        // 64-byte swizzle of the map, so no two lanes of a quarter-warp
+                        // share a bank
+                        staged = true;
+                        if (q * 32 < ti.valid) {    // a box starts on a row the GEMM writes; rows past M are clipped
+                            uint8_t *wbuf = sOut + (warp - 2) * 2 * C::kOutBuf;
+#pragma unroll
+                            for (int b = 0; b < 4; ++b) {
+                                uint8_t *buf = wbuf + (b & 1) * C::kOutBuf;
+                                if (lane == 0)
+                                    bulk_wait_group_read<1>();   // the store that last read this buffer is done
+                                __syncwarp();
+#pragma unroll
+                                for (int c = 0; c < 4; ++c)
+                                    *reinterpret_cast<uint4 *>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                                        make_uint4(o[16 * b + 4 * c], o[16 * b + 4 * c + 1], o[16 * b + 4 * c + 2],
+                                                   o[16 * b + 4 * c + 3]);
+                                fence_proxy_async_smem();
+                                __syncwarp();
+                                if (lane == 0) {
+                                    tma_store_2d(&map_out, ti.nt * BN + hf * kCols + b * 32, ti.row0_out + q * 32, buf);
+                                    bulk_commit_group();
+                                }
+                            }
+                        }
+                    }
+                }
+                if (!staged && valid) {
                     uint4 *dst = reinterpret_cast<uint4 *>(ga.out + static_cast<int64_t>(ti.row0_out + row) * ga.ldo +
                                                            static_cast<int64_t>(ti.nt) * BN + hf * kCols);
 #pragma unroll
@@ -1003,6 +1045,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    if (C::kOutStage && warp >= 2 && warp < 2 + kEpiWarps) {
+        if (lane == 0)
+            bulk_wait_group_all();  // this warp's output stores have completed and read their buffers
+        __syncwarp();
+    }
     if (p.pdl_wait_at_end)
         pdl_wait();                 // the kernel this one overlapped has finished: the next sees both
     pdl_trigger();                  // the next kernel may start launching during the teardown
@@ -1023,8 +1070,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int EPI, int CG, int FUSED, int SK = 0>
 static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
                               const GemmArgs &args, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
-                              const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream)
+                              const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream,
+                              const CUtensorMap *map_out = nullptr)
 {
+    if (args.out_tma && (map_out == nullptr || CG != 2 || EPI != EPI_BF16 || FUSED || SK))
+        return cudaErrorInvalidValue;
     const int smem = Cfg<BN, CG>::kSmem;
     static unsigned long long attr_done = 0;     // one bit per device
     const cudaError_t e =
@@ -1054,21 +1104,24 @@ static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a
         attr[cfg.numAttrs].val.clusterDim.z = 1;
         ++cfg.numAttrs;
     }
+    // without staged stores the output map is never read: any valid map fills the slot
     return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, CG, FUSED, SK>, map_a, map_a32, map_b, map_a2,
-                              map_a2_32, map_b2, args, args2);
+                              map_a2_32, map_b2, map_out != nullptr ? *map_out : map_a, args, args2);
 }
 
 template <int BN, int EPI, int CG>
 static cudaError_t launch_plain(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
-                                const GemmArgs &args, int grid, cudaStream_t stream)
+                                const GemmArgs &args, int grid, cudaStream_t stream, const CUtensorMap *map_out)
 {
-    return launch_one<BN, EPI, CG, 0>(map_a, map_a32, map_b, args, map_a, map_a32, map_b, args, grid, stream);
+    return launch_one<BN, EPI, CG, 0>(map_a, map_a32, map_b, args, map_a, map_a32, map_b, args, grid, stream,
+                                      map_out);
 }
 
 cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
-                        const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream)
+                        const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream,
+                        const CUtensorMap *map_out)
 {
-#define NVFP4_PLAIN(BN_, EPI_, CG_) launch_plain<BN_, EPI_, CG_>(map_a, map_a32, map_b, args, grid, stream)
+#define NVFP4_PLAIN(BN_, EPI_, CG_) launch_plain<BN_, EPI_, CG_>(map_a, map_a32, map_b, args, grid, stream, map_out)
     if (cg == 2) {
         if (bn != 256 || grid % 2 != 0)
             return cudaErrorInvalidValue;

@@ -87,6 +87,7 @@ struct GemmArgs {
     // bf16 epilogue
     __nv_bfloat16 *out;
     int64_t ldo;
+    int out_tma;              // pair tiles: store through shared memory with the output tensor map
     int32_t *err;             // device error word
     // fused grouped launches: the 1-CTA launch claims its tiles one at a time
     // from this counter (zeroed by the front launch); in pair mode 1 the pair
@@ -105,9 +106,12 @@ enum Epilogue { EPI_SWIGLU_QUANT = 0, EPI_BF16 = 1, EPI_SWIGLU_AMAX = 2 };
 // computing 256 x 256 tiles with pair MMAs (bn 256, grid even).  map_a /
 // map_a32: 2-D uint8 tensor maps over the A code matrix with boxes of 128 and
 // 32 rows; map_b: over the B code matrix with 128-row boxes; every box is 128
-// bytes wide with 128-byte swizzle.
+// bytes wide with 128-byte swizzle.  map_out (with args.out_tma = 1, bf16
+// pair tiles only): 2-D bf16 tensor map over out ([rows, ldo], the rows the
+// GEMM may write) with 32 x 32 boxes and 64-byte swizzle.
 cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
-                        const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream);
+                        const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream,
+                        const CUtensorMap *map_out = nullptr);
 // Dense bf16 GEMM with stream-K work split (256-wide tiles; cg 1 or 2):
 // args.sk_partials holds grid slots of 128 x 256 fp32 and args.sk_flags
 // one zeroed int per (tile, CTA of the pair).

@@ -193,3 +193,33 @@ def test_gemm_streamk_matches_oracle(M, N, K, segs):
     ref = O.gemm(ac[rows], asc[rows], a_gs, bc, bsc, bgs, segs)
     err = row_rel_l2(got[rows], ref)
     assert err.max() <= 5e-3, err.max()
+
+
+@pytest.mark.parametrize("M,N,K,segs", [
+    (257, 512, 256, [512]),      # pair tiles (staged stores): ragged last pair, 1 row in its odd half
+    (100, 384, 256, [384]),      # one-CTA tiles (direct stores)
+])
+def test_gemm_strided_output_leaves_the_rest(M, N, K, segs):
+    """The C ABI's ldo > N: out is a window [M, N] of a wider buffer.  The
+    window equals the contiguous call's result bit for bit; the columns past
+    N and the row past M keep their sentinel."""
+    import ctypes
+    from nvfp4_moe_expert_topk_b200 import lib
+    ac, asc, a_gs, bc, bsc, bgs = quantized_operands(M, N, K, M * 3 + N, segs)
+    d = [torch.from_numpy(ac).to(DEV), torch.from_numpy(to_mma_layout(asc)).to(DEV),
+         torch.tensor([a_gs], dtype=torch.float32, device=DEV), torch.from_numpy(bc).to(DEV),
+         torch.from_numpy(to_mma_layout(bsc)).to(DEV), torch.tensor(np.asarray(bgs, np.float32), device=DEV)]
+    plain = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    nvfp4_gemm(*d, segs, plain)
+    ldo = N + 72
+    buf = torch.full((M + 1, ldo), 7.0, dtype=torch.bfloat16, device=DEV)
+    seg = (ctypes.c_int64 * len(segs))(*segs)
+    st = lib().nvfp4_gemm(*[ctypes.c_void_p(t.data_ptr()) for t in d[:3]], M,
+                          *[ctypes.c_void_p(t.data_ptr()) for t in d[3:]], ctypes.cast(seg, ctypes.c_void_p), len(segs),
+                          N, K, ctypes.c_void_p(buf.data_ptr()), ldo,
+                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert st == 0
+    assert torch.equal(buf[:M, :N], plain)
+    assert bool((buf[:M, N:] == 7.0).all())
+    assert bool((buf[M] == 7.0).all())
