@@ -581,6 +581,33 @@ def graph_time(fns, reps, warmup, flush=None, region=None):
     return out
 
 
+def graph_time_seq(fn, reps, region=None):
+    """Mean milliseconds of one call of fn over `reps` calls issued back to
+    back in one CUDA graph (one event pair around the replay)."""
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for _ in range(reps):
+                fn()
+    stream.wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with clock_region(region) if region else contextlib.nullcontext():
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+    del g
+    return a.elapsed_time(b) / reps
+
+
 class L2Flush:
     """A 512 MB device buffer; calling the object overwrites it (4x the 126 MB L2)."""
 
@@ -713,11 +740,13 @@ def fp4_ceiling(dev, sms):
 def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
     """The MLA projections as separate dense NVFP4 GEMMs at M=2048 (weights
     quantised once; per step: activation global scale + quantisation + GEMM).
-    Device times from CUDA events inside a CUDA graph; the GEMM alone is
-    bracketed separately, hot (operands as the quantiser left them, weights
-    L2-resident where they fit) and cold (after a 512 MB L2 flush)."""
-    from nvfp4_moe_expert_topk_b200 import (NVFP4_SCALES_MMA, nvfp4_gemm_workspace_size, nvfp4_gemm_ws,
-                                            nvfp4_quantize, nvfp4_scales_bytes)
+    Device times from CUDA events around CUDA-graph replays.  gemm_ms: the
+    mean of `steps` GEMM calls issued back to back (hot: operands as the
+    quantiser left them, weights L2-resident where they fit; each call's
+    prologue overlaps the previous call's tail, as it overlaps the quantiser's
+    in a step); gemm_ms_isolated: one call between two event records, so
+    with no overlap; gemm_ms_cold: the same after a 512 MB L2 flush."""
+    from nvfp4_moe_expert_topk_b200 import NVFP4_SCALES_MMA, nvfp4_gemm, nvfp4_quantize, nvfp4_scales_bytes
     res = {}
     fp4_peak = peaks["bf16_tflops_sustained"] * BF16_TO_FP4_NOMINAL_RATIO
     ridge = fp4_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -746,13 +775,11 @@ def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
             nvfp4_global_scale(ad, a_gs)
             nvfp4_quantize(ad, a_gs, a_codes, a_sc, NVFP4_SCALES_MMA)
 
-        nbytes = nvfp4_gemm_workspace_size(M, N, K)     # > 0: stream-K split over the SMs
-        gws = torch.zeros(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
-
         def gemm():
-            nvfp4_gemm_ws(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out, gws)
+            nvfp4_gemm(a_codes, a_sc, a_gs, w_codes, w_sc, w_gs, segs, out)
 
-        quant_ms, gemm_ms = graph_time([quant, gemm], steps, warmup, region=f"mla_{name}")
+        quant_ms, gemm_iso_ms = graph_time([quant, gemm], steps, warmup, region=f"mla_{name}_isolated")
+        gemm_ms = graph_time_seq(gemm, steps, region=f"mla_{name}")
         _, gemm_cold_ms = graph_time([quant, gemm], steps, 0, flush, region=f"mla_{name}_cold")
         step_ms = quant_ms + gemm_ms
         flops = 2.0 * M * N * K
@@ -761,8 +788,8 @@ def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
         tflops = flops / (gemm_ms * 1e-3) / 1e12
         gbs = gbytes / (gemm_ms * 1e-3) / 1e9
         bound = "tensor" if ai >= ridge else "hbm"
-        res[name] = {"M": M, "N": N, "K": K, "stream_k": bool(nbytes), "ms_per_step": step_ms, "gemm_ms": gemm_ms,
-                     "tflops": tflops,
+        res[name] = {"M": M, "N": N, "K": K, "ms_per_step": step_ms, "gemm_ms": gemm_ms,
+                     "tflops": tflops, "gemm_ms_isolated": gemm_iso_ms,
                      "gemm_ms_cold": gemm_cold_ms, "tflops_cold": flops / (gemm_cold_ms * 1e-3) / 1e12,
                      "gbs": gbs, "arith_intensity": ai, "bound": bound,
                      "frac": (tflops / fp4_peak) if bound == "tensor" else (gbs / peaks["hbm_gbs"]),
@@ -770,7 +797,7 @@ def time_mla_gemms(dev, steps, warmup, peaks, flush, ceiling_tflops=None):
                      "sm_mhz": CLOCKS.mhz(f"mla_{name}") if CLOCKS else None}
         if ceiling_tflops:
             res[name]["fp4_ceiling_frac"] = tflops / ceiling_tflops
-        del ad, a_codes, a_sc, out, w_codes, w_sc, gws
+        del ad, a_codes, a_sc, out, w_codes, w_sc
         torch.cuda.empty_cache()
     return res
 

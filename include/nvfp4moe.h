@@ -108,31 +108,14 @@ int nvfp4_swizzle_scales(const uint8_t *in, int64_t batch, int64_t rows, int64_t
  * b_codes [N, K/2], b_scales NVFP4_SCALES_MMA, b_gs device [nseg];
  * seg_end HOST [nseg]: increasing column ends of the B segments, the last
  * equal to N, each a multiple of 32; rows of B in segment s use b_gs[s].
- * out [M, ldo] bf16, ldo >= N, ldo % 8 == 0.
+ * out [M, ldo] bf16, ldo >= N, ldo % 8 == 0; only the [M, N] window is
+ * written.  Each output element is one fp32 sum in a fixed k order, so
+ * repeated calls give identical results.
  * Constraints: M >= 1, N % 128 == 0, K % 64 == 0, 1 <= nseg <= 4. */
 int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs, int64_t M,
                const uint8_t *b_codes, const uint8_t *b_scales, const float *b_gs,
                const int64_t *seg_end, int nseg, int64_t N, int64_t K,
                uint16_t *out, int64_t ldo, void *stream);
-
-/* nvfp4_gemm with a caller-owned device workspace (16-byte aligned, at least
- * nvfp4_gemm_workspace_size(M, N, K) bytes, contents need not be kept
- * between calls).  When the tiles would fill the GPU unevenly with few tiles
- * per SM (e.g. 224 pair tiles over 74 SM pairs), the (tile, k-tile)
- * iterations are split evenly over the SMs ("stream-K"): a tile cut between
- * SMs is finished by the SM holding its first k-tile, which adds the others'
- * fp32 partial sums in a fixed order (deterministic; the rounding differs
- * from nvfp4_gemm's by the fp32 sum order).  Otherwise, or with workspace =
- * NULL, identical to nvfp4_gemm.  Calls sharing a workspace must not overlap
- * on the device.  A bounded device wait that gives up sets the workspace's
- * first int32 to NVFP4_ERR_TIMEOUT. */
-int nvfp4_gemm_ws(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs, int64_t M,
-                  const uint8_t *b_codes, const uint8_t *b_scales, const float *b_gs, const int64_t *seg_end, int nseg,
-                  int64_t N, int64_t K, uint16_t *out, int64_t ldo, void *workspace, size_t ws_bytes, void *stream);
-
-/* Workspace bytes nvfp4_gemm_ws uses for this shape on the current device
- * (0: the shape runs without a split; also 0 without a usable device). */
-size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* The routed-expert MoE block (page 1 "Phase 1" chain; page 3
  * "Architecture Notes" routing).  Shapes: T tokens, hidden H, expert

@@ -18,8 +18,8 @@ __all__ = [
     "nvfp4_swizzle_scales", "nvfp4_gemm", "nvfp4_moe_workspace_size", "nvfp4_moe_forward",
     "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc", "nvfp4_moe_forward_quantized",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
-    "nvfp4_moe_get_error", "nvfp4_moe_topk", "nvfp4_moe_topk_shared", "NVFP4_SCORING_SOFTMAX", "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax", "nvfp4_debug_bounded_wait", "nvfp4_gemm_ws",
-    "nvfp4_gemm_workspace_size",
+    "nvfp4_moe_get_error", "nvfp4_moe_topk", "nvfp4_moe_topk_shared", "NVFP4_SCORING_SOFTMAX",
+    "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax", "nvfp4_debug_bounded_wait",
     "MoeArgs",
 ]
 
@@ -81,9 +81,6 @@ def lib():
         L.nvfp4_moe_topk_shared.argtypes = [P, i64, i32, i32, i32, i32, P, P, P]
         L.nvfp4_amax.argtypes = [P, i64, P, P]
         L.nvfp4_debug_bounded_wait.argtypes = [P, i32, P, P]
-        L.nvfp4_gemm_ws.argtypes = [P, P, P, i64, P, P, P, P, i32, i64, i64, P, i64, P, ctypes.c_size_t, P]
-        L.nvfp4_gemm_workspace_size.argtypes = [i64, i64, i64]
-        L.nvfp4_gemm_workspace_size.restype = ctypes.c_size_t
         L.nvfp4_fp4_mma_ceiling.argtypes = [i32, i32, i32, P, P, P]
         L.nvfp4_moe_plan.argtypes = [i64, i32, i32, i64, i64, ctypes.POINTER(ctypes.c_int32),
                                      ctypes.POINTER(ctypes.c_int32)]
@@ -150,27 +147,6 @@ def nvfp4_gemm(a_codes, a_scales, a_gs, b_codes, b_scales, b_gs, seg_end, out, s
                             _dev(b_scales, "b_scales", torch.uint8), _dev(b_gs, "b_gs", torch.float32),
                             ctypes.cast(seg, ctypes.c_void_p), len(seg_end), N, K,
                             _dev(out, "out", torch.bfloat16), out.stride(0), _stream(stream)), "nvfp4_gemm")
-
-
-def nvfp4_gemm_workspace_size(M, N, K):
-    """Bytes of device workspace nvfp4_gemm_ws uses for this shape (0: none)."""
-    return int(lib().nvfp4_gemm_workspace_size(M, N, K))
-
-
-def nvfp4_gemm_ws(a_codes, a_scales, a_gs, b_codes, b_scales, b_gs, seg_end, out, workspace, stream=None):
-    """nvfp4_gemm with a workspace (uint8 CUDA tensor, or None): the stream-K
-    split for shapes whose tiles fill the GPU unevenly."""
-    M, K = a_codes.shape[0], a_codes.shape[1] * 2
-    N = b_codes.shape[0]
-    seg = (ctypes.c_int64 * len(seg_end))(*[int(v) for v in seg_end])
-    ws = None if workspace is None else _dev(workspace, "workspace", torch.uint8)
-    nbytes = 0 if workspace is None else workspace.numel()
-    _check(lib().nvfp4_gemm_ws(_dev(a_codes, "a_codes", torch.uint8), _dev(a_scales, "a_scales", torch.uint8),
-                               _dev(a_gs, "a_gs", torch.float32), M, _dev(b_codes, "b_codes", torch.uint8),
-                               _dev(b_scales, "b_scales", torch.uint8), _dev(b_gs, "b_gs", torch.float32),
-                               ctypes.cast(seg, ctypes.c_void_p), len(seg_end), N, K,
-                               _dev(out, "out", torch.bfloat16), out.stride(0), ws, nbytes, _stream(stream)),
-           "nvfp4_gemm_ws")
 
 
 def nvfp4_moe_workspace_size(T, k, E, H, I):

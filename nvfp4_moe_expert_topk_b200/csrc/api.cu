@@ -531,14 +531,13 @@ int nvfp4_swizzle_scales(const uint8_t *in, int64_t batch, int64_t rows, int64_t
 namespace {
 
 // Dense GEMM tile plan: pair tiles when there are at least two m-tiles and
-// the tiles are 256 wide; stream-K when there is at least one full round of
-// tiles and the last, partial round would leave more than 15 % of the
-// units' time idle (measured: with fewer tiles than units, splitting every
-// tile costs more in partial-sum traffic than the idle units lose).
+// the tiles are 256 wide, dealt round-robin over the resident units.  (A
+// stream-K split of the (tile, k-tile) iterations was measured against this
+// once the pair tiles stored their output through TMA: it lost on every shape
+// tried, since the launch is bound by the operand fill from L2 and a partial
+// last round runs its few tiles at a higher fill rate per SM.)
 struct DensePlan {
     int bn, cg, grid;
-    int64_t units, tiles;
-    bool streamk;
 };
 
 DensePlan dense_plan(int64_t M, int64_t N, int sms)
@@ -547,31 +546,13 @@ DensePlan dense_plan(int64_t M, int64_t N, int sms)
     d.bn = (N % 256 == 0) ? 256 : 128;
     d.cg = (M > 128 && d.bn == 256) ? 2 : 1;
     const int64_t m_units = d.cg == 2 ? (M + 255) / 256 : (M + 127) / 128;
-    d.tiles = m_units * (N / d.bn);
-    const int64_t max_units = d.cg == 2 ? gemm_pair_clusters(sms) : sms;
-    const int64_t rounds = (d.tiles + max_units - 1) / max_units;
-    const double idle = static_cast<double>(rounds * max_units - d.tiles) / static_cast<double>(rounds * max_units);
-    d.streamk = d.bn == 256 && d.tiles >= max_units && idle > 0.15;
-    if (d.streamk) {                      // every unit takes part in the split
-        d.units = max_units;
-        d.grid = static_cast<int>(max_units * d.cg);
-    } else {
-        d.grid = gemm_grid(d.cg, d.tiles, sms);
-        d.units = d.grid / d.cg;
-    }
+    d.grid = gemm_grid(d.cg, m_units * (N / d.bn), sms);
     return d;
-}
-
-int64_t dense_ws_bytes(const DensePlan &d)
-{
-    if (!d.streamk)
-        return 0;
-    return 256 + round_up(4 * d.tiles * d.cg, 256) + static_cast<int64_t>(d.grid) * 128 * 256 * 4;
 }
 
 int gemm_impl(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs, int64_t M, const uint8_t *b_codes,
               const uint8_t *b_scales, const float *b_gs, const int64_t *seg_end, int nseg, int64_t N, int64_t K,
-              uint16_t *out, int64_t ldo, void *workspace, size_t ws_bytes, void *stream)
+              uint16_t *out, int64_t ldo, void *stream)
 {
     if (a_codes == nullptr || a_scales == nullptr || a_gs == nullptr || b_codes == nullptr || b_scales == nullptr ||
         b_gs == nullptr || seg_end == nullptr || out == nullptr || M < 1 || N < 1 || K < 1 || nseg < 1 || ldo < N)
@@ -629,31 +610,16 @@ int gemm_impl(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs
     g.err = nullptr;            // no workspace: a timed-out wait ends the kernel without a report
     const DensePlan d = dense_plan(M, N, sms);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (d.streamk && workspace != nullptr) {
-        if (ws_bytes < static_cast<size_t>(dense_ws_bytes(d)))
-            return NVFP4_ERR_WORKSPACE_TOO_SMALL;
-        if (!aligned16(workspace))
-            return NVFP4_ERR_MISALIGNED;
-        uint8_t *ws = static_cast<uint8_t *>(workspace);
-        const int64_t flag_bytes = round_up(4 * d.tiles * d.cg, 256);
-        g.sk_flags = reinterpret_cast<int32_t *>(ws + 256);
-        g.sk_partials = reinterpret_cast<float *>(ws + 256 + flag_bytes);
-        g.err = reinterpret_cast<int32_t *>(ws);
-        if (cudaMemsetAsync(ws, 0, static_cast<size_t>(256 + flag_bytes), s) != cudaSuccess)
-            return NVFP4_ERR_CUDA;
-        return cuda_status(launch_gemm_streamk(d.cg, ma, ma32, mb, g, d.grid, s));
-    }
-    const int grid = gemm_grid(d.cg, d.tiles, sms);
+    // pair tiles write out through shared memory and TMA stores (rows >= M are not written)
+    CUtensorMap mo;
     if (d.cg == 2) {
-        // pair tiles write out through shared memory and TMA stores (rows >= M are not written)
-        CUtensorMap mo;
         st = make_out_map(&mo, out, M, N, ldo);
         if (st != NVFP4_OK)
             return st;
         g.out_tma = 1;
-        return cuda_status(launch_gemm(d.bn, EPI_BF16, d.cg, ma, ma32, mb, g, grid, s, &mo));
     }
-    return cuda_status(launch_gemm(d.bn, EPI_BF16, d.cg, ma, ma32, mb, g, grid, s));
+    const CUtensorMap *mo_ptr = d.cg == 2 ? &mo : nullptr;
+    return cuda_status(launch_gemm(d.bn, EPI_BF16, d.cg, ma, ma32, mb, g, d.grid, s, mo_ptr));
 }
 
 } // namespace
@@ -664,26 +630,7 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_g
                const uint8_t *b_scales, const float *b_gs, const int64_t *seg_end, int nseg, int64_t N, int64_t K,
                uint16_t *out, int64_t ldo, void *stream)
 {
-    return gemm_impl(a_codes, a_scales, a_gs, M, b_codes, b_scales, b_gs, seg_end, nseg, N, K, out, ldo, nullptr, 0,
-                     stream);
-}
-
-int nvfp4_gemm_ws(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_gs, int64_t M,
-                  const uint8_t *b_codes, const uint8_t *b_scales, const float *b_gs, const int64_t *seg_end, int nseg,
-                  int64_t N, int64_t K, uint16_t *out, int64_t ldo, void *workspace, size_t ws_bytes, void *stream)
-{
-    return gemm_impl(a_codes, a_scales, a_gs, M, b_codes, b_scales, b_gs, seg_end, nseg, N, K, out, ldo, workspace,
-                     ws_bytes, stream);
-}
-
-size_t nvfp4_gemm_workspace_size(int64_t M, int64_t N, int64_t K)
-{
-    if (M < 1 || N < 1 || K < 1 || N % 128 != 0 || K % 64 != 0)
-        return 0;
-    int sms = 0;
-    if (device_check(&sms) != NVFP4_OK)
-        return 0;
-    return static_cast<size_t>(dense_ws_bytes(dense_plan(M, N, sms)));
+    return gemm_impl(a_codes, a_scales, a_gs, M, b_codes, b_scales, b_gs, seg_end, nseg, N, K, out, ldo, stream);
 }
 
 size_t nvfp4_moe_workspace_size(int64_t T, int k, int E, int64_t H, int64_t I)

@@ -191,6 +191,31 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmArgs &p, const GemmArg
     return ti;
 }
 
+// One 32-row x 32-column bf16 box of a pair tile leaves through shared memory:
+// each lane's row (16 words of packed bf16 pairs) goes into `buf` as four
+// 16-byte chunks, chunk c at position c ^ ((row >> 1) & 3) (the 64-byte
+// swizzle the output map names, so that no two lanes of a quarter-warp share
+// a bank), then lane 0 stores the box at (x, y) with TMA.  The warp alternates
+// two buffers: before filling one it waits until the store issued from it
+// two boxes earlier has read it.
+__device__ __forceinline__ void store_box_staged(uint8_t *buf, const uint32_t (&v)[16], int lane,
+                                                 const CUtensorMap *map, int x, int y)
+{
+    if (lane == 0)
+        bulk_wait_group_read<1>();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4 *>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(map, x, y, buf);
+        bulk_commit_group();
+    }
+}
+
 // v[i] for a run-time i < 4 without indexing a register array
 __device__ __forceinline__ float pick4(const float (&v)[4], int i)
 {
@@ -258,51 +283,18 @@ __device__ __forceinline__ int dyn_next(uint64_t *q_full, uint64_t *q_empty, con
     return t >= 0 ? 1 : 0;
 }
 
-// Work cursor of a CTA (or pair) over its tiles.  SK = 0: whole tiles
-// t = unit, unit + units, ...  SK = 1 (stream-K, dense GEMMs): the
-// linearised (tile, k-tile) iterations are split evenly over the units, and
-// each unit walks its range as segments {tile, k-tiles [k0, k1)}: a segment
-// that is not a whole tile leaves a partial sum for the unit that holds the
-// tile's first k-tile (the head) to finish.
+// Work cursor of a CTA (or pair) that deals whole tiles round-robin:
+// t = unit, unit + units, ...
 struct Cursor {
-    int64_t it, end;
+    int it, end;
 };
 
-__device__ __forceinline__ int64_t sk_begin(int64_t unit, int64_t units, int64_t total)
-{
-    const int64_t q = total / units, r = total % units;
-    return unit * q + (unit < r ? unit : r);
-}
-
-template <int SK>
-__device__ __forceinline__ Cursor cursor_init(int unit, int units, int total_tiles, int kt_per_tile)
-{
-    if constexpr (SK) {
-        const int64_t total = static_cast<int64_t>(total_tiles) * kt_per_tile;
-        return Cursor{sk_begin(unit, units, total), sk_begin(unit + 1, units, total)};
-    } else {
-        return Cursor{unit, total_tiles};
-    }
-}
-
-// Next segment: tile t and k-tiles [k0, k1) (k1 < 0: all of the tile's).
-template <int SK>
-__device__ __forceinline__ bool cursor_next(Cursor &c, int units, int kt_per_tile, int &t, int &k0, int &k1)
+__device__ __forceinline__ bool cursor_next(Cursor &c, int units, int &t)
 {
     if (c.it >= c.end)
         return false;
-    if constexpr (SK) {
-        t = static_cast<int>(c.it / kt_per_tile);
-        k0 = static_cast<int>(c.it - static_cast<int64_t>(t) * kt_per_tile);
-        const int64_t left = c.end - c.it;
-        k1 = left < kt_per_tile - k0 ? k0 + static_cast<int>(left) : kt_per_tile;
-        c.it += k1 - k0;
-    } else {
-        t = static_cast<int>(c.it);
-        k0 = 0;
-        k1 = -1;
-        c.it += units;
-    }
+    t = c.it;
+    c.it += units;
     return true;
 }
 
@@ -335,7 +327,7 @@ cudaError_t launch_wait_probe(const int32_t *flag, int target, int32_t *err, cud
 // requirement); CG = 2 deals tiles round-robin over clusters that are all
 // resident (the launch follows the front on an idle GPU, one cluster per SM
 // pair).
-template <int BN, int EPI, int CG, int FUSED, int SK>
+template <int BN, int EPI, int CG, int FUSED>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a32,
                       const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_a2,
@@ -347,7 +339,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the fused 1-CTA launch claims its tiles one at a time (no residency
     // requirement); everything else deals tiles round-robin
     constexpr bool kDyn = FUSED && CG == 1;
-    static_assert(!SK || (!FUSED && EPI == EPI_BF16 && BN == 256), "stream-K: dense bf16 GEMMs");
     constexpr int kStages = C::kStages;
     constexpr int kHalves = C::kHalves;
     constexpr int kNumAcc = C::kNumAcc;
@@ -449,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0, pend_mask = 0, pend_par = 0;
             bool ok = true;
-            Cursor cur = cursor_init<SK>(unit, units, total, p.num_k_tiles);
-            int t = 0, kb0 = 0, kb1 = -1, pq = 0;
+            Cursor cur{unit, total};
+            int t = 0, pq = 0;
             while (ok) {
                 if constexpr (kDyn) {
                     // claim the next tile just before loading it, and queue its index for the other roles
@@ -469,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (tc < 0)
                         break;
                     t = tc;
-                } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+                } else if (!cursor_next(cur, units, t)) {
                     break;
                 }
                 const TileInfo ti = decode_tile<CG, FUSED>(p, p2, t, m_units, rank);
@@ -490,8 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t *sfa = q.sfa + static_cast<int64_t>(ti.row0 / kBM) * q.sfa_block_stride;
                 const uint8_t *sfb0 = q.sfb + (brow0 / 128) * q.sfb_block_stride;
                 const uint8_t *sfb1 = q.sfb + (brow1 / 128) * q.sfb_block_stride;
-                const int kend = kb1 < 0 ? q.num_k_tiles : kb1;
-                for (int kt = kb0; kt < kend; ++kt) {
+                for (int kt = 0; kt < q.num_k_tiles; ++kt) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) {
                         ok = false;
                         break;
@@ -556,8 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            Cursor cur = cursor_init<SK>(unit, units, total, p.num_k_tiles);
-            int t = 0, kb0 = 0, kb1 = -1, qi = 0;
+            Cursor cur{unit, total};
+            int t = 0, qi = 0;
             while (ok) {
                 if constexpr (kDyn) {
                     const int r = dyn_next(q_full, q_empty, tile_q, qi, t, false, abort_flag);
@@ -565,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                     if (r <= 0)
                         break;
-                } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+                } else if (!cursor_next(cur, units, t)) {
                     break;
                 }
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -575,8 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * BN);
                 const GemmArgs &q = (FUSED && t >= m_units * p.n_tiles) ? p2 : p;
-                const int kend = kb1 < 0 ? q.num_k_tiles : kb1;
-                for (int kt = kb0; kt < kend; ++kt) {
+                for (int kt = 0; kt < q.num_k_tiles; ++kt) {
                     // sf_ready completes only after every stager has seen its CTA's
                     // full barrier complete (all of the stage's copies landed), so
                     // one wait covers both the scales and the operand tiles
@@ -592,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kb = 0; kb < nkb; ++kb) {
                         const uint64_t ad = sdesc_kmajor_sw128(a_addr + kb * 32);
                         const uint64_t bd = sdesc_kmajor_sw128(b_addr + kb * 32);
-                        const uint32_t acc_flag = (kt != kb0 || kb != 0) ? 1u : 0u;
+                        const uint32_t acc_flag = (kt != 0 || kb != 0) ? 1u : 0u;
                         if constexpr (kPair)
                             tc_mma_nvf4_pair(d_tmem, ad, bd, idesc, t_sfa + kb * 4, t_sfa + 16 + kb * 4 * kHalves,
                                              acc_flag);
@@ -638,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        Cursor cur = cursor_init<SK>(unit, units, total, p.num_k_tiles);
-        int t = 0, kb0 = 0, kb1 = -1, qi = 0;
+        Cursor cur{unit, total};
+        int t = 0, qi = 0;
         while (ok) {
             if constexpr (kDyn) {
                 const int r = dyn_next(q_full, q_empty, tile_q, qi, t, true, abort_flag);
@@ -647,14 +636,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                 if (r <= 0)
                     break;
-            } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+            } else if (!cursor_next(cur, units, t)) {
                 break;
             }
             // an empty pair half has no A scales: its rows get scale 0
             const bool a_rows = !kPair || decode_tile<CG, FUSED>(p, p2, t, m_units, rank).valid > 0;
             const GemmArgs &q = (FUSED && t >= m_units * p.n_tiles) ? p2 : p;
-            const int kend = kb1 < 0 ? q.num_k_tiles : kb1;
-            for (int kt = kb0; kt < kend; ++kt) {
+            for (int kt = 0; kt < q.num_k_tiles; ++kt) {
                 const bool got = mbar_wait(&full[stage], phase, abort_flag);
                 if (!__all_sync(0xffffffffu, got)) {
                     ok = false;
@@ -725,8 +713,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
         int acc = 0;
         uint32_t acc_phase = 0;
-        Cursor cur = cursor_init<SK>(unit, units, total, p.num_k_tiles);
-        int t = 0, kb0 = 0, kb1 = -1, qi = 0;
+        Cursor cur{unit, total};
+        int t = 0, qi = 0;
         while (true) {
             if constexpr (kDyn) {
                 const int r = dyn_next(q_full, q_empty, tile_q, qi, t, true, abort_flag);
@@ -738,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (r <= 0)
                     break;
-            } else if (!cursor_next<SK>(cur, units, p.num_k_tiles, t, kb0, kb1)) {
+            } else if (!cursor_next(cur, units, t)) {
                 break;
             }
             // the tile's coordinates and global scales are read while its MMAs
@@ -846,122 +834,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 constexpr int kCols = BN / 2;
                 constexpr int kRound = kCols < 64 ? kCols : 64;
-                bool sk_segment = false;
-                if constexpr (SK) {
-                    // stream-K: a segment that is not a whole tile stores its fp32 sum in
-                    // this unit's slot (head: slot 0, other: slot 1); the head then adds
-                    // the later units' slots in unit order (a fixed order: deterministic)
-                    sk_segment = kb0 != 0 || kb1 < p.num_k_tiles;
-                    if (sk_segment) {
-                        // slot layout: per epilogue warp (q, hf), float4 i of lane l at
-                        // ((warp_role * kCols / 4 + i) * 32 + l): each store and load of a
-                        // warp is one contiguous 512-byte run
-                        constexpr int64_t kSlot4 = static_cast<int64_t>(kBM) * BN / 4;
-                        const int64_t lane_off4 = static_cast<int64_t>(q * 2 + hf) * (kCols / 4) * 32 + lane;
-                        if (kb0 != 0) {
-                            // not the tile's first k-tile: leave the partial sum in this
-                            // unit's slot and count it on the tile's flag
-                            float4 *mine = reinterpret_cast<float4 *>(p.sk_partials) +
-                                           static_cast<int64_t>(unit * CG + rank) * kSlot4 + lane_off4;
-#pragma unroll
-                            for (int r = 0; r < kCols / kRound; ++r) {
-                                uint32_t v[kRound];
-#pragma unroll
-                                for (int c = 0; c < kRound / 16; ++c)
-                                    tc_ld_32x32b_x16(t_acc + hf * kCols + r * kRound + c * 16,
-                                                     *reinterpret_cast<uint32_t(*)[16]>(&v[16 * c]));
-                                tc_wait_ld();
-#pragma unroll
-                                for (int i = 0; i < kRound / 4; ++i)
-                                    mine[static_cast<int64_t>(r * kRound / 4 + i) * 32] =
-                                        make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                    __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-                            }
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) {
-                                if constexpr (kPair)
-                                    mbar_arrive_cluster(acc_empty_lead + acc * 8);
-                                else
-                                    mbar_arrive(&acc_empty[acc]);
-                            }
-                            __threadfence();
-                            __syncwarp();
-                            if (lane == 0) {
-                                __threadfence();
-                                atomicAdd(p.sk_flags + t * CG + rank, 1);
-                            }
-                        } else {
-                            // the tile's first k-tiles, the unit's last segment: wait for
-                            // the later units' partial sums, then add them to this
-                            // accumulator in unit order (deterministic) while reading it
-                            // out of TMEM 16 columns at a time
-                            const int64_t total_it = static_cast<int64_t>(total) * p.num_k_tiles;
-                            const int64_t tile_end = static_cast<int64_t>(t + 1) * p.num_k_tiles;
-                            int n_other = 0;
-                            while (unit + 1 + n_other < units && sk_begin(unit + 1 + n_other, units, total_it) < tile_end)
-                                ++n_other;
-                            int ok_w = 1;
-                            if (lane == 0)
-                                ok_w = wait_counter(p.sk_flags + t * CG + rank, n_other * kEpiWarps, abort_flag) ? 1 : 0;
-                            ok_w = __shfl_sync(0xffffffffu, ok_w, 0);
-                            if (!ok_w) {
-                                *abort_flag = 1;
-                                record_error(p.err, NVFP4_ERR_TIMEOUT);
-                            } else {
-                                uint4 *dst = reinterpret_cast<uint4 *>(
-                                    ga.out + static_cast<int64_t>(ti.row0_out + row) * ga.ldo +
-                                    static_cast<int64_t>(ti.nt) * BN + hf * kCols);
-                                for (int c = 0; c < kCols / 16; ++c) {
-                                    uint32_t v[16];
-                                    tc_ld_32x32b_x16(t_acc + hf * kCols + c * 16, v);
-                                    tc_wait_ld();
-                                    float sum[16];
-#pragma unroll
-                                    for (int i = 0; i < 16; ++i)
-                                        sum[i] = __uint_as_float(v[i]);
-                                    for (int j = 0; j < n_other; ++j) {
-                                        const float4 *src = reinterpret_cast<const float4 *>(p.sk_partials) +
-                                                            static_cast<int64_t>((unit + 1 + j) * CG + rank) * kSlot4 +
-                                                            lane_off4;
-#pragma unroll
-                                        for (int i = 0; i < 4; ++i) {
-                                            const float4 f = __ldcg(src + static_cast<int64_t>(c * 4 + i) * 32);
-                                            sum[4 * i] += f.x;
-                                            sum[4 * i + 1] += f.y;
-                                            sum[4 * i + 2] += f.z;
-                                            sum[4 * i + 3] += f.w;
-                                        }
-                                    }
-                                    const int col = ti.nt * BN + hf * kCols + c * 16;
-                                    int seg = 0;
-#pragma unroll
-                                    for (int i = 0; i < 3; ++i)
-                                        if (i < ga.nseg - 1 && col >= ga.seg_end[i])
-                                            seg = i + 1;
-                                    const float alpha = pick4(alpha_seg, seg);
-                                    uint32_t o[8];
-#pragma unroll
-                                    for (int i = 0; i < 8; ++i)
-                                        o[i] = pack_bf16x2(sum[2 * i] * alpha, sum[2 * i + 1] * alpha);
-                                    if (valid) {
-                                        dst[2 * c] = make_uint4(o[0], o[1], o[2], o[3]);
-                                        dst[2 * c + 1] = make_uint4(o[4], o[5], o[6], o[7]);
-                                    }
-                                }
-                            }
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) {
-                                if constexpr (kPair)
-                                    mbar_arrive_cluster(acc_empty_lead + acc * 8);
-                                else
-                                    mbar_arrive(&acc_empty[acc]);
-                            }
-                        }
-                    }
-                }
-                if (!sk_segment) {
                 // drain columns [hf*BN/2, (hf+1)*BN/2) in rounds of 64 (one wait each),
                 // converting to bf16 as they arrive, then release the accumulator
                 uint32_t o[kCols / 2];
@@ -1001,30 +873,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (ga.out_tma) {
                         // four boxes of 32 rows x 32 columns through this warp's two
                         // buffers, written out by TMA stores (whole 64-byte row pieces
-                        // instead of one 16-byte piece per row per store instruction);
-                        // a row's 16-byte chunk c sits at c ^ ((row >> 1) & 3), the
-                        // 64-byte swizzle of the map, so no two lanes of a quarter-warp
-                        // share a bank
+                        // instead of one 16-byte piece per row per store instruction)
                         staged = true;
                         if (q * 32 < ti.valid) {    // a box starts on a row the GEMM writes; rows past M are clipped
-                            uint8_t *wbuf = sOut + (warp - 2) * 2 * C::kOutBuf;
 #pragma unroll
                             for (int b = 0; b < 4; ++b) {
-                                uint8_t *buf = wbuf + (b & 1) * C::kOutBuf;
-                                if (lane == 0)
-                                    bulk_wait_group_read<1>();   // the store that last read this buffer is done
-                                __syncwarp();
+                                uint32_t ob[16];
 #pragma unroll
-                                for (int c = 0; c < 4; ++c)
-                                    *reinterpret_cast<uint4 *>(buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
-                                        make_uint4(o[16 * b + 4 * c], o[16 * b + 4 * c + 1], o[16 * b + 4 * c + 2],
-                                                   o[16 * b + 4 * c + 3]);
-                                fence_proxy_async_smem();
-                                __syncwarp();
-                                if (lane == 0) {
-                                    tma_store_2d(&map_out, ti.nt * BN + hf * kCols + b * 32, ti.row0_out + q * 32, buf);
-                                    bulk_commit_group();
-                                }
+                                for (int i = 0; i < 16; ++i)
+                                    ob[i] = o[16 * b + i];
+                                store_box_staged(sOut + ((warp - 2) * 2 + (b & 1)) * C::kOutBuf, ob, lane, &map_out,
+                                                 ti.nt * BN + hf * kCols + b * 32, ti.row0_out + q * 32);
                             }
                         }
                     }
@@ -1035,7 +894,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < kCols / 8; ++i)
                         dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-                }
                 }
             }
             if (++acc == kNumAcc) {
@@ -1067,18 +925,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int BN, int EPI, int CG, int FUSED, int SK = 0>
+template <int BN, int EPI, int CG, int FUSED>
 static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a32, const CUtensorMap &map_b,
                               const GemmArgs &args, const CUtensorMap &map_a2, const CUtensorMap &map_a2_32,
                               const CUtensorMap &map_b2, const GemmArgs &args2, int grid, cudaStream_t stream,
                               const CUtensorMap *map_out = nullptr)
 {
-    if (args.out_tma && (map_out == nullptr || CG != 2 || EPI != EPI_BF16 || FUSED || SK))
+    if (args.out_tma && (map_out == nullptr || CG != 2 || EPI != EPI_BF16 || FUSED))
         return cudaErrorInvalidValue;
     const int smem = Cfg<BN, CG>::kSmem;
     static unsigned long long attr_done = 0;     // one bit per device
     const cudaError_t e =
-        ensure_smem_limit(reinterpret_cast<const void *>(nvfp4_gemm_kernel<BN, EPI, CG, FUSED, SK>), smem, &attr_done);
+        ensure_smem_limit(reinterpret_cast<const void *>(nvfp4_gemm_kernel<BN, EPI, CG, FUSED>), smem, &attr_done);
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
@@ -1105,7 +963,7 @@ static cudaError_t launch_one(const CUtensorMap &map_a, const CUtensorMap &map_a
         ++cfg.numAttrs;
     }
     // without staged stores the output map is never read: any valid map fills the slot
-    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, CG, FUSED, SK>, map_a, map_a32, map_b, map_a2,
+    return cudaLaunchKernelEx(&cfg, nvfp4_gemm_kernel<BN, EPI, CG, FUSED>, map_a, map_a32, map_b, map_a2,
                               map_a2_32, map_b2, map_out != nullptr ? *map_out : map_a, args, args2);
 }
 
@@ -1137,18 +995,6 @@ cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const
     default: return bn == 256 ? NVFP4_PLAIN(256, EPI_BF16, 1) : NVFP4_PLAIN(128, EPI_BF16, 1);
     }
 #undef NVFP4_PLAIN
-}
-
-cudaError_t launch_gemm_streamk(int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
-                                const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream)
-{
-    if (args.mtiles != nullptr || args.sk_partials == nullptr || args.sk_flags == nullptr)
-        return cudaErrorInvalidValue;
-    if (cg == 2)
-        return grid % 2 != 0 ? cudaErrorInvalidValue
-                             : launch_one<256, EPI_BF16, 2, 0, 1>(map_a, map_a32, map_b, args, map_a, map_a32, map_b,
-                                                                   args, grid, stream);
-    return launch_one<256, EPI_BF16, 1, 0, 1>(map_a, map_a32, map_b, args, map_a, map_a32, map_b, args, grid, stream);
 }
 
 cudaError_t launch_moe_fused(int cg, const CUtensorMap &map_a1, const CUtensorMap &map_a1_32,
@@ -1183,7 +1029,7 @@ int gemm_pair_clusters(int num_sms)
         return cached[dev];
     const int smem = Cfg<256, 2>::kSmem;
     int n = 0;
-    if (cudaFuncSetAttribute(nvfp4_gemm_kernel<256, EPI_BF16, 2, 0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(nvfp4_gemm_kernel<256, EPI_BF16, 2, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) == cudaSuccess) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(num_sms));
@@ -1196,7 +1042,7 @@ int gemm_pair_clusters(int num_sms)
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<256, EPI_BF16, 2, 0, 0>, &cfg) != cudaSuccess)
+        if (cudaOccupancyMaxActiveClusters(&n, nvfp4_gemm_kernel<256, EPI_BF16, 2, 0>, &cfg) != cudaSuccess)
             n = 0;
     }
     (void)cudaGetLastError();

@@ -62,8 +62,6 @@ struct GemmArgs {
     const int32_t *num_light_dev;
     const int32_t *light;     // 1-CTA tiles: the m-tiles not covered by pairs, by index into mtiles
     int32_t *ready;           // fused L1 -> L2 launch: per m-tile count of published L1 epilogue warps
-    float *sk_partials;       // stream-K: one slot of 128 x 256 fp32 per CTA
-    int32_t *sk_flags;        // stream-K: per (tile, CTA of the pair) count of published partial warps
     int dense_m_tiles;
     int dense_M;
     int n_tiles;
@@ -112,11 +110,6 @@ enum Epilogue { EPI_SWIGLU_QUANT = 0, EPI_BF16 = 1, EPI_SWIGLU_AMAX = 2 };
 cudaError_t launch_gemm(int bn, int epi, int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
                         const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream,
                         const CUtensorMap *map_out = nullptr);
-// Dense bf16 GEMM with stream-K work split (256-wide tiles; cg 1 or 2):
-// args.sk_partials holds grid slots of 128 x 256 fp32 and args.sk_flags
-// one zeroed int per (tile, CTA of the pair).
-cudaError_t launch_gemm_streamk(int cg, const CUtensorMap &map_a, const CUtensorMap &map_a32,
-                                const CUtensorMap &map_b, const GemmArgs &args, int grid, cudaStream_t stream);
 // One bounded counter wait (the fused launch's) in a one-thread kernel.
 cudaError_t launch_wait_probe(const int32_t *flag, int target, int32_t *err, cudaStream_t s);
 // Pair clusters that fit on the device at once (<= num_sms / 2).

@@ -157,38 +157,28 @@ def test_mla_projection_full_size(name):
 
 
 @pytest.mark.parametrize("M,N,K,segs", [
-    (256, 20480, 1024, [20480]),            # 80 pair tiles over 74 SM pairs
+    (256, 20480, 1024, [20480]),            # 80 pair tiles over 74 SM pairs: a second, nearly empty round
     (300, 10240, 512, [4096, 10240]),       # ragged M (empty half in each last pair), dual global scales
     (128, 40960, 512, [40960]),             # one m-tile: 160 one-CTA tiles over 148 SMs
     (2048, 7168, 8192, [7168]),             # o_b shape: 224 pair tiles over 74 pairs
 ])
-def test_gemm_streamk_matches_oracle(M, N, K, segs):
-    """nvfp4_gemm_ws splits the (tile, k-tile) iterations evenly over the SMs
-    when the tiles fill them unevenly: sampled rows against the oracle, the
-    whole result against nvfp4_gemm (same products, fp32 sums regrouped), and
-    two runs bit-identical (the partial sums are added in a fixed order)."""
-    from nvfp4_moe_expert_topk_b200 import nvfp4_gemm_workspace_size, nvfp4_gemm_ws
-    nbytes = nvfp4_gemm_workspace_size(M, N, K)
-    assert nbytes > 0
+def test_gemm_wide_shapes_match_oracle(M, N, K, segs):
+    """Shapes whose tiles fill the GPU unevenly: sampled rows against the
+    oracle, and two calls bit-identical (each element is one fp32 sum in a
+    fixed k order)."""
     ac, asc, a_gs, bc, bsc, bgs = quantized_operands(M, N, K, M + N + K, segs)
     dev_args = (torch.from_numpy(ac).to(DEV), torch.from_numpy(to_mma_layout(asc)).to(DEV),
                 torch.tensor([a_gs], dtype=torch.float32, device=DEV), torch.from_numpy(bc).to(DEV),
                 torch.from_numpy(to_mma_layout(bsc)).to(DEV), torch.tensor(np.asarray(bgs, np.float32), device=DEV))
-    ws = torch.zeros(nbytes, dtype=torch.uint8, device=DEV)
     outs = []
     for _ in range(2):
         out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
-        nvfp4_gemm_ws(*dev_args, segs, out, ws)
+        nvfp4_gemm(*dev_args, segs, out)
         torch.cuda.synchronize()
         outs.append(out)
-    assert ws[:4].view(torch.int32).item() == 0
     assert torch.equal(outs[0], outs[1])
-    plain = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
-    nvfp4_gemm(*dev_args, segs, plain)
-    torch.cuda.synchronize()
-    got, ref_dev = bf16_to_np(outs[0]), bf16_to_np(plain)
+    got = bf16_to_np(outs[0])
     assert np.all(np.isfinite(got))
-    assert row_rel_l2(got, ref_dev).max() <= 1e-2
     rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(M).choice(M, 6, replace=False)]))
     ref = O.gemm(ac[rows], asc[rows], a_gs, bc, bsc, bgs, segs)
     err = row_rel_l2(got[rows], ref)
