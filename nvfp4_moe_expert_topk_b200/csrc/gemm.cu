@@ -870,11 +870,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 bool staged = false;
                 if constexpr (C::kOutStage && kCols == 128) {
+                    staged = true;
                     if (ga.out_tma) {
                         // four boxes of 32 rows x 32 columns through this warp's two
                         // buffers, written out by TMA stores (whole 64-byte row pieces
                         // instead of one 16-byte piece per row per store instruction)
-                        staged = true;
                         if (q * 32 < ti.valid) {    // a box starts on a row the GEMM writes; rows past M are clipped
 #pragma unroll
                             for (int b = 0; b < 4; ++b) {
@@ -884,6 +884,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     ob[i] = o[16 * b + i];
                                 store_box_staged(sOut + ((warp - 2) * 2 + (b & 1)) * C::kOutBuf, ob, lane, &map_out,
                                                  ti.nt * BN + hf * kCols + b * 32, ti.row0_out + q * 32);
+                            }
+                        }
+                    } else if (q * 32 < ti.valid) {
+                        // grouped tiles: y's rows are compact, so the rows past an m-tile's
+                        // valid ones belong to the next expert and no box may cover them.
+                        // The warp stages 32 rows x 64 columns at a time in its 4 KB
+                        // (16-byte chunk c of row r at c ^ (r & 7): conflict-free both
+                        // ways) and writes them back as 4 rows x 128 bytes per store
+                        // instruction, each lane storing only for a valid row
+                        uint8_t *wbuf = sOut + (warp - 2) * 2 * C::kOutBuf;
+                        __nv_bfloat16 *ybase = ga.out + static_cast<int64_t>(ti.row0_out + q * 32) * ga.ldo +
+                                               static_cast<int64_t>(ti.nt) * BN + hf * kCols;
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            __syncwarp();           // the previous half has been read back
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                *reinterpret_cast<uint4 *>(wbuf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                                    make_uint4(o[32 * h2 + 4 * c], o[32 * h2 + 4 * c + 1], o[32 * h2 + 4 * c + 2],
+                                               o[32 * h2 + 4 * c + 3]);
+                            __syncwarp();
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int r = 4 * j + (lane >> 3), c = lane & 7;
+                                const uint4 v = *reinterpret_cast<const uint4 *>(wbuf + r * 128 + ((c ^ (r & 7)) << 4));
+                                if (q * 32 + r < ti.valid)
+                                    *reinterpret_cast<uint4 *>(ybase + static_cast<int64_t>(r) * ga.ldo + h2 * 64 + c * 8) = v;
                             }
                         }
                     }
