@@ -32,7 +32,10 @@
 //             EPI_SWIGLU_QUANT  h = SiLU(a_g*g) * (a_u*u), NVFP4-quantised
 //                               with the expert's inter_gs (L1),
 //             EPI_SWIGLU_AMAX   same h, max|h| per expert (warmup),
-//             EPI_BF16          y = alpha * acc -> bf16 (L2, dense GEMM).
+//             EPI_BF16          y = alpha * acc -> bf16 (L2, dense GEMM);
+//             pair tiles write bf16 through shared memory: the dense GEMM
+//             as 32 x 32 boxes with TMA stores, the grouped L2 (compact y
+//             rows) as 128-byte row pieces of its valid rows.
 // In the L1 tile the B tile is 128 gate rows stacked on the matching 128 up
 // rows of the stacked [gate; up] weight (two boxes), so TMEM columns 0-127
 // hold gate and 128-255 hold up of the same 128 h columns, and each
