@@ -924,10 +924,12 @@ def _run_all(args, world, rank, dev, peaks, peak_src, steps, warmup):
     torch.cuda.synchronize()
 
     mode = "eager" if args.eager else "timed"
-    ms_pre, stages_pre = time_steps(pre, steps, warmup, world, graph=not args.eager)
+    # decode first: timed right after the prefill it would run in the prefill's
+    # power-cap tail (a decode step alone draws ~300 W and keeps the full clock)
     ms_dec, stages_dec = time_steps(dec, steps, warmup, world, graph=not args.eager)
-    ms_pre_eager, _ = time_steps(pre, steps, warmup, world, graph=False, tag="eager")
     ms_dec_eager, _ = time_steps(dec, steps, warmup, world, graph=False, tag="eager")
+    ms_pre, stages_pre = time_steps(pre, steps, warmup, world, graph=not args.eager)
+    ms_pre_eager, _ = time_steps(pre, steps, warmup, world, graph=False, tag="eager")
     for wl in (pre, dec):
         err = nvfp4_moe_get_error(wl.ws)
         if err != 0:
