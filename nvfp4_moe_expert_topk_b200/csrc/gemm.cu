@@ -90,8 +90,9 @@ struct Cfg {
     static constexpr int kB = kA + kStages * kTileBytes;
     static constexpr int kSFA = kB + kStages * kTileBytes * kBBoxes;
     static constexpr int kSFB = kSFA + kStages * kSFStage;
-    // pair tiles with a bf16 epilogue may store through shared memory: per
-    // epilogue warp two buffers of 32 rows x 32 bf16 columns
+    // pair tiles store their bf16 tiles through shared memory: 4 KB per
+    // epilogue warp, two 2 KB boxes of 32 rows x 32 columns for TMA stores
+    // (dense) or one block of 32 rows x 64 columns (grouped y)
     static constexpr bool kOutStage = CG == 2;
     static constexpr int kOutBuf = 32 * 32 * 2;
     static constexpr int kOut = kSFB + kStages * kSFStage * kHalves;
