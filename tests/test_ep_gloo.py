@@ -1,5 +1,5 @@
-"""Expert parallelism on two gloo ranks (CPU): each rank owns half of the
-experts and its own batch; the dispatch / per-rank experts / combine result
+"""Expert parallelism on gloo ranks (CPU; two ranks, and four for a few
+scenarios): each rank owns an equal share of the experts and its own batch; the dispatch / per-rank experts / combine result
 equals the single-process oracle on the union batch with the union's global
 scale.  The per-rank expert computation here is the oracle (the library runs
 only on a GPU); the exchange logic is the product's (ep.py)."""
@@ -34,12 +34,12 @@ def rank_tokens(r, scenario):
     return CFG.T + 8 * r                                       # ranks hold different batch sizes
 
 
-def rank_batch(r, scenario):
+def rank_batch(r, scenario, world=WORLD):
     T = rank_tokens(r, scenario)
     x = W.activations(T, CFG.H, seed=100 + r)
     ids, w = W.routing(config(scenario), T, seed=200 + r)
     if scenario == "one_sided":                                # every slot on rank 0's experts
-        ids = ids % (CFG.E // WORLD)
+        ids = ids % (CFG.E // world)
     if scenario == "skips":
         ids[::5, 1] = -1                                       # skipped slots travel as -1
     return x, ids, w
@@ -55,13 +55,13 @@ def inter_gs_all(cfg):
     return np.array([O.global_scale_from_amax(a if a > 0 else amax.max()) for a in amax], np.float32)
 
 
-def worker(rank, port, scenario):
+def worker(rank, port, scenario, world=WORLD):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=WORLD)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         cfg = config(scenario)
-        El = CFG.E // WORLD                                    # routed experts per rank
+        El = CFG.E // world                                    # routed experts per rank
         shared = list(range(CFG.E, cfg.E))                     # replicated on every rank
         local = list(range(rank * El, (rank + 1) * El)) + shared
         ow = OracleWeights(cfg, local, "cpu")
@@ -83,11 +83,11 @@ def worker(rank, port, scenario):
 
         ep = ExpertParallelMoE(CFG.E, amax_fn=lambda x: O.amax_bf16(W.bf16_bits(x)), experts_fn=experts_fn,
                                num_shared=len(shared), quantize_fn=quantize_fn if "nvfp4" in scenario else None)
-        x, ids, w = rank_batch(rank, scenario)
+        x, ids, w = rank_batch(rank, scenario, world)
         got = ep.forward(x, ids, w, out_dtype=torch.float32).numpy()
 
         # reference: one process, all experts, the union batch
-        xs, idss, ws = zip(*(rank_batch(r, scenario) for r in range(WORLD)))
+        xs, idss, ws = zip(*(rank_batch(r, scenario, world) for r in range(world)))
         xu, idu, wu = torch.cat(xs), torch.cat(idss), torch.cat(ws)
         gs = global_scale_from_amax(max(O.amax_bf16(W.bf16_bits(xr)) if xr.numel() else 0.0 for xr in xs))
         assert gs == O.global_scale_bf16(W.bf16_bits(xu))
@@ -112,6 +112,13 @@ def free_port():
                                       "nvfp4_shared", "nvfp4_empty_rank"])
 def test_expert_parallel_two_ranks(scenario):
     mp.start_processes(worker, args=(free_port(), scenario), nprocs=WORLD, start_method="spawn")
+
+
+@pytest.mark.parametrize("scenario", ["plain", "nvfp4_shared", "one_sided"])
+def test_expert_parallel_four_ranks(scenario):
+    """Two experts per rank: every token's slots spread over up to four ranks
+    (one_sided: all on rank 0's two experts)."""
+    mp.start_processes(worker, args=(free_port(), scenario, 4), nprocs=4, start_method="spawn")
 
 
 def test_plan_rewrites_ids_per_rank():
