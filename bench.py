@@ -705,6 +705,40 @@ def time_shared_fold(dec, fold_cfg, dev, steps, warmup, hbm_gbs):
             "sm_mhz": CLOCKS.mhz(f"{fold_cfg.name}_folded") if CLOCKS else None}
 
 
+def tma_stream_ceiling(wl):
+    """The GEMM's weight-tile loads alone (nvfp4_tma_stream_ceiling): the
+    prefill workload's stacked W13 codes as the matrix ([E*2I, H/2], 8.5 GB,
+    the HBM read rate of the GEMM's access pattern), then its first 16384 rows
+    (59 MB, L2-resident: the L2 -> shared-memory rate); 4 stages of 32 KB per
+    SM as in the 1-CTA GEMM launch, 6 as a deeper ring."""
+    from nvfp4_moe_expert_topk_b200 import nvfp4_tma_stream_ceiling
+    c = wl.cfg
+    m = wl.weights.w13_codes.view(c.E * 2 * c.I, c.H // 2)
+    rows, row_bytes = m.shape
+    work = rows // 256                                      # one pass over the full matrix
+    err = torch.zeros(1, dtype=torch.int32, device=m.device)
+    res = {"row_bytes": row_bytes, "box": "2 x 128 rows x 128 B per step, 128-byte swizzle"}
+    for name, mat in (("hbm", m), ("l2", m[:16384])):
+        for stages in (4, 6):
+            region = f"tma_stream_{name}_{stages}"
+            nvfp4_tma_stream_ceiling(mat, work, stages, err)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ms = 1e9
+            with clock_region(region):
+                for _ in range(3):
+                    a.record()
+                    nvfp4_tma_stream_ceiling(mat, work, stages, err)
+                    b.record()
+                    torch.cuda.synchronize()
+                    ms = min(ms, a.elapsed_time(b))
+            res[f"{name}_{stages}_stages_gbs"] = work * 256 * row_bytes / (ms * 1e-3) / 1e9
+            res[f"{name}_{stages}_stages_sm_mhz"] = CLOCKS.mhz(region) if CLOCKS else None
+    if err.item() != 0:
+        raise RuntimeError(f"TMA stream probe error word {err.item()}")
+    return res
+
+
 def fp4_ceiling(dev, sms):
     """Tensor-pipe ceiling of the FP4 MMA (nvfp4_fp4_mma_ceiling): one block
     per SM issues k-tiles of four M=128 K=64 MMAs for ~20 ms (long enough to
@@ -940,6 +974,7 @@ def _run_all(args, world, rank, dev, peaks, peak_src, steps, warmup):
     flush = L2Flush(dev)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     ceiling = fp4_ceiling(dev, sms)
+    stream_ceiling = tma_stream_ceiling(pre)
     mla = time_mla_gemms(dev, min(steps, 50), warmup, peaks, flush, ceiling["n256"]["tflops"])
     router = time_router(pre.cfg, dev, 50, warmup, flush)
     pure = time_variant_routing(pre, W.MOE_CONFIGS["prefill_zipf_pure"], min(steps, 50), warmup, world)
@@ -1003,6 +1038,7 @@ def _run_all(args, world, rank, dev, peaks, peak_src, steps, warmup):
                     "decode": timed(ms_dec / steps, r_dec),
                     "decode_eager": timed(ms_dec_eager / steps, f"eager_{dec.cfg.name}")},
         "fp4_mma_ceiling": ceiling,
+        "tma_stream_ceiling": stream_ceiling,
         "mla_gemms": mla,
         "router": router,
         "prefill_pure_zipf": pure,

@@ -302,6 +302,22 @@ int nvfp4_moe_get_error(void *workspace, int32_t *err_host, void *stream);
  * 1 <= iters <= 1 << 24; 1 <= ctas <= 65535. */
 int nvfp4_fp4_mma_ceiling(int bn, int iters, int ctas, int64_t *cycles, int32_t *err, void *stream);
 
+/* Measurement hook, not a step of the method (the pages have no
+ * counterpart): TMA streaming probe.  The GEMM engine's weight-tile loads
+ * alone: one block per SM loads, per step, two 128-row x 128-byte boxes of
+ * the row-major uint8 matrix [rows, row_bytes] (device, 16-byte aligned; one
+ * k-tile of a 256-row weight tile, the GEMM's tensor map) into a `stages`-deep
+ * ring of 32 KB stages that another thread releases as soon as each lands.
+ * work_tiles tiles of 256 rows x row_bytes / 128 steps are dealt round-robin
+ * over the blocks; tile t reads the rows of tile t mod (rows / 256).  Bytes
+ * moved into shared memory = work_tiles * 256 * row_bytes: with a matrix
+ * larger than L2 the rate is the HBM read rate of the GEMM's access pattern,
+ * with a small one the L2 -> shared-memory rate.  Constraints: rows % 256 == 0,
+ * row_bytes % 128 == 0, 2 <= stages <= 6, work_tiles >= 1.  A bounded wait
+ * that gives up writes NVFP4_ERR_TIMEOUT to *err when err is not NULL. */
+int nvfp4_tma_stream_ceiling(const uint8_t *matrix, int64_t rows, int64_t row_bytes, int64_t work_tiles,
+                             int stages, int32_t *err, void *stream);
+
 /* Top-k router: the step that produces topk_ids / topk_weights for
  * nvfp4_moe_forward (page 3 "Architecture Notes": every token is routed to
  * 6 of 384 experts).  The pages name the routing but not the score function;

@@ -19,7 +19,7 @@ __all__ = [
     "nvfp4_moe_forward_timed", "nvfp4_moe_forward_noalloc", "nvfp4_moe_forward_quantized",
     "nvfp4_moe_calibrate", "nvfp4_moe_route_debug", "nvfp4_moe_workspace_region",
     "nvfp4_moe_get_error", "nvfp4_moe_topk", "nvfp4_moe_topk_shared", "NVFP4_SCORING_SOFTMAX",
-    "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_moe_plan", "nvfp4_amax", "nvfp4_debug_bounded_wait",
+    "NVFP4_SCORING_SIGMOID", "nvfp4_fp4_mma_ceiling", "nvfp4_tma_stream_ceiling", "nvfp4_moe_plan", "nvfp4_amax", "nvfp4_debug_bounded_wait",
     "MoeArgs",
 ]
 
@@ -82,6 +82,7 @@ def lib():
         L.nvfp4_amax.argtypes = [P, i64, P, P]
         L.nvfp4_debug_bounded_wait.argtypes = [P, i32, P, P]
         L.nvfp4_fp4_mma_ceiling.argtypes = [i32, i32, i32, P, P, P]
+        L.nvfp4_tma_stream_ceiling.argtypes = [P, i64, i64, i64, i32, P, P]
         L.nvfp4_moe_plan.argtypes = [i64, i32, i32, i64, i64, ctypes.POINTER(ctypes.c_int32),
                                      ctypes.POINTER(ctypes.c_int32)]
         _lib = L
@@ -296,6 +297,16 @@ def nvfp4_fp4_mma_ceiling(bn, iters, cycles, err=None, stream=None):
     _check(lib().nvfp4_fp4_mma_ceiling(bn, iters, cycles.numel(), _dev(cycles, "cycles", torch.int64),
                                        None if err is None else _dev(err, "err", torch.int32), _stream(stream)),
            "nvfp4_fp4_mma_ceiling")
+
+
+def nvfp4_tma_stream_ceiling(matrix, work_tiles, stages=4, err=None, stream=None):
+    """TMA streaming probe over a uint8 CUDA matrix [rows, row_bytes]: moves
+    work_tiles * 256 * row_bytes bytes into shared memory (see
+    nvfp4_tma_stream_ceiling in include/nvfp4moe.h)."""
+    rows, row_bytes = matrix.shape
+    _check(lib().nvfp4_tma_stream_ceiling(_dev(matrix, "matrix", torch.uint8), rows, row_bytes, work_tiles, stages,
+                                          None if err is None else _dev(err, "err", torch.int32), _stream(stream)),
+           "nvfp4_tma_stream_ceiling")
 
 
 def nvfp4_moe_plan(T, k, E, H, I):

@@ -903,6 +903,27 @@ int nvfp4_fp4_mma_ceiling(int bn, int iters, int ctas, int64_t *cycles, int32_t 
                                           static_cast<cudaStream_t>(stream)));
 }
 
+int nvfp4_tma_stream_ceiling(const uint8_t *matrix, int64_t rows, int64_t row_bytes, int64_t work_tiles,
+                             int stages, int32_t *err, void *stream)
+{
+    if (matrix == nullptr || rows < 256 || row_bytes < 128 || work_tiles < 1 || stages < 2)
+        return NVFP4_ERR_INVALID_ARG;
+    if (rows % 256 != 0 || row_bytes % 128 != 0 || stages > 6 || rows >= (1LL << 31) || row_bytes >= (1LL << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(matrix))
+        return NVFP4_ERR_MISALIGNED;
+    int sms = 0;
+    int st = device_check(&sms);
+    if (st != NVFP4_OK)
+        return st;
+    CUtensorMap map;
+    st = make_code_map(&map, matrix, rows, row_bytes, 128);
+    if (st != NVFP4_OK)
+        return st;
+    return cuda_status(launch_tma_stream(map, rows, row_bytes, work_tiles, stages, sms, err,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 int nvfp4_moe_get_error(void *workspace, int32_t *err_host, void *stream)
 {
     if (workspace == nullptr || err_host == nullptr)

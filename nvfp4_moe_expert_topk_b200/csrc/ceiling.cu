@@ -100,7 +100,110 @@ __global__ void __launch_bounds__(kCeilThreads, 1)
     (void)lane;
 }
 
+// TMA streaming probe: the GEMM engine's B-operand loads with nothing else.
+// One CTA per SM; one thread loads, per step, two 128-row x 128-byte boxes
+// (one k-tile of a 256-row weight tile, the map's 128-byte swizzle) into a
+// `stages`-deep ring of 32 KB stages, and another thread releases each stage
+// as soon as it has landed.  Tiles of 256 rows x (row_bytes / 128) steps are
+// dealt round-robin; tile t reads rows of tile t mod (rows / 256), so a matrix
+// larger than L2 measures the HBM read rate and a small one the L2 ->
+// shared-memory rate.
+constexpr int kStreamThreads = 64;
+constexpr int kStreamStage = 2 * 128 * 128;
+
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    tma_stream_kernel(const __grid_constant__ CUtensorMap map, int64_t work_tiles, int64_t tiles, int ksteps,
+                      int stages, int32_t *err)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + stages * kStreamStage);
+    uint64_t *empty = full + stages;
+    __shared__ int abort_flag;
+    __shared__ int never_abort;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        abort_flag = 0;
+        never_abort = 0;
+        fence_mbar_init();
+        tma_prefetch_map(&map);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int stage = 0;
+        uint32_t phase = 0, pend = 0, pend_par = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < work_tiles && ok; t += gridDim.x) {
+            const int64_t row0 = (t % tiles) * 256;
+            for (int k = 0; k < ksteps; ++k) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, &abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full[stage], kStreamStage);
+                for (int h = 0; h < 2; ++h)
+                    tma_load_2d(smem + stage * kStreamStage + h * (kStreamStage / 2), &map, k * 128,
+                                static_cast<int32_t>(row0 + 128 * h), &full[stage]);
+                pend |= 1u << stage;
+                pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
+                if (++stage == stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok) {
+            abort_flag = 1;
+            if (err != nullptr)
+                atomicCAS(err, 0, NVFP4_ERR_TIMEOUT);
+        }
+        for (int s = 0; s < stages; ++s)           // every copy has landed before the block exits
+            if ((pend >> s) & 1u)
+                mbar_wait(&full[s], (pend_par >> s) & 1u, &never_abort);
+    } else if (threadIdx.x == 32) {
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < work_tiles && ok; t += gridDim.x) {
+            for (int k = 0; k < ksteps; ++k) {
+                if (!mbar_wait(&full[stage], phase, &abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive(&empty[stage]);
+                if (++stage == stages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok) {
+            abort_flag = 1;
+            if (err != nullptr)
+                atomicCAS(err, 0, NVFP4_ERR_TIMEOUT);
+        }
+    }
+    __syncthreads();
+}
+
 } // namespace
+
+cudaError_t launch_tma_stream(const CUtensorMap &map, int64_t rows, int64_t row_bytes, int64_t work_tiles,
+                              int stages, int ctas, int32_t *err, cudaStream_t s)
+{
+    auto smem_of = [](int n) { return n * kStreamStage + 2 * n * 8 + 1024; };
+    const int smem = smem_of(stages);
+    static unsigned long long attr_done = 0;     // one bit per device; the limit allows the deepest ring
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(tma_stream_kernel), smem_of(6), &attr_done);
+    if (e != cudaSuccess)
+        return e;
+    tma_stream_kernel<<<ctas, kStreamThreads, smem, s>>>(map, work_tiles, rows / 256,
+                                                         static_cast<int>(row_bytes / 128), stages, err);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_mma_ceiling(int bn, int iters, int ctas, long long *cycles, int32_t *err, cudaStream_t s)
 {

@@ -174,6 +174,10 @@ cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *yrow, const fl
                            __nv_bfloat16 *out, cudaStream_t s);
 cudaError_t launch_finalize_inter_gs(const unsigned int *amax_bits, int E, float *inter_gs, cudaStream_t s);
 cudaError_t launch_mma_ceiling(int bn, int iters, int ctas, long long *cycles, int32_t *err, cudaStream_t s);
+// TMA streaming probe (ceiling.cu): map = the GEMM's 128-row B-box map over
+// a [rows, row_bytes] uint8 matrix (rows % 256 == 0, row_bytes % 128 == 0).
+cudaError_t launch_tma_stream(const CUtensorMap &map, int64_t rows, int64_t row_bytes, int64_t work_tiles,
+                              int stages, int ctas, int32_t *err, cudaStream_t s);
 cudaError_t launch_topk(const float *logits, int64_t T, int E, int k, int ns, int scoring, int32_t *ids,
                         float *weights, cudaStream_t s);
 

@@ -155,6 +155,15 @@ def test_ceiling_checks(L):
     assert L.nvfp4_fp4_mma_ceiling(192, 10, 148, F, None, None) == -1
     assert L.nvfp4_fp4_mma_ceiling(256, 0, 148, F, None, None) == -1
     assert L.nvfp4_fp4_mma_ceiling(256, (1 << 24) + 1, 148, F, None, None) == -2
+    # TMA streaming probe: shape and alignment checks before any device work
+    assert L.nvfp4_tma_stream_ceiling(None, 256, 128, 1, 4, None, None) == -1
+    assert L.nvfp4_tma_stream_ceiling(F, 128, 128, 1, 4, None, None) == -1        # rows < 256
+    assert L.nvfp4_tma_stream_ceiling(F, 256, 128, 0, 4, None, None) == -1        # no work
+    assert L.nvfp4_tma_stream_ceiling(F, 256, 128, 1, 1, None, None) == -1        # stages < 2
+    assert L.nvfp4_tma_stream_ceiling(F, 384, 128, 1, 4, None, None) == -2        # rows % 256
+    assert L.nvfp4_tma_stream_ceiling(F, 256, 192, 1, 4, None, None) == -2        # row_bytes % 128
+    assert L.nvfp4_tma_stream_ceiling(F, 256, 128, 1, 7, None, None) == -2        # stages > 6
+    assert L.nvfp4_tma_stream_ceiling(ctypes.c_void_p((1 << 40) + 8), 256, 128, 1, 4, None, None) == -3
 
 
 def test_moe_plan(L):
