@@ -66,14 +66,19 @@ def load_peaks():
 
 
 def gemm_source_sha():
-    """Hash of the GEMM sources' code, comments and layout whitespace removed
-    (a comment edit does not invalidate the captured traffic)."""
+    """Hash of the GEMM kernels' code: gemm.cu, ptx.cuh, quant.cuh and, of
+    internal.h, the GemmArgs struct the kernels take; comments and layout
+    whitespace removed (a comment edit, or a declaration of another kernel in
+    internal.h, does not invalidate the captured traffic)."""
     h = hashlib.sha256()
     for name in GEMM_SOURCES:
         with open(os.path.join(ROOT, "nvfp4_moe_expert_topk_b200", "csrc", name)) as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
         text = re.sub(r"//[^\n]*", "", text)
+        if name == "internal.h":
+            m = re.search(r"struct GemmArgs \{.*?\n\};", text, flags=re.S)
+            text = m.group(0) if m else text
         h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
