@@ -223,10 +223,9 @@ constexpr int64_t kSplitMinRows = 2048;
 // at once; the 1-CTA launch claims tiles, so CTAs that start late just take
 // fewer).  Measured on the B200 (prefill, CTA start / end stamps): running the
 // pair launch on fewer clusters beside the 1-CTA launch gains nothing -- with
-// both resident, the two compete for the same L2 -> shared-memory fill and the
-// pair of launches takes as long as one after the other (2.56 against 2.58 ms
-// with two streams; as a dependent launch the second kernel's resident CTAs
-// made no progress until the first kernel ended).
+// both resident the pair of launches takes as long as one after the other
+// (2.56 against 2.58 ms with two streams; as a dependent launch the second
+// kernel's resident CTAs made no progress until the first kernel ended).
 
 int gemm_grid(int cg, int64_t tiles, int num_sms)
 {
@@ -534,8 +533,8 @@ namespace {
 // the tiles are 256 wide, dealt round-robin over the resident units.  (A
 // stream-K split of the (tile, k-tile) iterations was measured against this
 // once the pair tiles stored their output through TMA: it lost on every shape
-// tried, since the launch is bound by the operand fill from L2 and a partial
-// last round runs its few tiles at a higher fill rate per SM.)
+// tried: a partial last round runs its few tiles faster per SM than a full
+// one, which the split's partial-sum traffic and waits do not beat.)
 struct DensePlan {
     int bn, cg, grid;
 };
