@@ -124,3 +124,19 @@ def test_clock_regions_summarise_only_their_samples():
     assert both["samples"] == 3 and both["sm_max_mhz"] == 1965.0
     t = bench.compact({"x": 3.14159265, "y": [2.718281828], "z": "s", "n": 7})
     assert t == {"x": 3.142, "y": [2.718], "z": "s", "n": 7}
+
+
+
+def test_source_hash_ignores_other_declarations_not_gemm_args(tmp_path, monkeypatch):
+    """Of internal.h only the GemmArgs struct the kernels take counts: a new
+    declaration of another kernel keeps the key, a GemmArgs field changes it."""
+    root, csrc = _copy_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h0 = bench.gemm_source_sha()
+    ih = csrc / "internal.h"
+    text = ih.read_text()
+    assert "struct GemmArgs {" in text
+    ih.write_text(text.replace("namespace nvfp4 {", "namespace nvfp4 {\nint another_kernel_launch(int n);", 1))
+    assert bench.gemm_source_sha() == h0
+    ih.write_text(text.replace("struct GemmArgs {", "struct GemmArgs {\n    int extra_field;", 1))
+    assert bench.gemm_source_sha() != h0
