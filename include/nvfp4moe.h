@@ -121,7 +121,9 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *a_g
  * "Architecture Notes" routing).  Shapes: T tokens, hidden H, expert
  * intermediate I, E experts, top-k.
  * Constraints: T >= 0, H % 128 == 0, I % 128 == 0, 1 <= E <= 1024,
- * 1 <= k <= 32, T*k < 2^31.  All pointers 16-B aligned. */
+ * 1 <= k <= 32, T*k < 2^31.  All pointers 16-B aligned.  With T = 0 the
+ * batch's pointers (x, x_gs when it is required, topk_ids, topk_weights,
+ * out) may be NULL: nothing of the batch is read or written. */
 typedef struct {
     const uint16_t *x;            /* [T, H] bf16 activations                          */
     int64_t T, H, I;

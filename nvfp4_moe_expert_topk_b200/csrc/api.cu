@@ -170,18 +170,25 @@ int check_moe_args(const nvfp4_moe_args *a, bool need_out, bool need_x = true)
     int st = check_moe_shape(a->T, a->k, a->E, a->H, a->I);
     if (st != NVFP4_OK)
         return st;
-    const void *ptrs[] = {need_x ? static_cast<const void *>(a->x) : static_cast<const void *>(a->x_gs), a->topk_ids, a->topk_weights, a->w13_codes, a->w13_scales,
-                          a->w13_gs, a->w2_codes, a->w2_scales, a->w2_gs};
-    for (const void *p : ptrs)
+    // an empty batch (T = 0) reads and writes nothing of the batch: its
+    // pointers (x or x_gs, topk_ids, topk_weights, out) may then be NULL
+    const bool batch = a->T > 0;
+    const void *batch_ptrs[] = {need_x ? static_cast<const void *>(a->x) : static_cast<const void *>(a->x_gs),
+                                a->topk_ids, a->topk_weights};
+    for (const void *p : batch_ptrs)
+        if (batch && p == nullptr)
+            return NVFP4_ERR_INVALID_ARG;
+    const void *weight_ptrs[] = {a->w13_codes, a->w13_scales, a->w13_gs, a->w2_codes, a->w2_scales, a->w2_gs};
+    for (const void *p : weight_ptrs)
         if (p == nullptr)
             return NVFP4_ERR_INVALID_ARG;
-    if (need_out && (a->out == nullptr || a->inter_gs == nullptr))
+    if (need_out && ((batch && a->out == nullptr) || a->inter_gs == nullptr))
         return NVFP4_ERR_INVALID_ARG;
-    const void *al[] = {need_x ? static_cast<const void *>(a->x) : static_cast<const void *>(a->w13_codes), a->w13_codes, a->w13_scales, a->w2_codes, a->w2_scales};
+    const void *al[] = {a->w13_codes, a->w13_scales, a->w2_codes, a->w2_scales};
     for (const void *p : al)
         if (!aligned16(p))
             return NVFP4_ERR_MISALIGNED;
-    if (need_out && !aligned16(a->out))
+    if (batch && ((need_x && !aligned16(a->x)) || (need_out && !aligned16(a->out))))
         return NVFP4_ERR_MISALIGNED;
     return NVFP4_OK;
 }
@@ -674,7 +681,7 @@ static int moe_forward_impl(const nvfp4_moe_args *a, void *workspace, size_t ws_
     int st = check_moe_args(a, true, xq_codes == nullptr);
     if (st != NVFP4_OK)
         return st;
-    if (xq_codes != nullptr && (!aligned16(xq_codes) || !aligned16(xq_scales)))
+    if (a->T > 0 && xq_codes != nullptr && (!aligned16(xq_codes) || !aligned16(xq_scales)))
         return NVFP4_ERR_MISALIGNED;
     if (workspace == nullptr)
         return NVFP4_ERR_INVALID_ARG;
@@ -783,7 +790,7 @@ int nvfp4_moe_forward(const nvfp4_moe_args *a, void *workspace, size_t ws_bytes,
 int nvfp4_moe_forward_quantized(const nvfp4_moe_args *a, const uint8_t *x_codes, const uint8_t *x_scales,
                                 void *workspace, size_t ws_bytes, void *stream)
 {
-    if (x_codes == nullptr || x_scales == nullptr)
+    if (a == nullptr || (a->T > 0 && (x_codes == nullptr || x_scales == nullptr)))
         return NVFP4_ERR_INVALID_ARG;
     return moe_forward_impl(a, workspace, ws_bytes, stream, nullptr, x_codes, x_scales);
 }

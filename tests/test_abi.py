@@ -129,6 +129,16 @@ def test_moe_forward_checks(L):
     a.x_gs = None
     assert L.nvfp4_moe_forward_quantized(ctypes.byref(a), ctypes.c_void_p(F), ctypes.c_void_p(F),
                                          ctypes.c_void_p(F), 1 << 40, None) == -1
+    # an empty batch: its pointers may be NULL (the checks pass; without a GPU the
+    # call then stops at the device check), the weights' may not
+    a.T = 0
+    a.x = a.topk_ids = a.topk_weights = a.x_gs = a.out = None
+    no_device = L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None)
+    assert no_device not in (-1, -2, -3, -4), no_device
+    assert L.nvfp4_moe_forward_quantized(ctypes.byref(a), None, None, ctypes.c_void_p(F), 1 << 40,
+                                         None) == no_device
+    a.w13_codes = None
+    assert L.nvfp4_moe_forward(ctypes.byref(a), ctypes.c_void_p(F), 1 << 40, None) == -1
 
 
 def test_topk_checks(L):

@@ -621,3 +621,32 @@ def test_cuda_graph_replay_split_plan_with_new_inputs():
         ref = O.moe_forward(xb, ids2.numpy(), p.w.numpy(), O.global_scale_bf16(xb), **p.ow.oracle_kwargs(),
                             inter_gs=p.inter_gs)
         check_output(out, ref)
+
+
+def test_empty_batch_runs_nothing():
+    """T = 0 through the Python API: the forward, the pre-quantised forward
+    and the calibration accept empty tensors (NULL batch pointers); the
+    forward writes nothing and sets no error, and the calibration of an
+    empty warmup batch gives every expert the global scale of amax = 0."""
+    from nvfp4_moe_expert_topk_b200 import nvfp4_moe_calibrate, nvfp4_moe_forward_quantized, prep
+    cfg = W.MOE_CONFIGS["tiny"]
+    p = Problem(cfg)
+    inputs = p.device_inputs()
+    H = cfg.H
+    ws = prep.workspace(0, cfg.k, cfg.E, H, cfg.I, DEV)
+    x0 = torch.empty(0, H, dtype=torch.bfloat16, device=DEV)
+    ids0 = torch.empty(0, cfg.k, dtype=torch.int32, device=DEV)
+    w0 = torch.empty(0, cfg.k, dtype=torch.float32, device=DEV)
+    out0 = torch.empty(0, H, dtype=torch.bfloat16, device=DEV)
+    args = {k: v for k, v in inputs.items() if k not in ("x", "topk_ids", "topk_weights", "x_gs")}
+    nvfp4_moe_forward(x0, ids0, w0, None, **args, out=out0, workspace=ws)
+    x_gs = torch.ones(1, dtype=torch.float32, device=DEV)
+    nvfp4_moe_forward_quantized(torch.empty(0, H // 2, dtype=torch.uint8, device=DEV),
+                                torch.empty(0, H // 16, dtype=torch.uint8, device=DEV), ids0, w0, x_gs, **args,
+                                out=out0, workspace=ws)
+    igs = torch.full((cfg.E,), -1.0, dtype=torch.float32, device=DEV)
+    cal = {k: v for k, v in args.items() if k != "inter_gs"}
+    nvfp4_moe_calibrate(x0, ids0, w0, x_gs, **cal, inter_gs_out=igs, workspace=ws)
+    torch.cuda.synchronize()
+    assert nvfp4_moe_get_error(ws) == 0
+    assert bool((igs == float(O.global_scale_from_amax(0.0))).all()), igs
