@@ -650,3 +650,32 @@ def test_empty_batch_runs_nothing():
     torch.cuda.synchronize()
     assert nvfp4_moe_get_error(ws) == 0
     assert bool((igs == float(O.global_scale_from_amax(0.0))).all()), igs
+
+
+def random_config(seed):
+    """A small MoE shape drawn from the seed: 2-40 experts, top-1..8, 1-1024
+    tokens, H in 128..512, I in 128..384, softmax or Zipf routing (some
+    experts empty), with or without outlier channels.  Large enough batches
+    reach the pair plans (R >= 2048, or R >= 256 E with H % 256 == 0), H not
+    a multiple of 256 the two-launch plan."""
+    rng = np.random.default_rng(1000 + seed)
+    E = int(rng.integers(2, 41))
+    k = int(rng.integers(1, min(8, E) + 1))
+    T = int(rng.choice([1, 7, 64, 129, 300, 600, 1024]))
+    H = int(rng.choice([128, 256, 256, 384, 512, 512]))
+    I = int(rng.choice([128, 256, 384]))
+    routing = str(rng.choice(["softmax", "zipf"]))
+    tail = int(min(2, E - k))
+    return W.MoeConfig(f"random{seed}", E=E, k=k, T=T, H=H, I=I, routing=routing, outliers=bool(rng.integers(2)),
+                       warmup_T=64, zipf_zero_tail=tail)
+
+
+@pytest.mark.parametrize("seed", range(48))
+def test_random_configs_match_oracle(seed):
+    """Every output row of a randomly drawn small config against the oracle,
+    whatever plan the forward picks for it."""
+    cfg = random_config(seed)
+    p = Problem(cfg)
+    out, ws = p.run()
+    assert nvfp4_moe_get_error(ws) == 0
+    check_output(out, p.oracle())
