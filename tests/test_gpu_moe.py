@@ -679,3 +679,26 @@ def test_random_configs_match_oracle(seed):
     out, ws = p.run()
     assert nvfp4_moe_get_error(ws) == 0
     check_output(out, p.oracle())
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_random_configs_with_shared_experts_and_skipped_slots(seed):
+    """Seeded random configs with one or two shared experts folded in (the
+    last slots, weight 1) and about a fifth of the routed slots skipped
+    (id -1): every output row against the oracle."""
+    base = random_config(100 + seed)
+    rng = np.random.default_rng(500 + seed)
+    shared = int(rng.integers(1, 3))
+    cfg = W.MoeConfig(f"random_shared{seed}", E=base.E + shared, k=base.k + shared, T=base.T, H=base.H, I=base.I,
+                      routing="softmax", outliers=base.outliers, warmup_T=64, shared=shared)
+    p = Problem(cfg)
+    ids = p.ids.clone()
+    skip = torch.from_numpy(rng.random((ids.shape[0], cfg.k - shared)) < 0.2)
+    ids[:, :cfg.k - shared][skip] = -1
+    inputs = p.device_inputs()
+    inputs["topk_ids"] = ids.to(DEV)
+    out, ws = p.run(inputs)
+    ref = O.moe_forward(W.bf16_bits(p.x), p.ow.remap_ids(ids.numpy()), p.w.numpy(), p.x_gs,
+                        **p.ow.oracle_kwargs(), inter_gs=p.inter_gs[p.ow.experts])
+    assert nvfp4_moe_get_error(ws) == 0
+    check_output(out, ref)
