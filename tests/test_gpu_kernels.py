@@ -146,3 +146,52 @@ def test_route_skipped_and_bad_ids():
     np.testing.assert_array_equal(inv.cpu().numpy(), ref["pos_padded"])
     assert nvfp4_moe_get_error(ws) == -8          # NVFP4_ERR_BAD_EXPERT_ID, sticky until read
     assert nvfp4_moe_get_error(ws) == 0           # read clears it
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_route_random_shapes(seed):
+    """Seeded random E (1-1024), k (1-min(32, E)), T (1-5000) with about a
+    tenth of the slots skipped (-1) and, every fourth seed, Zipf-like skew:
+    counts, padded offsets and every slot's padded row bit-exact."""
+    rng = np.random.default_rng(5000 + seed)
+    E = int(rng.integers(1, 1025))
+    k = int(rng.integers(1, min(32, E) + 1))
+    T = int(rng.integers(1, 5001))
+    if seed % 4 == 0:
+        p = 1.0 / np.arange(1, E + 1) ** 1.2
+        ids = rng.choice(E, size=(T, k), p=p / p.sum()).astype(np.int32)
+    else:
+        ids = rng.integers(0, E, (T, k)).astype(np.int32)
+    ids[rng.random((T, k)) < 0.1] = -1
+    ref = O.route(ids, E)
+    ws = prep.workspace(T, k, E, 128, 128, DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    poff = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    nvfp4_moe_route_debug(torch.from_numpy(ids).to(DEV), E, counts, poff, inv, ws)
+    np.testing.assert_array_equal(counts.cpu().numpy(), ref["counts"])
+    np.testing.assert_array_equal(poff.cpu().numpy(), ref["padded_offsets"])
+    np.testing.assert_array_equal(inv.cpu().numpy(), ref["pos_padded"])
+    assert nvfp4_moe_get_error(ws) == 0
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_quantize_random_shapes(seed):
+    """Seeded random rows (1-700) and columns (a multiple of 64 up to 8192) of
+    special values, both scale layouts: codes and scales bit-exact."""
+    rng = np.random.default_rng(6000 + seed)
+    rows = int(rng.integers(1, 701))
+    cols = 64 * int(rng.integers(1, 129))
+    x = special_matrix(rows, cols, 7000 + seed)
+    bits = W.bf16_bits(x)
+    gs = O.global_scale_bf16(bits)
+    want_c, want_s = O.quantize_bf16(bits, gs)
+    xd, g = x.to(DEV), torch.tensor([gs], device=DEV)
+    codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=DEV)
+    scales = torch.empty(rows, cols // 16, dtype=torch.uint8, device=DEV)
+    nvfp4_quantize(xd, g, codes, scales, NVFP4_SCALES_ROWMAJOR)
+    np.testing.assert_array_equal(codes.cpu().numpy(), want_c)
+    np.testing.assert_array_equal(scales.cpu().numpy(), want_s)
+    mma = torch.zeros(nvfp4_scales_bytes(rows, cols, NVFP4_SCALES_MMA), dtype=torch.uint8, device=DEV)
+    nvfp4_quantize(xd, g, codes, mma, NVFP4_SCALES_MMA)
+    np.testing.assert_array_equal(from_mma_layout(mma.cpu().numpy(), rows, cols), want_s)

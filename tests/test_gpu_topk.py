@@ -125,3 +125,19 @@ def test_topk_shared_feeds_forward():
     p.ids, p.w = ids.cpu(), w.cpu()
     out, _ = p.run()
     check_output(out, p.oracle())
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_topk_random_shapes(seed):
+    """Seeded random T (1-2000), E (1-1024), k (1-min(32, E)), scoring and
+    logit scale, a quarter of the logits quantised to a coarse grid so that
+    ties occur: ids bit-exact, weights within the bound."""
+    rng = np.random.default_rng(4000 + seed)
+    E = int(rng.integers(1, 1025))
+    k = int(rng.integers(1, min(32, E) + 1))
+    T = int(rng.integers(1, 2001))
+    scoring = str(rng.choice(["softmax", "sigmoid"]))
+    logits = rng.normal(0, float(rng.choice([0.3, 1.5, 6.0])), (T, E)).astype(np.float32)
+    coarse = rng.random((T, E)) < 0.25
+    logits[coarse] = np.round(logits[coarse] * 2) / 2
+    check(logits, k, scoring)
