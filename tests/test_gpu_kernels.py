@@ -195,3 +195,30 @@ def test_quantize_random_shapes(seed):
     mma = torch.zeros(nvfp4_scales_bytes(rows, cols, NVFP4_SCALES_MMA), dtype=torch.uint8, device=DEV)
     nvfp4_quantize(xd, g, codes, mma, NVFP4_SCALES_MMA)
     np.testing.assert_array_equal(from_mma_layout(mma.cpu().numpy(), rows, cols), want_s)
+
+
+@pytest.mark.parametrize("rows,cols,ldx", [(37, 256, 264), (130, 1024, 1536), (5, 64, 72)])
+def test_quantize_strided_rows(rows, cols, ldx):
+    """The C ABI's ldx > cols: x is a [rows, cols] window of a wider bf16
+    buffer (the columns past cols hold huge values that must not enter any
+    block's amax); codes and scales equal the contiguous window's, bit for bit."""
+    import ctypes
+    from nvfp4_moe_expert_topk_b200 import lib
+    x = special_matrix(rows, cols, rows + cols)
+    bits = W.bf16_bits(x)
+    gs = O.global_scale_bf16(bits)
+    want_c, want_s = O.quantize_bf16(bits, gs)
+    wide = torch.full((rows, ldx), 30000.0, dtype=torch.bfloat16)
+    wide[:, :cols] = x
+    wd = wide.to(DEV)
+    g = torch.tensor([gs], device=DEV)
+    codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=DEV)
+    scales = torch.empty(rows, cols // 16, dtype=torch.uint8, device=DEV)
+    P = ctypes.c_void_p
+    st = lib().nvfp4_quantize(P(wd.data_ptr()), rows, cols, ldx, P(g.data_ptr()), P(codes.data_ptr()),
+                              P(scales.data_ptr()), NVFP4_SCALES_ROWMAJOR,
+                              P(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert st == 0
+    np.testing.assert_array_equal(codes.cpu().numpy(), want_c)
+    np.testing.assert_array_equal(scales.cpu().numpy(), want_s)
