@@ -241,7 +241,8 @@ cudaError_t ensure_smem_limit(const void *kernel, int bytes, unsigned long long 
 // out[t] = bf16( sum_{j ascending} w[t,j] * y[yrow[t*k+j]] ) in fp32, where
 // yrow is the slot's row in the unpadded expert-major y buffer (-1: skipped).
 // One block per (token, 2048-column chunk); each thread owns 8 columns (16
-// bytes) and issues the loads of four slots before accumulating them in order.
+// bytes) and issues the loads of up to eight slots before accumulating them in
+// order.
 constexpr int kCombineThreads = 256;
 constexpr int kCombineCols = 8 * kCombineThreads;
 
@@ -267,15 +268,15 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __nv_bfl
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             acc[i] = 0.0f;
-        for (int j0 = 0; j0 < k; j0 += 4) {
-            uint4 v[4];
+        for (int j0 = 0; j0 < k; j0 += 8) {
+            uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int64_t row = j0 + u < k ? s_row[j0 + u] : -1;
                 v[u] = row >= 0 ? __ldg(reinterpret_cast<const uint4 *>(y + row * H + c)) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 if (j0 + u >= k || s_row[j0 + u] < 0)
                     continue;
                 const float wj = s_w[j0 + u];
