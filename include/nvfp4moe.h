@@ -171,7 +171,8 @@ int nvfp4_moe_forward(const nvfp4_moe_args *args, void *workspace, size_t ws_byt
  * a rank quantises its tokens once and sends 4-bit rows (H/2 + H/16 bytes
  * each) to the ranks owning their experts.  x_codes [T, H/2] and x_scales
  * [T, H/16] (NVFP4_SCALES_ROWMAJOR, as nvfp4_quantize writes them), both
- * 16-byte aligned, quantised with the global scale args->x_gs (required);
+ * 16-byte aligned (NULL allowed only when T = 0), quantised with the global
+ * scale args->x_gs (required when T > 0);
  * args->x is not read (may be NULL).  The front launch copies each row to its
  * slots' padded rows instead of quantising it; everything else is
  * nvfp4_moe_forward, so given the codes nvfp4_quantize makes from x with
@@ -194,7 +195,8 @@ int nvfp4_moe_forward_timed(const nvfp4_moe_args *args, void *workspace, size_t 
 /* Warmup (page 1 "Phase 1": warmup-based gs; page 2 "Option A": compute the
  * scale from a warmup pass): runs the chain up to h on args (a warmup batch;
  * inter_gs and out are ignored) and writes inter_gs_out[e] = 2688 / max|h|
- * over expert e's rows; experts without rows get 2688 / (max over experts).
+ * over expert e's rows; experts without rows get 2688 / (max over experts),
+ * and every expert 1.0 when no expert has a row (e.g. T = 0).
  * inter_gs_out: device [E]. */
 int nvfp4_moe_calibrate(const nvfp4_moe_args *args, float *inter_gs_out, void *workspace,
                         size_t ws_bytes, void *stream);
