@@ -234,3 +234,40 @@ def test_random_dense_shapes_match_oracle(seed):
     assert np.all(np.isfinite(out))
     assert row_rel_l2(out, ref).max() <= 5e-3
     assert cosine(out, ref) >= 0.99999
+
+
+def test_gemm_in_cuda_graph_with_new_inputs():
+    """nvfp4_gemm (pair tiles with staged TMA stores: the output's tensor map
+    is a launch parameter) captured once in a CUDA graph; replayed after new
+    operands are copied into the captured buffers, it equals an eager call on
+    those operands bit for bit."""
+    M, N, K, segs = 300, 1024, 512, [512, 1024]
+    first = quantized_operands(M, N, K, 11, segs)
+    second = quantized_operands(M, N, K, 12, segs)
+
+    def dev(ops):
+        ac, asc, a_gs, bc, bsc, bgs = ops
+        return [torch.from_numpy(ac).to(DEV), torch.from_numpy(to_mma_layout(asc)).to(DEV),
+                torch.tensor([a_gs], dtype=torch.float32, device=DEV), torch.from_numpy(bc).to(DEV),
+                torch.from_numpy(to_mma_layout(bsc)).to(DEV), torch.tensor(np.asarray(bgs, np.float32), device=DEV)]
+
+    bufs = dev(first)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device=DEV)
+    nvfp4_gemm(*bufs, segs, out)                      # eager call first (kernel attributes)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            nvfp4_gemm(*bufs, segs, out, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    for b, n in zip(bufs, dev(second)):
+        b.copy_(n)
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    ref = torch.empty_like(out)
+    nvfp4_gemm(*dev(second), segs, ref)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
